@@ -1,0 +1,131 @@
+"""fp64 CPU oracle for Sketch Attention -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s ``cpu_baseline`` /
+``--impl reference`` legs may import this package. The CUDA library never calls it
+and shares no code with it; the product path fails loudly when its CUDA extension
+is missing instead of falling back here.
+
+What it computes is written out in ``sa_oracle.cpp`` (plain C++, fp64, the
+unfolded definition K = X W_k, V = X W_v, prototype-wise softmax, mass-weighted
+mean). Sources: the "100,000 videos in your pocket" blog, section "1. Sketch
+Attention compresses the history"; the evolve.pub review of arXiv 2609.08443,
+"Summary" and the FAQ on how Sketch Attention differs from standard attention.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(closed forms, invariants, brute force at 50 digits, autograd and finite
+differences for the backward). The paper's analytic FLOP ratios (49.9x, 63.9x)
+are not computed here: parity unpinned, context only.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "sa_oracle.cpp")
+_LIB = os.path.join(_HERE, "libsa_oracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with g++ (OpenMP). Returns the path of the shared object."""
+    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
+        return _LIB
+    tmp = _LIB + f".tmp{os.getpid()}"
+    cmd = ["g++", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c++17", "-o", tmp, _SRC]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            # SA_ORACLE_LIB lets the mutation test load a deliberately broken build.
+            lib = ctypes.CDLL(os.environ.get("SA_ORACLE_LIB") or build())
+            dp = ctypes.POINTER(ctypes.c_double)
+            ip = ctypes.POINTER(ctypes.c_int64)
+            lib.sa_oracle_forward.restype = ctypes.c_int
+            lib.sa_oracle_forward.argtypes = [dp, ip, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                              dp, ctypes.c_int, dp, dp, dp, dp, dp, dp, ctypes.c_int]
+            lib.sa_oracle_backward.restype = ctypes.c_int
+            lib.sa_oracle_backward.argtypes = [dp, ip, ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                               dp, ctypes.c_int, dp, dp, dp, dp,
+                                               dp, dp, dp, dp, ctypes.c_int]
+            _lib = lib
+    return _lib
+
+
+def _f64(a) -> np.ndarray:
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _ptr(a: np.ndarray | None, ctype=ctypes.c_double):
+    if a is None:
+        return None
+    return a.ctypes.data_as(ctypes.POINTER(ctype))
+
+
+def _check_rc(rc: int) -> None:
+    if rc == 1:
+        raise ValueError("oracle: bad sizes")
+    if rc == 2:
+        raise ValueError("oracle: offsets must start at 0, be non-decreasing and end at n_total")
+    if rc != 0:
+        raise RuntimeError(f"oracle: error {rc}")
+
+
+def forward(X, offsets, P, Wk, Wv, nthreads: int = 0) -> dict:
+    """Sketch Attention forward in fp64.
+
+    X [n_total, d], offsets [R+1] (int64), P [k, d], Wk [d, d], Wv [d, d].
+    Returns a dict with sketch [R, k, d], mass [R, k], lse [n_total], xsketch [R, k, d].
+    """
+    X = _f64(X)
+    P, Wk, Wv = _f64(P), _f64(Wk), _f64(Wv)
+    off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int64))
+    n_total, d = X.shape
+    k = P.shape[0]
+    R = off.shape[0] - 1
+    assert P.shape == (k, d) and Wk.shape == (d, d) and Wv.shape == (d, d)
+    sketch = np.zeros((R, k, d))
+    mass = np.zeros((R, k))
+    lse = np.zeros(n_total)
+    xsk = np.zeros((R, k, d))
+    rc = _load().sa_oracle_forward(_ptr(X), _ptr(off, ctypes.c_int64), R, n_total, d, _ptr(P), k,
+                                   _ptr(Wk), _ptr(Wv), _ptr(sketch), _ptr(mass), _ptr(lse),
+                                   _ptr(xsk), int(nthreads))
+    _check_rc(rc)
+    return {"sketch": sketch, "mass": mass, "lse": lse, "xsketch": xsk}
+
+
+def backward(X, offsets, P, Wk, Wv, dsketch, dmass=None, nthreads: int = 0) -> dict:
+    """Gradients of L given dL/dsketch [R, k, d] and optional dL/dmass [R, k].
+
+    Returns dX [n_total, d] and dP [k, d], dWk [d, d], dWv [d, d] summed over users.
+    """
+    X = _f64(X)
+    P, Wk, Wv = _f64(P), _f64(Wk), _f64(Wv)
+    G = _f64(dsketch)
+    Gm = None if dmass is None else _f64(dmass)
+    off = np.ascontiguousarray(np.asarray(offsets, dtype=np.int64))
+    n_total, d = X.shape
+    k = P.shape[0]
+    R = off.shape[0] - 1
+    assert G.shape == (R, k, d)
+    assert Gm is None or Gm.shape == (R, k)
+    dX = np.zeros((n_total, d))
+    dP = np.zeros((k, d))
+    dWk = np.zeros((d, d))
+    dWv = np.zeros((d, d))
+    rc = _load().sa_oracle_backward(_ptr(X), _ptr(off, ctypes.c_int64), R, n_total, d, _ptr(P), k,
+                                    _ptr(Wk), _ptr(Wv), _ptr(G), _ptr(Gm), _ptr(dX), _ptr(dP),
+                                    _ptr(dWk), _ptr(dWv), int(nthreads))
+    _check_rc(rc)
+    return {"dX": dX, "dP": dP, "dWk": dWk, "dWv": dWv}
