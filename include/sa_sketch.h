@@ -1,0 +1,151 @@
+/*
+ * sa_sketch.h -- C ABI of libsa_sketch.so: Sketch Attention (SA) forward and
+ * backward on B200 (sm_100a).
+ *
+ * What SA computes. The sources are the "100,000 videos in your pocket" blog,
+ * section "1. Sketch Attention compresses the history", and the evolve.pub review
+ * of arXiv 2609.08443, "Summary" and its FAQ on how SA differs from standard
+ * attention. Per user u, with history tokens t in [offsets[u], offsets[u+1]):
+ *
+ *   K = X W_k,  V = X W_v                       learnable prototypes P (k x d)
+ *   s_jt = P_j . K_t / sqrt(d)                  prototypes score every token
+ *   A_jt = exp(s_jt) / sum_i exp(s_it)          normalised across prototypes:
+ *                                               each token spreads unit mass
+ *   mass_j   = sum_t A_jt
+ *   sketch_j = (sum_t A_jt V_t) / mass_j        fixed k x d, target-agnostic
+ *
+ * The pages give no equations. The projections, the 1/sqrt(d) scale, the softmax
+ * normaliser and the mass-weighted mean are the plainest reading of them.
+ * Several users of different lengths are processed in one call as a ragged batch.
+ * The batch is described by an offsets array (blog, "3. The system makes it cheap
+ * enough to matter": a fused kernel under ragged batches, with multi-request
+ * user-level batching).
+ *
+ * Conventions for every entry point:
+ *  - All pointer arguments are DEVICE pointers unless stated otherwise. All
+ *    matrices are dense and row-major. The caller allocates and owns every
+ *    buffer; these calls allocate nothing.
+ *  - Calls are asynchronous and stream-ordered on `stream`. A cudaStream_t is
+ *    passed as void*; NULL means the legacy default stream.
+ *  - Argument errors are detected on the host. They return a non-zero status
+ *    before anything is launched.
+ *  - Some errors are only visible on the device: offsets that are not
+ *    non-decreasing, offsets[0] != 0, offsets[R] != n_total, or a bounded wait
+ *    inside a kernel that gave up. These are latched in a status word inside the
+ *    workspace. sa_sketch_get_device_status() reads that word. When it is set,
+ *    the outputs of that call are unspecified. The kernels never trap.
+ *  - `workspace` must be at least sa_sketch_workspace_size(...) bytes, 256-byte
+ *    aligned, and not used by another call in flight. Its contents need no
+ *    initialisation; each call initialises what it uses.
+ */
+#ifndef SA_SKETCH_H
+#define SA_SKETCH_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element type of X, P, W_k and W_v (every output is fp32). */
+typedef enum { SA_F32 = 0, SA_BF16 = 1 } sa_dtype;
+
+typedef enum {
+  SA_OK = 0,
+  SA_ERR_INVALID_ARG = 1,   /* null pointer, negative size, misaligned pointer   */
+  SA_ERR_UNSUPPORTED = 2,   /* shape outside what the kernels implement          */
+  SA_ERR_WORKSPACE = 3,     /* workspace null, misaligned or too small           */
+  SA_ERR_CUDA = 4,          /* a CUDA runtime call failed (launch, copy, ...)     */
+  SA_ERR_TIMEOUT = 5,       /* device: a bounded wait inside a kernel gave up    */
+  SA_ERR_BAD_OFFSETS = 6,   /* device: offsets not a valid ragged partition      */
+  SA_ERR_NO_DEVICE = 7      /* no sm_100 device current                          */
+} sa_status;
+
+/* Limits. d must be 64 or 128. k may be 1..2048 for fp32 and bf16 alike; bf16
+ * runs on tcgen05 tensor cores in slices of 128 prototypes, with k padded up to a
+ * multiple of 128 inside the kernel. R may be 0..SA_MAX_USERS and n_total may be
+ * 0..2^31-1. */
+#define SA_MAX_K 2048
+#define SA_MAX_USERS (1 << 20)
+
+/*
+ * Bytes of device workspace that sa_sketch_forward (backward = 0) or
+ * sa_sketch_backward (backward = 1) needs for these sizes on the current device.
+ * The plan depends on the device's SM count, so query it with the device current
+ * that will run the call. Returns 0 if the sizes are unsupported.
+ */
+size_t sa_sketch_workspace_size(int R, int64_t n_total, int k, int d, sa_dtype dt,
+                                int backward);
+
+/*
+ * Forward. Sources: blog section "1. Sketch Attention compresses the history" and
+ * review "Summary" (prototype scoring, prototype-wise normalisation, k x d sketch).
+ *
+ *   X       [n_total, d]  dt    history tokens of all users, concatenated
+ *   offsets [R + 1]       int64 offsets[0] = 0, non-decreasing, offsets[R] = n_total
+ *   P       [k, d]        dt    prototypes, shared by all users
+ *   Wk, Wv  [d, d]        dt    key and value projections (K = X Wk, V = X Wv)
+ * Outputs (fp32, overwritten):
+ *   sketch  [R, k, d]     mass-weighted mean of values per prototype
+ *   mass    [R, k]        sum over the user's tokens of A_jt
+ *   lse     [n_total]     per-token log-sum-exp of the scores (natural log);
+ *                         nullable. Needed by the backward.
+ *   xsketch [R, k, d]     sum_t A_jt X_t (un-normalised, before W_v); nullable.
+ *                         Needed by the backward.
+ * A user with no tokens gets sketch = 0 and mass = 0. Results are deterministic:
+ * two calls on the same inputs give bitwise-equal outputs.
+ * Pointers must be 16-byte aligned.
+ */
+int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
+                      const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,
+                      float* sketch, float* mass, float* lse, float* xsketch,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Backward. SA is differentiable, so the ranking loss's gradient flows back
+ * through the compression (blog, "1. Sketch Attention compresses the history").
+ * Given G = dL/dsketch and optional Gm = dL/dmass, this writes the gradients with
+ * respect to X, P, Wk and Wv.
+ *
+ *   X, offsets, P, Wk, Wv, dt   as passed to the forward
+ *   sketch, mass, lse, xsketch  fp32 outputs of that forward (lse, xsketch required)
+ *   dsketch [R, k, d] fp32      G
+ *   dmass   [R, k]    fp32      Gm; nullable (NULL means zero)
+ * Outputs (fp32, overwritten, not accumulated into):
+ *   dX  [n_total, d]
+ *   dP  [k, d], dWk [d, d], dWv [d, d]   summed over all users
+ */
+int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
+                       const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,
+                       const float* sketch, const float* mass, const float* lse,
+                       const float* xsketch, const float* dsketch, const float* dmass,
+                       float* dX, float* dP, float* dWk, float* dWv,
+                       void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Reads the device status word that the last call using `workspace` left behind.
+ * It synchronises `stream` and returns SA_OK, SA_ERR_BAD_OFFSETS or SA_ERR_TIMEOUT,
+ * or SA_ERR_CUDA if the copy itself failed. The word is cleared at the start of
+ * every forward and backward call.
+ */
+int sa_sketch_get_device_status(const void* workspace, void* stream);
+
+/* Static, human-readable name of a status code. */
+const char* sa_status_string(int status);
+
+/*
+ * Test hook for the failure-detection path. It launches one block that waits on
+ * an mbarrier that nothing ever arrives on. The wait uses the same bounded-wait
+ * routine as the production kernels, with a limit of `budget_cycles` SM clocks.
+ * When the limit runs out the kernel latches SA_ERR_TIMEOUT in `workspace`
+ * (which needs >= 256 bytes) and returns. It never hangs and never traps.
+ * Read the result with sa_sketch_get_device_status().
+ */
+int sa_sketch_debug_wait_timeout(void* workspace, long long budget_cycles, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SA_SKETCH_H */

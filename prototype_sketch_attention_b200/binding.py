@@ -1,0 +1,182 @@
+"""ctypes binding of libsa_sketch.so (argument marshalling only).
+
+The functions named ``sa_*`` mirror the C ABI in include/sa_sketch.h one to one.
+They take raw device pointers (ints), sizes and a stream handle, and return the
+library's status code. ``forward`` and ``backward`` are conveniences for torch
+users: they allocate outputs and workspace with torch (the library itself
+allocates nothing), call the C ABI on the current stream and raise on errors.
+Every step of the computation runs in the library's CUDA kernels. There is no
+fallback: if the library is missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libsa_sketch.so")
+
+SA_F32 = 0
+SA_BF16 = 1
+SA_OK = 0
+SA_ERR_INVALID_ARG = 1
+SA_ERR_UNSUPPORTED = 2
+SA_ERR_WORKSPACE = 3
+SA_ERR_CUDA = 4
+SA_ERR_TIMEOUT = 5
+SA_ERR_BAD_OFFSETS = 6
+SA_ERR_NO_DEVICE = 7
+
+EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
+            "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout")
+
+
+class SketchAttentionError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {sa_status_string(status)} ({status})")
+
+
+def _load() -> ctypes.CDLL:
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(
+            f"{_LIB_PATH} is not built; run `python -m prototype_sketch_attention_b200.build`")
+    lib = ctypes.CDLL(_LIB_PATH)
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    lib.sa_sketch_workspace_size.restype = sz
+    lib.sa_sketch_workspace_size.argtypes = [i32, i64, i32, i32, i32, i32]
+    lib.sa_sketch_forward.restype = i32
+    lib.sa_sketch_forward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
+                                      vp, vp, vp, vp, vp, sz, vp]
+    lib.sa_sketch_backward.restype = i32
+    lib.sa_sketch_backward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
+                                       vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sa_sketch_get_device_status.restype = i32
+    lib.sa_sketch_get_device_status.argtypes = [vp, vp]
+    lib.sa_status_string.restype = ctypes.c_char_p
+    lib.sa_status_string.argtypes = [i32]
+    lib.sa_sketch_debug_wait_timeout.restype = i32
+    lib.sa_sketch_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+    return lib
+
+
+_lib = _load()
+
+
+# ---------------------------------------------------------------- raw C ABI
+def sa_sketch_workspace_size(R: int, n_total: int, k: int, d: int, dt: int, backward: int) -> int:
+    return int(_lib.sa_sketch_workspace_size(R, n_total, k, d, dt, backward))
+
+
+def sa_sketch_forward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass, lse, xsketch,
+                      workspace, ws_bytes, stream) -> int:
+    return int(_lib.sa_sketch_forward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass,
+                                      lse, xsketch, workspace, ws_bytes, stream))
+
+
+def sa_sketch_backward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass, lse, xsketch,
+                       dsketch, dmass, dX, dP, dWk, dWv, workspace, ws_bytes, stream) -> int:
+    return int(_lib.sa_sketch_backward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass,
+                                       lse, xsketch, dsketch, dmass, dX, dP, dWk, dWv, workspace,
+                                       ws_bytes, stream))
+
+
+def sa_sketch_get_device_status(workspace, stream) -> int:
+    return int(_lib.sa_sketch_get_device_status(workspace, stream))
+
+
+def sa_status_string(status: int) -> str:
+    return _lib.sa_status_string(int(status)).decode()
+
+
+def sa_sketch_debug_wait_timeout(workspace, budget_cycles: int, stream) -> int:
+    return int(_lib.sa_sketch_debug_wait_timeout(workspace, int(budget_cycles), stream))
+
+
+# ---------------------------------------------------------------- torch conveniences
+def _ptr(t: torch.Tensor | None):
+    return None if t is None else t.data_ptr()
+
+
+def _dt(x: torch.Tensor) -> int:
+    if x.dtype == torch.bfloat16:
+        return SA_BF16
+    if x.dtype == torch.float32:
+        return SA_F32
+    raise TypeError(f"X must be bfloat16 or float32, got {x.dtype}")
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def workspace(R: int, n_total: int, k: int, d: int, dtype: torch.dtype, backward: bool = False,
+              device=None) -> torch.Tensor:
+    """A workspace tensor large enough for one call with these sizes."""
+    dt = SA_BF16 if dtype == torch.bfloat16 else SA_F32
+    n = sa_sketch_workspace_size(R, n_total, k, d, dt, int(backward))
+    if n == 0:
+        raise SketchAttentionError(SA_ERR_UNSUPPORTED, "sa_sketch_workspace_size")
+    return torch.empty(n, dtype=torch.uint8, device=device or "cuda")
+
+
+def forward(X: torch.Tensor, offsets: torch.Tensor, P: torch.Tensor, Wk: torch.Tensor,
+            Wv: torch.Tensor, *, want_lse: bool = True, want_xsketch: bool = True,
+            ws: torch.Tensor | None = None, out: dict | None = None, stream=None) -> dict:
+    """Sketch Attention forward on the GPU. Returns sketch, mass (and lse, xsketch).
+
+    X [n_total, d] bf16/fp32, offsets [R+1] int64, P [k, d], Wk, Wv [d, d] (same dtype
+    as X), all contiguous on one CUDA device.
+    """
+    n_total, d = X.shape
+    k = P.shape[0]
+    R = offsets.shape[0] - 1
+    dt = _dt(X)
+    dev = X.device
+    if out is None:
+        out = {"sketch": torch.empty(R, k, d, device=dev, dtype=torch.float32),
+               "mass": torch.empty(R, k, device=dev, dtype=torch.float32)}
+        if want_lse:
+            out["lse"] = torch.empty(n_total, device=dev, dtype=torch.float32)
+        if want_xsketch:
+            out["xsketch"] = torch.empty(R, k, d, device=dev, dtype=torch.float32)
+    if ws is None:
+        ws = workspace(R, n_total, k, d, X.dtype, False, dev)
+    st = sa_sketch_forward(_ptr(X), _ptr(offsets), R, n_total, d, _ptr(P), k, _ptr(Wk), _ptr(Wv),
+                           dt, _ptr(out["sketch"]), _ptr(out["mass"]), _ptr(out.get("lse")),
+                           _ptr(out.get("xsketch")), _ptr(ws), ws.numel(), _stream(stream))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_forward")
+    out["_ws"] = ws
+    return out
+
+
+def backward(X, offsets, P, Wk, Wv, fwd: dict, dsketch: torch.Tensor, dmass=None, *,
+             ws: torch.Tensor | None = None, stream=None) -> dict:
+    """Gradients dX, dP, dWk, dWv given dL/dsketch (and optionally dL/dmass)."""
+    n_total, d = X.shape
+    k = P.shape[0]
+    R = offsets.shape[0] - 1
+    dt = _dt(X)
+    dev = X.device
+    out = {"dX": torch.empty(n_total, d, device=dev, dtype=torch.float32),
+           "dP": torch.empty(k, d, device=dev, dtype=torch.float32),
+           "dWk": torch.empty(d, d, device=dev, dtype=torch.float32),
+           "dWv": torch.empty(d, d, device=dev, dtype=torch.float32)}
+    if ws is None:
+        ws = workspace(R, n_total, k, d, X.dtype, True, dev)
+    st = sa_sketch_backward(_ptr(X), _ptr(offsets), R, n_total, d, _ptr(P), k, _ptr(Wk), _ptr(Wv),
+                            dt, _ptr(fwd["sketch"]), _ptr(fwd["mass"]), _ptr(fwd.get("lse")),
+                            _ptr(fwd["xsketch"]), _ptr(dsketch), _ptr(dmass), _ptr(out["dX"]),
+                            _ptr(out["dP"]), _ptr(out["dWk"]), _ptr(out["dWv"]), _ptr(ws),
+                            ws.numel(), _stream(stream))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_backward")
+    out["_ws"] = ws
+    return out
+
+
+def device_status(ws: torch.Tensor, stream=None) -> int:
+    return sa_sketch_get_device_status(_ptr(ws), _stream(stream))

@@ -1,0 +1,441 @@
+// Sketch Attention forward on tcgen05 tensor cores (sm_100a), bf16 in / fp32 accumulate.
+//
+// What is computed (blog "100,000 videos in your pocket", section "1. Sketch Attention
+// compresses the history"; evolve.pub review "Summary"): for every history token the k
+// prototypes' scores are normalised ACROSS PROTOTYPES (each token spreads unit mass),
+// and each prototype accumulates the mass-weighted sum of tokens. The projections are
+// folded away before this kernel: with P' = P W_k^T log2(e)/sqrt(d) (bf16, computed by
+// the fold kernel), the score of prototype j on token t in log2 units is P'_j . X_t, and
+// sum_t A_jt V_t = (sum_t A_jt X_t) W_v, applied later in the finalize kernel.
+//
+// Decomposition. A cluster of C = ceil(k/128) CTAs owns one slice of the token stream; CTA
+// of rank c owns prototypes [128c, 128c+128). Per tile of 128 tokens each CTA:
+//   1. TMA loads the X tile (128 x d bf16, 128B swizzle) into a shared-memory stage
+//      (every CTA loads it itself; no multicast, the C-fold re-read is served by L2).
+//   2. tcgen05.mma  S^T[tok, proto] = X_tile . P'_slice^T  into TMEM (fp32), so a
+//      token's scores sit in one TMEM lane and one thread owns one token.
+//   3. Softmax warps load their row, take the local max m_c and l_c = m_c + log2 sum
+//      2^(s - m_c), and send l_c to every CTA of the cluster with st.async (DSMEM).
+//      Once all C partials have arrived: lse2 = log2 sum_c 2^(l_c), A = 2^(s - lse2).
+//   4. A is written as bf16 into shared memory in the MN-major layout of the next MMA's
+//      A operand, then  U[proto, :] += A . X_tile  and  mass[proto] += A . 1
+//      (tcgen05, accumulators in TMEM).
+//   5. When the token stream crosses a user boundary (or the slice ends) the partial
+//      (U, mass) of that (slice, user) segment is written to the workspace; a separate
+//      kernel adds the segments of each user in a fixed order (deterministic).
+// All mbarrier waits are bounded (see sa_common.cuh).
+#include <cuda.h>
+
+#include "sa_common.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+namespace {
+
+constexpr int kProtoSlice = 128;              // prototypes per CTA (TMEM lanes / MMA M)
+constexpr int kXchSlots = 4;                  // exchange slots (tile index mod 4)
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS0 = 0, kColS1 = 128, kColU = 256;
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kStages = (D == 128) ? 3 : 4;
+  static constexpr int kBoxBytes = 128 * 64 * 2;            // one TMA box: 128 rows x 64 bf16
+  static constexpr int kXStage = 128 * D * 2;                // X tile
+  static constexpr int kPBytes = kProtoSlice * D * 2;        // P' slice
+  static constexpr int kABytes = kProtoSlice * kTileTokens * 2;  // A tile (bf16)
+  static constexpr int kOnesBytes = 512;
+  // byte offsets from the 1024-aligned base
+  static constexpr int oX = 0;
+  static constexpr int oP = oX + kStages * kXStage;
+  static constexpr int oA = oP + kPBytes;
+  static constexpr int oOnes = oA + 2 * kABytes;
+  static constexpr int oXch = oOnes + kOnesBytes;  // kXchSlots * C * 128 floats (runtime C)
+  static size_t bytes(int C) {
+    const size_t xch = (size_t)kXchSlots * C * 128 * 4;
+    const size_t bars = 64 * 8 + 16;
+    return 1024 + oXch + xch + bars;
+  }
+};
+
+struct Bars {
+  uint64_t x_full[4], x_empty[4];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t a_full[2], a_empty[2];
+  uint64_t u_full, u_empty;
+  uint64_t xch[kXchSlots];
+  uint64_t p_full, drain;
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
+  uint32_t r;
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];" : "=r"(r) : "r"(taddr) : "memory");
+  return __uint_as_float(r);
+}
+
+template <int D>
+__global__ void __launch_bounds__(192, 1)
+sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                    const __grid_constant__ CUtensorMap tmap_p,
+                    const int64_t* __restrict__ offsets, int R, int k_valid, int C, int k_pad,
+                    WsHeader* hdr, const long long* __restrict__ tile_start,
+                    float* __restrict__ part_u, float* __restrict__ part_m,
+                    float* __restrict__ lse_out, long long budget) {
+  using L = FwdSmem<D>;
+  constexpr int NS = L::kStages;
+  constexpr int KSTEPS1 = D / 16;           // MMA1 K steps (over d)
+  constexpr int KSTEPS2 = kTileTokens / 16;  // MMA2 K steps (over tokens)
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  float* xch = reinterpret_cast<float*>(smem + L::oXch);
+  Bars* bars = reinterpret_cast<Bars*>(smem + L::oXch + (size_t)kXchSlots * C * 128 * 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const uint32_t cid = cluster_id_x(), ncl = nclusters_x();
+  int* status = &hdr->status;
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_u32(&bars->x_full[s]), 1);
+      mbar_init(smem_u32(&bars->x_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->s_full[s]), 1);
+      mbar_init(smem_u32(&bars->s_empty[s]), 4);
+      mbar_init(smem_u32(&bars->a_full[s]), 4);
+      mbar_init(smem_u32(&bars->a_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->u_full), 1);
+    mbar_init(smem_u32(&bars->u_empty), 4);
+    for (int s = 0; s < kXchSlots; ++s) mbar_init(smem_u32(&bars->xch[s]), 1);
+    mbar_init(smem_u32(&bars->p_full), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp >= 2) {
+    // all-ones bf16 block: B operand of the mass MMA (16 x 16, K-major, no swizzle)
+    const int t = threadIdx.x - 64;
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + L::oOnes);
+    if (t < L::kOnesBytes / 4) ones[t] = 0x3F803F80u;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // peers' barriers are initialised before any st.async arrives
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  // this cluster's share of the token tiles
+  const long long T = read_status(status) == 0 ? hdr->total_tiles : 0;
+  const long long ta = (long long)cid * T / ncl, tb = (long long)(cid + 1) * T / ncl;
+
+  if (warp == 0) {
+    // ================= TMA producer
+    if (lane == 0 && ta < tb) {
+      tma_prefetch_desc(&tmap_x);
+      tma_prefetch_desc(&tmap_p);
+      const uint32_t pf = smem_u32(&bars->p_full);
+      mbar_arrive_expect_tx(pf, L::kPBytes);
+      for (int b = 0; b < D / 64; ++b)
+        tma_load_2d(sbase + L::oP + b * L::kBoxBytes, &tmap_p, b * 64, (int)rank * kProtoSlice, pf);
+      TileIter it;
+      it.init(tile_start, offsets, R, ta, tb);
+      long long i = 0;
+      for (; it.valid(); it.next(), ++i) {
+        const int st = (int)(i % NS);
+        const uint32_t par = (uint32_t)((i / NS) & 1);
+        if (!mbar_wait(smem_u32(&bars->x_empty[st]), par ^ 1u, status, budget)) break;
+        const uint32_t fb = smem_u32(&bars->x_full[st]);
+        mbar_arrive_expect_tx(fb, L::kXStage);
+        const int y = (int)it.t0();
+        for (int b = 0; b < D / 64; ++b)
+          tma_load_2d(sbase + L::oX + st * L::kXStage + b * L::kBoxBytes, &tmap_x, b * 64, y, fb);
+      }
+      // drain: the loads of the last NS tiles issued must have landed before exit
+      for (long long j = (i > NS ? i - NS : 0); j < i; ++j)
+        mbar_wait_drain(smem_u32(&bars->x_full[j % NS]), (uint32_t)((j / NS) & 1), budget);
+      mbar_wait_drain(pf, 0, budget);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer
+    if (lane == 0 && ta < tb) {
+      const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);  // S^T = X . P'^T
+      const uint32_t idesc2 = idesc_bf16_f32(128, D, 1, 1);            // U += A . X
+      const uint32_t idescm = idesc_bf16_f32(128, 16, 1, 0);           // mass += A . 1
+      const uint64_t ones_desc = smem_desc(sbase + L::oOnes, 128, 256, kSwizzleNone);
+      bool ok = mbar_wait(smem_u32(&bars->p_full), 0, status, budget);
+      TileIter it;
+      it.init(tile_start, offsets, R, ta, tb);
+      long long i = 0;
+      int seg = -1;
+      // pending MMA2 (one tile behind MMA1)
+      long long pj = -1;
+      bool pfirst = false, plast = false;
+      int pseg = 0;
+      auto issue_mma2 = [&](long long j, bool first, bool last, int sg) -> bool {
+        const int ab = (int)(j & 1);
+        const int st = (int)(j % NS);
+        if (!mbar_wait(smem_u32(&bars->a_full[ab]), (uint32_t)((j >> 1) & 1), status, budget))
+          return false;
+        if (first && !mbar_wait(smem_u32(&bars->u_empty), (uint32_t)((sg & 1) ^ 1), status, budget))
+          return false;
+        tc_fence_after();
+        const uint32_t a_base = sbase + L::oA + ab * L::kABytes;
+        const uint32_t x_base = sbase + L::oX + st * L::kXStage;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS2; ++ks) {
+          const uint64_t ad = smem_desc(a_base + ks * 2048, L::kBoxBytes, 1024, kSwizzle128B);
+          const uint64_t bd = smem_desc(x_base + ks * 2048, L::kBoxBytes, 1024, kSwizzle128B);
+          const uint32_t acc = (first && ks == 0) ? 0u : 1u;
+          tc_mma_f16(tmem + kColU, ad, bd, idesc2, acc);
+          tc_mma_f16(tmem + kColU + D, ad, ones_desc, idescm, acc);
+        }
+        tc_commit(smem_u32(&bars->x_empty[st]));
+        tc_commit(smem_u32(&bars->a_empty[ab]));
+        if (last) tc_commit(smem_u32(&bars->u_full));
+        return true;
+      };
+      for (; ok && it.valid(); it.next(), ++i) {
+        const bool first = it.first(), last = it.last();
+        if (first) ++seg;
+        const int st = (int)(i % NS);
+        const int sb = (int)(i & 1);
+        ok = mbar_wait(smem_u32(&bars->x_full[st]), (uint32_t)((i / NS) & 1), status, budget) &&
+             mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t x_base = sbase + L::oX + st * L::kXStage;
+        const uint32_t p_base = sbase + L::oP;
+#pragma unroll
+        for (int ks = 0; ks < KSTEPS1; ++ks) {
+          const uint32_t koff = (ks >> 2) * L::kBoxBytes + (ks & 3) * 32;
+          const uint64_t ad = smem_desc(x_base + koff, 16, 1024, kSwizzle128B);
+          const uint64_t bd = smem_desc(p_base + koff, 16, 1024, kSwizzle128B);
+          tc_mma_f16(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc1, ks > 0 ? 1u : 0u);
+        }
+        tc_commit(smem_u32(&bars->s_full[sb]));
+        if (pj >= 0) {
+          ok = issue_mma2(pj, pfirst, plast, pseg);
+          if (!ok) break;
+        }
+        pj = i; pfirst = first; plast = last; pseg = seg;
+      }
+      if (ok && pj >= 0) issue_mma2(pj, pfirst, plast, pseg);
+      // drain every tcgen05 op this thread issued before the CTA tears down
+      tc_commit(smem_u32(&bars->drain));
+      mbar_wait_drain(smem_u32(&bars->drain), 0, budget);
+    }
+  } else {
+    // ================= softmax + epilogue warpgroup (warps 2..5; TMEM lane quadrant = warp % 4)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;              // token row in the tile == TMEM lane
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool leader = (threadIdx.x == 64);
+    const int pbase = (int)rank * kProtoSlice;
+    TileIter it;
+    it.init(tile_start, offsets, R, ta, tb);
+    long long i = 0;
+    int seg = -1;
+    bool ok = true;
+    for (; ok && it.valid(); it.next(), ++i) {
+      if (it.first()) ++seg;
+      const int sb = (int)(i & 1);
+      if (!mbar_wait_warp(smem_u32(&bars->s_full[sb]), (uint32_t)((i >> 1) & 1), status, budget)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      float e[kProtoSlice];
+#pragma unroll
+      for (int c = 0; c < kProtoSlice / 32; ++c) {
+        float v[32];
+        tmem_ld32(tmem + lane_off + (sb ? kColS1 : kColS0) + c * 32, v);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) e[c * 32 + x] = v[x];
+      }
+      tc_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[sb]));
+
+      // local (this slice) max and log2-sum-exp2
+      float m = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < kProtoSlice; ++c) {
+        if (pbase + c >= k_valid) e[c] = -INFINITY;
+        m = fmaxf(m, e[c]);
+      }
+      float z = 0.f;
+#pragma unroll
+      for (int c = 0; c < kProtoSlice; ++c) {
+        e[c] = ex2_approx(e[c] - m);
+        z += e[c];
+      }
+      const int nv = it.nvalid();
+      const bool valid = r < nv;
+      const float l = valid ? m + lg2_approx(z) : 0.f;
+
+      // exchange l with every CTA of the cluster (4 tokens per 16-byte st.async)
+      const int qs = (int)(i & (kXchSlots - 1));
+      const uint32_t xbar = smem_u32(&bars->xch[qs]);
+      {
+        const int g0 = lane & ~3;
+        const float v0 = __shfl_sync(0xffffffffu, l, g0 + 0);
+        const float v1 = __shfl_sync(0xffffffffu, l, g0 + 1);
+        const float v2 = __shfl_sync(0xffffffffu, l, g0 + 2);
+        const float v3 = __shfl_sync(0xffffffffu, l, g0 + 3);
+        const uint32_t laddr = smem_u32(xch + ((qs * C + (int)rank) * 128 + q * 32 + g0));
+        for (int p = lane & 3; p < C; p += 4)
+          st_async_v4(mapa(laddr, (uint32_t)p), v0, v1, v2, v3, mapa(xbar, (uint32_t)p));
+      }
+      if (leader) mbar_arrive_expect_tx(xbar, (uint32_t)C * 128u * 4u);
+      if (!mbar_wait_warp<true>(xbar, (uint32_t)((i >> 2) & 1), status, budget)) {
+        ok = false;
+        break;
+      }
+      float lmax = -INFINITY;
+      for (int p = 0; p < C; ++p) lmax = fmaxf(lmax, xch[(qs * C + p) * 128 + r]);
+      float zs = 0.f;
+      for (int p = 0; p < C; ++p) zs += ex2_approx(xch[(qs * C + p) * 128 + r] - lmax);
+      const float lse2 = lmax + lg2_approx(zs);
+      const float scale = valid ? ex2_approx(m - lse2) : 0.f;
+      if (rank == 0 && valid && lse_out != nullptr)
+        lse_out[it.t0() + r] = lse2 * 0.69314718055994530942f;
+
+      // A (bf16) into the MN-major, 128B-swizzled A operand: row = token, 64 prototypes
+      // per 128-byte row, two 16 KB blocks for prototypes [0,64) and [64,128).
+      const int ab = (int)(i & 1);
+      if (!mbar_wait_warp(smem_u32(&bars->a_empty[ab]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget)) {
+        ok = false;
+        break;
+      }
+      uint8_t* arow = smem + L::oA + ab * L::kABytes + r * 128;
+#pragma unroll
+      for (int mb = 0; mb < 2; ++mb) {
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          const int c0 = mb * 64 + ch * 8;
+          uint4 w;
+          w.x = pack_bf16x2(e[c0 + 0] * scale, e[c0 + 1] * scale);
+          w.y = pack_bf16x2(e[c0 + 2] * scale, e[c0 + 3] * scale);
+          w.z = pack_bf16x2(e[c0 + 4] * scale, e[c0 + 5] * scale);
+          w.w = pack_bf16x2(e[c0 + 6] * scale, e[c0 + 7] * scale);
+          *reinterpret_cast<uint4*>(arow + mb * 16384 + ((ch ^ (r & 7)) << 4)) = w;
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->a_full[ab]));
+
+      if (it.last()) {
+        // ---- epilogue: this segment's partial (U, mass) for our 128 prototypes
+        if (!mbar_wait_warp(smem_u32(&bars->u_full), (uint32_t)(seg & 1), status, budget)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const long long sgid = (long long)cid + it.u;
+        float* dst = part_u + ((size_t)sgid * k_pad + pbase + r) * D;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          float v[32];
+          tmem_ld32(tmem + lane_off + kColU + c * 32, v);
+          tc_wait_ld();
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            *reinterpret_cast<float4*>(dst + c * 32 + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
+        }
+        const float ms = tmem_ld1(tmem + lane_off + kColU + D);
+        tc_wait_ld();
+        part_m[(size_t)sgid * k_pad + pbase + r] = ms;
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&bars->u_empty));
+      }
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();  // no peer touches our shared memory after this point
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D>
+cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
+  auto kern = sa_fwd_sm100_kernel<D>;
+  const size_t smem = FwdSmem<D>::bytes(a.C);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (a.C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(a.G * a.C));
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)a.C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, *a.tmap_x, *a.tmap_p, a.offsets, a.R, a.k_valid, a.C,
+                            a.k_pad, a.hdr, a.tile_start, a.part_u, a.part_m, a.lse, a.budget);
+}
+
+template <int D>
+cudaError_t max_clusters_t(int C, int* n) {
+  auto kern = sa_fwd_sm100_kernel<D>;
+  const size_t smem = FwdSmem<D>::bytes(C);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  if (C > 8) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
+    if (e != cudaSuccess) return e;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)C);
+  cfg.blockDim = dim3(192);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = (unsigned)C;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaOccupancyMaxActiveClusters(n, kern, &cfg);
+}
+
+}  // namespace
+
+size_t fwd_sm100_smem_bytes(int d, int C) {
+  return d == 128 ? FwdSmem<128>::bytes(C) : FwdSmem<64>::bytes(C);
+}
+
+cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
+  return d == 128 ? max_clusters_t<128>(C, n) : max_clusters_t<64>(C, n);
+}
+
+cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream) {
+  return a.d == 128 ? launch_fwd_sm100_t<128>(a, stream) : launch_fwd_sm100_t<64>(a, stream);
+}
+
+}  // namespace sa

@@ -1,0 +1,377 @@
+// C ABI of libsa_sketch.so: argument checks, the workspace plan, tensor maps and the
+// launch sequence of Sketch Attention's forward and backward. See include/sa_sketch.h
+// for the contract of every entry point.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <cstring>
+#include <map>
+#include <mutex>
+#include <tuple>
+
+#include "sa_common.cuh"
+#include "sa_internal.h"
+#include "sa_sketch.h"
+
+namespace sa {
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr float kLog2e = 1.4426950408889634f;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Device {
+  int id = -1;
+  int sms = 0;
+  bool ok = false;
+};
+
+sa_status current_device(Device* dev) {
+  int id = 0;
+  if (cudaGetDevice(&id) != cudaSuccess) return SA_ERR_NO_DEVICE;
+  int major = 0, minor = 0, sms = 0;
+  if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, id) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, id) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, id) != cudaSuccess)
+    return SA_ERR_NO_DEVICE;
+  if (major != 10 || minor != 0) return SA_ERR_NO_DEVICE;  // built for sm_100a only
+  dev->id = id;
+  dev->sms = sms;
+  dev->ok = true;
+  return SA_OK;
+}
+
+// Co-resident clusters of the tcgen05 forward, cached per (device, d, C).
+sa_status tc_clusters(const Device& dev, int d, int C, int* G) {
+  static std::mutex mu;
+  static std::map<std::tuple<int, int, int>, int> cache;
+  std::lock_guard<std::mutex> lock(mu);
+  const auto key = std::make_tuple(dev.id, d, C);
+  auto it = cache.find(key);
+  if (it == cache.end()) {
+    int n = 0;
+    if (fwd_sm100_max_clusters(d, C, &n) != cudaSuccess) {
+      cudaGetLastError();
+      return SA_ERR_CUDA;
+    }
+    it = cache.emplace(key, n).first;
+  }
+  *G = it->second;
+  return *G > 0 ? SA_OK : SA_ERR_UNSUPPORTED;
+}
+
+struct Plan {
+  bool tc = false;  // tcgen05 path
+  int C = 0, k_pad = 0, G = 0, Gb = 0;
+  size_t hdr = 0, ts = 0, pf = 0, pu = 0, pm = 0, lse2 = 0;
+  size_t pn = 0, gt = 0, gh = 0, cj = 0, lseb = 0, db = 0, dppp = 0, dpp = 0, wvp = 0;
+  size_t total = 0;
+};
+
+sa_status check_sizes(int R, int64_t n_total, int k, int d, sa_dtype dt) {
+  if (R < 0 || R > SA_MAX_USERS || n_total < 0 || n_total > INT32_MAX) return SA_ERR_INVALID_ARG;
+  if (dt != SA_F32 && dt != SA_BF16) return SA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+  if (k < 1 || k > SA_MAX_K) return SA_ERR_UNSUPPORTED;
+  return SA_OK;
+}
+
+sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_dtype dt,
+                    bool backward, Plan* p) {
+  sa_status st = check_sizes(R, n_total, k, d, dt);
+  if (st != SA_OK) return st;
+  Plan q;
+  q.tc = (dt == SA_BF16) && !backward;
+  if (q.tc) {
+    q.C = (k + 127) / 128;
+    q.k_pad = q.C * 128;
+    if ((st = tc_clusters(dev, d, q.C, &q.G)) != SA_OK) return st;
+  } else {
+    q.k_pad = (k + 31) / 32 * 32;
+    const int pblocks = q.k_pad / 32;
+    q.G = dev.sms * 4 / pblocks;
+    if (q.G < 1) q.G = 1;
+  }
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + bytes);
+    return at;
+  };
+  q.hdr = take(sizeof(WsHeader));
+  q.ts = take((size_t)(R + 1) * sizeof(long long));
+  if (!backward) {
+    q.pf = take((size_t)q.k_pad * d * (dt == SA_BF16 ? 2 : 4));
+    const size_t segs = (size_t)q.G + (size_t)R;
+    q.pu = take(segs * q.k_pad * d * sizeof(float));
+    q.pm = take(segs * q.k_pad * sizeof(float));
+    if (!q.tc) q.lse2 = take((size_t)n_total * sizeof(float));
+  } else {
+    q.Gb = q.G;
+    q.pn = take((size_t)q.k_pad * d * sizeof(float));
+    q.gt = take((size_t)R * q.k_pad * d * sizeof(float));
+    q.gh = take((size_t)R * q.k_pad * d * sizeof(float));
+    q.cj = take((size_t)R * q.k_pad * sizeof(float));
+    q.lseb = take((size_t)n_total * sizeof(float));
+    q.db = take((size_t)n_total * sizeof(float));
+    q.dppp = take((size_t)q.Gb * q.k_pad * d * sizeof(float));
+    q.dpp = take((size_t)q.k_pad * d * sizeof(float));
+    q.wvp = take(bwd_wv_chunks(R, k) * d * d * sizeof(float));
+  }
+  q.total = o;
+  *p = q;
+  return SA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda needed).
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// Row-major [rows, d] bf16 matrix, boxes of 128 rows x 64 columns, 128-byte swizzle.
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
+                        strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+sa_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SA_OK;
+  cudaGetLastError();
+  return SA_ERR_CUDA;
+}
+
+}  // namespace
+}  // namespace sa
+
+using namespace sa;
+
+extern "C" {
+
+size_t sa_sketch_workspace_size(int R, int64_t n_total, int k, int d, sa_dtype dt, int backward) {
+  Device dev;
+  if (current_device(&dev) != SA_OK) return 0;
+  Plan p;
+  if (make_plan(dev, R, n_total, k, d, dt, backward != 0, &p) != SA_OK) return 0;
+  return p.total;
+}
+
+int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
+                      const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,
+                      float* sketch, float* mass, float* lse, float* xsketch, void* workspace,
+                      size_t ws_bytes, void* stream_) {
+  sa_status st = check_sizes(R, n_total, k, d, dt);
+  if (st != SA_OK) return st;
+  if (!offsets || !P || !Wk || !Wv || (n_total > 0 && !X) || (R > 0 && (!sketch || !mass)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(P) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(sketch) ||
+      !aligned16(mass) || !aligned16(lse) || !aligned16(xsketch) || !aligned16(offsets))
+    return SA_ERR_INVALID_ARG;
+  Device dev;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  Plan p;
+  if ((st = make_plan(dev, R, n_total, k, d, dt, false, &p)) != SA_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || ws_bytes < p.total)
+    return SA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  WsHeader* hdr = at<WsHeader>(workspace, p.hdr);
+  long long* ts = at<long long>(workspace, p.ts);
+  float* pu = at<float>(workspace, p.pu);
+  float* pm = at<float>(workspace, p.pm);
+
+  if ((st = cuda_status(launch_schedule(offsets, R, n_total, hdr, ts, s))) != SA_OK) return st;
+  const float scale = kLog2e / std::sqrt((float)d);
+  if ((st = cuda_status(launch_fold(P, Wk, dt, k, p.k_pad, d, scale, at<void>(workspace, p.pf),
+                                    p.tc, s))) != SA_OK)
+    return st;
+  if (n_total > 0) {
+    if (p.tc) {
+      CUtensorMap tx, tp;
+      if (!make_tmap_bf16(&tx, X, (uint64_t)n_total, d) ||
+          !make_tmap_bf16(&tp, at<void>(workspace, p.pf), (uint64_t)p.k_pad, d))
+        return SA_ERR_CUDA;
+      FwdSm100Args a;
+      a.tmap_x = &tx;
+      a.tmap_p = &tp;
+      a.offsets = offsets;
+      a.R = R;
+      a.k_valid = k;
+      a.C = p.C;
+      a.k_pad = p.k_pad;
+      a.d = d;
+      a.G = p.G;
+      a.hdr = hdr;
+      a.tile_start = ts;
+      a.part_u = pu;
+      a.part_m = pm;
+      a.lse = lse;
+      a.budget = kDefaultWaitBudget;
+      if ((st = cuda_status(launch_fwd_sm100(a, s))) != SA_OK) return st;
+    } else {
+      FwdSimtArgs a;
+      a.X = static_cast<const float*>(X);
+      a.offsets = offsets;
+      a.R = R;
+      a.k = k;
+      a.k_pad = p.k_pad;
+      a.d = d;
+      a.G = p.G;
+      a.Pf = at<float>(workspace, p.pf);
+      a.hdr = hdr;
+      a.tile_start = ts;
+      a.lse2 = at<float>(workspace, p.lse2);
+      a.lse = lse;
+      a.n_total = n_total;
+      a.part_u = pu;
+      a.part_m = pm;
+      if ((st = cuda_status(launch_fwd_simt(a, s))) != SA_OK) return st;
+    }
+  }
+  FinalizeArgs f;
+  f.hdr = hdr;
+  f.tile_start = ts;
+  f.part_u = pu;
+  f.part_m = pm;
+  f.Wv = Wv;
+  f.dt = dt;
+  f.R = R;
+  f.k = k;
+  f.k_pad = p.k_pad;
+  f.d = d;
+  f.G = p.G;
+  f.sketch = sketch;
+  f.mass = mass;
+  f.xsketch = xsketch;
+  return cuda_status(launch_finalize(f, s));
+}
+
+int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
+                       const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,
+                       const float* sketch, const float* mass, const float* lse,
+                       const float* xsketch, const float* dsketch, const float* dmass, float* dX,
+                       float* dP, float* dWk, float* dWv, void* workspace, size_t ws_bytes,
+                       void* stream_) {
+  (void)lse;  // per-token statistics are recomputed in fp32
+  sa_status st = check_sizes(R, n_total, k, d, dt);
+  if (st != SA_OK) return st;
+  if (!offsets || !P || !Wk || !Wv || !dP || !dWk || !dWv ||
+      (n_total > 0 && (!X || !dX)) ||
+      (R > 0 && (!sketch || !mass || !xsketch || !dsketch)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(X) || !aligned16(P) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(sketch) ||
+      !aligned16(mass) || !aligned16(xsketch) || !aligned16(dsketch) || !aligned16(dmass) ||
+      !aligned16(dX) || !aligned16(dP) || !aligned16(dWk) || !aligned16(dWv) || !aligned16(offsets))
+    return SA_ERR_INVALID_ARG;
+  Device dev;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  Plan p;
+  if ((st = make_plan(dev, R, n_total, k, d, dt, true, &p)) != SA_OK) return st;
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || ws_bytes < p.total)
+    return SA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  WsHeader* hdr = at<WsHeader>(workspace, p.hdr);
+  long long* ts = at<long long>(workspace, p.ts);
+  if ((st = cuda_status(launch_schedule(offsets, R, n_total, hdr, ts, s))) != SA_OK) return st;
+  if ((st = cuda_status(launch_fold(P, Wk, dt, k, p.k_pad, d, 1.0f / std::sqrt((float)d),
+                                    at<void>(workspace, p.pn), false, s))) != SA_OK)
+    return st;
+  BwdArgs a;
+  a.X = X;
+  a.dt = dt;
+  a.offsets = offsets;
+  a.R = R;
+  a.k = k;
+  a.k_pad = p.k_pad;
+  a.d = d;
+  a.G = p.Gb;
+  a.n_total = n_total;
+  a.P = P;
+  a.Wk = Wk;
+  a.Wv = Wv;
+  a.sketch = sketch;
+  a.mass = mass;
+  a.xsketch = xsketch;
+  a.dsketch = dsketch;
+  a.dmass = dmass;
+  a.hdr = hdr;
+  a.tile_start = ts;
+  a.Pn = at<float>(workspace, p.pn);
+  a.Gt = at<float>(workspace, p.gt);
+  a.Gh = at<float>(workspace, p.gh);
+  a.cj = at<float>(workspace, p.cj);
+  a.lseb = at<float>(workspace, p.lseb);
+  a.Db = at<float>(workspace, p.db);
+  a.dpp_part = at<float>(workspace, p.dppp);
+  a.dpp = at<float>(workspace, p.dpp);
+  a.wv_part = at<float>(workspace, p.wvp);
+  a.dX = dX;
+  a.dP = dP;
+  a.dWk = dWk;
+  a.dWv = dWv;
+  return cuda_status(launch_bwd_simt(a, s));
+}
+
+int sa_sketch_get_device_status(const void* workspace, void* stream_) {
+  if (!workspace) return SA_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream_);
+  int h = 0;
+  if (cudaMemcpyAsync(&h, workspace, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return SA_ERR_CUDA;
+  }
+  return h;
+}
+
+const char* sa_status_string(int status) {
+  switch (status) {
+    case SA_OK: return "SA_OK";
+    case SA_ERR_INVALID_ARG: return "SA_ERR_INVALID_ARG: null, negative or misaligned argument";
+    case SA_ERR_UNSUPPORTED: return "SA_ERR_UNSUPPORTED: shape outside the implemented range";
+    case SA_ERR_WORKSPACE: return "SA_ERR_WORKSPACE: workspace null, misaligned or too small";
+    case SA_ERR_CUDA: return "SA_ERR_CUDA: a CUDA call failed";
+    case SA_ERR_TIMEOUT: return "SA_ERR_TIMEOUT: a bounded wait inside a kernel gave up";
+    case SA_ERR_BAD_OFFSETS: return "SA_ERR_BAD_OFFSETS: offsets are not a ragged partition";
+    case SA_ERR_NO_DEVICE: return "SA_ERR_NO_DEVICE: no sm_100 device is current";
+    default: return "unknown sa_status";
+  }
+}
+
+int sa_sketch_debug_wait_timeout(void* workspace, long long budget_cycles, void* stream_) {
+  if (!workspace || budget_cycles <= 0) return SA_ERR_INVALID_ARG;
+  Device dev;
+  sa_status st = current_device(&dev);
+  if (st != SA_OK) return st;
+  return cuda_status(launch_debug_wait_timeout(static_cast<WsHeader*>(workspace), budget_cycles,
+                                               static_cast<cudaStream_t>(stream_)));
+}
+
+}  // extern "C"

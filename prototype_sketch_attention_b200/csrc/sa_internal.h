@@ -1,0 +1,110 @@
+// Internal (host-side) interface between the C-ABI layer and the kernel files.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "sa_sketch.h"
+
+namespace sa {
+
+struct WsHeader;
+
+// ---- schedule: validates offsets, clears the status word, tile prefix sums
+cudaError_t launch_schedule(const int64_t* offsets, int R, int64_t n_total, WsHeader* hdr,
+                            long long* tile_start, cudaStream_t s);
+
+// ---- fold: Pf[j][c] = scale * sum_e P[j][e] Wk[c][e] for j < k, 0 for k <= j < k_pad
+cudaError_t launch_fold(const void* P, const void* Wk, sa_dtype dt, int k, int k_pad, int d,
+                        float scale, void* Pf, bool out_bf16, cudaStream_t s);
+
+// ---- finalize: sums a user's segment partials in order, then sketch = (U Wv) / mass
+struct FinalizeArgs {
+  const WsHeader* hdr;
+  const long long* tile_start;
+  const float* part_u;  // [segments, k_pad, d]
+  const float* part_m;  // [segments, k_pad]
+  const void* Wv;
+  sa_dtype dt;
+  int R, k, k_pad, d, G;
+  float* sketch;
+  float* mass;
+  float* xsketch;  // nullable
+};
+cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
+
+// ---- tcgen05 forward (bf16)
+struct FwdSm100Args {
+  const CUtensorMap* tmap_x;
+  const CUtensorMap* tmap_p;
+  const int64_t* offsets;
+  int R, k_valid, C, k_pad, d, G;
+  WsHeader* hdr;
+  const long long* tile_start;
+  float* part_u;
+  float* part_m;
+  float* lse;
+  long long budget;
+};
+size_t fwd_sm100_smem_bytes(int d, int C);
+cudaError_t fwd_sm100_max_clusters(int d, int C, int* n);
+cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream);
+
+// ---- SIMT fp32 forward
+struct FwdSimtArgs {
+  const float* X;
+  const int64_t* offsets;
+  int R, k, k_pad, d, G;
+  const float* Pf;  // folded prototypes [k_pad, d], log2 units
+  WsHeader* hdr;
+  const long long* tile_start;
+  float* lse2;      // [n_total] workspace, log2 units
+  float* lse;       // [n_total] user output (natural log), nullable
+  int64_t n_total;
+  float* part_u;
+  float* part_m;
+};
+cudaError_t launch_fwd_simt(const FwdSimtArgs& a, cudaStream_t s);
+
+// ---- SIMT backward
+struct BwdArgs {
+  const void* X;
+  sa_dtype dt;
+  const int64_t* offsets;
+  int R, k, k_pad, d, G;
+  int64_t n_total;
+  const void* P;
+  const void* Wk;
+  const void* Wv;
+  const float* sketch;
+  const float* mass;
+  const float* xsketch;
+  const float* dsketch;
+  const float* dmass;  // nullable
+  WsHeader* hdr;
+  const long long* tile_start;
+  // workspace
+  float* Pn;      // [k_pad, d]  P W_k^T / sqrt(d)
+  float* Gt;      // [R, k_pad, d]  G / mass
+  float* Gh;      // [R, k_pad, d]  (G / mass) W_v^T
+  float* cj;      // [R, k_pad]     (G / mass) . sketch - dmass
+  float* lseb;    // [n_total]      fp32 per-token log-sum-exp (natural)
+  float* Db;      // [n_total]      sum_j A_jt dA_jt
+  float* dpp_part;  // [G, k_pad, d]
+  float* dpp;       // [k_pad, d]
+  float* wv_part;   // [nchunks, d, d]
+  // outputs
+  float* dX;
+  float* dP;
+  float* dWk;
+  float* dWv;
+};
+size_t bwd_wv_chunks(int R, int k);
+cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t s);
+
+// ---- failure-detection test hook
+cudaError_t launch_debug_wait_timeout(WsHeader* hdr, long long budget, cudaStream_t s);
+
+}  // namespace sa

@@ -1,0 +1,83 @@
+"""C-ABI library: builds, loads, exports every symbol include/sa_sketch.h declares,
+and rejects bad arguments on the host before touching a GPU (no compute calls here)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "sa_sketch.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from prototype_sketch_attention_b200 import build
+    path = build.build()
+    return ctypes.CDLL(path)
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(sa_[a-z_0-9]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_expected_entry_points():
+    names = declared_functions()
+    for n in ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
+              "sa_sketch_get_device_status", "sa_status_string"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for n in declared_functions():
+        assert hasattr(lib, n), f"{n} declared in sa_sketch.h but not exported"
+
+
+def test_status_strings(lib):
+    lib.sa_status_string.restype = ctypes.c_char_p
+    lib.sa_status_string.argtypes = [ctypes.c_int]
+    for code in range(8):
+        s = lib.sa_status_string(code).decode()
+        assert s.startswith("SA_"), s
+    assert "unknown" in lib.sa_status_string(99).decode()
+
+
+def _fwd(lib, **kw):
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    lib.sa_sketch_forward.restype = i32
+    lib.sa_sketch_forward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
+                                      vp, vp, vp, vp, vp, sz, vp]
+    a = dict(X=16, offsets=16, R=1, n_total=10, d=128, P=16, k=1024, Wk=16, Wv=16, dt=1,
+             sketch=16, mass=16, lse=None, xsketch=None, ws=256, ws_bytes=1 << 30, stream=None)
+    a.update(kw)
+    return lib.sa_sketch_forward(a["X"], a["offsets"], a["R"], a["n_total"], a["d"], a["P"], a["k"],
+                                 a["Wk"], a["Wv"], a["dt"], a["sketch"], a["mass"], a["lse"],
+                                 a["xsketch"], a["ws"], a["ws_bytes"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(d=0), 2), (dict(k=0), 2), (dict(k=4096), 2),
+    (dict(R=-1), 1), (dict(n_total=-5), 1), (dict(dt=7), 1),
+    (dict(offsets=None), 1), (dict(X=None), 1), (dict(P=None), 1), (dict(sketch=None), 1),
+    (dict(X=18), 1), (dict(mass=20), 1),
+])
+def test_forward_rejects_bad_arguments_on_host(lib, kw, code):
+    """Argument errors return before any CUDA call (these run without a GPU)."""
+    assert _fwd(lib, **kw) == code
+
+
+def test_workspace_size_zero_for_unsupported(lib):
+    lib.sa_sketch_workspace_size.restype = ctypes.c_size_t
+    lib.sa_sketch_workspace_size.argtypes = [ctypes.c_int, ctypes.c_int64, ctypes.c_int,
+                                             ctypes.c_int, ctypes.c_int, ctypes.c_int]
+    assert lib.sa_sketch_workspace_size(1, 10, 1024, 96, 1, 0) == 0
+    assert lib.sa_sketch_workspace_size(1, 10, 0, 128, 1, 0) == 0
+
+
+def test_binding_names_match_header():
+    from prototype_sketch_attention_b200 import binding
+    for n in declared_functions():
+        assert n in binding.EXPORTED and hasattr(binding, n), n

@@ -1,0 +1,126 @@
+"""GPU forward parity: the CUDA path through the C ABI vs the fp64 oracle.
+
+Small cases compare every output element; they span several 128-token tiles, a ragged
+tail, empty users, users shorter than a tile, k not a multiple of 128, and every
+cluster size (k = 64 .. 2048). The full-size configurations run in the same launch
+configuration that bench.py times and are compared on sampled users (the oracle
+recomputes those users exactly), plus the unit-mass property on every user.
+"""
+import numpy as np
+import pytest
+import torch
+
+from parity_util import check_forward, gpu_forward, rel_l2
+from prototype_sketch_attention_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.mark.parametrize("lengths,k,d", [
+    ([300, 0, 1037], 128, 128),
+    ([1, 127, 128, 129], 256, 128),
+    ([2000, 55], 1024, 128),
+    ([700], 2048, 128),
+    ([513, 9], 200, 128),
+    ([640, 77], 1024, 64),
+    ([130], 64, 64),
+    ([4100, 3], 512, 128),
+])
+def test_bf16_small_full_compare(lengths, k, d):
+    w = inputs.make_workload(lengths, d, k, "bf16", seed=11 + k + d + len(lengths))
+    _, out = gpu_forward(w)
+    check_forward(w, out)
+
+
+@pytest.mark.parametrize("lengths,k,d", [
+    ([300, 0, 77], 64, 64),
+    ([1000], 1000, 128),
+    ([129, 5], 2048, 64),
+])
+def test_fp32_small_full_compare(lengths, k, d):
+    w = inputs.make_workload(lengths, d, k, "f32", seed=5 + k)
+    _, out = gpu_forward(w)
+    check_forward(w, out)
+
+
+def test_config1_fp32():
+    w = inputs.make_config(1)
+    _, out = gpu_forward(w)
+    check_forward(w, out)
+
+
+def test_config2_full_user():
+    w = inputs.make_config(2)
+    _, out = gpu_forward(w)
+    check_forward(w, out)
+
+
+def _unit_mass_all_users(w, out):
+    mass = out["mass"].double().sum(dim=1).cpu().numpy()
+    n = np.diff(w.offsets.numpy())
+    np.testing.assert_allclose(mass, n, rtol=2e-3)
+
+
+def test_config3_sampled_users():
+    w = inputs.make_config(3)
+    _, out = gpu_forward(w)
+    _unit_mass_all_users(w, out)
+    order = np.argsort(w.lengths)
+    check_forward(w, out, users=[int(order[0]), int(order[len(order) // 2])])
+
+
+@pytest.mark.parametrize("k", [256, 512, 1024, 2048])
+def test_config4_sampled_users(k):
+    w = inputs.make_config(4, k=k)
+    _, out = gpu_forward(w)
+    _unit_mass_all_users(w, out)
+    order = np.argsort(w.lengths)
+    check_forward(w, out, users=[int(order[0]), int(order[1]), int(order[150])])
+
+
+def test_deterministic_bitwise():
+    w = inputs.make_workload([5000, 123, 30000, 1], 128, 512, "bf16", seed=77)
+    g, a = gpu_forward(w)
+    from prototype_sketch_attention_b200 import binding
+    b = binding.forward(g["X"], g["offsets"], g["P"], g["Wk"], g["Wv"])
+    for key in ("sketch", "mass", "lse", "xsketch"):
+        assert torch.equal(a[key], b[key]), key
+
+
+def test_empty_batches():
+    from prototype_sketch_attention_b200 import binding
+    w = inputs.make_workload([0, 0], 128, 256, "bf16", seed=3)
+    _, out = gpu_forward(w)
+    assert not out["sketch"].any() and not out["mass"].any()
+    w0 = inputs.make_workload([], 128, 256, "bf16", seed=3)
+    g = {k: v.cuda() for k, v in dict(X=w0.X, offsets=w0.offsets, P=w0.P, Wk=w0.Wk, Wv=w0.Wv).items()}
+    out0 = binding.forward(g["X"], g["offsets"], g["P"], g["Wk"], g["Wv"])
+    assert out0["sketch"].shape == (0, 256, 128)
+
+
+def test_bad_offsets_latched_on_device():
+    from prototype_sketch_attention_b200 import binding
+    w = inputs.make_workload([200, 300], 128, 256, "bf16", seed=4)
+    g = {k: v.cuda() for k, v in dict(X=w.X, P=w.P, Wk=w.Wk, Wv=w.Wv).items()}
+    bad = torch.tensor([0, 400, 300], dtype=torch.int64, device="cuda")  # decreasing
+    out = binding.forward(g["X"], bad, g["P"], g["Wk"], g["Wv"])
+    assert binding.device_status(out["_ws"]) == binding.SA_ERR_BAD_OFFSETS
+    bad2 = torch.tensor([0, 200, 499], dtype=torch.int64, device="cuda")  # != n_total
+    out = binding.forward(g["X"], bad2, g["P"], g["Wk"], g["Wv"])
+    assert binding.device_status(out["_ws"]) == binding.SA_ERR_BAD_OFFSETS
+    # the next good call clears the status and is correct
+    _, ok = gpu_forward(w)
+    check_forward(w, ok)
+
+
+def test_bounded_wait_times_out_and_context_survives():
+    """The bounded-wait routine gives up on a barrier nothing arrives on, latches
+    SA_ERR_TIMEOUT, and the context stays usable."""
+    from prototype_sketch_attention_b200 import binding
+    ws = torch.zeros(256, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.current_stream().cuda_stream
+    assert binding.sa_sketch_debug_wait_timeout(ws.data_ptr(), 2_000_000, s) == 0
+    assert binding.sa_sketch_get_device_status(ws.data_ptr(), s) == binding.SA_ERR_TIMEOUT
+    w = inputs.make_workload([300, 40], 128, 256, "bf16", seed=8)
+    _, out = gpu_forward(w)
+    check_forward(w, out)
