@@ -1,0 +1,398 @@
+#!/usr/bin/env python
+"""Benchmark of the Sketch Attention forward (history tokens/s, fraction of bf16 peak).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+    torchrun --nproc-per-node N bench.py --gpus N ...      (one process per GPU)
+
+Workload: config 3, the training batch: R=40 users with lengths uniform in
+[10000, 100000], d=128, k=1024, bf16 inputs / fp32 accumulate, synthetic N(0,1)
+inputs from the seeded generator. One step = one sa_sketch_forward call over the
+batch (schedule, fold, tcgen05 forward, finalize). Inputs stay resident in HBM
+during the timed region, and X (453 MB) is larger than L2. With N GPUs each rank
+runs its own batch (users are independent; no collective on the data path), so
+scaling is weak and `value` is total tokens / max-over-ranks time.
+
+The JSON line also carries:
+  roofline      the tcgen05 forward kernel alone: algorithmic FLOP per launch
+                (4*k*d per token) / its CUDA-event duration vs the measured bf16 peak
+  e2e           the same metric through the public API from pinned host buffers,
+                with the per-step H2D of X and offsets and the D2H of sketch and mass
+  cpu_baseline  the fp64 oracle on the host cores, on a bounded sample (rank 0, N=1)
+  clocks        SM clock median and throttle reasons sampled during the timed region
+`--impl reference` times the oracle (the reference arm here) on the same config.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "history tokens/s of SA sketch (k=1024,d=128) and % of bf16 tensor-core peak"
+UNIT = "tokens/s"
+FALLBACK_PEAK_TFLOPS = 1590.0
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sa_fwd_sm100_config3.md")
+KERNEL_SOURCES = [os.path.join(ROOT, "prototype_sketch_attention_b200", "csrc", f)
+                  for f in ("sa_fwd_sm100.cu", "sa_common.cuh")]
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        with open(f, "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["bf16_tflops"]), "measured (MEASURED_PEAKS.json bf16_tflops, burst)"
+    except Exception:
+        return FALLBACK_PEAK_TFLOPS, "fallback (1.59 PFLOP/s, profiling recipe)"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the
+    current kernel source (null otherwise)."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith(("source_sha256", "dram_bytes_per_launch")):
+            key, v = line.strip().split(":", 1)
+            vals[key.strip()] = v.strip().strip("`")
+    if vals.get("source_sha256") != kernel_source_hash():
+        return None
+    try:
+        return int(float(vals["dram_bytes_per_launch"]))
+    except (KeyError, ValueError):
+        return None
+
+
+def event_ms(a, b) -> float:
+    """Milliseconds between two torch.cuda.Event objects that the library recorded
+    itself (cudaEventRecord inside libsa_sketch.so), read through the CUDA runtime."""
+    import ctypes
+    lib = ctypes.CDLL("libcudart.so.12")
+    ms = ctypes.c_float(0.0)
+    rc = lib.cudaEventElapsedTime(ctypes.byref(ms), ctypes.c_void_p(a.cuda_event),
+                                  ctypes.c_void_p(b.cuda_event))
+    if rc != 0:
+        raise RuntimeError(f"cudaEventElapsedTime failed: {rc}")
+    return float(ms.value)
+
+
+# ------------------------------------------------------------------ clocks
+THROTTLE_BITS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap",
+                 0x8: "hw_slowdown", 0x10: "sync_boost", 0x20: "sw_thermal_slowdown",
+                 0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons with NVML while the timed region runs."""
+
+    def __init__(self, torch_device_index: int):
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._h = None
+        try:
+            import pynvml
+            import torch
+            pynvml.nvmlInit()
+            props = torch.cuda.get_device_properties(torch_device_index)
+            bus = "%08x:%02x:%02x.0" % (props.pci_domain_id, props.pci_bus_id, props.pci_device_id)
+            try:
+                self._h = pynvml.nvmlDeviceGetHandleByPciBusId(bus)
+            except Exception:
+                self._h = pynvml.nvmlDeviceGetHandleByIndex(torch_device_index)
+            self._nv = pynvml
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # no NVML: clocks stay empty and are reported as such
+            self.error = repr(e)
+        self._t = threading.Thread(target=self._run, daemon=True)
+
+    def _reasons(self):
+        nv = self._nv
+        for fn in ("nvmlDeviceGetCurrentClocksEventReasons", "nvmlDeviceGetCurrentClocksThrottleReasons"):
+            if hasattr(nv, fn):
+                return getattr(nv, fn)(self._h)
+        return 0
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self._nv.nvmlDeviceGetClockInfo(self._h, self._nv.NVML_CLOCK_SM))
+                self.reasons |= int(self._reasons())
+            except Exception:
+                pass
+            time.sleep(0.002)
+
+    def __enter__(self):
+        if self._h is not None:
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t.is_alive():
+            self._t.join()
+
+    def summary(self) -> dict:
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": [], "samples": 0}
+        names = [n for b, n in THROTTLE_BITS.items() if self.reasons & b and n != "gpu_idle"]
+        return {"sm_mhz": float(statistics.median(self.samples)), "sm_max_mhz": self.max_mhz,
+                "reasons": names, "samples": len(self.samples)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_sample_rate(w, target_s: float, max_tokens: int = 200_000):
+    """Times the fp64 oracle on the first S tokens of user 0 (S sized for ~target_s).
+    Returns (tokens/s, tokens, seconds, threads)."""
+    import numpy as np
+    import oracle
+    threads = os.cpu_count() or 1
+    off = w.offsets.numpy()
+    n0 = int(off[1] - off[0])
+    P = w.P.double().numpy()
+    Wk = w.Wk.double().numpy()
+    Wv = w.Wv.double().numpy()
+
+    def run(S):
+        X = w.X[:S].double().numpy()
+        t0 = time.perf_counter()
+        oracle.forward(X, np.array([0, S], dtype=np.int64), P, Wk, Wv, nthreads=threads)
+        return time.perf_counter() - t0
+
+    probe = min(n0, 2048)
+    tp = run(probe)
+    S = int(min(n0, max_tokens, max(probe, probe * target_s / max(tp, 1e-6))))
+    t = run(S) if S != probe else tp
+    used = min(threads, math.ceil(S / 1024))  # the oracle parallelises over 1024-token chunks
+    return S / t, S, t, used
+
+
+# ------------------------------------------------------------------ reference arm
+def run_reference(args) -> None:
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    from prototype_sketch_attention_b200 import inputs
+    w = inputs.make_config(3)
+    import numpy as np
+    import oracle
+    threads = os.cpu_count() or 1
+    # each step: the oracle on a bounded sample of user 0 (whole run within a few minutes)
+    per_step_target = max(0.5, 150.0 / max(1, args.steps + args.warmup))
+    rate, S, t, used = oracle_sample_rate(w, per_step_target)
+    P, Wk, Wv = (w.P.double().numpy(), w.Wk.double().numpy(), w.Wv.double().numpy())
+    X = w.X[:S].double().numpy()
+    off = np.array([0, S], dtype=np.int64)
+    for _ in range(args.warmup):
+        oracle.forward(X, off, P, Wk, Wv, nthreads=threads)
+    times = []
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        oracle.forward(X, off, P, Wk, Wv, nthreads=threads)
+        times.append(time.perf_counter() - t0)
+    step_s = sum(times) / len(times)
+    value = S / step_s
+    sample = f"first {S} tokens of user 0 of config 3 per step (k=1024, d=128), fp64 oracle"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic",
+        "config": {"workload": w.meta["desc"], "n_total": w.n_total, "sample_tokens": S},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, math.ceil(S / 1024)),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args) -> None:
+    import torch
+    import torch.distributed as dist
+    from prototype_sketch_attention_b200 import binding, inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != args.gpus:
+        raise SystemExit(f"--gpus {args.gpus} but WORLD_SIZE={world}: launch N>1 with torchrun")
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    w = inputs.make_config(3)
+    if rank > 0:  # each rank its own batch of users, same length recipe
+        gen = torch.Generator().manual_seed(1003 + 7919 * rank)
+        lengths = inputs.draw_lengths(inputs.CONFIGS[3]["lengths"], 40, gen)
+        w = inputs.make_workload(lengths, 128, 1024, "bf16", seed=0, gen=gen, name="config3")
+    X = w.X.to(dev)
+    off = w.offsets.to(dev)
+    P, Wk, Wv = w.P.to(dev), w.Wk.to(dev), w.Wv.to(dev)
+    n_total, d, k, R = w.n_total, w.d, w.k, w.R
+    out = binding.forward(X, off, P, Wk, Wv)
+    ws = out["_ws"]
+    st = binding.device_status(ws)
+    if st != 0:
+        raise SystemExit(f"forward failed on device: {binding.sa_status_string(st)}")
+    stream = torch.cuda.current_stream()
+
+    def step():
+        binding.forward(X, off, P, Wk, Wv, ws=ws, out=out)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for a, b in ev_k:  # torch creates the CUDA event on first record: materialise the handles
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            binding.sa_sketch_profile_events(ev_k[i][0].cuda_event, ev_k[i][1].cuda_event)
+            step()
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    binding.sa_sketch_profile_events(None, None)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    kern_ms = sum(event_ms(a, b) for a, b in ev_k) / args.steps
+    st = binding.device_status(ws)
+    if st != 0:
+        raise SystemExit(f"forward failed on device: {binding.sa_status_string(st)}")
+
+    # ---- e2e through the public API: pinned host inputs -> device -> forward -> host
+    Xh = w.X.pin_memory()
+    offh = w.offsets.pin_memory()
+    Xd = torch.empty_like(X)
+    offd = torch.empty_like(off)
+    sk_h = torch.empty(R, k, d, dtype=torch.float32).pin_memory()
+    ms_h = torch.empty(R, k, dtype=torch.float32).pin_memory()
+    e2e_steps = max(3, min(args.steps, 20))
+
+    def e2e_step():
+        Xd.copy_(Xh, non_blocking=True)
+        offd.copy_(offh, non_blocking=True)
+        binding.forward(Xd, offd, P, Wk, Wv, ws=ws, out=out)
+        sk_h.copy_(out["sketch"], non_blocking=True)
+        ms_h.copy_(out["mass"], non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+
+    # ---- max over ranks
+    t = torch.tensor([elapsed_ms, e2e_ms, kern_ms, float(n_total)], dtype=torch.float64, device=dev)
+    if world > 1:
+        tmax = t[:3].clone()
+        dist.all_reduce(tmax, op=dist.ReduceOp.MAX)
+        tot = t[3:].clone()
+        dist.all_reduce(tot, op=dist.ReduceOp.SUM)
+        elapsed_ms, e2e_ms, kern_ms = tmax.tolist()
+        total_tokens = tot.item()
+    else:
+        total_tokens = float(n_total)
+    ms_per_step = elapsed_ms / args.steps
+    value = total_tokens / (ms_per_step / 1e3)
+    peak, peak_src = measured_peak()
+    flop_per_launch = 4.0 * k * d * n_total
+    achieved = flop_per_launch / (kern_ms / 1e3) / 1e12
+    step_tflops = 4.0 * k * d * total_tokens / (ms_per_step / 1e3) / 1e12
+    h2d = X.numel() * X.element_size() + off.numel() * 8
+    d2h = sk_h.numel() * 4 + ms_h.numel() * 4
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, S, secs, used = oracle_sample_rate(w, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle",
+               "sample": f"first {S} tokens of user 0 of config 3 (k=1024, d=128), fp64 oracle, "
+                         f"{secs:.1f} s wall"}
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": "config3: R=40 users, n~U[10000,100000], d=128, k=1024, bf16 in / "
+                               "fp32 accumulate, forward",
+                   "n_total_per_gpu": n_total, "R": R, "k": k, "d": d,
+                   "l2": "inputs larger than L2 (X is %.0f MB per GPU)" % (h2d / 1e6),
+                   "parallelism": f"users sharded, {world} independent batch(es)"},
+        "pct_of_peak": step_tflops / peak,
+        "step_tflops": step_tflops,
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": profiled_traffic(),
+                     "kernel": "sa_fwd_sm100_kernel<128>", "kernel_ms": kern_ms,
+                     "peak_source": peak_src, "flop_per_launch": flop_per_launch},
+        "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if cpu is not None:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None) -> int:
+    ap = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -109,7 +109,10 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
  * respect to X, P, Wk and Wv.
  *
  *   X, offsets, P, Wk, Wv, dt   as passed to the forward
- *   sketch, mass, lse, xsketch  fp32 outputs of that forward (lse, xsketch required)
+ *   sketch, mass, xsketch       fp32 outputs of that forward (required)
+ *   lse                         the forward's lse; nullable and not read: this
+ *                               implementation recomputes the per-token statistics
+ *                               it needs in fp32
  *   dsketch [R, k, d] fp32      G
  *   dmass   [R, k]    fp32      Gm; nullable (NULL means zero)
  * Outputs (fp32, overwritten, not accumulated into):
@@ -130,6 +133,17 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
  * every forward and backward call.
  */
 int sa_sketch_get_device_status(const void* workspace, void* stream);
+
+/*
+ * Measurement hook. When both handles are non-null, every later sa_sketch_forward
+ * call made by this host thread records `start_event` on its stream just before the
+ * main forward kernel (the tcgen05 kernel for bf16, the SIMT kernels for fp32) and
+ * `stop_event` just after it. The caller then reads that kernel's own duration with
+ * cudaEventElapsedTime. Both handles are cudaEvent_t passed as void*; the caller owns
+ * them. Passing two nulls turns the hook off. Returns SA_OK, or SA_ERR_INVALID_ARG if
+ * exactly one handle is null.
+ */
+int sa_sketch_profile_events(void* start_event, void* stop_event);
 
 /* Static, human-readable name of a status code. */
 const char* sa_status_string(int status);

@@ -29,7 +29,8 @@ SA_ERR_BAD_OFFSETS = 6
 SA_ERR_NO_DEVICE = 7
 
 EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
-            "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout")
+            "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
+            "sa_sketch_profile_events")
 
 
 class SketchAttentionError(RuntimeError):
@@ -58,6 +59,8 @@ def _load() -> ctypes.CDLL:
     lib.sa_status_string.argtypes = [i32]
     lib.sa_sketch_debug_wait_timeout.restype = i32
     lib.sa_sketch_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
+    lib.sa_sketch_profile_events.restype = i32
+    lib.sa_sketch_profile_events.argtypes = [vp, vp]
     return lib
 
 
@@ -92,6 +95,10 @@ def sa_status_string(status: int) -> str:
 
 def sa_sketch_debug_wait_timeout(workspace, budget_cycles: int, stream) -> int:
     return int(_lib.sa_sketch_debug_wait_timeout(workspace, int(budget_cycles), stream))
+
+
+def sa_sketch_profile_events(start_event, stop_event) -> int:
+    return int(_lib.sa_sketch_profile_events(start_event, stop_event))
 
 
 # ---------------------------------------------------------------- torch conveniences

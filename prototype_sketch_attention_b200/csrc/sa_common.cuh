@@ -245,9 +245,38 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32]) {
   for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+// 32 lanes x 32 columns into raw registers (no wait); pair with tmem_wait_tie.
+__device__ __forceinline__ void tmem_ld32_raw(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15,"
+      " %16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr)
+      : "memory");
+}
+
+// tcgen05.wait::ld that also carries the loaded registers as in/out operands, so no
+// use of them can be scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_tie(uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]),
+        "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]),
+        "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+      :
+      : "memory");
+}
+
 // Shared-memory matrix descriptor for tcgen05 (start, leading and stride byte
 // offsets in 16-byte units; version 1; swizzle mode in bits 61..63).
-enum : uint32_t { kSwizzleNone = 0, kSwizzle128B = 2 };
+enum : uint32_t { kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle32B = 6 };
 
 __device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo,
                                               uint32_t swizzle) {
@@ -269,6 +298,90 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, int a_mn, in
          | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16)
          | ((uint32_t)(N >> 3) << 17)   // N / 8
          | ((uint32_t)(M >> 4) << 24);  // M / 16
+}
+
+// ---------------------------------------------------------------- packed fp32 (sm_100)
+// Two fp32 lanes in one 64-bit register pair: one instruction, two results.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.ftz.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("mul.rn.ftz.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+__device__ __forceinline__ uint32_t cvt_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// 2^x for two packed fp32 values x <= 0, on the FMA pipe instead of the MUFU.
+// x = n + f with n = round(x) (add and subtract 1.5 * 2^23), f in [-1/2, 1/2];
+// 2^f by a degree-4 polynomial (relative error 2.7e-6 in fp32 Horner; coefficients
+// from csrc/gen_exp2_poly.py, a relative-error least-squares fit refined toward
+// minimax by Lawson reweighting); 2^n by adding n to the exponent field.
+// Inputs below -125 are clamped (2^-125 is ~2e-38, below every other term).
+__device__ __forceinline__ uint64_t exp2_poly2(uint64_t x2) {
+  constexpr float kC0 = 0.9999992847442627f;
+  constexpr float kC1 = 0.6931217908859253f;
+  constexpr float kC2 = 0.240247443318367f;
+  constexpr float kC3 = 0.05591785907745361f;
+  constexpr float kC4 = 0.009570096619427204f;
+  constexpr float kMagic = 12582912.0f;  // 1.5 * 2^23
+  float a, b;
+  f2_unpack(x2, a, b);
+  const uint64_t x = f2_pack(fmaxf(a, -125.f), fmaxf(b, -125.f));
+  const uint64_t t = f2_add(x, f2_pack(kMagic, kMagic));      // magic + n
+  const uint64_t n = f2_add(t, f2_pack(-kMagic, -kMagic));    // n as float
+  const uint64_t f = f2_fma(n, f2_pack(-1.f, -1.f), x);       // x - n
+  uint64_t p = f2_fma(f2_pack(kC4, kC4), f, f2_pack(kC3, kC3));
+  p = f2_fma(p, f, f2_pack(kC2, kC2));
+  p = f2_fma(p, f, f2_pack(kC1, kC1));
+  p = f2_fma(p, f, f2_pack(kC0, kC0));
+  float pa, pb, ta, tb;
+  f2_unpack(p, pa, pb);
+  f2_unpack(t, ta, tb);
+  const float ra = __int_as_float(__float_as_int(pa) + (__float_as_int(ta) << 23));
+  const float rb = __int_as_float(__float_as_int(pb) + (__float_as_int(tb) << 23));
+  return f2_pack(ra, rb);
+}
+
+// Non-blocking probe of an mbarrier phase (for issue loops that poll several barriers).
+__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+  return ok != 0;
+}
+
+// Pull one TMA box into L2 ahead of its load (no shared memory involved).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const void* tmap, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global [%0, {%1, %2}];"
+               ::"l"(reinterpret_cast<uint64_t>(tmap)), "r"(x), "r"(y) : "memory");
 }
 
 // ---------------------------------------------------------------- math

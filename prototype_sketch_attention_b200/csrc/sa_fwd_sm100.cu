@@ -37,20 +37,21 @@ constexpr int kXchSlots = 4;                  // exchange slots (tile index mod 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColU = 256;
 
-template <int D>
+template <int D, int NS>
 struct FwdSmem {
-  static constexpr int kStages = (D == 128) ? 3 : 4;
-  static constexpr int kBoxBytes = 128 * 64 * 2;            // one TMA box: 128 rows x 64 bf16
-  static constexpr int kXStage = 128 * D * 2;                // X tile
+  static constexpr int kStages = NS;
+  static constexpr int kBoxBytes = 128 * 16 * 2;             // X TMA box: 128 rows x 16 bf16 (32B swizzle)
+  static constexpr int kXBytes = 128 * D * 2;                // X tile
+  static constexpr int kOnesBytes = 128 * 16 * 2;            // all-ones 16-column atom after X
+  static constexpr int kXStage = kXBytes + kOnesBytes;
+  static constexpr int kPBox = 128 * 64 * 2;                 // P' TMA box: 128 rows x 64 bf16 (128B swizzle)
   static constexpr int kPBytes = kProtoSlice * D * 2;        // P' slice
   static constexpr int kABytes = kProtoSlice * kTileTokens * 2;  // A tile (bf16)
-  static constexpr int kOnesBytes = 512;
   // byte offsets from the 1024-aligned base
   static constexpr int oX = 0;
   static constexpr int oP = oX + kStages * kXStage;
   static constexpr int oA = oP + kPBytes;
-  static constexpr int oOnes = oA + 2 * kABytes;
-  static constexpr int oXch = oOnes + kOnesBytes;  // kXchSlots * C * 128 floats (runtime C)
+  static constexpr int oXch = oA + 2 * kABytes;  // kXchSlots * C * 128 floats (runtime C)
   static size_t bytes(int C) {
     const size_t xch = (size_t)kXchSlots * C * 128 * 4;
     const size_t bars = 64 * 8 + 16;
@@ -62,7 +63,7 @@ struct Bars {
   uint64_t x_full[4], x_empty[4];
   uint64_t s_full[2], s_empty[2];
   uint64_t a_full[2], a_empty[2];
-  uint64_t u_full, u_empty;
+  uint64_t u_full[2], u_empty;  // u_full[w]: segments whose last tile warpgroup w owns
   uint64_t xch[kXchSlots];
   uint64_t p_full, drain;
   uint32_t tmem_base;
@@ -74,16 +75,21 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
   return __uint_as_float(r);
 }
 
-template <int D>
-__global__ void __launch_bounds__(192, 1)
+constexpr int kNWG = 2;                        // softmax warpgroups (ping-pong on tiles)
+// warps 0-3: TMA producer (0), TMEM allocator and MMA issuer (1), idle (2, 3);
+// warps 4-11: the two softmax warpgroups
+constexpr int kThreads = 128 + 128 * kNWG;
+constexpr int kPrefetchAhead = 4;               // tiles prefetched into L2 ahead of the load
+
+template <int D, int NS>
+__global__ void __launch_bounds__(kThreads, 1)
 sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_p,
                     const int64_t* __restrict__ offsets, int R, int k_valid, int C, int k_pad,
                     WsHeader* hdr, const long long* __restrict__ tile_start,
                     float* __restrict__ part_u, float* __restrict__ part_m,
                     float* __restrict__ lse_out, long long budget) {
-  using L = FwdSmem<D>;
-  constexpr int NS = L::kStages;
+  using L = FwdSmem<D, NS>;
   constexpr int KSTEPS1 = D / 16;           // MMA1 K steps (over d)
   constexpr int KSTEPS2 = kTileTokens / 16;  // MMA2 K steps (over tokens)
   extern __shared__ uint8_t smem_raw[];
@@ -110,7 +116,8 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
       mbar_init(smem_u32(&bars->a_full[s]), 4);
       mbar_init(smem_u32(&bars->a_empty[s]), 1);
     }
-    mbar_init(smem_u32(&bars->u_full), 1);
+    mbar_init(smem_u32(&bars->u_full[0]), 1);
+    mbar_init(smem_u32(&bars->u_full[1]), 1);
     mbar_init(smem_u32(&bars->u_empty), 4);
     for (int s = 0; s < kXchSlots; ++s) mbar_init(smem_u32(&bars->xch[s]), 1);
     mbar_init(smem_u32(&bars->p_full), 1);
@@ -121,11 +128,14 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
     tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
     tmem_relinquish();
   }
-  if (warp >= 2) {
-    // all-ones bf16 block: B operand of the mass MMA (16 x 16, K-major, no swizzle)
-    const int t = threadIdx.x - 64;
-    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + L::oOnes);
-    if (t < L::kOnesBytes / 4) ones[t] = 0x3F803F80u;
+  if (warp >= 4) {
+    // the all-ones atom after every X stage: MMA2 runs with N = d + 16, so the 16
+    // extra output columns accumulate sum_t A_jt (the mass) next to U
+    const int t = threadIdx.x - 128;
+    for (int s2 = 0; s2 < NS; ++s2) {
+      uint32_t* ones = reinterpret_cast<uint32_t*>(smem + L::oX + s2 * L::kXStage + L::kXBytes);
+      for (int w = t; w < L::kOnesBytes / 4; w += kThreads - 128) ones[w] = 0x3F803F80u;
+    }
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -139,26 +149,35 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
   const long long ta = (long long)cid * T / ncl, tb = (long long)(cid + 1) * T / ncl;
 
   if (warp == 0) {
-    // ================= TMA producer
+    // ================= TMA producer (+ L2 prefetch of upcoming tiles by rank 0)
     if (lane == 0 && ta < tb) {
       tma_prefetch_desc(&tmap_x);
       tma_prefetch_desc(&tmap_p);
       const uint32_t pf = smem_u32(&bars->p_full);
       mbar_arrive_expect_tx(pf, L::kPBytes);
       for (int b = 0; b < D / 64; ++b)
-        tma_load_2d(sbase + L::oP + b * L::kBoxBytes, &tmap_p, b * 64, (int)rank * kProtoSlice, pf);
-      TileIter it;
+        tma_load_2d(sbase + L::oP + b * L::kPBox, &tmap_p, b * 64, (int)rank * kProtoSlice, pf);
+      TileIter it, ahead;
       it.init(tile_start, offsets, R, ta, tb);
+      ahead.init(tile_start, offsets, R, ta, tb);
+      if (rank == 0) {
+        for (int j = 0; j < kPrefetchAhead && ahead.valid(); ++j, ahead.next())
+          for (int b = 0; b < D / 16; ++b) tma_prefetch_l2_2d(&tmap_x, b * 16, (int)ahead.t0());
+      }
       long long i = 0;
       for (; it.valid(); it.next(), ++i) {
         const int st = (int)(i % NS);
         const uint32_t par = (uint32_t)((i / NS) & 1);
         if (!mbar_wait(smem_u32(&bars->x_empty[st]), par ^ 1u, status, budget)) break;
         const uint32_t fb = smem_u32(&bars->x_full[st]);
-        mbar_arrive_expect_tx(fb, L::kXStage);
+        mbar_arrive_expect_tx(fb, L::kXBytes);
         const int y = (int)it.t0();
-        for (int b = 0; b < D / 64; ++b)
-          tma_load_2d(sbase + L::oX + st * L::kXStage + b * L::kBoxBytes, &tmap_x, b * 64, y, fb);
+        for (int b = 0; b < D / 16; ++b)
+          tma_load_2d(sbase + L::oX + st * L::kXStage + b * L::kBoxBytes, &tmap_x, b * 16, y, fb);
+        if (rank == 0 && ahead.valid()) {
+          for (int b = 0; b < D / 16; ++b) tma_prefetch_l2_2d(&tmap_x, b * 16, (int)ahead.t0());
+          ahead.next();
+        }
       }
       // drain: the loads of the last NS tiles issued must have landed before exit
       for (long long j = (i > NS ? i - NS : 0); j < i; ++j)
@@ -166,120 +185,174 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
       mbar_wait_drain(pf, 0, budget);
     }
   } else if (warp == 1) {
-    // ================= MMA issuer
+    // ================= MMA issuer: MMA1 (scores) and MMA2 (accumulate) issued in
+    // whatever order their inputs become ready, each stream in tile order.
     if (lane == 0 && ta < tb) {
       const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);  // S^T = X . P'^T
-      const uint32_t idesc2 = idesc_bf16_f32(128, D, 1, 1);            // U += A . X
-      const uint32_t idescm = idesc_bf16_f32(128, 16, 1, 0);           // mass += A . 1
-      const uint64_t ones_desc = smem_desc(sbase + L::oOnes, 128, 256, kSwizzleNone);
+      const uint32_t idesc2 = idesc_bf16_f32(128, D + 16, 1, 1);       // [U | mass] += A . [X | 1]
       bool ok = mbar_wait(smem_u32(&bars->p_full), 0, status, budget);
+      struct Info {
+        int st, seg;
+        bool first, last;
+      } ring[4];
       TileIter it;
       it.init(tile_start, offsets, R, ta, tb);
-      long long i = 0;
+      const long long ntile = tb - ta;
+      long long i1 = 0, i2 = 0;
       int seg = -1;
-      // pending MMA2 (one tile behind MMA1)
-      long long pj = -1;
-      bool pfirst = false, plast = false;
-      int pseg = 0;
-      auto issue_mma2 = [&](long long j, bool first, bool last, int sg) -> bool {
-        const int ab = (int)(j & 1);
-        const int st = (int)(j % NS);
-        if (!mbar_wait(smem_u32(&bars->a_full[ab]), (uint32_t)((j >> 1) & 1), status, budget))
-          return false;
-        if (first && !mbar_wait(smem_u32(&bars->u_empty), (uint32_t)((sg & 1) ^ 1), status, budget))
-          return false;
-        tc_fence_after();
-        const uint32_t a_base = sbase + L::oA + ab * L::kABytes;
-        const uint32_t x_base = sbase + L::oX + st * L::kXStage;
+      long long t_prog = clock64();
+      uint32_t spins = 0;
+      while (ok && i2 < ntile) {
+        bool prog = false;
+        if (i1 < ntile) {
+          const int st = (int)(i1 % NS);
+          const int sb = (int)(i1 & 1);
+          if (mbar_test(smem_u32(&bars->x_full[st]), (uint32_t)((i1 / NS) & 1)) &&
+              mbar_test(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i1 >> 1) & 1) ^ 1))) {
+            tc_fence_after();
+            const uint32_t x_base = sbase + L::oX + st * L::kXStage;
+            const uint32_t p_base = sbase + L::oP;
 #pragma unroll
-        for (int ks = 0; ks < KSTEPS2; ++ks) {
-          const uint64_t ad = smem_desc(a_base + ks * 2048, L::kBoxBytes, 1024, kSwizzle128B);
-          const uint64_t bd = smem_desc(x_base + ks * 2048, L::kBoxBytes, 1024, kSwizzle128B);
-          const uint32_t acc = (first && ks == 0) ? 0u : 1u;
-          tc_mma_f16(tmem + kColU, ad, bd, idesc2, acc);
-          tc_mma_f16(tmem + kColU + D, ad, ones_desc, idescm, acc);
+            for (int ks = 0; ks < KSTEPS1; ++ks) {
+              // A = X tile, K-major, 32B swizzle: one 16-wide K step per 4 KB atom column
+              const uint64_t ad = smem_desc(x_base + ks * L::kBoxBytes, 16, 256, kSwizzle32B);
+              // B = P' slice, K-major, 128B swizzle: four 16-wide K steps per 16 KB box
+              const uint32_t koff = (ks >> 2) * L::kPBox + (ks & 3) * 32;
+              const uint64_t bd = smem_desc(p_base + koff, 16, 1024, kSwizzle128B);
+              tc_mma_f16(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc1, ks > 0 ? 1u : 0u);
+            }
+            tc_commit(smem_u32(&bars->s_full[sb]));
+            const bool first = it.first();
+            if (first) ++seg;
+            ring[i1 & 3] = Info{st, seg, first, it.last()};
+            it.next();
+            ++i1;
+            prog = true;
+          }
         }
-        tc_commit(smem_u32(&bars->x_empty[st]));
-        tc_commit(smem_u32(&bars->a_empty[ab]));
-        if (last) tc_commit(smem_u32(&bars->u_full));
-        return true;
-      };
-      for (; ok && it.valid(); it.next(), ++i) {
-        const bool first = it.first(), last = it.last();
-        if (first) ++seg;
-        const int st = (int)(i % NS);
-        const int sb = (int)(i & 1);
-        ok = mbar_wait(smem_u32(&bars->x_full[st]), (uint32_t)((i / NS) & 1), status, budget) &&
-             mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget);
-        if (!ok) break;
-        tc_fence_after();
-        const uint32_t x_base = sbase + L::oX + st * L::kXStage;
-        const uint32_t p_base = sbase + L::oP;
+        if (i2 < i1) {
+          const Info f = ring[i2 & 3];
+          const int ab = (int)(i2 & 1);
+          if (mbar_test(smem_u32(&bars->a_full[ab]), (uint32_t)((i2 >> 1) & 1)) &&
+              (!f.first || mbar_test(smem_u32(&bars->u_empty), (uint32_t)((f.seg & 1) ^ 1)))) {
+            tc_fence_after();
+            const uint32_t a_base = sbase + L::oA + ab * L::kABytes;
+            const uint32_t x_base = sbase + L::oX + f.st * L::kXStage;
 #pragma unroll
-        for (int ks = 0; ks < KSTEPS1; ++ks) {
-          const uint32_t koff = (ks >> 2) * L::kBoxBytes + (ks & 3) * 32;
-          const uint64_t ad = smem_desc(x_base + koff, 16, 1024, kSwizzle128B);
-          const uint64_t bd = smem_desc(p_base + koff, 16, 1024, kSwizzle128B);
-          tc_mma_f16(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc1, ks > 0 ? 1u : 0u);
+            for (int ks = 0; ks < KSTEPS2; ++ks) {
+              // A = A tile, MN-major (prototypes contiguous), 128B swizzle
+              const uint64_t ad = smem_desc(a_base + ks * 2048, L::kPBox, 1024, kSwizzle128B);
+              // B = [X | 1], MN-major (d contiguous), 32B swizzle: 16-wide N atoms 4 KB apart
+              const uint64_t bd = smem_desc(x_base + ks * 512, L::kBoxBytes, 256, kSwizzle32B);
+              const uint32_t acc = (f.first && ks == 0) ? 0u : 1u;
+              tc_mma_f16(tmem + kColU, ad, bd, idesc2, acc);
+            }
+            tc_commit(smem_u32(&bars->x_empty[f.st]));
+            tc_commit(smem_u32(&bars->a_empty[ab]));
+            if (f.last) tc_commit(smem_u32(&bars->u_full[i2 & 1]));
+            ++i2;
+            prog = true;
+          }
         }
-        tc_commit(smem_u32(&bars->s_full[sb]));
-        if (pj >= 0) {
-          ok = issue_mma2(pj, pfirst, plast, pseg);
-          if (!ok) break;
+        if (prog) {
+          t_prog = clock64();
+          spins = 0;
+        } else if ((++spins & 63u) == 0u) {
+          if (read_status(status) != 0) ok = false;
+          else if (clock64() - t_prog > budget) {
+            latch_status(status, SA_ERR_TIMEOUT);
+            ok = false;
+          }
         }
-        pj = i; pfirst = first; plast = last; pseg = seg;
       }
-      if (ok && pj >= 0) issue_mma2(pj, pfirst, plast, pseg);
       // drain every tcgen05 op this thread issued before the CTA tears down
       tc_commit(smem_u32(&bars->drain));
       mbar_wait_drain(smem_u32(&bars->drain), 0, budget);
     }
-  } else {
-    // ================= softmax + epilogue warpgroup (warps 2..5; TMEM lane quadrant = warp % 4)
-    const int q = warp & 3;
+  } else if (warp >= 4) {
+    // ================= softmax + epilogue: warpgroup wg takes the tiles i with i % 2 == wg
+    const int wg = (warp >> 2) - 1;
+    const int q = warp & 3;                   // TMEM lane quadrant of this warp
     const int r = q * 32 + lane;              // token row in the tile == TMEM lane
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    const bool leader = (threadIdx.x == 64);
+    const bool leader = (threadIdx.x & 127) == 0;
     const int pbase = (int)rank * kProtoSlice;
+    const bool partial_slice = pbase + kProtoSlice > k_valid;
     TileIter it;
     it.init(tile_start, offsets, R, ta, tb);
     long long i = 0;
-    int seg = -1;
+    int useg = 0;  // segments whose last tile this warpgroup owned so far (u_full[wg] phases)
     bool ok = true;
     for (; ok && it.valid(); it.next(), ++i) {
-      if (it.first()) ++seg;
-      const int sb = (int)(i & 1);
+      if ((int)(i & 1) != wg) continue;
+      const int sb = wg;
       if (!mbar_wait_warp(smem_u32(&bars->s_full[sb]), (uint32_t)((i >> 1) & 1), status, budget)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      float e[kProtoSlice];
+      float v[kProtoSlice];
+      {
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        const uint32_t ta0 = tmem + lane_off + (sb ? kColS1 : kColS0);
+        tmem_ld32_raw(ta0 + 0, r0);
+        tmem_ld32_raw(ta0 + 32, r1);
+        tmem_ld32_raw(ta0 + 64, r2);
+        tmem_ld32_raw(ta0 + 96, r3);
+        tmem_wait_tie(r0);
+        tmem_wait_tie(r1);
+        tmem_wait_tie(r2);
+        tmem_wait_tie(r3);
 #pragma unroll
-      for (int c = 0; c < kProtoSlice / 32; ++c) {
-        float v[32];
-        tmem_ld32(tmem + lane_off + (sb ? kColS1 : kColS0) + c * 32, v);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) e[c * 32 + x] = v[x];
+        for (int x = 0; x < 32; ++x) {
+          v[x] = __uint_as_float(r0[x]);
+          v[32 + x] = __uint_as_float(r1[x]);
+          v[64 + x] = __uint_as_float(r2[x]);
+          v[96 + x] = __uint_as_float(r3[x]);
+        }
       }
-      tc_wait_ld();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[sb]));
 
-      // local (this slice) max and log2-sum-exp2
-      float m = -INFINITY;
+      if (partial_slice) {
 #pragma unroll
-      for (int c = 0; c < kProtoSlice; ++c) {
-        if (pbase + c >= k_valid) e[c] = -INFINITY;
-        m = fmaxf(m, e[c]);
+        for (int c = 0; c < kProtoSlice; ++c)
+          if (pbase + c >= k_valid) v[c] = -INFINITY;
       }
-      float z = 0.f;
+      // local max: four independent chains of 3-input max
+      float mc[4];
 #pragma unroll
-      for (int c = 0; c < kProtoSlice; ++c) {
-        e[c] = ex2_approx(e[c] - m);
-        z += e[c];
+      for (int j = 0; j < 4; ++j) {
+        float a = fmaxf(v[32 * j], v[32 * j + 31]);
+#pragma unroll
+        for (int c = 1; c < 31; c += 2) a = fmax3(a, v[32 * j + c], v[32 * j + c + 1]);
+        mc[j] = a;
       }
+      const float m = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+      // e = 2^(s - m) and its sum (packed subtract, four packed accumulators)
+      const uint64_t nm2 = f2_pack(-m, -m);
+      uint64_t za[4] = {0ull, 0ull, 0ull, 0ull};
+      // prototypes [0, 64) on the MUFU, [64, 128) on the FMA pipe: the MUFU's 16
+      // results per clock per SM would otherwise match the tensor core's time per tile
+#pragma unroll
+      for (int p = 0; p < kProtoSlice / 2; ++p) {
+        float a, b;
+        const uint64_t xm = f2_add(f2_pack(v[2 * p], v[2 * p + 1]), nm2);
+        if (p < kProtoSlice / 4) {
+          f2_unpack(xm, a, b);
+          a = ex2_approx(a);
+          b = ex2_approx(b);
+        } else {
+          f2_unpack(exp2_poly2(xm), a, b);
+        }
+        v[2 * p] = a;
+        v[2 * p + 1] = b;
+        za[p & 3] = f2_add(za[p & 3], f2_pack(a, b));
+      }
+      float z0, z1;
+      f2_unpack(f2_add(f2_add(za[0], za[1]), f2_add(za[2], za[3])), z0, z1);
+      const float z = z0 + z1;
       const int nv = it.nvalid();
       const bool valid = r < nv;
       const float l = valid ? m + lg2_approx(z) : 0.f;
@@ -313,23 +386,27 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
 
       // A (bf16) into the MN-major, 128B-swizzled A operand: row = token, 64 prototypes
       // per 128-byte row, two 16 KB blocks for prototypes [0,64) and [64,128).
-      const int ab = (int)(i & 1);
+      const int ab = wg;
       if (!mbar_wait_warp(smem_u32(&bars->a_empty[ab]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget)) {
         ok = false;
         break;
       }
       uint8_t* arow = smem + L::oA + ab * L::kABytes + r * 128;
+      const uint64_t sc2 = f2_pack(scale, scale);
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
 #pragma unroll
         for (int ch = 0; ch < 8; ++ch) {
           const int c0 = mb * 64 + ch * 8;
-          uint4 w;
-          w.x = pack_bf16x2(e[c0 + 0] * scale, e[c0 + 1] * scale);
-          w.y = pack_bf16x2(e[c0 + 2] * scale, e[c0 + 3] * scale);
-          w.z = pack_bf16x2(e[c0 + 4] * scale, e[c0 + 5] * scale);
-          w.w = pack_bf16x2(e[c0 + 6] * scale, e[c0 + 7] * scale);
-          *reinterpret_cast<uint4*>(arow + mb * 16384 + ((ch ^ (r & 7)) << 4)) = w;
+          uint32_t w4[4];
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            float a, b;
+            f2_unpack(f2_mul(f2_pack(v[c0 + 2 * h], v[c0 + 2 * h + 1]), sc2), a, b);
+            w4[h] = cvt_bf16x2(a, b);
+          }
+          *reinterpret_cast<uint4*>(arow + mb * 16384 + ((ch ^ (r & 7)) << 4)) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
       fence_proxy_async_smem();
@@ -338,21 +415,24 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
 
       if (it.last()) {
         // ---- epilogue: this segment's partial (U, mass) for our 128 prototypes
-        if (!mbar_wait_warp(smem_u32(&bars->u_full), (uint32_t)(seg & 1), status, budget)) {
+        if (!mbar_wait_warp(smem_u32(&bars->u_full[wg]), (uint32_t)(useg & 1), status, budget)) {
           ok = false;
           break;
         }
+        ++useg;
         tc_fence_after();
         const long long sgid = (long long)cid + it.u;
         float* dst = part_u + ((size_t)sgid * k_pad + pbase + r) * D;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c) {
-          float v[32];
-          tmem_ld32(tmem + lane_off + kColU + c * 32, v);
-          tc_wait_ld();
+          uint32_t u32[32];
+          tmem_ld32_raw(tmem + lane_off + kColU + c * 32, u32);
+          tmem_wait_tie(u32);
 #pragma unroll
           for (int x = 0; x < 32; x += 4)
-            *reinterpret_cast<float4*>(dst + c * 32 + x) = make_float4(v[x], v[x + 1], v[x + 2], v[x + 3]);
+            *reinterpret_cast<float4*>(dst + c * 32 + x) =
+                make_float4(__uint_as_float(u32[x]), __uint_as_float(u32[x + 1]),
+                            __uint_as_float(u32[x + 2]), __uint_as_float(u32[x + 3]));
         }
         const float ms = tmem_ld1(tmem + lane_off + kColU + D);
         tc_wait_ld();
@@ -374,10 +454,10 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
   }
 }
 
-template <int D>
+template <int D, int NS>
 cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
-  auto kern = sa_fwd_sm100_kernel<D>;
-  const size_t smem = FwdSmem<D>::bytes(a.C);
+  auto kern = sa_fwd_sm100_kernel<D, NS>;
+  const size_t smem = FwdSmem<D, NS>::bytes(a.C);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -386,7 +466,7 @@ cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)(a.G * a.C));
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -400,10 +480,10 @@ cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
                             a.k_pad, a.hdr, a.tile_start, a.part_u, a.part_m, a.lse, a.budget);
 }
 
-template <int D>
+template <int D, int NS>
 cudaError_t max_clusters_t(int C, int* n) {
-  auto kern = sa_fwd_sm100_kernel<D>;
-  const size_t smem = FwdSmem<D>::bytes(C);
+  auto kern = sa_fwd_sm100_kernel<D, NS>;
+  const size_t smem = FwdSmem<D, NS>::bytes(C);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (C > 8) {
@@ -412,7 +492,7 @@ cudaError_t max_clusters_t(int C, int* n) {
   }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3((unsigned)C);
-  cfg.blockDim = dim3(192);
+  cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -424,18 +504,27 @@ cudaError_t max_clusters_t(int C, int* n) {
   return cudaOccupancyMaxActiveClusters(n, kern, &cfg);
 }
 
+// X stages: 3 while the exchange slots leave room (C <= 8 at d = 128), else 2; 4 at d = 64.
+int stages_for(int d, int C) { return d == 64 ? 4 : (C <= 8 ? 3 : 2); }
+
 }  // namespace
 
 size_t fwd_sm100_smem_bytes(int d, int C) {
-  return d == 128 ? FwdSmem<128>::bytes(C) : FwdSmem<64>::bytes(C);
+  const int ns = stages_for(d, C);
+  if (d == 64) return FwdSmem<64, 4>::bytes(C);
+  return ns == 3 ? FwdSmem<128, 3>::bytes(C) : FwdSmem<128, 2>::bytes(C);
 }
 
 cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
-  return d == 128 ? max_clusters_t<128>(C, n) : max_clusters_t<64>(C, n);
+  const int ns = stages_for(d, C);
+  if (d == 64) return max_clusters_t<64, 4>(C, n);
+  return ns == 3 ? max_clusters_t<128, 3>(C, n) : max_clusters_t<128, 2>(C, n);
 }
 
 cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream) {
-  return a.d == 128 ? launch_fwd_sm100_t<128>(a, stream) : launch_fwd_sm100_t<64>(a, stream);
+  const int ns = stages_for(a.d, a.C);
+  if (a.d == 64) return launch_fwd_sm100_t<64, 4>(a, stream);
+  return ns == 3 ? launch_fwd_sm100_t<128, 3>(a, stream) : launch_fwd_sm100_t<128, 2>(a, stream);
 }
 
 }  // namespace sa

@@ -143,17 +143,19 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// Row-major [rows, d] bf16 matrix, boxes of 128 rows x 64 columns, 128-byte swizzle.
-bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, int d) {
+// Row-major [rows, d] bf16 matrix, boxes of 128 rows x `box_cols` columns; the swizzle
+// width equals the box row (64 columns: 128B swizzle, 16 columns: 32B swizzle).
+bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_cols) {
   auto fn = encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
-  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t box[2] = {(cuuint32_t)box_cols, 128};
   const cuuint32_t estr[2] = {1, 1};
   const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims,
                         strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        box_cols == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_32B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
@@ -161,6 +163,13 @@ bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, int d) {
 template <typename T>
 T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+thread_local cudaEvent_t g_prof_start = nullptr;
+thread_local cudaEvent_t g_prof_stop = nullptr;
+
+cudaError_t prof_mark(cudaEvent_t ev, cudaStream_t s) {
+  return ev ? cudaEventRecord(ev, s) : cudaSuccess;
 }
 
 sa_status cuda_status(cudaError_t e) {
@@ -215,8 +224,8 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   if (n_total > 0) {
     if (p.tc) {
       CUtensorMap tx, tp;
-      if (!make_tmap_bf16(&tx, X, (uint64_t)n_total, d) ||
-          !make_tmap_bf16(&tp, at<void>(workspace, p.pf), (uint64_t)p.k_pad, d))
+      if (!make_tmap_bf16(&tx, X, (uint64_t)n_total, d, 16) ||
+          !make_tmap_bf16(&tp, at<void>(workspace, p.pf), (uint64_t)p.k_pad, d, 64))
         return SA_ERR_CUDA;
       FwdSm100Args a;
       a.tmap_x = &tx;
@@ -234,7 +243,9 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
       a.part_m = pm;
       a.lse = lse;
       a.budget = kDefaultWaitBudget;
+      if ((st = cuda_status(prof_mark(g_prof_start, s))) != SA_OK) return st;
       if ((st = cuda_status(launch_fwd_sm100(a, s))) != SA_OK) return st;
+      if ((st = cuda_status(prof_mark(g_prof_stop, s))) != SA_OK) return st;
     } else {
       FwdSimtArgs a;
       a.X = static_cast<const float*>(X);
@@ -252,7 +263,9 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
       a.n_total = n_total;
       a.part_u = pu;
       a.part_m = pm;
+      if ((st = cuda_status(prof_mark(g_prof_start, s))) != SA_OK) return st;
       if ((st = cuda_status(launch_fwd_simt(a, s))) != SA_OK) return st;
+      if ((st = cuda_status(prof_mark(g_prof_stop, s))) != SA_OK) return st;
     }
   }
   FinalizeArgs f;
@@ -349,6 +362,13 @@ int sa_sketch_get_device_status(const void* workspace, void* stream_) {
     return SA_ERR_CUDA;
   }
   return h;
+}
+
+int sa_sketch_profile_events(void* start_event, void* stop_event) {
+  if ((start_event == nullptr) != (stop_event == nullptr)) return SA_ERR_INVALID_ARG;
+  g_prof_start = static_cast<cudaEvent_t>(start_event);
+  g_prof_stop = static_cast<cudaEvent_t>(stop_event);
+  return SA_OK;
 }
 
 const char* sa_status_string(int status) {

@@ -25,6 +25,7 @@ pytestmark = pytest.mark.gpu
     ([640, 77], 1024, 64),
     ([130], 64, 64),
     ([4100, 3], 512, 128),
+    ([100, 200, 129, 60, 300, 1, 128, 257, 90, 5000, 2, 383, 384, 385], 1024, 128),
 ])
 def test_bf16_small_full_compare(lengths, k, d):
     w = inputs.make_workload(lengths, d, k, "bf16", seed=11 + k + d + len(lengths))
