@@ -274,6 +274,54 @@ __device__ __forceinline__ void tmem_wait_tie(uint32_t (&r)[32]) {
       : "memory");
 }
 
+// 32 lanes x 32 consecutive columns from registers (thread i of the warp -> lane i).
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]),
+        "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]),
+        "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+// 16-column variants (fewer live registers).
+__device__ __forceinline__ void tmem_ld16_raw(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait_tie16(uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]),
+        "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]),
+        "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+  asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor for tcgen05 (start, leading and stride byte
 // offsets in 16-byte units; version 1; swizzle mode in bits 61..63).
 enum : uint32_t { kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle32B = 6 };
@@ -414,30 +462,29 @@ __device__ __forceinline__ int user_of_tile(const long long* tile_start, int R, 
 }
 
 // Walks the tiles [a, b) of the global tile sequence (users' tiles concatenated).
+// Tile indices fit in 32 bits: n_total < 2^31 tokens gives fewer than 2^31 tiles.
 struct TileIter {
   const long long* ts;
   const int64_t* off;
-  int R;
-  long long g, a, end;
-  int u;
-  __device__ void init(const long long* ts_, const int64_t* off_, int R_, long long a_,
+  int g, a, end, u;
+  __device__ void init(const long long* ts_, const int64_t* off_, int R, long long a_,
                        long long b_) {
-    ts = ts_; off = off_; R = R_; g = a_; a = a_; end = b_; u = 0;
+    ts = ts_; off = off_; g = (int)a_; a = (int)a_; end = (int)b_; u = 0;
     if (a_ < b_) u = user_of_tile(ts, R, a_);
   }
   __device__ bool valid() const { return g < end; }
-  __device__ long long local() const { return g - ts[u]; }
-  __device__ long long t0() const { return off[u] + local() * kTileTokens; }
+  __device__ int local() const { return g - (int)ts[u]; }
+  __device__ long long t0() const { return off[u] + (long long)local() * kTileTokens; }
   __device__ int nvalid() const {
-    const long long n = off[u + 1] - off[u] - local() * kTileTokens;
+    const long long n = off[u + 1] - off[u] - (long long)local() * kTileTokens;
     return n >= kTileTokens ? kTileTokens : (int)n;
   }
-  __device__ bool first() const { return g == a || g == ts[u]; }
-  __device__ bool last() const { return g == end - 1 || g == ts[u + 1] - 1; }
+  __device__ bool first() const { return g == a || g == (int)ts[u]; }
+  __device__ bool last() const { return g == end - 1 || g == (int)ts[u + 1] - 1; }
   __device__ void next() {
     ++g;
     if (g < end)
-      while (ts[u + 1] <= g) ++u;
+      while ((int)ts[u + 1] <= g) ++u;
   }
 };
 

@@ -10,20 +10,26 @@
 //
 // Decomposition. A cluster of C = ceil(k/128) CTAs owns one slice of the token stream; CTA
 // of rank c owns prototypes [128c, 128c+128). Per tile of 128 tokens each CTA:
-//   1. TMA loads the X tile (128 x d bf16, 128B swizzle) into a shared-memory stage
-//      (every CTA loads it itself; no multicast, the C-fold re-read is served by L2).
-//   2. tcgen05.mma  S^T[tok, proto] = X_tile . P'_slice^T  into TMEM (fp32), so a
-//      token's scores sit in one TMEM lane and one thread owns one token.
-//   3. Softmax warps load their row, take the local max m_c and l_c = m_c + log2 sum
-//      2^(s - m_c), and send l_c to every CTA of the cluster with st.async (DSMEM).
-//      Once all C partials have arrived: lse2 = log2 sum_c 2^(l_c), A = 2^(s - lse2).
+//   1. TMA loads the X tile (128 x d bf16, 32B swizzle, 16-column boxes) into one of NS
+//      shared-memory stages; each stage is followed by an all-ones 16-column block.
+//      Every CTA loads the tile itself (no multicast; the C-fold re-read is served by L2,
+//      and rank 0 prefetches upcoming tiles into L2).
+//   2. tcgen05.mma  S^T[tok, proto] = X_tile . P'_slice^T  into TMEM (fp32, two
+//      buffers), so a token's scores sit in one TMEM lane and one thread owns one token.
+//   3. Two softmax warpgroups take alternate tiles. Each thread loads its token's row,
+//      takes the local max m and l = m + log2 sum 2^(s - m), and sends l to every CTA of
+//      the cluster with st.async (DSMEM); once all C partials are in,
+//      lse2 = log2 sum_c 2^(l_c) and A = 2^(s - lse2).
 //   4. A is written as bf16 into shared memory in the MN-major layout of the next MMA's
-//      A operand, then  U[proto, :] += A . X_tile  and  mass[proto] += A . 1
-//      (tcgen05, accumulators in TMEM).
+//      A operand, then  [U | mass] += A . [X_tile | 1]  (one tcgen05.mma with N = d + 16,
+//      accumulator in TMEM): the 16 extra columns read the all-ones block and carry the
+//      per-prototype mass sum_t A_jt.
 //   5. When the token stream crosses a user boundary (or the slice ends) the partial
-//      (U, mass) of that (slice, user) segment is written to the workspace; a separate
+//      (U, mass) of that (cluster, user) segment is written to the workspace; the finalize
 //      kernel adds the segments of each user in a fixed order (deterministic).
-// All mbarrier waits are bounded (see sa_common.cuh).
+// Roles: warp 0 TMA producer, warp 1 allocates TMEM and issues the score MMAs, warp 2 the
+// accumulate MMAs, warp 3 idle, warps 4-11 the softmax warpgroups. All mbarrier waits are
+// bounded (see sa_common.cuh).
 #include <cuda.h>
 
 #include "sa_common.cuh"
@@ -65,7 +71,7 @@ struct Bars {
   uint64_t a_full[2], a_empty[2];
   uint64_t u_full[2], u_empty;  // u_full[w]: segments whose last tile warpgroup w owns
   uint64_t xch[kXchSlots];
-  uint64_t p_full, drain;
+  uint64_t p_full, drain, drain2;
   uint32_t tmem_base;
 };
 
@@ -76,8 +82,8 @@ __device__ __forceinline__ float tmem_ld1(uint32_t taddr) {
 }
 
 constexpr int kNWG = 2;                        // softmax warpgroups (ping-pong on tiles)
-// warps 0-3: TMA producer (0), TMEM allocator and MMA issuer (1), idle (2, 3);
-// warps 4-11: the two softmax warpgroups
+// warps 0-3: TMA producer (0), TMEM allocator and MMA1 issuer (1), MMA2 issuer (2),
+// idle (3); warps 4-11: the two softmax warpgroups
 constexpr int kThreads = 128 + 128 * kNWG;
 constexpr int kPrefetchAhead = 4;               // tiles prefetched into L2 ahead of the load
 
@@ -122,6 +128,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
     for (int s = 0; s < kXchSlots; ++s) mbar_init(smem_u32(&bars->xch[s]), 1);
     mbar_init(smem_u32(&bars->p_full), 1);
     mbar_init(smem_u32(&bars->drain), 1);
+    mbar_init(smem_u32(&bars->drain2), 1);
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -184,90 +191,58 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         mbar_wait_drain(smem_u32(&bars->x_full[j % NS]), (uint32_t)((j / NS) & 1), budget);
       mbar_wait_drain(pf, 0, budget);
     }
-  } else if (warp == 1) {
-    // ================= MMA issuer: MMA1 (scores) and MMA2 (accumulate) issued in
-    // whatever order their inputs become ready, each stream in tile order.
+  } else if (warp == 1 || warp == 2) {
+    // ================= MMA issuers: warp 1 issues MMA1 (scores), warp 2 MMA2 (accumulate)
     if (lane == 0 && ta < tb) {
-      const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);  // S^T = X . P'^T
-      const uint32_t idesc2 = idesc_bf16_f32(128, D + 16, 1, 1);       // [U | mass] += A . [X | 1]
+      const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);
+      const uint32_t idesc2 = idesc_bf16_f32(128, D + 16, 1, 1);
       bool ok = mbar_wait(smem_u32(&bars->p_full), 0, status, budget);
-      struct Info {
-        int st, seg;
-        bool first, last;
-      } ring[4];
       TileIter it;
       it.init(tile_start, offsets, R, ta, tb);
-      const long long ntile = tb - ta;
-      long long i1 = 0, i2 = 0;
+      long long i = 0;
       int seg = -1;
-      long long t_prog = clock64();
-      uint32_t spins = 0;
-      while (ok && i2 < ntile) {
-        bool prog = false;
-        if (i1 < ntile) {
-          const int st = (int)(i1 % NS);
-          const int sb = (int)(i1 & 1);
-          if (mbar_test(smem_u32(&bars->x_full[st]), (uint32_t)((i1 / NS) & 1)) &&
-              mbar_test(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i1 >> 1) & 1) ^ 1))) {
-            tc_fence_after();
-            const uint32_t x_base = sbase + L::oX + st * L::kXStage;
-            const uint32_t p_base = sbase + L::oP;
+      for (; ok && it.valid(); it.next(), ++i) {
+        const bool first = it.first(), last = it.last();
+        if (first) ++seg;
+        const int st = (int)(i % NS);
+        const int sb = (int)(i & 1);
+        if (warp == 1) {
+          ok = mbar_wait(smem_u32(&bars->x_full[st]), (uint32_t)((i / NS) & 1), status, budget) &&
+               mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget);
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t x_base = sbase + L::oX + st * L::kXStage;
+          const uint32_t p_base = sbase + L::oP;
 #pragma unroll
-            for (int ks = 0; ks < KSTEPS1; ++ks) {
-              // A = X tile, K-major, 32B swizzle: one 16-wide K step per 4 KB atom column
-              const uint64_t ad = smem_desc(x_base + ks * L::kBoxBytes, 16, 256, kSwizzle32B);
-              // B = P' slice, K-major, 128B swizzle: four 16-wide K steps per 16 KB box
-              const uint32_t koff = (ks >> 2) * L::kPBox + (ks & 3) * 32;
-              const uint64_t bd = smem_desc(p_base + koff, 16, 1024, kSwizzle128B);
-              tc_mma_f16(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc1, ks > 0 ? 1u : 0u);
-            }
-            tc_commit(smem_u32(&bars->s_full[sb]));
-            const bool first = it.first();
-            if (first) ++seg;
-            ring[i1 & 3] = Info{st, seg, first, it.last()};
-            it.next();
-            ++i1;
-            prog = true;
+          for (int ks = 0; ks < KSTEPS1; ++ks) {
+            const uint64_t ad = smem_desc(x_base + ks * L::kBoxBytes, 16, 256, kSwizzle32B);
+            const uint32_t koff = (ks >> 2) * L::kPBox + (ks & 3) * 32;
+            const uint64_t bd = smem_desc(p_base + koff, 16, 1024, kSwizzle128B);
+            tc_mma_f16(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc1, ks > 0 ? 1u : 0u);
           }
-        }
-        if (i2 < i1) {
-          const Info f = ring[i2 & 3];
-          const int ab = (int)(i2 & 1);
-          if (mbar_test(smem_u32(&bars->a_full[ab]), (uint32_t)((i2 >> 1) & 1)) &&
-              (!f.first || mbar_test(smem_u32(&bars->u_empty), (uint32_t)((f.seg & 1) ^ 1)))) {
-            tc_fence_after();
-            const uint32_t a_base = sbase + L::oA + ab * L::kABytes;
-            const uint32_t x_base = sbase + L::oX + f.st * L::kXStage;
+          tc_commit(smem_u32(&bars->s_full[sb]));
+        } else {
+          const int ab = sb;
+          ok = mbar_wait(smem_u32(&bars->a_full[ab]), (uint32_t)((i >> 1) & 1), status, budget) &&
+               (!first || mbar_wait(smem_u32(&bars->u_empty), (uint32_t)((seg & 1) ^ 1), status, budget));
+          if (!ok) break;
+          tc_fence_after();
+          const uint32_t a_base = sbase + L::oA + ab * L::kABytes;
+          const uint32_t x_base = sbase + L::oX + st * L::kXStage;
 #pragma unroll
-            for (int ks = 0; ks < KSTEPS2; ++ks) {
-              // A = A tile, MN-major (prototypes contiguous), 128B swizzle
-              const uint64_t ad = smem_desc(a_base + ks * 2048, L::kPBox, 1024, kSwizzle128B);
-              // B = [X | 1], MN-major (d contiguous), 32B swizzle: 16-wide N atoms 4 KB apart
-              const uint64_t bd = smem_desc(x_base + ks * 512, L::kBoxBytes, 256, kSwizzle32B);
-              const uint32_t acc = (f.first && ks == 0) ? 0u : 1u;
-              tc_mma_f16(tmem + kColU, ad, bd, idesc2, acc);
-            }
-            tc_commit(smem_u32(&bars->x_empty[f.st]));
-            tc_commit(smem_u32(&bars->a_empty[ab]));
-            if (f.last) tc_commit(smem_u32(&bars->u_full[i2 & 1]));
-            ++i2;
-            prog = true;
+          for (int ks = 0; ks < KSTEPS2; ++ks) {
+            const uint64_t ad = smem_desc(a_base + ks * 2048, L::kPBox, 1024, kSwizzle128B);
+            const uint64_t bd = smem_desc(x_base + ks * 512, L::kBoxBytes, 256, kSwizzle32B);
+            tc_mma_f16(tmem + kColU, ad, bd, idesc2, (first && ks == 0) ? 0u : 1u);
           }
-        }
-        if (prog) {
-          t_prog = clock64();
-          spins = 0;
-        } else if ((++spins & 63u) == 0u) {
-          if (read_status(status) != 0) ok = false;
-          else if (clock64() - t_prog > budget) {
-            latch_status(status, SA_ERR_TIMEOUT);
-            ok = false;
-          }
+          tc_commit(smem_u32(&bars->x_empty[st]));
+          tc_commit(smem_u32(&bars->a_empty[ab]));
+          if (last) tc_commit(smem_u32(&bars->u_full[i & 1]));
         }
       }
-      // drain every tcgen05 op this thread issued before the CTA tears down
-      tc_commit(smem_u32(&bars->drain));
-      mbar_wait_drain(smem_u32(&bars->drain), 0, budget);
+      const uint32_t db = smem_u32(warp == 1 ? &bars->drain : &bars->drain2);
+      tc_commit(db);
+      mbar_wait_drain(db, 0, budget);
     }
   } else if (warp >= 4) {
     // ================= softmax + epilogue: warpgroup wg takes the tiles i with i % 2 == wg
@@ -333,19 +308,15 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
       // e = 2^(s - m) and its sum (packed subtract, four packed accumulators)
       const uint64_t nm2 = f2_pack(-m, -m);
       uint64_t za[4] = {0ull, 0ull, 0ull, 0ull};
-      // prototypes [0, 64) on the MUFU, [64, 128) on the FMA pipe: the MUFU's 16
-      // results per clock per SM would otherwise match the tensor core's time per tile
+      // All on the MUFU: measured, moving half of them to the polynomial exp2_poly2 on
+      // the FMA pipe made the tile slower, as this loop is bound by latency and
+      // instruction count rather than by MUFU throughput.
 #pragma unroll
       for (int p = 0; p < kProtoSlice / 2; ++p) {
         float a, b;
-        const uint64_t xm = f2_add(f2_pack(v[2 * p], v[2 * p + 1]), nm2);
-        if (p < kProtoSlice / 4) {
-          f2_unpack(xm, a, b);
-          a = ex2_approx(a);
-          b = ex2_approx(b);
-        } else {
-          f2_unpack(exp2_poly2(xm), a, b);
-        }
+        f2_unpack(f2_add(f2_pack(v[2 * p], v[2 * p + 1]), nm2), a, b);
+        a = ex2_approx(a);
+        b = ex2_approx(b);
         v[2 * p] = a;
         v[2 * p + 1] = b;
         za[p & 3] = f2_add(za[p & 3], f2_pack(a, b));

@@ -280,6 +280,7 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   f.k_pad = p.k_pad;
   f.d = d;
   f.G = p.G;
+  f.mass_lanes = 1;
   f.sketch = sketch;
   f.mass = mass;
   f.xsketch = xsketch;

@@ -25,10 +25,11 @@ struct FinalizeArgs {
   const WsHeader* hdr;
   const long long* tile_start;
   const float* part_u;  // [segments, k_pad, d]
-  const float* part_m;  // [segments, k_pad]
+  const float* part_m;  // [segments, k_pad, mass_lanes]
   const void* Wv;
   sa_dtype dt;
   int R, k, k_pad, d, G;
+  int mass_lanes;       // partial masses per prototype and segment, summed in order
   float* sketch;
   float* mass;
   float* xsketch;  // nullable

@@ -135,7 +135,12 @@ __global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a, const TIn
       const size_t seg = (size_t)g + u;
       const float* src = a.part_u + (seg * a.k_pad + j0) * d;
       for (int i = threadIdx.x; i < 32 * d; i += blockDim.x) us[i] += src[i];
-      if (threadIdx.x < 32) ms[threadIdx.x] += a.part_m[seg * a.k_pad + j0 + threadIdx.x];
+      if (threadIdx.x < 32) {
+        const float* pm = a.part_m + (seg * a.k_pad + j0 + threadIdx.x) * a.mass_lanes;
+        float v = 0.f;
+        for (int l = 0; l < a.mass_lanes; ++l) v += pm[l];
+        ms[threadIdx.x] += v;
+      }
     }
   }
   for (int i = threadIdx.x; i < d * d; i += blockDim.x) wv[i] = to_f(Wv[i]);
