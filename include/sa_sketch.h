@@ -127,6 +127,33 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Forward without a workspace, for callers that cannot allocate device memory (for
+ * example a serving process whose allocator reserved all of its memory at start-up and
+ * forbids new allocations, or code running where cudaMalloc may not be called). The
+ * pages describe no such interface; it has no counterpart in the paper.
+ *
+ * Same arguments, results and conventions as sa_sketch_forward, minus the workspace.
+ * The scratch space is one device array of SA_NOALLOC_SCRATCH_BYTES per GPU, reserved
+ * when this entry point is first used on that GPU and held until the process exits.
+ *  - The first call on each device looks up the array's device address (set-up, with
+ *    that device current). Make that first call before any stream capture begins.
+ *  - Every call on a device shares the one array: calls whose work overlaps on the GPU
+ *    (different streams, or different host threads) race and give wrong results.
+ *    Serialise them, for instance on one stream.
+ *  - Sizes whose plan needs more than SA_NOALLOC_SCRATCH_BYTES are rejected with
+ *    SA_ERR_WORKSPACE before anything is launched (at k = 1024, d = 128 on a B200 about 48 users).
+ *  - It calls no cudaMalloc, cudaFree or allocating library routine.
+ *  - device_status: nullable HOST pointer. When given, the call waits for `stream` and
+ *    stores the device status word there (SA_OK, SA_ERR_BAD_OFFSETS, SA_ERR_TIMEOUT), since
+ *    the caller cannot name the scratch array in sa_sketch_get_device_status.
+ */
+#define SA_NOALLOC_SCRATCH_BYTES (32u << 20)
+int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, int R, int64_t n_total,
+                              int d, const void* P, int k, const void* Wk, const void* Wv,
+                              sa_dtype dt, float* sketch, float* mass, float* lse,
+                              float* xsketch, int* device_status, void* stream);
+
+/*
  * Reads the device status word that the last call using `workspace` left behind.
  * It synchronises `stream` and returns SA_OK, SA_ERR_BAD_OFFSETS or SA_ERR_TIMEOUT,
  * or SA_ERR_CUDA if the copy itself failed. The word is cleared at the start of

@@ -30,7 +30,7 @@ SA_ERR_NO_DEVICE = 7
 
 EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
             "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
-            "sa_sketch_profile_events")
+            "sa_sketch_profile_events", "sa_sketch_forward_noalloc")
 
 
 class SketchAttentionError(RuntimeError):
@@ -61,6 +61,9 @@ def _load() -> ctypes.CDLL:
     lib.sa_sketch_debug_wait_timeout.argtypes = [vp, ctypes.c_longlong, vp]
     lib.sa_sketch_profile_events.restype = i32
     lib.sa_sketch_profile_events.argtypes = [vp, vp]
+    lib.sa_sketch_forward_noalloc.restype = i32
+    lib.sa_sketch_forward_noalloc.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
+                                              vp, vp, vp, vp, vp, vp]
     return lib
 
 
@@ -95,6 +98,14 @@ def sa_status_string(status: int) -> str:
 
 def sa_sketch_debug_wait_timeout(workspace, budget_cycles: int, stream) -> int:
     return int(_lib.sa_sketch_debug_wait_timeout(workspace, int(budget_cycles), stream))
+
+
+def sa_sketch_forward_noalloc(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass, lse,
+                              xsketch, device_status, stream) -> int:
+    """Forward without a workspace (see include/sa_sketch.h). `device_status` is a host
+    pointer (ctypes) or None."""
+    return int(_lib.sa_sketch_forward_noalloc(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch,
+                                              mass, lse, xsketch, device_status, stream))
 
 
 def sa_sketch_profile_events(start_event, stop_event) -> int:
