@@ -57,9 +57,8 @@ __global__ void __launch_bounds__(1024) schedule_kernel(const int64_t* __restric
   }
 }
 
-// ------------------------------------------------------------------ fold
+// ------------------------------------------------------------------ fold (helpers)
 // Pf[j][c] = scale * sum_e P[j][e] Wk[c][e]   (so P_j . (X_t Wk) = X_t . Pf_j / scale).
-// Block: 32 prototypes x all d outputs; Wk staged transposed-free with a padded stride.
 template <typename TIn>
 __device__ __forceinline__ float to_f(TIn v);
 template <>
@@ -67,40 +66,10 @@ __device__ __forceinline__ float to_f<float>(float v) { return v; }
 template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
-template <typename TIn>
-__global__ void __launch_bounds__(256) fold_kernel(const TIn* __restrict__ P, const TIn* __restrict__ Wk,
-                                                   int k, int k_pad, int d, float scale,
-                                                   void* __restrict__ out, int out_bf16) {
-  extern __shared__ float fsm[];
-  float* wk = fsm;                      // [d][d+1]
-  float* ps = fsm + d * (d + 1);        // [32][d]
-  const int j0 = blockIdx.x * 32;
-  for (int i = threadIdx.x; i < d * d; i += blockDim.x) {
-    const int c = i / d, e = i % d;
-    wk[c * (d + 1) + e] = to_f(Wk[i]);
-  }
-  for (int i = threadIdx.x; i < 32 * d; i += blockDim.x) {
-    const int jj = i / d, e = i % d;
-    ps[i] = (j0 + jj < k) ? to_f(P[(size_t)(j0 + jj) * d + e]) : 0.f;
-  }
-  __syncthreads();
-  for (int i = threadIdx.x; i < 32 * d; i += blockDim.x) {
-    const int jj = i / d, c = i % d;
-    float acc = 0.f;
-    for (int e = 0; e < d; ++e) acc = fmaf(ps[jj * d + e], wk[c * (d + 1) + e], acc);
-    acc *= scale;
-    const size_t o = (size_t)(j0 + jj) * d + c;
-    if (j0 + jj < k_pad) {
-      if (out_bf16) reinterpret_cast<__nv_bfloat16*>(out)[o] = __float2bfloat16_rn(acc);
-      else reinterpret_cast<float*>(out)[o] = acc;
-    }
-  }
-}
-
-// ------------------------------------------------------------------ finalize
-// Block (user u, 32 prototypes). The user's segments are the clusters whose tile range
-// intersects the user's tiles; their partials are added in cluster order, so the
-// result does not depend on timing. Then sketch_j = (U_j Wv) / mass_j, mass_j = 0 -> 0.
+// ------------------------------------------------------------------ finalize (helpers)
+// A user's segments are the clusters whose tile range intersects the user's tiles; their
+// partials are added in cluster order, so the result does not depend on timing. Then
+// sketch_j = (U_j Wv) / mass_j, with mass_j = 0 -> 0.
 __device__ __forceinline__ long long range_start(long long g, long long T, int G) {
   return g * T / G;
 }
@@ -113,52 +82,166 @@ __device__ int cluster_of_tile(long long x, long long T, int G) {
   return (int)g;
 }
 
-template <typename TIn>
-__global__ void __launch_bounds__(256) finalize_kernel(FinalizeArgs a, const TIn* __restrict__ Wv) {
-  extern __shared__ float fsm[];
-  const int d = a.d;
-  float* wv = fsm;              // [d][d]
-  float* us = fsm + d * d;      // [32][d]
-  float* ms = us + 32 * d;      // [32]
+// ------------------------------------------------------------------ tiled row GEMM
+// out[j][e] = sum_c lr[j][c] * rm[c][e] for a tile of 64 rows j and D columns e, both
+// operands in shared memory with row stride D+4 floats. 256 threads: kTE = D/4 threads
+// across e (4 columns each) and 256/kTE across rows, kJPT rows each. Per 4 values of c a
+// thread reads kJPT float4 of lr (the same address across a warp's e lanes) and 4 float4
+// of rm, then issues 16*kJPT FMAs.
+constexpr int kRowTile = 64;
+
+template <int D>
+struct TileShape {
+  static constexpr int kLd = D + 4;
+  static constexpr int kTE = D / 4;
+  static constexpr int kTJ = 256 / kTE;
+  static constexpr int kJPT = kRowTile / kTJ;
+};
+
+template <int D>
+__device__ __forceinline__ void tile_gemm(const float* __restrict__ lr, const float* __restrict__ rm,
+                                          float (&acc)[TileShape<D>::kJPT][4]) {
+  using S = TileShape<D>;
+  const int te = threadIdx.x % S::kTE, tj = threadIdx.x / S::kTE;
+#pragma unroll
+  for (int r = 0; r < S::kJPT; ++r)
+#pragma unroll
+    for (int x = 0; x < 4; ++x) acc[r][x] = 0.f;
+#pragma unroll 2
+  for (int c = 0; c < D; c += 4) {
+    float4 w[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) w[q] = *reinterpret_cast<const float4*>(rm + (c + q) * S::kLd + te * 4);
+#pragma unroll
+    for (int r = 0; r < S::kJPT; ++r) {
+      const float4 l = *reinterpret_cast<const float4*>(lr + (tj * S::kJPT + r) * S::kLd + c);
+      const float lv[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        acc[r][0] = fmaf(lv[q], w[q].x, acc[r][0]);
+        acc[r][1] = fmaf(lv[q], w[q].y, acc[r][1]);
+        acc[r][2] = fmaf(lv[q], w[q].z, acc[r][2]);
+        acc[r][3] = fmaf(lv[q], w[q].w, acc[r][3]);
+      }
+    }
+  }
+}
+
+// fold, tiled: block = 64 prototypes; Pf[j][c] = scale * sum_e P[j][e] Wk[c][e].
+template <int D, typename TIn>
+__global__ void __launch_bounds__(256) fold_tiled_kernel(const TIn* __restrict__ P,
+                                                         const TIn* __restrict__ Wk, int k,
+                                                         int k_pad, float scale,
+                                                         void* __restrict__ out, int out_bf16) {
+  using S = TileShape<D>;
+  extern __shared__ __align__(16) float tsm[];
+  float* lr = tsm;                  // [64][D+4]  lr[j][e] = P[j0 + j][e]
+  float* rm = tsm + kRowTile * S::kLd;  // [D][D+4]   rm[e][c] = Wk[c][e]
+  const int j0 = blockIdx.x * kRowTile;
+  for (int i = threadIdx.x; i < kRowTile * D; i += blockDim.x) {
+    const int j = i / D, e = i % D;
+    lr[j * S::kLd + e] = (j0 + j < k) ? to_f(P[(size_t)(j0 + j) * D + e]) : 0.f;
+  }
+  for (int i = threadIdx.x; i < D * D; i += blockDim.x) {
+    const int c = i / D, e = i % D;
+    rm[e * S::kLd + c] = to_f(Wk[i]);
+  }
+  __syncthreads();
+  float acc[S::kJPT][4];
+  tile_gemm<D>(lr, rm, acc);
+  const int te = threadIdx.x % S::kTE, tj = threadIdx.x / S::kTE;
+#pragma unroll
+  for (int r = 0; r < S::kJPT; ++r) {
+    const int j = j0 + tj * S::kJPT + r;
+    if (j >= k_pad) continue;
+    const size_t o = (size_t)j * D + te * 4;
+    if (out_bf16) {
+      __nv_bfloat16* ob = reinterpret_cast<__nv_bfloat16*>(out) + o;
+      ob[0] = __float2bfloat16_rn(acc[r][0] * scale);
+      ob[1] = __float2bfloat16_rn(acc[r][1] * scale);
+      ob[2] = __float2bfloat16_rn(acc[r][2] * scale);
+      ob[3] = __float2bfloat16_rn(acc[r][3] * scale);
+    } else {
+      *reinterpret_cast<float4*>(reinterpret_cast<float*>(out) + o) =
+          make_float4(acc[r][0] * scale, acc[r][1] * scale, acc[r][2] * scale, acc[r][3] * scale);
+    }
+  }
+}
+
+// finalize, tiled: block = (user u, 64 prototypes). Adds the user's segment partials in
+// cluster order (deterministic), writes xsketch = U and mass, then sketch = U Wv / mass.
+template <int D, typename TIn>
+__global__ void __launch_bounds__(256) finalize_tiled_kernel(FinalizeArgs a, const TIn* __restrict__ Wv) {
+  using S = TileShape<D>;
+  extern __shared__ __align__(16) float tsm[];
+  float* lr = tsm;                      // [64][D+4]  lr[j][c] = U[j0 + j][c]
+  float* rm = tsm + kRowTile * S::kLd;  // [D][D+4]   rm[c][e] = Wv[c][e]
+  float* ms = rm + D * S::kLd;          // [64]
+  constexpr int kV = D / 4;             // float4 per row
   const int u = blockIdx.x;
-  const int j0 = blockIdx.y * 32;
+  const int j0 = blockIdx.y * kRowTile;
   if (read_status(&a.hdr->status) != 0) return;
   const long long T = a.hdr->total_tiles;
   const long long x0 = a.tile_start[u], x1 = a.tile_start[u + 1];
-  for (int i = threadIdx.x; i < 32 * d; i += blockDim.x) us[i] = 0.f;
-  if (threadIdx.x < 32) ms[threadIdx.x] = 0.f;
-  __syncthreads();
+  float4 us[kRowTile * kV / 256];       // this thread's float4 of the U tile
+  float mv = 0.f;                       // thread t < 64: mass of row t
+#pragma unroll
+  for (int q = 0; q < kRowTile * kV / 256; ++q) us[q] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (x1 > x0) {
     const int g0 = cluster_of_tile(x0, T, a.G), g1 = cluster_of_tile(x1 - 1, T, a.G);
     for (int g = g0; g <= g1; ++g) {
       if (range_start(g, T, a.G) == range_start(g + 1, T, a.G)) continue;  // empty range
       const size_t seg = (size_t)g + u;
-      const float* src = a.part_u + (seg * a.k_pad + j0) * d;
-      for (int i = threadIdx.x; i < 32 * d; i += blockDim.x) us[i] += src[i];
-      if (threadIdx.x < 32) {
+      const float4* src = reinterpret_cast<const float4*>(a.part_u + (seg * a.k_pad + j0) * D);
+#pragma unroll
+      for (int q = 0; q < kRowTile * kV / 256; ++q) {
+        const int i = threadIdx.x + q * 256;
+        if (j0 + i / kV < a.k_pad) {
+          const float4 v = src[i];
+          us[q].x += v.x; us[q].y += v.y; us[q].z += v.z; us[q].w += v.w;
+        }
+      }
+      if (threadIdx.x < kRowTile && j0 + (int)threadIdx.x < a.k_pad) {
         const float* pm = a.part_m + (seg * a.k_pad + j0 + threadIdx.x) * a.mass_lanes;
         float v = 0.f;
         for (int l = 0; l < a.mass_lanes; ++l) v += pm[l];
-        ms[threadIdx.x] += v;
+        mv += v;
       }
     }
   }
-  for (int i = threadIdx.x; i < d * d; i += blockDim.x) wv[i] = to_f(Wv[i]);
-  __syncthreads();
-  // outputs
-  for (int i = threadIdx.x; i < 32 * d; i += blockDim.x) {
-    const int jj = i / d, e = i % d;
-    if (j0 + jj < a.k && a.xsketch) a.xsketch[((size_t)u * a.k + j0 + jj) * d + e] = us[i];
+#pragma unroll
+  for (int q = 0; q < kRowTile * kV / 256; ++q) {
+    const int i = threadIdx.x + q * 256;
+    const int j = i / kV, c4 = i % kV;
+    *reinterpret_cast<float4*>(lr + j * S::kLd + c4 * 4) = us[q];
+    if (a.xsketch && j0 + j < a.k)
+      reinterpret_cast<float4*>(a.xsketch + ((size_t)u * a.k + j0 + j) * D)[c4] = us[q];
   }
-  if (threadIdx.x < 32 && j0 + threadIdx.x < a.k) a.mass[(size_t)u * a.k + j0 + threadIdx.x] = ms[threadIdx.x];
-  const int e = threadIdx.x % d;
-  const int jstep = blockDim.x / d;
-  for (int jj = threadIdx.x / d; jj < 32; jj += jstep) {
-    if (j0 + jj >= a.k) break;
-    float acc = 0.f;
-    for (int c = 0; c < d; ++c) acc = fmaf(us[jj * d + c], wv[c * d + e], acc);
+  if (threadIdx.x < kRowTile) {
+    ms[threadIdx.x] = mv;
+    if (j0 + (int)threadIdx.x < a.k) a.mass[(size_t)u * a.k + j0 + threadIdx.x] = mv;
+  }
+  for (int i = threadIdx.x; i < D * kV; i += blockDim.x) {
+    const int c = i / kV, e4 = i % kV;
+    float4 w;
+    w.x = to_f(Wv[c * D + e4 * 4]);
+    w.y = to_f(Wv[c * D + e4 * 4 + 1]);
+    w.z = to_f(Wv[c * D + e4 * 4 + 2]);
+    w.w = to_f(Wv[c * D + e4 * 4 + 3]);
+    *reinterpret_cast<float4*>(rm + c * S::kLd + e4 * 4) = w;
+  }
+  __syncthreads();
+  float acc[S::kJPT][4];
+  tile_gemm<D>(lr, rm, acc);
+  const int te = threadIdx.x % S::kTE, tj = threadIdx.x / S::kTE;
+#pragma unroll
+  for (int r = 0; r < S::kJPT; ++r) {
+    const int jj = tj * S::kJPT + r, j = j0 + jj;
+    if (j >= a.k) continue;
     const float m = ms[jj];
-    a.sketch[((size_t)u * a.k + j0 + jj) * d + e] = m > 0.f ? acc / m : 0.f;
+    const float inv = m > 0.f ? 1.f / m : 0.f;
+    *reinterpret_cast<float4*>(a.sketch + ((size_t)u * a.k + j) * D + te * 4) =
+        make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
   }
 }
 
@@ -186,42 +269,44 @@ cudaError_t launch_schedule(const int64_t* offsets, int R, int64_t n_total, WsHe
   return cudaGetLastError();
 }
 
+template <int D, typename TIn>
+cudaError_t launch_fold_t(const void* P, const void* Wk, int k, int k_pad, float scale, void* Pf,
+                          bool out_bf16, cudaStream_t s) {
+  auto kern = fold_tiled_kernel<D, TIn>;
+  const size_t smem = (size_t)(kRowTile + D) * TileShape<D>::kLd * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)((k_pad + kRowTile - 1) / kRowTile));
+  kern<<<grid, 256, smem, s>>>(static_cast<const TIn*>(P), static_cast<const TIn*>(Wk), k, k_pad,
+                               scale, Pf, out_bf16 ? 1 : 0);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fold(const void* P, const void* Wk, sa_dtype dt, int k, int k_pad, int d,
                         float scale, void* Pf, bool out_bf16, cudaStream_t s) {
-  const size_t smem = (size_t)(d * (d + 1) + 32 * d) * sizeof(float);
-  const dim3 grid((unsigned)((k_pad + 31) / 32));
-  cudaError_t e;
-  if (dt == SA_BF16) {
-    e = cudaFuncSetAttribute(fold_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fold_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(
-        static_cast<const __nv_bfloat16*>(P), static_cast<const __nv_bfloat16*>(Wk), k, k_pad, d,
-        scale, Pf, out_bf16 ? 1 : 0);
-  } else {
-    e = cudaFuncSetAttribute(fold_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    fold_kernel<float><<<grid, 256, smem, s>>>(static_cast<const float*>(P),
-                                               static_cast<const float*>(Wk), k, k_pad, d, scale,
-                                               Pf, out_bf16 ? 1 : 0);
-  }
+  if (dt == SA_BF16)
+    return d == 128 ? launch_fold_t<128, __nv_bfloat16>(P, Wk, k, k_pad, scale, Pf, out_bf16, s)
+                    : launch_fold_t<64, __nv_bfloat16>(P, Wk, k, k_pad, scale, Pf, out_bf16, s);
+  return d == 128 ? launch_fold_t<128, float>(P, Wk, k, k_pad, scale, Pf, out_bf16, s)
+                  : launch_fold_t<64, float>(P, Wk, k, k_pad, scale, Pf, out_bf16, s);
+}
+
+template <int D, typename TIn>
+cudaError_t launch_finalize_t(const FinalizeArgs& a, cudaStream_t s) {
+  auto kern = finalize_tiled_kernel<D, TIn>;
+  const size_t smem = ((size_t)(kRowTile + D) * TileShape<D>::kLd + kRowTile) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)a.R, (unsigned)((a.k + kRowTile - 1) / kRowTile));
+  kern<<<grid, 256, smem, s>>>(a, static_cast<const TIn*>(a.Wv));
   return cudaGetLastError();
 }
 
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s) {
   if (a.R == 0) return cudaSuccess;
-  const size_t smem = (size_t)(a.d * a.d + 32 * a.d + 32) * sizeof(float);
-  const dim3 grid((unsigned)a.R, (unsigned)((a.k + 31) / 32));
-  cudaError_t e;
-  if (a.dt == SA_BF16) {
-    e = cudaFuncSetAttribute(finalize_kernel<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    finalize_kernel<__nv_bfloat16><<<grid, 256, smem, s>>>(a, static_cast<const __nv_bfloat16*>(a.Wv));
-  } else {
-    e = cudaFuncSetAttribute(finalize_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    finalize_kernel<float><<<grid, 256, smem, s>>>(a, static_cast<const float*>(a.Wv));
-  }
-  return cudaGetLastError();
+  if (a.dt == SA_BF16)
+    return a.d == 128 ? launch_finalize_t<128, __nv_bfloat16>(a, s) : launch_finalize_t<64, __nv_bfloat16>(a, s);
+  return a.d == 128 ? launch_finalize_t<128, float>(a, s) : launch_finalize_t<64, float>(a, s);
 }
 
 cudaError_t launch_debug_wait_timeout(WsHeader* hdr, long long budget, cudaStream_t s) {
