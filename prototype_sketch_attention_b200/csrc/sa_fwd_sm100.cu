@@ -39,6 +39,7 @@ namespace sa {
 namespace {
 
 constexpr int kProtoSlice = 128;              // prototypes per CTA (TMEM lanes / MMA M)
+constexpr int kMaxCluster = SA_MAX_K / kProtoSlice;  // CTAs per cluster at most
 constexpr int kXchSlots = 4;                  // exchange slots (tile index mod 4)
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColU = 256;
@@ -86,6 +87,75 @@ constexpr int kNWG = 2;                        // softmax warpgroups (ping-pong 
 // idle (3); warps 4-11: the two softmax warpgroups
 constexpr int kThreads = 128 + 128 * kNWG;
 constexpr int kPrefetchAhead = 4;               // tiles prefetched into L2 ahead of the load
+
+// Scores of this thread's token (one TMEM lane) for the CTA's 128 prototypes.
+__device__ __forceinline__ void load_scores(uint32_t taddr, float (&v)[kProtoSlice]) {
+  uint32_t r0[32], r1[32], r2[32], r3[32];
+  tmem_ld32_raw(taddr + 0, r0);
+  tmem_ld32_raw(taddr + 32, r1);
+  tmem_ld32_raw(taddr + 64, r2);
+  tmem_ld32_raw(taddr + 96, r3);
+  tmem_wait_tie(r0);
+  tmem_wait_tie(r1);
+  tmem_wait_tie(r2);
+  tmem_wait_tie(r3);
+#pragma unroll
+  for (int x = 0; x < 32; ++x) {
+    v[x] = __uint_as_float(r0[x]);
+    v[32 + x] = __uint_as_float(r1[x]);
+    v[64 + x] = __uint_as_float(r2[x]);
+    v[96 + x] = __uint_as_float(r3[x]);
+  }
+}
+
+// v <- 2^v in place; returns the sum (four packed accumulators, then a tree).
+__device__ __forceinline__ float exp2_and_sum(float (&v)[kProtoSlice]) {
+  uint64_t za[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int p = 0; p < kProtoSlice / 2; ++p) {
+    v[2 * p] = ex2_approx(v[2 * p]);
+    v[2 * p + 1] = ex2_approx(v[2 * p + 1]);
+    za[p & 3] = f2_add(za[p & 3], f2_pack(v[2 * p], v[2 * p + 1]));
+  }
+  float z0, z1;
+  f2_unpack(f2_add(f2_add(za[0], za[1]), f2_add(za[2], za[3])), z0, z1);
+  return z0 + z1;
+}
+
+// Maximum of the 128 scores: four independent chains of 3-input max.
+__device__ __forceinline__ float row_max(const float (&v)[kProtoSlice]) {
+  float mc[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    float a = fmaxf(v[32 * j], v[32 * j + 31]);
+#pragma unroll
+    for (int c = 1; c < 31; c += 2) a = fmax3(a, v[32 * j + c], v[32 * j + c + 1]);
+    mc[j] = a;
+  }
+  return fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+}
+
+// log2 of the sum of 2^x[p * 128] over the C partials of one token (C <= kMaxCluster).
+// Every load and exponential is independent; max and sum are trees.
+__device__ __forceinline__ float combine_partials(const float* x, int C) {
+  float lp[kMaxCluster], t[kMaxCluster];
+#pragma unroll
+  for (int p = 0; p < kMaxCluster; ++p) lp[p] = p < C ? x[p * 128] : -INFINITY;
+#pragma unroll
+  for (int p = 0; p < kMaxCluster; ++p) t[p] = lp[p];
+#pragma unroll
+  for (int w = kMaxCluster / 2; w >= 1; w /= 2)
+#pragma unroll
+    for (int p = 0; p < w; ++p) t[p] = fmaxf(t[p], t[p + w]);
+  const float mx = t[0];
+#pragma unroll
+  for (int p = 0; p < kMaxCluster; ++p) t[p] = p < C ? ex2_approx(lp[p] - mx) : 0.f;
+#pragma unroll
+  for (int w = kMaxCluster / 2; w >= 1; w /= 2)
+#pragma unroll
+    for (int p = 0; p < w; ++p) t[p] += t[p + w];
+  return mx + lg2_approx(t[0]);
+}
 
 template <int D, int NS>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -196,6 +266,14 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
     if (lane == 0 && ta < tb) {
       const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);
       const uint32_t idesc2 = idesc_bf16_f32(128, D + 16, 1, 1);
+      // Shared-memory descriptors for stage 0 / A buffer 0, built once: a later operand
+      // address is the same descriptor plus (byte offset >> 4) in its 14-bit address
+      // field (every operand lies below 256 KB, so the field never carries). Building
+      // each descriptor from scratch right before its MMA made issue the bottleneck.
+      const uint64_t dx1 = smem_desc(sbase + L::oX, 16, 256, kSwizzle32B);            // X, K-major
+      const uint64_t dp1 = smem_desc(sbase + L::oP, 16, 1024, kSwizzle128B);          // P', K-major
+      const uint64_t da2 = smem_desc(sbase + L::oA, L::kPBox, 1024, kSwizzle128B);    // A, MN-major
+      const uint64_t dx2 = smem_desc(sbase + L::oX, L::kBoxBytes, 256, kSwizzle32B);  // [X|1], MN-major
       bool ok = mbar_wait(smem_u32(&bars->p_full), 0, status, budget);
       TileIter it;
       it.init(tile_start, offsets, R, ta, tb);
@@ -211,14 +289,12 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget);
           if (!ok) break;
           tc_fence_after();
-          const uint32_t x_base = sbase + L::oX + st * L::kXStage;
-          const uint32_t p_base = sbase + L::oP;
+          const uint64_t xd = dx1 + (uint64_t)((st * L::kXStage) >> 4);
 #pragma unroll
           for (int ks = 0; ks < KSTEPS1; ++ks) {
-            const uint64_t ad = smem_desc(x_base + ks * L::kBoxBytes, 16, 256, kSwizzle32B);
             const uint32_t koff = (ks >> 2) * L::kPBox + (ks & 3) * 32;
-            const uint64_t bd = smem_desc(p_base + koff, 16, 1024, kSwizzle128B);
-            tc_mma_f16(tmem + (sb ? kColS1 : kColS0), ad, bd, idesc1, ks > 0 ? 1u : 0u);
+            tc_mma_f16(tmem + (sb ? kColS1 : kColS0), xd + (uint64_t)((ks * L::kBoxBytes) >> 4),
+                       dp1 + (uint64_t)(koff >> 4), idesc1, ks > 0 ? 1u : 0u);
           }
           tc_commit(smem_u32(&bars->s_full[sb]));
         } else {
@@ -227,14 +303,12 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                (!first || mbar_wait(smem_u32(&bars->u_empty), (uint32_t)((seg & 1) ^ 1), status, budget));
           if (!ok) break;
           tc_fence_after();
-          const uint32_t a_base = sbase + L::oA + ab * L::kABytes;
-          const uint32_t x_base = sbase + L::oX + st * L::kXStage;
+          const uint64_t ad0 = da2 + (uint64_t)((ab * L::kABytes) >> 4);
+          const uint64_t xd = dx2 + (uint64_t)((st * L::kXStage) >> 4);
 #pragma unroll
-          for (int ks = 0; ks < KSTEPS2; ++ks) {
-            const uint64_t ad = smem_desc(a_base + ks * 2048, L::kPBox, 1024, kSwizzle128B);
-            const uint64_t bd = smem_desc(x_base + ks * 512, L::kBoxBytes, 256, kSwizzle32B);
-            tc_mma_f16(tmem + kColU, ad, bd, idesc2, (first && ks == 0) ? 0u : 1u);
-          }
+          for (int ks = 0; ks < KSTEPS2; ++ks)
+            tc_mma_f16(tmem + kColU, ad0 + (uint64_t)((ks * 2048) >> 4), xd + (uint64_t)((ks * 512) >> 4),
+                       idesc2, (first && ks == 0) ? 0u : 1u);
           tc_commit(smem_u32(&bars->x_empty[st]));
           tc_commit(smem_u32(&bars->a_empty[ab]));
           if (last) tc_commit(smem_u32(&bars->u_full[i & 1]));
@@ -266,64 +340,35 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         break;
       }
       tc_fence_after();
+      const uint32_t s_tmem = tmem + lane_off + (sb ? kColS1 : kColS0);
       float v[kProtoSlice];
-      {
-        uint32_t r0[32], r1[32], r2[32], r3[32];
-        const uint32_t ta0 = tmem + lane_off + (sb ? kColS1 : kColS0);
-        tmem_ld32_raw(ta0 + 0, r0);
-        tmem_ld32_raw(ta0 + 32, r1);
-        tmem_ld32_raw(ta0 + 64, r2);
-        tmem_ld32_raw(ta0 + 96, r3);
-        tmem_wait_tie(r0);
-        tmem_wait_tie(r1);
-        tmem_wait_tie(r2);
-        tmem_wait_tie(r3);
-#pragma unroll
-        for (int x = 0; x < 32; ++x) {
-          v[x] = __uint_as_float(r0[x]);
-          v[32 + x] = __uint_as_float(r1[x]);
-          v[64 + x] = __uint_as_float(r2[x]);
-          v[96 + x] = __uint_as_float(r3[x]);
-        }
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[sb]));
-
+      load_scores(s_tmem, v);
       if (partial_slice) {
 #pragma unroll
         for (int c = 0; c < kProtoSlice; ++c)
           if (pbase + c >= k_valid) v[c] = -INFINITY;
       }
-      // local max: four independent chains of 3-input max
-      float mc[4];
+      // e = 2^s and z = sum e without a max shift: exact whenever z stays within
+      // [2^-100, 2^100], which holds unless a token's scores are extreme. A warp with
+      // any lane outside that range reloads its scores and takes the shifted path.
+      float m = 0.f;
+      float z = exp2_and_sum(v);
+      const bool in_range = z >= 0x1p-100f && z <= 0x1p100f;
+      if (!__all_sync(0xffffffffu, in_range)) {
+        load_scores(s_tmem, v);
+        if (partial_slice) {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float a = fmaxf(v[32 * j], v[32 * j + 31]);
+          for (int c = 0; c < kProtoSlice; ++c)
+            if (pbase + c >= k_valid) v[c] = -INFINITY;
+        }
+        m = row_max(v);
 #pragma unroll
-        for (int c = 1; c < 31; c += 2) a = fmax3(a, v[32 * j + c], v[32 * j + c + 1]);
-        mc[j] = a;
+        for (int c = 0; c < kProtoSlice; ++c) v[c] -= m;
+        z = exp2_and_sum(v);
       }
-      const float m = fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
-      // e = 2^(s - m) and its sum (packed subtract, four packed accumulators)
-      const uint64_t nm2 = f2_pack(-m, -m);
-      uint64_t za[4] = {0ull, 0ull, 0ull, 0ull};
-      // All on the MUFU: measured, moving half of them to the polynomial exp2_poly2 on
-      // the FMA pipe made the tile slower, as this loop is bound by latency and
-      // instruction count rather than by MUFU throughput.
-#pragma unroll
-      for (int p = 0; p < kProtoSlice / 2; ++p) {
-        float a, b;
-        f2_unpack(f2_add(f2_pack(v[2 * p], v[2 * p + 1]), nm2), a, b);
-        a = ex2_approx(a);
-        b = ex2_approx(b);
-        v[2 * p] = a;
-        v[2 * p + 1] = b;
-        za[p & 3] = f2_add(za[p & 3], f2_pack(a, b));
-      }
-      float z0, z1;
-      f2_unpack(f2_add(f2_add(za[0], za[1]), f2_add(za[2], za[3])), z0, z1);
-      const float z = z0 + z1;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[sb]));
       const int nv = it.nvalid();
       const bool valid = r < nv;
       const float l = valid ? m + lg2_approx(z) : 0.f;
@@ -346,11 +391,8 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         ok = false;
         break;
       }
-      float lmax = -INFINITY;
-      for (int p = 0; p < C; ++p) lmax = fmaxf(lmax, xch[(qs * C + p) * 128 + r]);
-      float zs = 0.f;
-      for (int p = 0; p < C; ++p) zs += ex2_approx(xch[(qs * C + p) * 128 + r] - lmax);
-      const float lse2 = lmax + lg2_approx(zs);
+      // lse over the C partials: all loads and exponentials independent (tree reductions)
+      const float lse2 = combine_partials(xch + qs * C * 128 + r, C);
       const float scale = valid ? ex2_approx(m - lse2) : 0.f;
       if (rank == 0 && valid && lse_out != nullptr)
         lse_out[it.t0() + r] = lse2 * 0.69314718055994530942f;
