@@ -127,6 +127,26 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Epilogue for a user whose tokens were split across calls (for example across GPUs,
+ * one part per rank). The forward's accumulation is a plain sum over tokens, so the
+ * parts' xsketch and mass outputs add up to the whole user's (the sketch's definition
+ * as a mass-weighted mean of V over tokens; blog "1. Sketch Attention compresses the
+ * history"). After the caller has summed them (an all-reduce), this writes
+ *   sketch_j = (xsketch_j Wv) / mass_j   (0 where mass_j = 0)
+ * exactly as the forward's own last step does.
+ *
+ *   xsketch [R, k, d] fp32, device   sums of the parts' xsketch outputs
+ *   mass    [R, k]    fp32, device   sums of the parts' mass outputs
+ *   Wv      [d, d]    dt, device     as passed to the forward
+ *   sketch  [R, k, d] fp32, device   output (overwritten)
+ * d in {64, 128}; k >= 1. Pointers 16-byte aligned. Needs no workspace, allocates
+ * nothing, enqueues one kernel on `stream` and does not synchronise. Returns SA_OK,
+ * SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED or SA_ERR_CUDA.
+ */
+int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int d,
+                      const void* Wv, sa_dtype dt, float* sketch, void* stream);
+
+/*
  * Forward without a workspace, for callers that cannot allocate device memory (for
  * example a serving process whose allocator reserved all of its memory at start-up and
  * forbids new allocations, or code running where cudaMalloc may not be called). The

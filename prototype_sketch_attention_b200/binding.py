@@ -30,7 +30,7 @@ SA_ERR_NO_DEVICE = 7
 
 EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
             "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
-            "sa_sketch_profile_events", "sa_sketch_forward_noalloc")
+            "sa_sketch_profile_events", "sa_sketch_forward_noalloc", "sa_sketch_combine")
 
 
 class SketchAttentionError(RuntimeError):
@@ -53,6 +53,8 @@ def _load() -> ctypes.CDLL:
     lib.sa_sketch_backward.restype = i32
     lib.sa_sketch_backward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
                                        vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sa_sketch_combine.restype = i32
+    lib.sa_sketch_combine.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp, vp]
     lib.sa_sketch_get_device_status.restype = i32
     lib.sa_sketch_get_device_status.argtypes = [vp, vp]
     lib.sa_status_string.restype = ctypes.c_char_p
@@ -86,6 +88,10 @@ def sa_sketch_backward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass
     return int(_lib.sa_sketch_backward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass,
                                        lse, xsketch, dsketch, dmass, dX, dP, dWk, dWv, workspace,
                                        ws_bytes, stream))
+
+
+def sa_sketch_combine(xsketch, mass, R, k, d, Wv, dt, sketch, stream) -> int:
+    return int(_lib.sa_sketch_combine(xsketch, mass, R, k, d, Wv, dt, sketch, stream))
 
 
 def sa_sketch_get_device_status(workspace, stream) -> int:
@@ -193,6 +199,21 @@ def backward(X, offsets, P, Wk, Wv, fwd: dict, dsketch: torch.Tensor, dmass=None
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_sketch_backward")
     out["_ws"] = ws
+    return out
+
+
+def combine(xsketch: torch.Tensor, mass: torch.Tensor, Wv: torch.Tensor, *,
+            out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """sketch = (xsketch Wv) / mass for users whose partial xsketch and mass (from
+    forward calls over parts of their tokens) have been summed. xsketch [R, k, d] and
+    mass [R, k] fp32, Wv [d, d] bf16/fp32, all on one CUDA device."""
+    R, k, d = xsketch.shape
+    if out is None:
+        out = torch.empty(R, k, d, device=xsketch.device, dtype=torch.float32)
+    st = sa_sketch_combine(_ptr(xsketch), _ptr(mass), R, k, d, _ptr(Wv), _dt(Wv), _ptr(out),
+                           _stream(stream))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_combine")
     return out
 
 

@@ -353,6 +353,22 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
   return cuda_status(launch_bwd_simt(a, s));
 }
 
+int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int d, const void* Wv,
+                      sa_dtype dt, float* sketch, void* stream_) {
+  if (R < 0 || R > SA_MAX_USERS || k < 1 || k > SA_MAX_K) return SA_ERR_INVALID_ARG;
+  if (dt != SA_F32 && dt != SA_BF16) return SA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+  if (R == 0) return SA_OK;
+  if (!xsketch || !mass || !Wv || !sketch) return SA_ERR_INVALID_ARG;
+  if (!aligned16(xsketch) || !aligned16(mass) || !aligned16(Wv) || !aligned16(sketch))
+    return SA_ERR_INVALID_ARG;
+  Device dev;
+  sa_status st = current_device(&dev);
+  if (st != SA_OK) return st;
+  return cuda_status(launch_combine(xsketch, mass, R, k, d, Wv, dt, sketch,
+                                    static_cast<cudaStream_t>(stream_)));
+}
+
 int sa_sketch_get_device_status(const void* workspace, void* stream_) {
   if (!workspace) return SA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream_);

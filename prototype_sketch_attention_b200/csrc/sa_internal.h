@@ -36,6 +36,10 @@ struct FinalizeArgs {
 };
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
 
+// ---- combine: sketch = (U Wv) / mass from already summed U [R, k, d] and mass [R, k]
+cudaError_t launch_combine(const float* U, const float* mass, int R, int k, int d, const void* Wv,
+                           sa_dtype dt, float* sketch, cudaStream_t s);
+
 // ---- tcgen05 forward (bf16)
 struct FwdSm100Args {
   const CUtensorMap* tmap_x;

@@ -245,6 +245,54 @@ __global__ void __launch_bounds__(256) finalize_tiled_kernel(FinalizeArgs a, con
   }
 }
 
+// combine, tiled: block = (user u, 64 prototypes). U and mass are already summed (over
+// the parts of a user that was split across calls); sketch = U Wv / mass.
+template <int D, typename TIn>
+__global__ void __launch_bounds__(256) combine_tiled_kernel(const float* __restrict__ U,
+                                                            const float* __restrict__ mass, int k,
+                                                            const TIn* __restrict__ Wv,
+                                                            float* __restrict__ sketch) {
+  using S = TileShape<D>;
+  extern __shared__ __align__(16) float tsm[];
+  float* lr = tsm;                      // [64][D+4]
+  float* rm = tsm + kRowTile * S::kLd;  // [D][D+4]
+  float* ms = rm + D * S::kLd;          // [64]
+  constexpr int kV = D / 4;
+  const int u = blockIdx.x;
+  const int j0 = blockIdx.y * kRowTile;
+  for (int i = threadIdx.x; i < kRowTile * kV; i += blockDim.x) {
+    const int j = i / kV, c4 = i % kV;
+    const float4 v = (j0 + j < k)
+        ? reinterpret_cast<const float4*>(U + ((size_t)u * k + j0 + j) * D)[c4]
+        : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4*>(lr + j * S::kLd + c4 * 4) = v;
+  }
+  if (threadIdx.x < kRowTile)
+    ms[threadIdx.x] = (j0 + (int)threadIdx.x < k) ? mass[(size_t)u * k + j0 + threadIdx.x] : 0.f;
+  for (int i = threadIdx.x; i < D * kV; i += blockDim.x) {
+    const int c = i / kV, e4 = i % kV;
+    float4 w;
+    w.x = to_f(Wv[c * D + e4 * 4]);
+    w.y = to_f(Wv[c * D + e4 * 4 + 1]);
+    w.z = to_f(Wv[c * D + e4 * 4 + 2]);
+    w.w = to_f(Wv[c * D + e4 * 4 + 3]);
+    *reinterpret_cast<float4*>(rm + c * S::kLd + e4 * 4) = w;
+  }
+  __syncthreads();
+  float acc[S::kJPT][4];
+  tile_gemm<D>(lr, rm, acc);
+  const int te = threadIdx.x % S::kTE, tj = threadIdx.x / S::kTE;
+#pragma unroll
+  for (int r = 0; r < S::kJPT; ++r) {
+    const int jj = tj * S::kJPT + r, j = j0 + jj;
+    if (j >= k) continue;
+    const float m = ms[jj];
+    const float inv = m > 0.f ? 1.f / m : 0.f;
+    *reinterpret_cast<float4*>(sketch + ((size_t)u * k + j) * D + te * 4) =
+        make_float4(acc[r][0] * inv, acc[r][1] * inv, acc[r][2] * inv, acc[r][3] * inv);
+  }
+}
+
 // ------------------------------------------------------------------ test hook
 __global__ void debug_wait_timeout_kernel(WsHeader* hdr, long long budget) {
   __shared__ alignas(8) uint64_t bar;
@@ -307,6 +355,28 @@ cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s) {
   if (a.dt == SA_BF16)
     return a.d == 128 ? launch_finalize_t<128, __nv_bfloat16>(a, s) : launch_finalize_t<64, __nv_bfloat16>(a, s);
   return a.d == 128 ? launch_finalize_t<128, float>(a, s) : launch_finalize_t<64, float>(a, s);
+}
+
+template <int D, typename TIn>
+cudaError_t launch_combine_t(const float* U, const float* mass, int R, int k, const void* Wv,
+                             float* sketch, cudaStream_t s) {
+  auto kern = combine_tiled_kernel<D, TIn>;
+  const size_t smem = ((size_t)(kRowTile + D) * TileShape<D>::kLd + kRowTile) * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((unsigned)R, (unsigned)((k + kRowTile - 1) / kRowTile));
+  kern<<<grid, 256, smem, s>>>(U, mass, k, static_cast<const TIn*>(Wv), sketch);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_combine(const float* U, const float* mass, int R, int k, int d, const void* Wv,
+                           sa_dtype dt, float* sketch, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  if (dt == SA_BF16)
+    return d == 128 ? launch_combine_t<128, __nv_bfloat16>(U, mass, R, k, Wv, sketch, s)
+                    : launch_combine_t<64, __nv_bfloat16>(U, mass, R, k, Wv, sketch, s);
+  return d == 128 ? launch_combine_t<128, float>(U, mass, R, k, Wv, sketch, s)
+                  : launch_combine_t<64, float>(U, mass, R, k, Wv, sketch, s);
 }
 
 cudaError_t launch_debug_wait_timeout(WsHeader* hdr, long long budget, cudaStream_t s) {

@@ -81,3 +81,16 @@ def test_binding_names_match_header():
     from prototype_sketch_attention_b200 import binding
     for n in declared_functions():
         assert n in binding.EXPORTED and hasattr(binding, n), n
+
+
+def test_combine_rejects_bad_arguments_on_host(lib):
+    vp, i32 = ctypes.c_void_p, ctypes.c_int
+    f = lib.sa_sketch_combine
+    f.restype = i32
+    f.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp, vp]
+    assert f(None, None, -1, 8, 64, None, 0, None, None) == 1   # R < 0
+    assert f(None, None, 1, 0, 64, None, 0, None, None) == 1    # k < 1
+    assert f(None, None, 1, 8, 64, None, 7, None, None) == 1    # bad dtype
+    assert f(None, None, 1, 8, 100, None, 0, None, None) == 2   # d not in {64, 128}
+    assert f(None, None, 1, 8, 64, None, 0, None, None) == 1    # null pointers
+    assert f(None, None, 0, 8, 64, None, 0, None, None) == 0    # no users: nothing to do
