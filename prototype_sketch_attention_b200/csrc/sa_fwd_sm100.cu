@@ -10,8 +10,8 @@
 //
 // Decomposition. A cluster of C = ceil(k/128) CTAs owns one slice of the token stream; CTA
 // of rank c owns prototypes [128c, 128c+128). Per tile of 128 tokens each CTA:
-//   1. TMA loads the X tile (128 x d bf16, 32B swizzle, 16-column boxes) into one of NS
-//      shared-memory stages; each stage is followed by an all-ones 16-column block.
+//   1. TMA loads the X tile (128 x d bf16, 128B swizzle, 64-column boxes) into one of NS
+//      shared-memory stages; the stages share one all-ones atom (see FwdSmem).
 //      Every CTA loads the tile itself (no multicast; the C-fold re-read is served by L2,
 //      and rank 0 prefetches upcoming tiles into L2).
 //   2. tcgen05.mma  S^T[tok, proto] = X_tile . P'_slice^T  into TMEM (fp32, two
@@ -22,7 +22,7 @@
 //      lse2 = log2 sum_c 2^(l_c) and A = 2^(s - lse2).
 //   4. A is written as bf16 into shared memory in the MN-major layout of the next MMA's
 //      A operand, then  [U | mass] += A . [X_tile | 1]  (one tcgen05.mma with N = d + 16,
-//      accumulator in TMEM): the 16 extra columns read the all-ones block and carry the
+//      accumulator in TMEM): the 16 extra columns read the all-ones atom and carry the
 //      per-prototype mass sum_t A_jt.
 //   5. When the token stream crosses a user boundary (or the slice ends) the partial
 //      (U, mass) of that (cluster, user) segment is written to the workspace; the finalize
@@ -44,21 +44,41 @@ constexpr int kXchSlots = 4;                  // exchange slots (tile index mod 
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS0 = 0, kColS1 = 128, kColU = 256;
 
+// Shared memory in 16 KB slots (one 128-row x 128-byte swizzled atom column each).
+//
+// X arrives in boxes of 64 columns with the 128-byte swizzle (a 32 KB tile moves in
+// two TMA boxes; measured on B200, that lands in under half the time of eight 16-column
+// boxes). MMA2 reads [X | 1] as one MN-major operand of width d + 16: its 64-column
+// atoms sit LBO bytes apart and the all-ones block is the atom after the last X atom.
+// The descriptor's LBO is per stage, so every stage can end on ONE shared ones atom:
+// stage s puts X box b at slot kOnes - (d/64 - b) * a_s and uses LBO = a_s slots, with
+// the a_s chosen so that no two stages share a slot (d = 128: a = 1, 3, 4 -> slots
+// {6,7}, {2,5}, {0,4}; the free slots 1 and 3 hold an A buffer).
 template <int D, int NS>
 struct FwdSmem {
-  static constexpr int kStages = NS;
-  static constexpr int kBoxBytes = 128 * 16 * 2;             // X TMA box: 128 rows x 16 bf16 (32B swizzle)
+  static constexpr int kSlot = 16384;
+  static constexpr int kXBoxes = D / 64;
   static constexpr int kXBytes = 128 * D * 2;                // X tile
-  static constexpr int kOnesBytes = 128 * 16 * 2;            // all-ones 16-column atom after X
-  static constexpr int kXStage = kXBytes + kOnesBytes;
-  static constexpr int kPBox = 128 * 64 * 2;                 // P' TMA box: 128 rows x 64 bf16 (128B swizzle)
   static constexpr int kPBytes = kProtoSlice * D * 2;        // P' slice
   static constexpr int kABytes = kProtoSlice * kTileTokens * 2;  // A tile (bf16)
-  // byte offsets from the 1024-aligned base
-  static constexpr int oX = 0;
-  static constexpr int oP = oX + kStages * kXStage;
-  static constexpr int oA = oP + kPBytes;
-  static constexpr int oXch = oA + 2 * kABytes;  // kXchSlots * C * 128 floats (runtime C)
+  static_assert((D == 128 && (NS == 3 || NS == 2)) || (D == 64 && NS == 4), "layout");
+  static constexpr int kOnes = D == 128 ? 8 : 4;
+  // stage spacing a_s (in slots): d = 128: 1, 3, 4; d = 64: 1, 2, 3, 4
+  __host__ __device__ static constexpr int stage_a(int s) {
+    return D == 128 ? (s == 0 ? 1 : s == 1 ? 3 : 4) : s + 1;
+  }
+  // byte offset of X box b of stage s; of the A buffer's two 64-prototype atoms
+  __host__ __device__ static constexpr int xbox(int s, int b) {
+    return (kOnes - (kXBoxes - b) * stage_a(s)) * kSlot;
+  }
+  __host__ __device__ static constexpr int abox(int buf, int mb) {
+    return (D == 128 ? (NS == 3 ? (buf == 0 ? (mb == 0 ? 1 : 3) : (mb == 0 ? 9 : 10))
+                                : (buf == 0 ? (mb == 0 ? 0 : 1) : (mb == 0 ? 3 : 4)))
+                     : (buf == 0 ? (mb == 0 ? 5 : 6) : (mb == 0 ? 7 : 8))) * kSlot;
+  }
+  static constexpr int oOnes = kOnes * kSlot;
+  static constexpr int oP = (D == 128 ? (NS == 3 ? 11 : 9) : 9) * kSlot;
+  static constexpr int oXch = oP + kPBytes;  // kXchSlots * C * 128 floats (runtime C)
   static size_t bytes(int C) {
     const size_t xch = (size_t)kXchSlots * C * 128 * 4;
     const size_t bars = 64 * 8 + 16;
@@ -206,13 +226,10 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
     tmem_relinquish();
   }
   if (warp >= 4) {
-    // the all-ones atom after every X stage: MMA2 runs with N = d + 16, so the 16
-    // extra output columns accumulate sum_t A_jt (the mass) next to U
-    const int t = threadIdx.x - 128;
-    for (int s2 = 0; s2 < NS; ++s2) {
-      uint32_t* ones = reinterpret_cast<uint32_t*>(smem + L::oX + s2 * L::kXStage + L::kXBytes);
-      for (int w = t; w < L::kOnesBytes / 4; w += kThreads - 128) ones[w] = 0x3F803F80u;
-    }
+    // the shared all-ones atom read by MMA2 after the X atoms (N = d + 16): its 16 extra
+    // output columns accumulate sum_t A_jt (the mass) next to U
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + L::oOnes);
+    for (int w = threadIdx.x - 128; w < L::kSlot / 4; w += kThreads - 128) ones[w] = 0x3F803F80u;
     fence_proxy_async_smem();
   }
   tc_fence_before();
@@ -233,13 +250,13 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
       const uint32_t pf = smem_u32(&bars->p_full);
       mbar_arrive_expect_tx(pf, L::kPBytes);
       for (int b = 0; b < D / 64; ++b)
-        tma_load_2d(sbase + L::oP + b * L::kPBox, &tmap_p, b * 64, (int)rank * kProtoSlice, pf);
+        tma_load_2d(sbase + L::oP + b * L::kSlot, &tmap_p, b * 64, (int)rank * kProtoSlice, pf);
       TileIter it, ahead;
       it.init(tile_start, offsets, R, ta, tb);
       ahead.init(tile_start, offsets, R, ta, tb);
       if (rank == 0) {
         for (int j = 0; j < kPrefetchAhead && ahead.valid(); ++j, ahead.next())
-          for (int b = 0; b < D / 16; ++b) tma_prefetch_l2_2d(&tmap_x, b * 16, (int)ahead.t0());
+          for (int b = 0; b < L::kXBoxes; ++b) tma_prefetch_l2_2d(&tmap_x, b * 64, (int)ahead.t0());
       }
       long long i = 0;
       for (; it.valid(); it.next(), ++i) {
@@ -249,10 +266,10 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const uint32_t fb = smem_u32(&bars->x_full[st]);
         mbar_arrive_expect_tx(fb, L::kXBytes);
         const int y = (int)it.t0();
-        for (int b = 0; b < D / 16; ++b)
-          tma_load_2d(sbase + L::oX + st * L::kXStage + b * L::kBoxBytes, &tmap_x, b * 16, y, fb);
+        for (int b = 0; b < L::kXBoxes; ++b)
+          tma_load_2d(sbase + L::xbox(st, b), &tmap_x, b * 64, y, fb);
         if (rank == 0 && ahead.valid()) {
-          for (int b = 0; b < D / 16; ++b) tma_prefetch_l2_2d(&tmap_x, b * 16, (int)ahead.t0());
+          for (int b = 0; b < L::kXBoxes; ++b) tma_prefetch_l2_2d(&tmap_x, b * 64, (int)ahead.t0());
           ahead.next();
         }
       }
@@ -266,14 +283,14 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
     if (lane == 0 && ta < tb) {
       const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);
       const uint32_t idesc2 = idesc_bf16_f32(128, D + 16, 1, 1);
-      // Shared-memory descriptors for stage 0 / A buffer 0, built once: a later operand
-      // address is the same descriptor plus (byte offset >> 4) in its 14-bit address
-      // field (every operand lies below 256 KB, so the field never carries). Building
-      // each descriptor from scratch right before its MMA made issue the bottleneck.
-      const uint64_t dx1 = smem_desc(sbase + L::oX, 16, 256, kSwizzle32B);            // X, K-major
-      const uint64_t dp1 = smem_desc(sbase + L::oP, 16, 1024, kSwizzle128B);          // P', K-major
-      const uint64_t da2 = smem_desc(sbase + L::oA, L::kPBox, 1024, kSwizzle128B);    // A, MN-major
-      const uint64_t dx2 = smem_desc(sbase + L::oX, L::kBoxBytes, 256, kSwizzle32B);  // [X|1], MN-major
+      // Shared-memory descriptors built once per operand base; a later operand address is
+      // the same descriptor plus (byte offset >> 4) in its 14-bit address field (every
+      // operand lies below 256 KB, so the field never carries).
+      const uint64_t dp1 = smem_desc(sbase + L::oP, 16, 1024, kSwizzle128B);  // P', K-major
+      const uint64_t da2_0 =                                                  // A, MN-major
+          smem_desc(sbase + L::abox(0, 0), L::abox(0, 1) - L::abox(0, 0), 1024, kSwizzle128B);
+      const uint64_t da2_1 =
+          smem_desc(sbase + L::abox(1, 0), L::abox(1, 1) - L::abox(1, 0), 1024, kSwizzle128B);
       bool ok = mbar_wait(smem_u32(&bars->p_full), 0, status, budget);
       TileIter it;
       it.init(tile_start, offsets, R, ta, tb);
@@ -289,11 +306,15 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget);
           if (!ok) break;
           tc_fence_after();
-          const uint64_t xd = dx1 + (uint64_t)((st * L::kXStage) >> 4);
+          // A = X tile, K-major, 128B swizzle: four 16-wide K steps per 64-column box
+          uint64_t xd[L::kXBoxes];
+#pragma unroll
+          for (int b = 0; b < L::kXBoxes; ++b)
+            xd[b] = smem_desc(sbase + L::xbox(st, b), 16, 1024, kSwizzle128B);
 #pragma unroll
           for (int ks = 0; ks < KSTEPS1; ++ks) {
-            const uint32_t koff = (ks >> 2) * L::kPBox + (ks & 3) * 32;
-            tc_mma_f16(tmem + (sb ? kColS1 : kColS0), xd + (uint64_t)((ks * L::kBoxBytes) >> 4),
+            const uint32_t koff = (ks >> 2) * L::kSlot + (ks & 3) * 32;
+            tc_mma_f16(tmem + (sb ? kColS1 : kColS0), xd[ks >> 2] + (uint64_t)(((ks & 3) * 32) >> 4),
                        dp1 + (uint64_t)(koff >> 4), idesc1, ks > 0 ? 1u : 0u);
           }
           tc_commit(smem_u32(&bars->s_full[sb]));
@@ -303,11 +324,15 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                (!first || mbar_wait(smem_u32(&bars->u_empty), (uint32_t)((seg & 1) ^ 1), status, budget));
           if (!ok) break;
           tc_fence_after();
-          const uint64_t ad0 = da2 + (uint64_t)((ab * L::kABytes) >> 4);
-          const uint64_t xd = dx2 + (uint64_t)((st * L::kXStage) >> 4);
+          // A = A tile, MN-major (prototypes contiguous); B = [X | 1], MN-major (d contiguous),
+          // its atoms LBO = a_s slots apart ending on the shared ones atom; both 128B swizzle,
+          // a 16-token K step is two 8-row groups (2048 bytes)
+          const uint64_t ad0 = ab ? da2_1 : da2_0;
+          const uint64_t xd = smem_desc(sbase + L::xbox(st, 0), L::stage_a(st) * L::kSlot, 1024,
+                                        kSwizzle128B);
 #pragma unroll
           for (int ks = 0; ks < KSTEPS2; ++ks)
-            tc_mma_f16(tmem + kColU, ad0 + (uint64_t)((ks * 2048) >> 4), xd + (uint64_t)((ks * 512) >> 4),
+            tc_mma_f16(tmem + kColU, ad0 + (uint64_t)((ks * 2048) >> 4), xd + (uint64_t)((ks * 2048) >> 4),
                        idesc2, (first && ks == 0) ? 0u : 1u);
           tc_commit(smem_u32(&bars->x_empty[st]));
           tc_commit(smem_u32(&bars->a_empty[ab]));
@@ -404,7 +429,8 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         ok = false;
         break;
       }
-      uint8_t* arow = smem + L::oA + ab * L::kABytes + r * 128;
+      uint8_t* arow0 = smem + L::abox(ab, 0) + r * 128;
+      uint8_t* arow1 = smem + L::abox(ab, 1) + r * 128;
       const uint64_t sc2 = f2_pack(scale, scale);
 #pragma unroll
       for (int mb = 0; mb < 2; ++mb) {
@@ -418,7 +444,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
             f2_unpack(f2_mul(f2_pack(v[c0 + 2 * h], v[c0 + 2 * h + 1]), sc2), a, b);
             w4[h] = cvt_bf16x2(a, b);
           }
-          *reinterpret_cast<uint4*>(arow + mb * 16384 + ((ch ^ (r & 7)) << 4)) =
+          *reinterpret_cast<uint4*>((mb ? arow1 : arow0) + ((ch ^ (r & 7)) << 4)) =
               make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }

@@ -224,7 +224,7 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   if (n_total > 0) {
     if (p.tc) {
       CUtensorMap tx, tp;
-      if (!make_tmap_bf16(&tx, X, (uint64_t)n_total, d, 16) ||
+      if (!make_tmap_bf16(&tx, X, (uint64_t)n_total, d, 64) ||
           !make_tmap_bf16(&tp, at<void>(workspace, p.pf), (uint64_t)p.k_pad, d, 64))
         return SA_ERR_CUDA;
       FwdSm100Args a;
