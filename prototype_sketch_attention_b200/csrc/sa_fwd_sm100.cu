@@ -52,32 +52,36 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColU = 256;
 // atoms sit LBO bytes apart and the all-ones block is the atom after the last X atom.
 // The descriptor's LBO is per stage, so every stage can end on ONE shared ones atom:
 // stage s puts X box b at slot kOnes - (d/64 - b) * a_s and uses LBO = a_s slots, with
-// the a_s chosen so that no two stages share a slot (d = 128: a = 1, 3, 4 -> slots
-// {6,7}, {2,5}, {0,4}; the free slots 1 and 3 hold an A buffer).
-template <int D, int NS>
+// the a_s chosen so that no two stages share a slot (d = 128: a = 1, 3, 4, 5 -> slots
+// {8,9}, {4,7}, {2,6}, {0,5}; the free slots 1 and 3 hold the A tile).
+//
+// The A tile is single-buffered at d = 128 (NA = 1): it lives from the softmax's store
+// to the end of the accumulate MMA, well under one tile period, and the slots it frees
+// buy a fourth X stage, which is what bounds the tile rate (an X stage is held from its
+// load through the scores, the softmax and the accumulate MMA).
+template <int D, int NS, int NA>
 struct FwdSmem {
   static constexpr int kSlot = 16384;
   static constexpr int kXBoxes = D / 64;
   static constexpr int kXBytes = 128 * D * 2;                // X tile
   static constexpr int kPBytes = kProtoSlice * D * 2;        // P' slice
-  static constexpr int kABytes = kProtoSlice * kTileTokens * 2;  // A tile (bf16)
-  static_assert((D == 128 && (NS == 3 || NS == 2)) || (D == 64 && NS == 4), "layout");
-  static constexpr int kOnes = D == 128 ? 8 : 4;
-  // stage spacing a_s (in slots): d = 128: 1, 3, 4; d = 64: 1, 2, 3, 4
+  static_assert((D == 128 && NA == 1 && (NS == 4 || NS == 3)) || (D == 64 && NS == 4 && NA == 2),
+                "layout");
+  static constexpr int kOnes = D == 128 ? (NS == 4 ? 10 : 8) : 4;
+  // stage spacing a_s (in slots): d = 128: 1, 3, 4, 5; d = 64: 1, 2, 3, 4
   __host__ __device__ static constexpr int stage_a(int s) {
-    return D == 128 ? (s == 0 ? 1 : s == 1 ? 3 : 4) : s + 1;
+    return D == 128 ? (s == 0 ? 1 : s == 1 ? 3 : s == 2 ? 4 : 5) : s + 1;
   }
   // byte offset of X box b of stage s; of the A buffer's two 64-prototype atoms
   __host__ __device__ static constexpr int xbox(int s, int b) {
     return (kOnes - (kXBoxes - b) * stage_a(s)) * kSlot;
   }
   __host__ __device__ static constexpr int abox(int buf, int mb) {
-    return (D == 128 ? (NS == 3 ? (buf == 0 ? (mb == 0 ? 1 : 3) : (mb == 0 ? 9 : 10))
-                                : (buf == 0 ? (mb == 0 ? 0 : 1) : (mb == 0 ? 3 : 4)))
+    return (D == 128 ? (NS == 4 ? (mb == 0 ? 1 : 3) : (mb == 0 ? 1 : 3))
                      : (buf == 0 ? (mb == 0 ? 5 : 6) : (mb == 0 ? 7 : 8))) * kSlot;
   }
   static constexpr int oOnes = kOnes * kSlot;
-  static constexpr int oP = (D == 128 ? (NS == 3 ? 11 : 9) : 9) * kSlot;
+  static constexpr int oP = (D == 128 ? (NS == 4 ? 11 : 9) : 9) * kSlot;
   static constexpr int oXch = oP + kPBytes;  // kXchSlots * C * 128 floats (runtime C)
   static size_t bytes(int C) {
     const size_t xch = (size_t)kXchSlots * C * 128 * 4;
@@ -177,7 +181,7 @@ __device__ __forceinline__ float combine_partials(const float* x, int C) {
   return mx + lg2_approx(t[0]);
 }
 
-template <int D, int NS>
+template <int D, int NS, int NA>
 __global__ void __launch_bounds__(kThreads, 1)
 sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const __grid_constant__ CUtensorMap tmap_p,
@@ -185,7 +189,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     WsHeader* hdr, const long long* __restrict__ tile_start,
                     float* __restrict__ part_u, float* __restrict__ part_m,
                     float* __restrict__ lse_out, long long budget) {
-  using L = FwdSmem<D, NS>;
+  using L = FwdSmem<D, NS, NA>;
   constexpr int KSTEPS1 = D / 16;           // MMA1 K steps (over d)
   constexpr int KSTEPS2 = kTileTokens / 16;  // MMA2 K steps (over tokens)
   extern __shared__ uint8_t smem_raw[];
@@ -319,8 +323,9 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
           }
           tc_commit(smem_u32(&bars->s_full[sb]));
         } else {
-          const int ab = sb;
-          ok = mbar_wait(smem_u32(&bars->a_full[ab]), (uint32_t)((i >> 1) & 1), status, budget) &&
+          const int ab = NA == 2 ? sb : 0;
+          const uint32_t apar = NA == 2 ? (uint32_t)((i >> 1) & 1) : (uint32_t)(i & 1);
+          ok = mbar_wait(smem_u32(&bars->a_full[ab]), apar, status, budget) &&
                (!first || mbar_wait(smem_u32(&bars->u_empty), (uint32_t)((seg & 1) ^ 1), status, budget));
           if (!ok) break;
           tc_fence_after();
@@ -424,8 +429,9 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
 
       // A (bf16) into the MN-major, 128B-swizzled A operand: row = token, 64 prototypes
       // per 128-byte row, two 16 KB blocks for prototypes [0,64) and [64,128).
-      const int ab = wg;
-      if (!mbar_wait_warp(smem_u32(&bars->a_empty[ab]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget)) {
+      const int ab = NA == 2 ? wg : 0;
+      const uint32_t epar = NA == 2 ? (uint32_t)(((i >> 1) & 1) ^ 1) : (uint32_t)((i & 1) ^ 1);
+      if (!mbar_wait_warp(smem_u32(&bars->a_empty[ab]), epar, status, budget)) {
         ok = false;
         break;
       }
@@ -493,10 +499,10 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
   }
 }
 
-template <int D, int NS>
+template <int D, int NS, int NA>
 cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
-  auto kern = sa_fwd_sm100_kernel<D, NS>;
-  const size_t smem = FwdSmem<D, NS>::bytes(a.C);
+  auto kern = sa_fwd_sm100_kernel<D, NS, NA>;
+  const size_t smem = FwdSmem<D, NS, NA>::bytes(a.C);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (a.C > 8) {
@@ -519,10 +525,10 @@ cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
                             a.k_pad, a.hdr, a.tile_start, a.part_u, a.part_m, a.lse, a.budget);
 }
 
-template <int D, int NS>
+template <int D, int NS, int NA>
 cudaError_t max_clusters_t(int C, int* n) {
-  auto kern = sa_fwd_sm100_kernel<D, NS>;
-  const size_t smem = FwdSmem<D, NS>::bytes(C);
+  auto kern = sa_fwd_sm100_kernel<D, NS, NA>;
+  const size_t smem = FwdSmem<D, NS, NA>::bytes(C);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   if (C > 8) {
@@ -543,27 +549,27 @@ cudaError_t max_clusters_t(int C, int* n) {
   return cudaOccupancyMaxActiveClusters(n, kern, &cfg);
 }
 
-// X stages: 3 while the exchange slots leave room (C <= 8 at d = 128), else 2; 4 at d = 64.
-int stages_for(int d, int C) { return d == 64 ? 4 : (C <= 8 ? 3 : 2); }
+// X stages: 4 at d = 128 while the exchange slots leave room (C <= 8), else 3; 4 at d = 64.
+int stages_for(int d, int C) { return d == 64 ? 4 : (C <= 8 ? 4 : 3); }
 
 }  // namespace
 
 size_t fwd_sm100_smem_bytes(int d, int C) {
   const int ns = stages_for(d, C);
-  if (d == 64) return FwdSmem<64, 4>::bytes(C);
-  return ns == 3 ? FwdSmem<128, 3>::bytes(C) : FwdSmem<128, 2>::bytes(C);
+  if (d == 64) return FwdSmem<64, 4, 2>::bytes(C);
+  return ns == 4 ? FwdSmem<128, 4, 1>::bytes(C) : FwdSmem<128, 3, 1>::bytes(C);
 }
 
 cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
   const int ns = stages_for(d, C);
-  if (d == 64) return max_clusters_t<64, 4>(C, n);
-  return ns == 3 ? max_clusters_t<128, 3>(C, n) : max_clusters_t<128, 2>(C, n);
+  if (d == 64) return max_clusters_t<64, 4, 2>(C, n);
+  return ns == 4 ? max_clusters_t<128, 4, 1>(C, n) : max_clusters_t<128, 3, 1>(C, n);
 }
 
 cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream) {
   const int ns = stages_for(a.d, a.C);
-  if (a.d == 64) return launch_fwd_sm100_t<64, 4>(a, stream);
-  return ns == 3 ? launch_fwd_sm100_t<128, 3>(a, stream) : launch_fwd_sm100_t<128, 2>(a, stream);
+  if (a.d == 64) return launch_fwd_sm100_t<64, 4, 2>(a, stream);
+  return ns == 4 ? launch_fwd_sm100_t<128, 4, 1>(a, stream) : launch_fwd_sm100_t<128, 3, 1>(a, stream);
 }
 
 }  // namespace sa
