@@ -464,46 +464,43 @@ __device__ __forceinline__ int user_of_tile(const long long* tile_start, int R, 
 // Walks the tiles [a, b) of the global tile sequence (users' tiles concatenated).
 // Tile indices fit in 32 bits: n_total < 2^31 tokens gives fewer than 2^31 tiles.
 struct TileIter {
-  // Walks the tiles [a, end) of the concatenated per-user tile lists. The current
-  // user's tile and token ranges live in registers; global memory (tile_start,
+  // Walks the tiles [g0, end) of the concatenated per-user tile lists. The current
+  // user's tile and token bounds live in registers; global memory (tile_start,
   // offsets) is read only when the walk crosses into the next user, so the per-tile
   // queries below cost no memory round trip.
   const long long* ts;
   const int64_t* off;
-  int g, a, end, u;
-  int ts_u, ts_u1;          // tiles [ts_u, ts_u1) belong to user u
-  int off_u, off_u1;        // tokens [off_u, off_u1) belong to user u (n_total < 2^31)
+  int g, end, u;
+  int ts_u1;    // first tile of the next user (tiles of user u end there)
+  int t0b;      // first token of tile g is t0b + 128 g (n_total < 2^31)
+  int tok_end;  // one past the last token of user u
   __device__ void init(const long long* ts_, const int64_t* off_, int R, long long a_,
                        long long b_) {
-    ts = ts_; off = off_; g = (int)a_; a = (int)a_; end = (int)b_; u = 0;
-    ts_u = ts_u1 = 0;
-    off_u = off_u1 = 0;
+    ts = ts_; off = off_; g = (int)a_; end = (int)b_; u = 0;
+    ts_u1 = t0b = tok_end = 0;
     if (a_ < b_) {
       u = user_of_tile(ts, R, a_);
-      ts_u = (int)ts[u];
+      const int ts_u = (int)ts[u];
       ts_u1 = (int)ts[u + 1];
-      off_u = (int)off[u];
-      off_u1 = (int)off[u + 1];
+      t0b = (int)off[u] - ts_u * kTileTokens;
+      tok_end = (int)off[u + 1];
     }
   }
   __device__ bool valid() const { return g < end; }
-  __device__ int local() const { return g - ts_u; }
-  __device__ long long t0() const { return (long long)off_u + local() * kTileTokens; }
+  __device__ long long t0() const { return (long long)t0b + g * kTileTokens; }
   __device__ int nvalid() const {
-    const int n = off_u1 - off_u - local() * kTileTokens;
+    const int n = tok_end - (t0b + g * kTileTokens);
     return n >= kTileTokens ? kTileTokens : n;
   }
-  __device__ bool first() const { return g == a || g == ts_u; }
   __device__ bool last() const { return g == end - 1 || g == ts_u1 - 1; }
   __device__ void next() {
     ++g;
     if (g < end) {
-      while (ts_u1 <= g) {
+      while (ts_u1 <= g) {  // next user (users without tiles are skipped)
         ++u;
-        ts_u = ts_u1;
+        t0b = tok_end - ts_u1 * kTileTokens;
         ts_u1 = (int)ts[u + 1];
-        off_u = off_u1;
-        off_u1 = (int)off[u + 1];
+        tok_end = (int)off[u + 1];
       }
     }
   }

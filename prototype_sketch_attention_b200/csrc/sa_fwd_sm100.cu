@@ -159,23 +159,25 @@ __device__ __forceinline__ float row_max(const float (&v)[kProtoSlice]) {
   return fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
 }
 
-// log2 of the sum of 2^x[p * 128] over the C partials of one token (C <= kMaxCluster).
-// Every load and exponential is independent; max and sum are trees.
+// log2 of the sum of 2^x[p * 128] over the C partials of one token (C <= MAXC).
+// Every load and exponential is independent; max and sum are trees. MAXC is the
+// kernel's cluster-size bound, which keeps the register footprint at MAXC.
+template <int MAXC>
 __device__ __forceinline__ float combine_partials(const float* x, int C) {
-  float lp[kMaxCluster], t[kMaxCluster];
+  float lp[MAXC], t[MAXC];
 #pragma unroll
-  for (int p = 0; p < kMaxCluster; ++p) lp[p] = p < C ? x[p * 128] : -INFINITY;
+  for (int p = 0; p < MAXC; ++p) lp[p] = p < C ? x[p * 128] : -INFINITY;
 #pragma unroll
-  for (int p = 0; p < kMaxCluster; ++p) t[p] = lp[p];
+  for (int p = 0; p < MAXC; ++p) t[p] = lp[p];
 #pragma unroll
-  for (int w = kMaxCluster / 2; w >= 1; w /= 2)
+  for (int w = MAXC / 2; w >= 1; w /= 2)
 #pragma unroll
     for (int p = 0; p < w; ++p) t[p] = fmaxf(t[p], t[p + w]);
   const float mx = t[0];
 #pragma unroll
-  for (int p = 0; p < kMaxCluster; ++p) t[p] = p < C ? ex2_approx(lp[p] - mx) : 0.f;
+  for (int p = 0; p < MAXC; ++p) t[p] = p < C ? ex2_approx(lp[p] - mx) : 0.f;
 #pragma unroll
-  for (int w = kMaxCluster / 2; w >= 1; w /= 2)
+  for (int w = MAXC / 2; w >= 1; w /= 2)
 #pragma unroll
     for (int p = 0; p < w; ++p) t[p] += t[p + w];
   return mx + lg2_approx(t[0]);
@@ -192,6 +194,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
   using L = FwdSmem<D, NS, NA>;
   constexpr int KSTEPS1 = D / 16;           // MMA1 K steps (over d)
   constexpr int KSTEPS2 = kTileTokens / 16;  // MMA2 K steps (over tokens)
+  constexpr int kMaxC = (D == 128 && NS == 4) ? 8 : kMaxCluster;  // cluster-size bound
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
@@ -262,7 +265,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         for (int j = 0; j < kPrefetchAhead && ahead.valid(); ++j, ahead.next())
           for (int b = 0; b < L::kXBoxes; ++b) tma_prefetch_l2_2d(&tmap_x, b * 64, (int)ahead.t0());
       }
-      long long i = 0;
+      int i = 0;
       for (; it.valid(); it.next(), ++i) {
         const int st = (int)(i % NS);
         const uint32_t par = (uint32_t)((i / NS) & 1);
@@ -298,10 +301,11 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
       bool ok = mbar_wait(smem_u32(&bars->p_full), 0, status, budget);
       TileIter it;
       it.init(tile_start, offsets, R, ta, tb);
-      long long i = 0;
-      int seg = -1;
+      int i = 0;
+      int seg = -1, prev_u = -1;
       for (; ok && it.valid(); it.next(), ++i) {
-        const bool first = it.first(), last = it.last();
+        const bool first = it.u != prev_u, last = it.last();  // first tile of a segment
+        prev_u = it.u;
         if (first) ++seg;
         const int st = (int)(i % NS);
         const int sb = (int)(i & 1);
@@ -359,7 +363,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
     const bool partial_slice = pbase + kProtoSlice > k_valid;
     TileIter it;
     it.init(tile_start, offsets, R, ta, tb);
-    long long i = 0;
+    int i = 0;
     int useg = 0;  // segments whose last tile this warpgroup owned so far (u_full[wg] phases)
     bool ok = true;
     for (; ok && it.valid(); it.next(), ++i) {
@@ -422,7 +426,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         break;
       }
       // lse over the C partials: all loads and exponentials independent (tree reductions)
-      const float lse2 = combine_partials(xch + qs * C * 128 + r, C);
+      const float lse2 = combine_partials<kMaxC>(xch + qs * C * 128 + r, C);
       const float scale = valid ? ex2_approx(m - lse2) : 0.f;
       if (rank == 0 && valid && lse_out != nullptr)
         lse_out[it.t0() + r] = lse2 * 0.69314718055994530942f;
