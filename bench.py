@@ -38,6 +38,8 @@ sys.path.insert(0, ROOT)
 
 METRIC = "history tokens/s of SA sketch (k=1024,d=128) and % of bf16 tensor-core peak"
 UNIT = "tokens/s"
+WORKLOAD = ("config3: R=40 users, n~U[10000,100000], d=128, k=1024, bf16 in / fp32 accumulate, "
+            "forward")
 FALLBACK_PEAK_TFLOPS = 1590.0
 PROFILE_SUMMARY = os.path.join(ROOT, "profiles", "sa_fwd_sm100_config3.md")
 KERNEL_SOURCES = [os.path.join(ROOT, "prototype_sketch_attention_b200", "csrc", f)
@@ -161,30 +163,37 @@ class ClockSampler:
 
 
 # ------------------------------------------------------------------ CPU oracle baseline
-def oracle_sample_rate(w, target_s: float, max_tokens: int = 200_000):
-    """Times the fp64 oracle on the first S tokens of user 0 (S sized for ~target_s).
-    Returns (tokens/s, tokens, seconds, threads)."""
+def oracle_sample(w, S: int):
+    """The first S tokens of the batch (spanning users 0, 1, ... with their own offsets),
+    as fp64 arrays for the oracle."""
     import numpy as np
+    off = w.offsets.numpy()
+    S = int(min(S, off[-1]))
+    cut = np.minimum(off, S)
+    last = int(np.searchsorted(cut, S, side="left"))  # users [0, last) hold the sample
+    sub_off = cut[:last + 1].astype(np.int64) if last > 0 else np.array([0, S], dtype=np.int64)
+    return (w.X[:S].double().numpy(), sub_off, w.P.double().numpy(), w.Wk.double().numpy(),
+            w.Wv.double().numpy())
+
+
+def oracle_sample_rate(w, target_s: float, max_tokens: int = 2_000_000):
+    """Times the fp64 oracle on the first S tokens of the batch (S sized for ~target_s of
+    wall time). Returns (tokens/s, tokens, seconds, threads, users)."""
     import oracle
     threads = os.cpu_count() or 1
-    off = w.offsets.numpy()
-    n0 = int(off[1] - off[0])
-    P = w.P.double().numpy()
-    Wk = w.Wk.double().numpy()
-    Wv = w.Wv.double().numpy()
 
     def run(S):
-        X = w.X[:S].double().numpy()
+        X, off, P, Wk, Wv = oracle_sample(w, S)
         t0 = time.perf_counter()
-        oracle.forward(X, np.array([0, S], dtype=np.int64), P, Wk, Wv, nthreads=threads)
-        return time.perf_counter() - t0
+        oracle.forward(X, off, P, Wk, Wv, nthreads=threads)
+        return time.perf_counter() - t0, len(off) - 1
 
-    probe = min(n0, 2048)
-    tp = run(probe)
-    S = int(min(n0, max_tokens, max(probe, probe * target_s / max(tp, 1e-6))))
-    t = run(S) if S != probe else tp
+    probe = 8192
+    tp, _ = run(probe)
+    S = int(min(w.n_total, max_tokens, max(probe, probe * target_s / max(tp, 1e-6))))
+    t, users = run(S)
     used = min(threads, math.ceil(S / 1024))  # the oracle parallelises over 1024-token chunks
-    return S / t, S, t, used
+    return S / t, S, t, used, users
 
 
 # ------------------------------------------------------------------ reference arm
@@ -197,12 +206,10 @@ def run_reference(args) -> None:
     import numpy as np
     import oracle
     threads = os.cpu_count() or 1
-    # each step: the oracle on a bounded sample of user 0 (whole run within a few minutes)
+    # each step: the oracle on a bounded sample of the batch (whole run within a few minutes)
     per_step_target = max(0.5, 150.0 / max(1, args.steps + args.warmup))
-    rate, S, t, used = oracle_sample_rate(w, per_step_target)
-    P, Wk, Wv = (w.P.double().numpy(), w.Wk.double().numpy(), w.Wv.double().numpy())
-    X = w.X[:S].double().numpy()
-    off = np.array([0, S], dtype=np.int64)
+    rate, S, t, used, users = oracle_sample_rate(w, per_step_target)
+    X, off, P, Wk, Wv = oracle_sample(w, S)
     for _ in range(args.warmup):
         oracle.forward(X, off, P, Wk, Wv, nthreads=threads)
     times = []
@@ -212,13 +219,15 @@ def run_reference(args) -> None:
         times.append(time.perf_counter() - t0)
     step_s = sum(times) / len(times)
     value = S / step_s
-    sample = f"first {S} tokens of user 0 of config 3 per step (k=1024, d=128), fp64 oracle"
+    sample = (f"first {S} tokens of config 3 ({users} users) per step (k=1024, d=128), "
+              "fp64 oracle")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic",
-        "config": {"workload": w.meta["desc"], "n_total": w.n_total, "sample_tokens": S},
+        "config": {"workload": WORKLOAD, "n_total_per_gpu": w.n_total, "R": w.R, "k": w.k, "d": w.d,
+                   "sample_tokens": S, "parallelism": "host cores, rank 0 only"},
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": min(threads, math.ceil(S / 1024)),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -342,10 +351,10 @@ def run_ours(args) -> None:
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, S, secs, used = oracle_sample_rate(w, args.cpu_seconds)
+        rate, S, secs, used, users = oracle_sample_rate(w, args.cpu_seconds)
         cpu = {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle",
-               "sample": f"first {S} tokens of user 0 of config 3 (k=1024, d=128), fp64 oracle, "
-                         f"{secs:.1f} s wall"}
+               "sample": f"first {S} tokens of config 3 ({users} users; k=1024, d=128), "
+                         f"fp64 oracle, {secs:.1f} s wall"}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
@@ -355,8 +364,7 @@ def run_ours(args) -> None:
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": "config3: R=40 users, n~U[10000,100000], d=128, k=1024, bf16 in / "
-                               "fp32 accumulate, forward",
+        "config": {"workload": WORKLOAD,
                    "n_total_per_gpu": n_total, "R": R, "k": k, "d": d,
                    "l2": "inputs larger than L2 (X is %.0f MB per GPU)" % (h2d / 1e6),
                    "parallelism": f"users sharded, {world} independent batch(es)"},
