@@ -55,7 +55,9 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a, const TIn* __r
     const int jj = i / d, c = i % d;
     float acc = 0.f;
     for (int e = 0; e < d; ++e) acc = fmaf(gt[jj * d + e], wv[c * ld + e], acc);
-    a.Gh[((size_t)u * a.k_pad + j0 + jj) * d + c] = acc;
+    const size_t o = ((size_t)u * a.k_pad + j0 + jj) * d + c;
+    if (a.Gh) a.Gh[o] = acc;
+    if (a.Ghb) a.Ghb[o] = __float2bfloat16_rn(acc);
   }
   if (threadIdx.x < kCP) {
     const int j = j0 + threadIdx.x;
@@ -385,18 +387,50 @@ cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t s) {
 }
 
 template <typename TIn>
+static cudaError_t launch_prep(const BwdArgs& a, cudaStream_t s) {
+  if (a.R == 0) return cudaSuccess;
+  const int d = a.d;
+  const size_t smem = (size_t)(d * (d + 1) + kCP * d) * sizeof(float);
+  cudaError_t e =
+      cudaFuncSetAttribute(bwd_prep_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  bwd_prep_kernel<TIn><<<dim3((unsigned)a.R, (unsigned)(a.k_pad / kCP)), 256, smem, s>>>(
+      a, static_cast<const TIn*>(a.Wv));
+  return cudaGetLastError();
+}
+
+// dPn = sum of a.G partials (fixed order), dW_v chunks, then dW_v, dP, dW_k.
+template <typename TIn>
+static cudaError_t launch_tail(const BwdArgs& a, cudaStream_t s) {
+  cudaError_t e;
+  const int d = a.d;
+  bwd_reduce_dpp_kernel<<<256, 256, 0, s>>>(a);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const int nch = (int)bwd_wv_chunks(a.R, a.k);
+  if (nch > 0) {
+    const size_t smem_w = (size_t)(64 * d) * sizeof(float);
+    bwd_wv_part_kernel<<<(unsigned)nch, 256, smem_w, s>>>(a);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  bwd_finish_kernel<TIn><<<dim3((unsigned)d, 3), 128, 0, s>>>(
+      a, static_cast<const TIn*>(a.P), static_cast<const TIn*>(a.Wk), nch, 1.0f / sqrtf((float)d));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_bwd_prep(const BwdArgs& a, cudaStream_t s) {
+  return a.dt == SA_BF16 ? launch_prep<__nv_bfloat16>(a, s) : launch_prep<float>(a, s);
+}
+
+cudaError_t launch_bwd_tail(const BwdArgs& a, cudaStream_t s) {
+  return a.dt == SA_BF16 ? launch_tail<__nv_bfloat16>(a, s) : launch_tail<float>(a, s);
+}
+
+template <typename TIn>
 static cudaError_t launch_all(const BwdArgs& a, cudaStream_t s) {
   cudaError_t e;
   const int d = a.d;
   const TIn* X = static_cast<const TIn*>(a.X);
-  if (a.R > 0) {
-    const size_t smem = (size_t)(d * (d + 1) + kCP * d) * sizeof(float);
-    e = cudaFuncSetAttribute(bwd_prep_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    bwd_prep_kernel<TIn><<<dim3((unsigned)a.R, (unsigned)(a.k_pad / kCP)), 256, smem, s>>>(
-        a, static_cast<const TIn*>(a.Wv));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
+  if ((e = launch_prep<TIn>(a, s)) != cudaSuccess) return e;
   if (a.n_total > 0) {
     const long long max_tiles = a.n_total / kTileTokens + a.R + 1;
     const size_t smem_t =
@@ -413,18 +447,8 @@ static cudaError_t launch_all(const BwdArgs& a, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     bwd_proto_kernel<TIn><<<dim3((unsigned)a.G, (unsigned)(a.k_pad / kCP)), 256, smem_p, s>>>(a, X);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    bwd_reduce_dpp_kernel<<<256, 256, 0, s>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  const int nch = (int)bwd_wv_chunks(a.R, a.k);
-  if (nch > 0) {
-    const size_t smem_w = (size_t)(64 * d) * sizeof(float);
-    bwd_wv_part_kernel<<<(unsigned)nch, 256, smem_w, s>>>(a);
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-  bwd_finish_kernel<TIn><<<dim3((unsigned)d, 3), 128, 0, s>>>(
-      a, static_cast<const TIn*>(a.P), static_cast<const TIn*>(a.Wk), nch, 1.0f / sqrtf((float)d));
-  return cudaGetLastError();
+  return launch_tail<TIn>(a, s);
 }
 
 }  // namespace sa

@@ -1,0 +1,238 @@
+// Sketch Attention backward on tcgen05 tensor cores (bf16 inputs, fp32 accumulate).
+//
+// The gradient of the sketch (blog "100,000 videos in your pocket", section "1. Sketch
+// Attention compresses the history": the compression is differentiable) with
+// Pn = P W_k^T / sqrt(d), G = dL/dsketch, Gm = dL/dmass and, per user u,
+//   Gt = G / mass,  Gh = Gt W_v^T,  c_j = Gt_j . sketch_j - Gm_j,
+//   A_jt = exp(Pn_j . X_t - lse_t),  dA_jt = Gh_j . X_t - c_j,
+//   D_t = sum_j A_jt dA_jt,  dS_jt = A_jt (dA_jt - D_t),
+//   dX_t = sum_j dS_jt Pn_j + sum_j A_jt Gh_j,   dPn = sum_t dS_t^T X_t,
+// then dP = dPn W_k / sqrt(d), dW_k = dPn^T P / sqrt(d), dW_v = sum_u U_u^T Gt_u.
+//
+// Every contraction over d, k or the tokens runs as a tensor-core GEMM
+// (sa_gemm_sm100.cu) with the elementwise work fused into its epilogue; the token x
+// prototype intermediates (A, Q = A (dA) and dS) live in the workspace:
+//   prep (CUDA cores)   Gt, bf16 Gh, c per user
+//   fold                pn2 = bf16(Pn log2 e), pnn = bf16(Pn)
+//   [lse not given]     GEMM S2 = X pn2^T -> per-tile log2-sum-exp -> lse2 per token
+//   GEMM (plain tiles)  A = 2^(X pn2^T - lse2)                          bf16 [n, k_pad]
+//   GEMM (user tiles)   Q = A (X Gh_u^T - c_u), per-tile row sums of Q   fp32 [n, k_pad]
+//   CUDA cores          D_t = sum of the row sums, dS = Q - A D_t        bf16 [n, k_pad]
+//   GEMM (user tiles)   dX = dS pnn + A Gh_u  (two operand pairs, one accumulator)
+//   GEMM (split-K)      partials of dPn = dS^T X over token ranges
+//   tail (CUDA cores)   dPn = sum of partials (fixed order), dW_v, dP, dW_k
+// 10 k d FLOP per token on the tensor cores (12 when the lse is recomputed).
+#include <cmath>
+
+#include "sa_common.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+namespace {
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// D_t = sum of the row's per-tile partial sums of Q; dS = Q - A D_t (bf16).
+// One warp per token row, 8 columns per lane and step.
+__global__ void __launch_bounds__(256) bwd_ds_kernel(const float* __restrict__ Q,
+                                                     const __nv_bfloat16* __restrict__ A,
+                                                     const float* __restrict__ dpart, int ntiles,
+                                                     int k_pad, long long n_total,
+                                                     __nv_bfloat16* __restrict__ dS,
+                                                     const WsHeader* hdr) {
+  if (read_status(&hdr->status) != 0) return;
+  const int lane = threadIdx.x & 31;
+  const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long t = w0; t < n_total; t += nw) {
+    float D = 0.f;
+    for (int i = lane; i < ntiles; i += 32) D += dpart[t * ntiles + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
+    const float* q = Q + t * k_pad;
+    const __nv_bfloat16* a = A + t * k_pad;
+    __nv_bfloat16* o = dS + t * k_pad;
+    for (int c = lane * 8; c < k_pad; c += 256) {
+      const float4 q0 = *reinterpret_cast<const float4*>(q + c);
+      const float4 q1 = *reinterpret_cast<const float4*>(q + c + 4);
+      const uint4 av = *reinterpret_cast<const uint4*>(a + c);
+      const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+      uint32_t w[4];
+#pragma unroll
+      for (int h = 0; h < 4; ++h) {
+        const float a0 = __uint_as_float(aw[h] << 16), a1 = __uint_as_float(aw[h] & 0xFFFF0000u);
+        w[h] = cvt_bf16x2(fmaf(-a0, D, qv[2 * h]), fmaf(-a1, D, qv[2 * h + 1]));
+      }
+      *reinterpret_cast<uint4*>(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+  }
+}
+
+// lse2_t = log2 sum over the row's tiles of 2^(partial).  One thread per token.
+__global__ void bwd_lse_kernel(const float* __restrict__ dpart, int ntiles, long long n_total,
+                               float* __restrict__ lse2, const WsHeader* hdr) {
+  if (read_status(&hdr->status) != 0) return;
+  for (long long t = blockIdx.x * (long long)blockDim.x + threadIdx.x; t < n_total;
+       t += (long long)gridDim.x * blockDim.x) {
+    const float* p = dpart + t * ntiles;
+    float m = -INFINITY;
+    for (int i = 0; i < ntiles; ++i) m = fmaxf(m, p[i]);
+    float z = 0.f;
+    for (int i = 0; i < ntiles; ++i) z += ex2_approx(p[i] - m);
+    lse2[t] = m + lg2_approx(z);
+  }
+}
+
+GemmOperandDesc op(const void* base, uint64_t rows, uint64_t cols, bool mn_major) {
+  GemmOperandDesc o;
+  o.base = base;
+  o.rows = rows;
+  o.cols = cols;
+  o.mn_major = mn_major;
+  return o;
+}
+
+}  // namespace
+
+// Split-K count of the dPn GEMM: about two CTAs per SM, at most one split per K tile.
+int bwd_tc_splits(int sms, int k_pad, int d, long long n_total) {
+  const int tiles = (k_pad / 128) * ((d + 127) / 128);
+  const long long kt = (n_total + 63) / 64;
+  long long s = (2LL * sms + tiles - 1) / tiles;
+  if (s > kt) s = kt;
+  if (s < 1) s = 1;
+  return (int)s;
+}
+
+cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
+  const BwdArgs& b = a.b;
+  cudaError_t e;
+  const int d = b.d, k = b.k, k_pad = b.k_pad, R = b.R;
+  const long long n = b.n_total;
+  const int ntiles = k_pad / 128;
+  if ((e = launch_bwd_prep(b, s)) != cudaSuccess) return e;
+  const float isd = 1.0f / std::sqrt((float)d);
+  if ((e = launch_fold(b.P, b.Wk, SA_BF16, k, k_pad, d, kLog2e * isd, a.pn2, true, s)) != cudaSuccess)
+    return e;
+  if ((e = launch_fold(b.P, b.Wk, SA_BF16, k, k_pad, d, isd, a.pnn, true, s)) != cudaSuccess)
+    return e;
+  if (n == 0) {
+    e = cudaMemsetAsync(b.dpp_part, 0, (size_t)a.splits * k_pad * d * sizeof(float), s);
+    if (e != cudaSuccess) return e;
+    return launch_bwd_tail(b, s);
+  }
+  const int m_plain = (int)((n + 127) / 128);
+  const int m_user = (int)(n / 128 + R + 1);
+  const GemmOperandDesc X_k = op(b.X, (uint64_t)n, (uint64_t)d, false);       // [n][d], K = d
+  const GemmOperandDesc pn2_k = op(a.pn2, (uint64_t)k_pad, (uint64_t)d, false);
+  const GemmOperandDesc gh_k = op(b.Ghb, (uint64_t)R * k_pad, (uint64_t)d, false);
+
+  GemmArgs g = {};
+  g.hdr = b.hdr;
+  g.tile_start = b.tile_start;
+  g.offsets = b.offsets;
+  g.R = R;
+  g.k_pad = k_pad;
+  g.k_valid = k;
+  g.splits = 1;
+
+  // lse2 per token (log2 units): the forward's lse, or recomputed here
+  const float* lse_src = a.lse;
+  float lse_scale = kLog2e;
+  if (!lse_src) {
+    GemmArgs l = g;
+    l.phases = 1;
+    l.a[0] = X_k;
+    l.b[0] = pn2_k;
+    l.k_tiles[0] = (d + 63) / 64;
+    l.user_mode = 0;
+    l.M = (int)n;
+    l.N = k_pad;
+    l.m_tiles_bound = m_plain;
+    l.epi = kEpiLse;
+    l.dpart = a.dpart;
+    l.dpart_ld = ntiles;
+    if ((e = launch_gemm(l, s)) != cudaSuccess) return e;
+    bwd_lse_kernel<<<1024, 256, 0, s>>>(a.dpart, ntiles, n, a.lse2, b.hdr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    lse_src = a.lse2;
+    lse_scale = 1.f;
+  }
+  {  // A = 2^(X pn2^T - lse2)
+    GemmArgs t = g;
+    t.phases = 1;
+    t.a[0] = X_k;
+    t.b[0] = pn2_k;
+    t.k_tiles[0] = (d + 63) / 64;
+    t.user_mode = 0;
+    t.M = (int)n;
+    t.N = k_pad;
+    t.m_tiles_bound = m_plain;
+    t.epi = kEpiAExp;
+    t.out_bf16 = a.A;
+    t.ld_out = k_pad;
+    t.lse2 = lse_src;
+    t.lse_scale = lse_scale;
+    if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
+  }
+  {  // Q = A (X Gh_u^T - c_u) and its per-tile row sums
+    GemmArgs t = g;
+    t.phases = 1;
+    t.a[0] = X_k;
+    t.b[0] = gh_k;
+    t.b_user_rows[0] = k_pad;
+    t.k_tiles[0] = (d + 63) / 64;
+    t.user_mode = 1;
+    t.N = k_pad;
+    t.m_tiles_bound = m_user;
+    t.epi = kEpiQ;
+    t.out_f32 = a.Q;
+    t.ld_out = k_pad;
+    t.a_in = a.A;
+    t.ld_a_in = k_pad;
+    t.c_user = b.cj;
+    t.dpart = a.dpart;
+    t.dpart_ld = ntiles;
+    if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
+  }
+  bwd_ds_kernel<<<2048, 256, 0, s>>>(a.Q, a.A, a.dpart, ntiles, k_pad, n, a.dS, b.hdr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {  // dX = dS pnn + A Gh_u
+    GemmArgs t = g;
+    t.phases = 2;
+    t.a[0] = op(a.dS, (uint64_t)n, (uint64_t)k_pad, false);
+    t.b[0] = op(a.pnn, (uint64_t)k_pad, (uint64_t)d, true);
+    t.a[1] = op(a.A, (uint64_t)n, (uint64_t)k_pad, false);
+    t.b[1] = op(b.Ghb, (uint64_t)R * k_pad, (uint64_t)d, true);
+    t.b_user_rows[1] = k_pad;
+    t.k_tiles[0] = t.k_tiles[1] = k_pad / 64;
+    t.user_mode = 1;
+    t.N = d;
+    t.m_tiles_bound = m_user;
+    t.epi = kEpiStoreF32;
+    t.out_f32 = b.dX;
+    t.ld_out = d;
+    if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
+  }
+  {  // dPn partials = dS^T X, split over token ranges
+    GemmArgs t = g;
+    t.phases = 1;
+    t.a[0] = op(a.dS, (uint64_t)n, (uint64_t)k_pad, true);
+    t.b[0] = op(b.X, (uint64_t)n, (uint64_t)d, true);
+    t.k_tiles[0] = (int)((n + 63) / 64);
+    t.user_mode = 0;
+    t.M = k_pad;
+    t.N = d;
+    t.m_tiles_bound = ntiles;
+    t.splits = a.splits;
+    t.epi = kEpiStoreF32;
+    t.out_f32 = b.dpp_part;
+    t.ld_out = d;
+    t.split_stride = (long long)k_pad * d;
+    if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
+  }
+  return launch_bwd_tail(b, s);
+}
+
+}  // namespace sa

@@ -1,0 +1,353 @@
+// Tensor-core GEMM building block for the Sketch Attention backward (sm_100a).
+//
+//   C[128 x 128 tile] = sum over phases p, K tiles k of  A_p[m, k] . B_p[n, k]
+//
+// bf16 operands arrive by TMA in 128-byte-swizzled boxes; tcgen05.mma (kind::f16, fp32
+// accumulate) runs from one thread into TMEM; four epilogue warps read the accumulator
+// (thread = output row = TMEM lane) and apply one of the fused epilogues below. Each
+// operand is either K-major (stored [M or N rows][K], K contiguous) or MN-major (stored
+// [K rows][M or N], M/N contiguous), so A B^T, A^T B and A B are all one kernel.
+//
+// Row tiles are either plain (128 consecutive rows of M) or user tiles: tile g covers
+// the tokens of one user only (the forward's schedule: tile_start prefix sums), so an
+// operand that depends on the user (B_p with a per-user row offset) is well defined.
+//
+// Epilogues:
+//   kEpiStoreF32  out[row][n] = acc (fp32), or a split-K partial at split * split_stride
+//   kEpiAExp      out_bf16[row][n] = bf16(2^(acc - lse_scale * lse[row])) (A = softmax),
+//                 0 for columns n >= k_valid
+//   kEpiLse       dpart[row][tile] = log2 sum over the tile's columns n < k_valid of 2^acc
+//   kEpiQ         q = A[row][n] (acc - c[user][n]); out[row][n] = q (fp32) and the
+//                 row sum of q over the tile's 128 columns into dpart[row][tile]
+// Waits on mbarriers are bounded like every other kernel of the library.
+#include <cuda.h>
+
+#include "sa_common.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+namespace {
+
+constexpr int kBM = 128, kBN = 128, kBK = 64;
+constexpr int kStages = 3;
+constexpr int kStageBytes = (kBM + kBN) * kBK * 2;  // 32 KB
+constexpr int kGemmThreads = 192;                   // producer, MMA, 4 epilogue warps
+
+struct GemmParams {
+  CUtensorMap ta[2], tb[2];
+  int a_mn[2], b_mn[2];
+  int k_tiles[2];
+  int b_user_rows[2];
+  int phases;
+  int user_mode;
+  int M, N;
+  int splits;
+  const WsHeader* hdr;
+  const long long* tile_start;
+  const int64_t* offsets;
+  int R;
+  float* out_f32;
+  long long ld_out;
+  long long split_stride;
+  __nv_bfloat16* out_bf16;
+  const float* lse2;
+  float lse_scale;
+  int k_valid;
+  const __nv_bfloat16* a_in;
+  long long ld_a_in;
+  const float* c_user;
+  int k_pad;
+  float* dpart;
+  int dpart_ld;
+  long long budget;
+};
+
+struct GemmBars {
+  uint64_t full[kStages], empty[kStages], done, drain;
+  uint32_t tmem_base;
+};
+
+// One operand tile (128 rows of M or N by 64 of K) of the given layout into smem.
+__device__ __forceinline__ void load_operand(uint32_t dst, const CUtensorMap* tm, int mn_major,
+                                             int mn0, int k0, uint32_t bar) {
+  if (!mn_major) {
+    tma_load_2d(dst, tm, k0, mn0, bar);  // box {64 K, 128 rows}
+  } else {
+    tma_load_2d(dst, tm, mn0, k0, bar);              // box {64 M/N, 64 K}
+    tma_load_2d(dst + 8192, tm, mn0 + 64, k0, bar);  // the second 64 M/N columns
+  }
+}
+
+// Shared-memory descriptor of K step ks (16 wide) of an operand tile.
+__device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, int ks) {
+  return mn_major ? smem_desc(base + ks * 2048, 8192, 1024, kSwizzle128B)
+                  : smem_desc(base + ks * 32, 16, 1024, kSwizzle128B);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(kGemmThreads)
+sa_gemm_kernel(const __grid_constant__ GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  GemmBars* bars = reinterpret_cast<GemmBars*>(smem + kStages * kStageBytes);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = const_cast<int*>(&p.hdr->status);
+
+  // ---- which output tile
+  int row0 = 0, nrows = 0, user = 0;
+  if (p.user_mode) {
+    const long long T = p.hdr->total_tiles;
+    const long long g = blockIdx.x;
+    if (g >= T || read_status(status) != 0) return;
+    user = user_of_tile(p.tile_start, p.R, g);
+    const long long local = g - p.tile_start[user];
+    row0 = (int)(p.offsets[user] + local * kBM);
+    const long long n = p.offsets[user + 1] - row0;
+    nrows = n >= kBM ? kBM : (int)n;
+  } else {
+    row0 = blockIdx.x * kBM;
+    nrows = min(kBM, p.M - row0);
+    if (nrows <= 0) return;
+  }
+  const int n0 = blockIdx.y * kBN;
+  // K tiles of this CTA: phase 0 is split evenly across gridDim.z; phase 1 is not split
+  const int z = blockIdx.z;
+  const int kt0 = (int)((long long)p.k_tiles[0] * z / p.splits);
+  const int kt1 = (int)((long long)p.k_tiles[0] * (z + 1) / p.splits);
+  const int total_kt = (kt1 - kt0) + (p.phases > 1 ? p.k_tiles[1] : 0);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&bars->full[s]), 1);
+      mbar_init(smem_u32(&bars->empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->done), 1);
+    mbar_init(smem_u32(&bars->drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kBN);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ================= TMA producer
+    if (lane == 0 && total_kt > 0) {
+      for (int ph = 0; ph < p.phases; ++ph) {
+        tma_prefetch_desc(&p.ta[ph]);
+        tma_prefetch_desc(&p.tb[ph]);
+      }
+      for (int j = 0; j < total_kt; ++j) {
+        const int st = j % kStages;
+        if (!mbar_wait(smem_u32(&bars->empty[st]), (uint32_t)(((j / kStages) & 1) ^ 1), status,
+                       p.budget))
+          break;
+        const int ph = j < kt1 - kt0 ? 0 : 1;
+        const int kt = ph == 0 ? kt0 + j : j - (kt1 - kt0);
+        const uint32_t fb = smem_u32(&bars->full[st]);
+        mbar_arrive_expect_tx(fb, kStageBytes);
+        const uint32_t sa = sbase + st * kStageBytes;
+        const int bu = p.b_user_rows[ph] * user;
+        load_operand(sa, &p.ta[ph], p.a_mn[ph], row0, kt * kBK, fb);
+        // B's per-user offset applies to its row dimension: N for K-major, K for MN-major
+        if (!p.b_mn[ph]) load_operand(sa + kBM * kBK * 2, &p.tb[ph], 0, bu + n0, kt * kBK, fb);
+        else load_operand(sa + kBM * kBK * 2, &p.tb[ph], 1, n0, bu + kt * kBK, fb);
+      }
+      // the last stages' loads must land before exit
+      for (int j = total_kt > kStages ? total_kt - kStages : 0; j < total_kt; ++j)
+        mbar_wait_drain(smem_u32(&bars->full[j % kStages]), (uint32_t)((j / kStages) & 1), p.budget);
+    }
+  } else if (warp == 1) {
+    // ================= MMA issuer
+    if (lane == 0 && total_kt > 0) {
+      const uint32_t idesc0 = idesc_bf16_f32(kBM, kBN, p.a_mn[0], p.b_mn[0]);
+      const uint32_t idesc1 = idesc_bf16_f32(kBM, kBN, p.a_mn[1], p.b_mn[1]);
+      bool ok = true;
+      for (int j = 0; j < total_kt && ok; ++j) {
+        const int st = j % kStages;
+        ok = mbar_wait(smem_u32(&bars->full[st]), (uint32_t)((j / kStages) & 1), status, p.budget);
+        if (!ok) break;
+        tc_fence_after();
+        const int ph = j < kt1 - kt0 ? 0 : 1;
+        const uint32_t sa = sbase + st * kStageBytes, sb = sa + kBM * kBK * 2;
+#pragma unroll
+        for (int ks = 0; ks < kBK / 16; ++ks)
+          tc_mma_f16(tmem, operand_desc(sa, p.a_mn[ph], ks), operand_desc(sb, p.b_mn[ph], ks),
+                     ph ? idesc1 : idesc0, (j > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&bars->empty[st]));
+      }
+      tc_commit(smem_u32(&bars->done));
+      mbar_wait_drain(smem_u32(&bars->done), 0, p.budget);
+    }
+  } else {
+    // ================= epilogue: thread = output row (TMEM lane)
+    const int q = warp & 3;
+    const int r = q * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    const bool have = total_kt > 0 &&
+                      mbar_wait_warp(smem_u32(&bars->done), 0, status, p.budget);
+    if (have) {
+      tc_fence_after();
+      const bool valid = r < nrows;
+      const long long row = (long long)row0 + r;
+      float lse2 = 0.f;
+      if (EPI == kEpiAExp && valid) lse2 = p.lse2[row] * p.lse_scale;
+      float qsum = 0.f, lmax = -INFINITY, lsum = 0.f;
+#pragma unroll 1
+      for (int c = 0; c < kBN / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32_raw(tmem + lane_off + c * 32, u);
+        tmem_wait_tie(u);
+        const int nb = n0 + c * 32;
+        if (!valid || nb >= p.N) continue;
+        if (EPI == kEpiStoreF32) {
+          float* dst = p.out_f32 + (long long)z * p.split_stride + row * p.ld_out + nb;
+#pragma unroll
+          for (int x = 0; x < 32; x += 4)
+            if (nb + x < p.N)
+              *reinterpret_cast<float4*>(dst + x) =
+                  make_float4(__uint_as_float(u[x]), __uint_as_float(u[x + 1]),
+                              __uint_as_float(u[x + 2]), __uint_as_float(u[x + 3]));
+        } else if (EPI == kEpiAExp) {
+          __nv_bfloat16* dst = p.out_bf16 + row * p.ld_out + nb;
+#pragma unroll
+          for (int x = 0; x < 32; x += 8) {
+            uint32_t w[4];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const int n = nb + x + 2 * h;
+              w[h] = cvt_bf16x2(n < p.k_valid ? ex2_approx(__uint_as_float(u[x + 2 * h]) - lse2) : 0.f,
+                                n + 1 < p.k_valid ? ex2_approx(__uint_as_float(u[x + 2 * h + 1]) - lse2) : 0.f);
+            }
+            if (nb + x < p.N) *reinterpret_cast<uint4*>(dst + x) = make_uint4(w[0], w[1], w[2], w[3]);
+          }
+        } else if (EPI == kEpiLse) {
+          // running log2-sum-exp2 over this row's columns (a fresh max per 32 columns)
+          float cm = -INFINITY;
+#pragma unroll
+          for (int x = 0; x < 32; ++x)
+            if (nb + x < p.k_valid) cm = fmaxf(cm, __uint_as_float(u[x]));
+          if (cm > -INFINITY) {
+            float cs = 0.f;
+#pragma unroll
+            for (int x = 0; x < 32; ++x)
+              if (nb + x < p.k_valid) cs += ex2_approx(__uint_as_float(u[x]) - cm);
+            const float nm = fmaxf(lmax, cm);
+            lsum = lsum * ex2_approx(lmax - nm) + cs * ex2_approx(cm - nm);
+            lmax = nm;
+          }
+        } else {  // kEpiQ
+          const __nv_bfloat16* ain = p.a_in + row * p.ld_a_in + nb;
+          const float* cu = p.c_user + (long long)user * p.k_pad + nb;
+          float* dst = p.out_f32 + row * p.ld_out + nb;
+#pragma unroll
+          for (int x = 0; x < 32; x += 8) {
+            if (nb + x >= p.N) break;
+            const uint4 av = *reinterpret_cast<const uint4*>(ain + x);
+            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
+            float qv[8];
+#pragma unroll
+            for (int h = 0; h < 4; ++h) {
+              const float a0 = __uint_as_float(aw[h] << 16), a1 = __uint_as_float(aw[h] & 0xFFFF0000u);
+              qv[2 * h] = a0 * (__uint_as_float(u[x + 2 * h]) - cu[x + 2 * h]);
+              qv[2 * h + 1] = a1 * (__uint_as_float(u[x + 2 * h + 1]) - cu[x + 2 * h + 1]);
+            }
+            *reinterpret_cast<float4*>(dst + x) = make_float4(qv[0], qv[1], qv[2], qv[3]);
+            *reinterpret_cast<float4*>(dst + x + 4) = make_float4(qv[4], qv[5], qv[6], qv[7]);
+            qsum += ((qv[0] + qv[1]) + (qv[2] + qv[3])) + ((qv[4] + qv[5]) + (qv[6] + qv[7]));
+          }
+        }
+      }
+      if (EPI == kEpiQ && valid) p.dpart[row * p.dpart_ld + blockIdx.y] = qsum;
+      if (EPI == kEpiLse && valid)
+        p.dpart[row * p.dpart_ld + blockIdx.y] = lmax > -INFINITY ? lmax + lg2_approx(lsum) : -INFINITY;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kBN);
+  }
+}
+
+// Row-major bf16 matrix [rows][cols] with boxes of box_cols x box_rows (128B swizzle).
+bool make_operand_map(CUtensorMap* m, const GemmOperandDesc& o) {
+  auto fn = tmap_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {o.cols, o.rows};
+  const cuuint64_t strides[1] = {o.cols * 2};
+  const cuuint32_t box[2] = {64, o.mn_major ? 64u : 128u};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(o.base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int EPI>
+cudaError_t launch_t(const GemmParams& p, dim3 grid, cudaStream_t s) {
+  const size_t smem = 1024 + kStages * kStageBytes + sizeof(GemmBars);
+  cudaError_t e = cudaFuncSetAttribute(sa_gemm_kernel<EPI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  sa_gemm_kernel<EPI><<<grid, kGemmThreads, smem, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
+  GemmParams p = {};
+  for (int ph = 0; ph < g.phases; ++ph) {
+    if (!make_operand_map(&p.ta[ph], g.a[ph]) || !make_operand_map(&p.tb[ph], g.b[ph]))
+      return cudaErrorInvalidValue;
+    p.a_mn[ph] = g.a[ph].mn_major ? 1 : 0;
+    p.b_mn[ph] = g.b[ph].mn_major ? 1 : 0;
+    p.k_tiles[ph] = g.k_tiles[ph];
+    p.b_user_rows[ph] = g.b_user_rows[ph];
+  }
+  if (g.phases == 1) {
+    p.ta[1] = p.ta[0];
+    p.tb[1] = p.tb[0];
+  }
+  p.phases = g.phases;
+  p.user_mode = g.user_mode;
+  p.M = g.M;
+  p.N = g.N;
+  p.splits = g.splits < 1 ? 1 : g.splits;
+  p.hdr = g.hdr;
+  p.tile_start = g.tile_start;
+  p.offsets = g.offsets;
+  p.R = g.R;
+  p.out_f32 = g.out_f32;
+  p.ld_out = g.ld_out;
+  p.split_stride = g.split_stride;
+  p.out_bf16 = g.out_bf16;
+  p.lse2 = g.lse2;
+  p.lse_scale = g.lse_scale;
+  p.k_valid = g.k_valid;
+  p.a_in = g.a_in;
+  p.ld_a_in = g.ld_a_in;
+  p.c_user = g.c_user;
+  p.k_pad = g.k_pad;
+  p.dpart = g.dpart;
+  p.dpart_ld = g.dpart_ld;
+  p.budget = kDefaultWaitBudget;
+  const dim3 grid((unsigned)g.m_tiles_bound, (unsigned)((g.N + kBN - 1) / kBN), (unsigned)p.splits);
+  if (grid.x == 0) return cudaSuccess;
+  switch (g.epi) {
+    case kEpiStoreF32: return launch_t<kEpiStoreF32>(p, grid, s);
+    case kEpiAExp: return launch_t<kEpiAExp>(p, grid, s);
+    case kEpiQ: return launch_t<kEpiQ>(p, grid, s);
+    case kEpiLse: return launch_t<kEpiLse>(p, grid, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace sa

@@ -69,6 +69,10 @@ struct Plan {
   int C = 0, k_pad = 0, G = 0, Gb = 0;
   size_t hdr = 0, ts = 0, pf = 0, pu = 0, pm = 0, lse2 = 0;
   size_t pn = 0, gt = 0, gh = 0, cj = 0, lseb = 0, db = 0, dppp = 0, dpp = 0, wvp = 0;
+  // tensor-core backward (bf16)
+  bool btc = false;
+  int splits = 0;
+  size_t ghb = 0, pn2 = 0, pnn = 0, ab = 0, qb = 0, dsb = 0, dpart = 0, lse2b = 0;
   size_t total = 0;
 };
 
@@ -110,6 +114,26 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
     q.pu = take(segs * q.k_pad * d * sizeof(float));
     q.pm = take(segs * q.k_pad * sizeof(float));
     if (!q.tc) q.lse2 = take((size_t)n_total * sizeof(float));
+  } else if (dt == SA_BF16) {
+    // tensor-core backward: token x prototype intermediates in the workspace
+    q.btc = true;
+    q.k_pad = (k + 127) / 128 * 128;
+    q.splits = bwd_tc_splits(dev.sms, q.k_pad, d, n_total);
+    q.Gb = q.splits;
+    const size_t nk = (size_t)n_total * q.k_pad;
+    q.gt = take((size_t)R * q.k_pad * d * sizeof(float));
+    q.ghb = take((size_t)R * q.k_pad * d * 2);
+    q.cj = take((size_t)R * q.k_pad * sizeof(float));
+    q.pn2 = take((size_t)q.k_pad * d * 2);
+    q.pnn = take((size_t)q.k_pad * d * 2);
+    q.ab = take(nk * 2);
+    q.qb = take(nk * sizeof(float));
+    q.dsb = take(nk * 2);
+    q.dpart = take((size_t)n_total * (q.k_pad / 128) * sizeof(float));
+    q.lse2b = take((size_t)n_total * sizeof(float));
+    q.dppp = take((size_t)q.splits * q.k_pad * d * sizeof(float));
+    q.dpp = take((size_t)q.k_pad * d * sizeof(float));
+    q.wvp = take(bwd_wv_chunks(R, k) * d * d * sizeof(float));
   } else {
     q.Gb = q.G;
     q.pn = take((size_t)q.k_pad * d * sizeof(float));
@@ -129,24 +153,10 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda needed).
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
-  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void* p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
-  });
-  return fn;
-}
-
 // Row-major [rows, d] bf16 matrix, boxes of 128 rows x `box_cols` columns; the swizzle
 // width equals the box row (64 columns: 128B swizzle, 16 columns: 32B swizzle).
 bool make_tmap_bf16(CUtensorMap* m, const void* base, uint64_t rows, int d, int box_cols) {
-  auto fn = encode_fn();
+  auto fn = tmap_encode_fn();
   if (!fn) return false;
   const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
   const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
@@ -179,6 +189,22 @@ sa_status cuda_status(cudaError_t e) {
 }
 
 }  // namespace
+}  // namespace sa
+
+namespace sa {
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda needed).
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
 }  // namespace sa
 
 using namespace sa;
@@ -293,7 +319,6 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
                        const float* xsketch, const float* dsketch, const float* dmass, float* dX,
                        float* dP, float* dWk, float* dWv, void* workspace, size_t ws_bytes,
                        void* stream_) {
-  (void)lse;  // per-token statistics are recomputed in fp32
   sa_status st = check_sizes(R, n_total, k, d, dt);
   if (st != SA_OK) return st;
   if (!offsets || !P || !Wk || !Wv || !dP || !dWk || !dWv ||
@@ -302,7 +327,8 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
     return SA_ERR_INVALID_ARG;
   if (!aligned16(X) || !aligned16(P) || !aligned16(Wk) || !aligned16(Wv) || !aligned16(sketch) ||
       !aligned16(mass) || !aligned16(xsketch) || !aligned16(dsketch) || !aligned16(dmass) ||
-      !aligned16(dX) || !aligned16(dP) || !aligned16(dWk) || !aligned16(dWv) || !aligned16(offsets))
+      !aligned16(dX) || !aligned16(dP) || !aligned16(dWk) || !aligned16(dWv) || !aligned16(offsets) ||
+      !aligned16(lse))
     return SA_ERR_INVALID_ARG;
   Device dev;
   if ((st = current_device(&dev)) != SA_OK) return st;
@@ -314,10 +340,11 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
   WsHeader* hdr = at<WsHeader>(workspace, p.hdr);
   long long* ts = at<long long>(workspace, p.ts);
   if ((st = cuda_status(launch_schedule(offsets, R, n_total, hdr, ts, s))) != SA_OK) return st;
-  if ((st = cuda_status(launch_fold(P, Wk, dt, k, p.k_pad, d, 1.0f / std::sqrt((float)d),
+  if (!p.btc &&
+      (st = cuda_status(launch_fold(P, Wk, dt, k, p.k_pad, d, 1.0f / std::sqrt((float)d),
                                     at<void>(workspace, p.pn), false, s))) != SA_OK)
     return st;
-  BwdArgs a;
+  BwdArgs a = {};
   a.X = X;
   a.dt = dt;
   a.offsets = offsets;
@@ -350,7 +377,25 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
   a.dP = dP;
   a.dWk = dWk;
   a.dWv = dWv;
-  return cuda_status(launch_bwd_simt(a, s));
+  if (!p.btc) return cuda_status(launch_bwd_simt(a, s));
+  // bf16: tensor-core backward (the SIMT-only buffers are unused)
+  a.Pn = nullptr;
+  a.Gh = nullptr;
+  a.Ghb = at<__nv_bfloat16>(workspace, p.ghb);
+  a.lseb = nullptr;
+  a.Db = nullptr;
+  BwdTcArgs t;
+  t.b = a;
+  t.lse = lse;
+  t.pn2 = at<__nv_bfloat16>(workspace, p.pn2);
+  t.pnn = at<__nv_bfloat16>(workspace, p.pnn);
+  t.A = at<__nv_bfloat16>(workspace, p.ab);
+  t.Q = at<float>(workspace, p.qb);
+  t.dS = at<__nv_bfloat16>(workspace, p.dsb);
+  t.dpart = at<float>(workspace, p.dpart);
+  t.lse2 = at<float>(workspace, p.lse2b);
+  t.splits = p.splits;
+  return cuda_status(launch_bwd_tc(t, s));
 }
 
 int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int d, const void* Wv,

@@ -5,6 +5,8 @@
 #include <cstdint>
 #include <cuda.h>
 #include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <cudaTypedefs.h>
 
 #include "sa_sketch.h"
 
@@ -93,7 +95,8 @@ struct BwdArgs {
   // workspace
   float* Pn;      // [k_pad, d]  P W_k^T / sqrt(d)
   float* Gt;      // [R, k_pad, d]  G / mass
-  float* Gh;      // [R, k_pad, d]  (G / mass) W_v^T
+  float* Gh;      // [R, k_pad, d]  (G / mass) W_v^T (nullable)
+  __nv_bfloat16* Ghb;  // the same in bf16 (nullable; the tensor-core backward)
   float* cj;      // [R, k_pad]     (G / mass) . sketch - dmass
   float* lseb;    // [n_total]      fp32 per-token log-sum-exp (natural)
   float* Db;      // [n_total]      sum_j A_jt dA_jt
@@ -108,6 +111,64 @@ struct BwdArgs {
 };
 size_t bwd_wv_chunks(int R, int k);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t s);
+cudaError_t launch_bwd_prep(const BwdArgs& a, cudaStream_t s);  // Gt, Gh, c per user
+cudaError_t launch_bwd_tail(const BwdArgs& a, cudaStream_t s);  // dPn reduce, dW_v, dP, dW_k
+
+// ---- tensor-core backward (bf16 inputs; sa_bwd_tc.cu)
+struct BwdTcArgs {
+  BwdArgs b;                 // shared inputs, outputs and SIMT-stage workspace
+  const float* lse;          // forward's lse (natural log); null: recomputed here
+  __nv_bfloat16* pn2;        // [k_pad, d] P W_k^T log2(e)/sqrt(d)
+  __nv_bfloat16* pnn;        // [k_pad, d] P W_k^T / sqrt(d)
+  __nv_bfloat16* A;          // [n_total, k_pad]
+  float* Q;                  // [n_total, k_pad]
+  __nv_bfloat16* dS;         // [n_total, k_pad]
+  float* dpart;              // [n_total, k_pad / 128]
+  float* lse2;               // [n_total] (when lse is null)
+  int splits;                // split-K of dPn (== b.G)
+};
+cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s);
+int bwd_tc_splits(int sms, int k_pad, int d, long long n_total);
+
+// ---- tensor-core GEMM (backward building block, sa_gemm_sm100.cu)
+enum GemmEpi { kEpiStoreF32 = 0, kEpiAExp = 1, kEpiQ = 2, kEpiLse = 3 };
+struct GemmOperandDesc {  // one bf16 operand, row-major in memory
+  const void* base;
+  uint64_t rows, cols;
+  bool mn_major;  // false: rows = M (or N), cols = K; true: rows = K, cols = M (or N)
+};
+struct GemmArgs {
+  GemmOperandDesc a[2], b[2];  // operand pairs, accumulated into one result
+  int phases;                  // 1 or 2
+  int k_tiles[2];              // 64-wide K tiles of each pair
+  int b_user_rows[2];          // user tiles: B's row offset per user (0: shared B)
+  int user_mode;               // 0: plain 128-row tiles of M; 1: one user per tile
+  int M, N;                    // rows (plain mode) and output columns
+  int m_tiles_bound;           // grid x (user mode: an upper bound; extra CTAs exit)
+  int splits;                  // split-K over pair 0's K tiles (grid z)
+  int epi;
+  const WsHeader* hdr;         // status word (and the tile count in user mode)
+  const long long* tile_start;
+  const int64_t* offsets;
+  int R;
+  float* out_f32;
+  long long ld_out;
+  long long split_stride;
+  __nv_bfloat16* out_bf16;
+  const float* lse2;
+  float lse_scale;             // kEpiAExp: lse2 = lse_scale * lse2[row]
+  int k_valid;                 // kEpiAExp / kEpiLse: columns n >= k_valid are padding
+  const __nv_bfloat16* a_in;
+  long long ld_a_in;
+  const float* c_user;
+  int k_pad;
+  float* dpart;
+  int dpart_ld;
+};
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable)
+PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();
 
 // ---- failure-detection test hook
 cudaError_t launch_debug_wait_timeout(WsHeader* hdr, long long budget, cudaStream_t s);
