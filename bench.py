@@ -329,6 +329,33 @@ def run_ours(args) -> None:
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
 
+    # ---- the backward on the same batch (bf16 tensor-core path), reported alongside
+    bwd = None
+    if not args.no_backward and world == 1:
+        gen = torch.Generator().manual_seed(4242)
+        G = torch.randn(R, k, d, generator=gen).to(dev)
+        bout = binding.backward(X, off, P, Wk, Wv, out, G)
+        bws = bout["_ws"]
+        for _ in range(2):
+            binding.backward(X, off, P, Wk, Wv, out, G, ws=bws)
+        torch.cuda.synchronize()
+        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nb = 5
+        b0.record(stream)
+        for _ in range(nb):
+            binding.backward(X, off, P, Wk, Wv, out, G, ws=bws)
+        b1.record(stream)
+        torch.cuda.synchronize()
+        st = binding.device_status(bws)
+        if st != 0:
+            raise SystemExit(f"backward failed on device: {binding.sa_status_string(st)}")
+        bwd_ms = b0.elapsed_time(b1) / nb
+        del bws, bout
+        bwd = {"ms": bwd_ms, "tokens_per_s": n_total / (bwd_ms / 1e3),
+               "tflops_algorithmic": 10.0 * k * d * n_total / (bwd_ms / 1e3) / 1e12,
+               "note": "sa_sketch_backward on the same batch, dL/dsketch ~ N(0,1); "
+                       "10kd FLOP per token"}
+
     # ---- max over ranks
     t = torch.tensor([elapsed_ms, e2e_ms, kern_ms, float(n_total)], dtype=torch.float64, device=dev)
     if world > 1:
@@ -381,6 +408,8 @@ def run_ours(args) -> None:
     }
     if cpu is not None:
         line["cpu_baseline"] = cpu
+    if bwd is not None and world == 1:
+        line["backward"] = bwd
     print(json.dumps(line), flush=True)
 
 
@@ -391,6 +420,7 @@ def main(argv=None) -> int:
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:

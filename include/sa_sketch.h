@@ -110,14 +110,19 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
  *
  *   X, offsets, P, Wk, Wv, dt   as passed to the forward
  *   sketch, mass, xsketch       fp32 outputs of that forward (required)
- *   lse                         the forward's lse; nullable and not read: this
- *                               implementation recomputes the per-token statistics
- *                               it needs in fp32
+ *   lse                         the forward's lse for the same inputs, nullable. The
+ *                               bf16 path uses it when given (else it recomputes it, one
+ *                               more k x n x d contraction); the fp32 path recomputes
+ *                               the per-token statistics and does not read it
  *   dsketch [R, k, d] fp32      G
  *   dmass   [R, k]    fp32      Gm; nullable (NULL means zero)
  * Outputs (fp32, overwritten, not accumulated into):
  *   dX  [n_total, d]
  *   dP  [k, d], dWk [d, d], dWv [d, d]   summed over all users
+ * bf16 inputs run on the tensor cores: the token x prototype intermediates (the softmax
+ * A, A * dA and its gradient dS; 8 bytes per token and prototype) live in the workspace,
+ * which sa_sketch_workspace_size(..., backward = 1) sizes accordingly (about 14 GB at
+ * 1.8 M tokens and k = 1024). fp32 inputs run on CUDA cores with a small workspace.
  */
 int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
                        const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,

@@ -4,7 +4,7 @@ import pytest
 import torch
 
 import oracle
-from parity_util import check_grads, gpu_forward, nthreads
+from parity_util import check_grads, gpu_forward, nthreads, rel_l2
 from prototype_sketch_attention_b200 import binding, inputs
 
 pytestmark = pytest.mark.gpu
@@ -56,3 +56,34 @@ def test_config5_full_size_one_user_gradient():
     rest = np.concatenate([got["dX"][:off[u]], got["dX"][off[u + 1]:]])
     assert not rest.any()
     check_grads({"dX": dX_u, "dP": got["dP"], "dWk": got["dWk"], "dWv": got["dWv"]}, ref, fp32=False)
+
+
+@pytest.mark.parametrize("lengths,k,d", [([300, 0, 1037], 256, 128), ([129, 5], 384, 64)])
+def test_backward_recomputes_lse_when_not_given(lengths, k, d):
+    """The bf16 backward uses the forward's lse when passed and otherwise recomputes it
+    (its own log-sum-exp pass). Both must match the oracle, and each other closely."""
+    w = inputs.make_workload(lengths, d, k, "bf16", seed=31 + k, with_grad=True)
+    g, fwd = gpu_forward(w)
+    G = w.G.numpy().astype(np.float64)
+    with_lse = _run(w, g, fwd, G)
+    no_lse = {key: v for key, v in fwd.items() if key != "lse"}
+    without = _run(w, g, no_lse, G)
+    sub = w.to_f64()
+    ref = oracle.backward(sub["X"], sub["offsets"], sub["P"], sub["Wk"], sub["Wv"], G,
+                          nthreads=nthreads())
+    check_grads(with_lse, ref, fp32=False)
+    check_grads(without, ref, fp32=False)
+    for key in ("dX", "dP", "dWk", "dWv"):
+        assert rel_l2(without[key], with_lse[key]) <= 2e-3, key
+
+
+def test_backward_bf16_k_not_multiple_of_128():
+    """k = 200: the last 128-prototype tile is partly padding, which every epilogue masks."""
+    w = inputs.make_workload([700, 260], 128, 200, "bf16", seed=77, with_grad=True)
+    g, fwd = gpu_forward(w)
+    G = w.G.numpy().astype(np.float64)
+    got = _run(w, g, fwd, G)
+    sub = w.to_f64()
+    ref = oracle.backward(sub["X"], sub["offsets"], sub["P"], sub["Wk"], sub["Wv"], G,
+                          nthreads=nthreads())
+    check_grads(got, ref, fp32=False)
