@@ -120,8 +120,8 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
  *   dX  [n_total, d]
  *   dP  [k, d], dWk [d, d], dWv [d, d]   summed over all users
  * bf16 inputs run on the tensor cores: the token x prototype intermediates (the softmax
- * A, A * dA and its gradient dS; 8 bytes per token and prototype) live in the workspace,
- * which sa_sketch_workspace_size(..., backward = 1) sizes accordingly (about 14 GB at
+ * A and its gradient dS, bf16: 4 bytes per token and prototype) live in the workspace,
+ * which sa_sketch_workspace_size(..., backward = 1) sizes accordingly (about 8 GB at
  * 1.8 M tokens and k = 1024). fp32 inputs run on CUDA cores with a small workspace.
  */
 int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,

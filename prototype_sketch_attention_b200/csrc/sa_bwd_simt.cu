@@ -49,6 +49,7 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a, const TIn* __r
     }
     gt[i] = v;
     a.Gt[((size_t)u * a.k_pad + j) * d + e] = v;
+    if (a.Gtb) a.Gtb[((size_t)u * a.k_pad + j) * d + e] = __float2bfloat16_rn(v);
   }
   __syncthreads();
   for (int i = threadIdx.x; i < kCP * d; i += blockDim.x) {
@@ -399,15 +400,16 @@ static cudaError_t launch_prep(const BwdArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
-// dPn = sum of a.G partials (fixed order), dW_v chunks, then dW_v, dP, dW_k.
+// dPn = sum of a.G partials (fixed order), dW_v chunks (unless wv_parts partials are
+// already in a.wv_part), then dW_v, dP, dW_k.
 template <typename TIn>
-static cudaError_t launch_tail(const BwdArgs& a, cudaStream_t s) {
+static cudaError_t launch_tail(const BwdArgs& a, int wv_parts, cudaStream_t s) {
   cudaError_t e;
   const int d = a.d;
   bwd_reduce_dpp_kernel<<<256, 256, 0, s>>>(a);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  const int nch = (int)bwd_wv_chunks(a.R, a.k);
-  if (nch > 0) {
+  const int nch = wv_parts > 0 ? wv_parts : (int)bwd_wv_chunks(a.R, a.k);
+  if (wv_parts == 0 && nch > 0) {
     const size_t smem_w = (size_t)(64 * d) * sizeof(float);
     bwd_wv_part_kernel<<<(unsigned)nch, 256, smem_w, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -421,8 +423,9 @@ cudaError_t launch_bwd_prep(const BwdArgs& a, cudaStream_t s) {
   return a.dt == SA_BF16 ? launch_prep<__nv_bfloat16>(a, s) : launch_prep<float>(a, s);
 }
 
-cudaError_t launch_bwd_tail(const BwdArgs& a, cudaStream_t s) {
-  return a.dt == SA_BF16 ? launch_tail<__nv_bfloat16>(a, s) : launch_tail<float>(a, s);
+cudaError_t launch_bwd_tail(const BwdArgs& a, int wv_parts, cudaStream_t s) {
+  return a.dt == SA_BF16 ? launch_tail<__nv_bfloat16>(a, wv_parts, s)
+                         : launch_tail<float>(a, wv_parts, s);
 }
 
 template <typename TIn>
@@ -448,7 +451,7 @@ static cudaError_t launch_all(const BwdArgs& a, cudaStream_t s) {
     bwd_proto_kernel<TIn><<<dim3((unsigned)a.G, (unsigned)(a.k_pad / kCP)), 256, smem_p, s>>>(a, X);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  return launch_tail<TIn>(a, s);
+  return launch_tail<TIn>(a, 0, s);
 }
 
 }  // namespace sa

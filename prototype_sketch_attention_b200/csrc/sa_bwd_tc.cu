@@ -10,17 +10,20 @@
 // then dP = dPn W_k / sqrt(d), dW_k = dPn^T P / sqrt(d), dW_v = sum_u U_u^T Gt_u.
 //
 // Every contraction over d, k or the tokens runs as a tensor-core GEMM
-// (sa_gemm_sm100.cu) with the elementwise work fused into its epilogue; the token x
-// prototype intermediates (A, Q = A (dA) and dS) live in the workspace:
-//   prep (CUDA cores)   Gt, bf16 Gh, c per user
+// (sa_gemm_sm100.cu) with the elementwise work fused into its epilogue. D_t uses
+// sum_j A_jt dA_jt = X_t . Y_t - sum_j A_jt c_j with Y = A Gh (which dX needs anyway), so
+// dS comes straight out of one GEMM epilogue and no fp32 token x prototype matrix exists:
+//   prep (CUDA cores)   Gt (fp32, bf16), bf16 Gh, c per user; bf16 U
 //   fold                pn2 = bf16(Pn log2 e), pnn = bf16(Pn)
 //   [lse not given]     GEMM S2 = X pn2^T -> per-tile log2-sum-exp -> lse2 per token
-//   GEMM (plain tiles)  A = 2^(X pn2^T - lse2)                          bf16 [n, k_pad]
-//   GEMM (user tiles)   Q = A (X Gh_u^T - c_u), per-tile row sums of Q   fp32 [n, k_pad]
-//   CUDA cores          D_t = sum of the row sums, dS = Q - A D_t        bf16 [n, k_pad]
-//   GEMM (user tiles)   dX = dS pnn + A Gh_u  (two operand pairs, one accumulator)
+//   GEMM (user tiles)   A = 2^(X pn2^T - lse2) (bf16) and per-tile sums of A c_u
+//   GEMM (user tiles)   Y = A Gh_u                                     fp32 [n, d]
+//   CUDA cores          D_t = X_t . Y_t - sum_j A_jt c_j
+//   GEMM (user tiles)   dS = A (X Gh_u^T - c_u - D_t)                  bf16 [n, k_pad]
+//   GEMM (user tiles)   dX = dS pnn + Y
 //   GEMM (split-K)      partials of dPn = dS^T X over token ranges
-//   tail (CUDA cores)   dPn = sum of partials (fixed order), dW_v, dP, dW_k
+//   GEMM (split-K)      partials of dW_v = U^T Gt over (user, prototype) rows
+//   tail (CUDA cores)   sums of the partials (fixed order), dP, dW_k
 // 10 k d FLOP per token on the tensor cores (12 when the lse is recomputed).
 #include <cmath>
 
@@ -32,40 +35,42 @@ namespace {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
-// D_t = sum of the row's per-tile partial sums of Q; dS = Q - A D_t (bf16).
-// One warp per token row, 8 columns per lane and step.
-__global__ void __launch_bounds__(256) bwd_ds_kernel(const float* __restrict__ Q,
-                                                     const __nv_bfloat16* __restrict__ A,
-                                                     const float* __restrict__ dpart, int ntiles,
-                                                     int k_pad, long long n_total,
-                                                     __nv_bfloat16* __restrict__ dS,
-                                                     const WsHeader* hdr) {
+// D_t = X_t . Y_t - sum of the row's per-tile partials of sum_j A_jt c_j.
+// One warp per token row.
+__global__ void __launch_bounds__(256) bwd_d_kernel(const __nv_bfloat16* __restrict__ X,
+                                                    const float* __restrict__ Y, int d,
+                                                    const float* __restrict__ cpart, int ntiles,
+                                                    long long n_total, float* __restrict__ D,
+                                                    const WsHeader* hdr) {
   if (read_status(&hdr->status) != 0) return;
   const int lane = threadIdx.x & 31;
   const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
   const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
   for (long long t = w0; t < n_total; t += nw) {
-    float D = 0.f;
-    for (int i = lane; i < ntiles; i += 32) D += dpart[t * ntiles + i];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) D += __shfl_xor_sync(0xffffffffu, D, o);
-    const float* q = Q + t * k_pad;
-    const __nv_bfloat16* a = A + t * k_pad;
-    __nv_bfloat16* o = dS + t * k_pad;
-    for (int c = lane * 8; c < k_pad; c += 256) {
-      const float4 q0 = *reinterpret_cast<const float4*>(q + c);
-      const float4 q1 = *reinterpret_cast<const float4*>(q + c + 4);
-      const uint4 av = *reinterpret_cast<const uint4*>(a + c);
-      const float qv[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-      const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-      uint32_t w[4];
-#pragma unroll
-      for (int h = 0; h < 4; ++h) {
-        const float a0 = __uint_as_float(aw[h] << 16), a1 = __uint_as_float(aw[h] & 0xFFFF0000u);
-        w[h] = cvt_bf16x2(fmaf(-a0, D, qv[2 * h]), fmaf(-a1, D, qv[2 * h + 1]));
-      }
-      *reinterpret_cast<uint4*>(o + c) = make_uint4(w[0], w[1], w[2], w[3]);
+    float acc = 0.f;
+    for (int c = lane * 4; c < d; c += 128) {
+      const float4 y = *reinterpret_cast<const float4*>(Y + t * d + c);
+      const uint2 xv = *reinterpret_cast<const uint2*>(X + t * d + c);
+      acc = fmaf(__uint_as_float(xv.x << 16), y.x, acc);
+      acc = fmaf(__uint_as_float(xv.x & 0xFFFF0000u), y.y, acc);
+      acc = fmaf(__uint_as_float(xv.y << 16), y.z, acc);
+      acc = fmaf(__uint_as_float(xv.y & 0xFFFF0000u), y.w, acc);
     }
+    for (int i = lane; i < ntiles; i += 32) acc -= cpart[t * ntiles + i];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) D[t] = acc;
+  }
+}
+
+// U (the forward's xsketch, fp32 [R, k, d]) as bf16 [R, k_pad, d] with zero padding rows.
+__global__ void bwd_u_bf16_kernel(const float* __restrict__ U, int R, int k, int k_pad, int d,
+                                  __nv_bfloat16* __restrict__ Ub) {
+  const long long n = (long long)R * k_pad * d;
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n;
+       i += (long long)gridDim.x * blockDim.x) {
+    const long long e = i % d, rj = i / d, j = rj % k_pad, u = rj / k_pad;
+    Ub[i] = __float2bfloat16_rn(j < k ? U[(u * k + j) * d + e] : 0.f);
   }
 }
 
@@ -105,28 +110,63 @@ int bwd_tc_splits(int sms, int k_pad, int d, long long n_total) {
   return (int)s;
 }
 
+// Split-K count of the dW_v GEMM (one 128 x 128 output tile): about two CTAs per SM.
+int bwd_tc_wv_splits(int sms, int R, int k_pad) {
+  const long long kt = ((long long)R * k_pad + 63) / 64;
+  long long s = 2LL * sms;
+  if (s > kt) s = kt;
+  if (s < 1) s = 1;
+  return (int)s;
+}
+
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
   const BwdArgs& b = a.b;
   cudaError_t e;
   const int d = b.d, k = b.k, k_pad = b.k_pad, R = b.R;
   const long long n = b.n_total;
   const int ntiles = k_pad / 128;
+  const int nparts = 2 * ntiles;  // per-row partials: two column halves per tile
   if ((e = launch_bwd_prep(b, s)) != cudaSuccess) return e;
   const float isd = 1.0f / std::sqrt((float)d);
   if ((e = launch_fold(b.P, b.Wk, SA_BF16, k, k_pad, d, kLog2e * isd, a.pn2, true, s)) != cudaSuccess)
     return e;
   if ((e = launch_fold(b.P, b.Wk, SA_BF16, k, k_pad, d, isd, a.pnn, true, s)) != cudaSuccess)
     return e;
+  if (R > 0) {  // dW_v = sum over (user, prototype) rows of U^T Gt, split-K
+    bwd_u_bf16_kernel<<<1024, 256, 0, s>>>(b.xsketch, R, k, k_pad, d, a.Ub);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    GemmArgs t = {};
+    t.hdr = b.hdr;
+    t.phases = 1;
+    t.a[0] = op(a.Ub, (uint64_t)R * k_pad, (uint64_t)d, true);
+    t.b[0] = op(b.Gtb, (uint64_t)R * k_pad, (uint64_t)d, true);
+    t.k_tiles[0] = (int)(((long long)R * k_pad + 63) / 64);
+    t.user_mode = 0;
+    t.M = d;
+    t.N = d;
+    t.m_tiles_bound = 1;
+    t.splits = a.wv_splits;
+    t.epi = kEpiStoreF32;
+    t.out_f32 = b.wv_part;
+    t.ld_out = d;
+    t.split_stride = (long long)d * d;
+    if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
+  } else {
+    e = cudaMemsetAsync(b.wv_part, 0, (size_t)d * d * sizeof(float), s);
+    if (e != cudaSuccess) return e;
+  }
+  const int wv_parts = R > 0 ? a.wv_splits : 1;
   if (n == 0) {
     e = cudaMemsetAsync(b.dpp_part, 0, (size_t)a.splits * k_pad * d * sizeof(float), s);
     if (e != cudaSuccess) return e;
-    return launch_bwd_tail(b, s);
+    return launch_bwd_tail(b, wv_parts, s);
   }
   const int m_plain = (int)((n + 127) / 128);
   const int m_user = (int)(n / 128 + R + 1);
   const GemmOperandDesc X_k = op(b.X, (uint64_t)n, (uint64_t)d, false);       // [n][d], K = d
   const GemmOperandDesc pn2_k = op(a.pn2, (uint64_t)k_pad, (uint64_t)d, false);
   const GemmOperandDesc gh_k = op(b.Ghb, (uint64_t)R * k_pad, (uint64_t)d, false);
+  const GemmOperandDesc gh_mn = op(b.Ghb, (uint64_t)R * k_pad, (uint64_t)d, true);
 
   GemmArgs g = {};
   g.hdr = b.hdr;
@@ -152,31 +192,51 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
     l.m_tiles_bound = m_plain;
     l.epi = kEpiLse;
     l.dpart = a.dpart;
-    l.dpart_ld = ntiles;
+    l.dpart_ld = nparts;
     if ((e = launch_gemm(l, s)) != cudaSuccess) return e;
-    bwd_lse_kernel<<<1024, 256, 0, s>>>(a.dpart, ntiles, n, a.lse2, b.hdr);
+    bwd_lse_kernel<<<1024, 256, 0, s>>>(a.dpart, nparts, n, a.lse2, b.hdr);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     lse_src = a.lse2;
     lse_scale = 1.f;
   }
-  {  // A = 2^(X pn2^T - lse2)
+  {  // A = 2^(X pn2^T - lse2), and per-tile sums of A c_u
     GemmArgs t = g;
     t.phases = 1;
     t.a[0] = X_k;
     t.b[0] = pn2_k;
     t.k_tiles[0] = (d + 63) / 64;
-    t.user_mode = 0;
-    t.M = (int)n;
+    t.user_mode = 1;
     t.N = k_pad;
-    t.m_tiles_bound = m_plain;
+    t.m_tiles_bound = m_user;
     t.epi = kEpiAExp;
     t.out_bf16 = a.A;
     t.ld_out = k_pad;
     t.lse2 = lse_src;
     t.lse_scale = lse_scale;
+    t.c_user = b.cj;
+    t.dpart = a.dpart;
+    t.dpart_ld = nparts;
     if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
   }
-  {  // Q = A (X Gh_u^T - c_u) and its per-tile row sums
+  {  // Y = A Gh_u
+    GemmArgs t = g;
+    t.phases = 1;
+    t.a[0] = op(a.A, (uint64_t)n, (uint64_t)k_pad, false);
+    t.b[0] = gh_mn;
+    t.b_user_rows[0] = k_pad;
+    t.k_tiles[0] = k_pad / 64;
+    t.user_mode = 1;
+    t.N = d;
+    t.m_tiles_bound = m_user;
+    t.epi = kEpiStoreF32;
+    t.out_f32 = a.Y;
+    t.ld_out = d;
+    if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
+  }
+  bwd_d_kernel<<<2048, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(b.X), a.Y, d, a.dpart, nparts,
+                                    n, a.D, b.hdr);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  {  // dS = A (X Gh_u^T - c_u - D)
     GemmArgs t = g;
     t.phases = 1;
     t.a[0] = X_k;
@@ -186,33 +246,29 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
     t.user_mode = 1;
     t.N = k_pad;
     t.m_tiles_bound = m_user;
-    t.epi = kEpiQ;
-    t.out_f32 = a.Q;
+    t.epi = kEpiDS;
+    t.out_bf16 = a.dS;
     t.ld_out = k_pad;
     t.a_in = a.A;
     t.ld_a_in = k_pad;
     t.c_user = b.cj;
-    t.dpart = a.dpart;
-    t.dpart_ld = ntiles;
+    t.drow = a.D;
     if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
   }
-  bwd_ds_kernel<<<2048, 256, 0, s>>>(a.Q, a.A, a.dpart, ntiles, k_pad, n, a.dS, b.hdr);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  {  // dX = dS pnn + A Gh_u
+  {  // dX = dS pnn + Y
     GemmArgs t = g;
-    t.phases = 2;
+    t.phases = 1;
     t.a[0] = op(a.dS, (uint64_t)n, (uint64_t)k_pad, false);
     t.b[0] = op(a.pnn, (uint64_t)k_pad, (uint64_t)d, true);
-    t.a[1] = op(a.A, (uint64_t)n, (uint64_t)k_pad, false);
-    t.b[1] = op(b.Ghb, (uint64_t)R * k_pad, (uint64_t)d, true);
-    t.b_user_rows[1] = k_pad;
-    t.k_tiles[0] = t.k_tiles[1] = k_pad / 64;
+    t.k_tiles[0] = k_pad / 64;
     t.user_mode = 1;
     t.N = d;
     t.m_tiles_bound = m_user;
     t.epi = kEpiStoreF32;
     t.out_f32 = b.dX;
     t.ld_out = d;
+    t.add_in = a.Y;
+    t.ld_add = d;
     if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
   }
   {  // dPn partials = dS^T X, split over token ranges
@@ -232,7 +288,7 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
     t.split_stride = (long long)k_pad * d;
     if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
   }
-  return launch_bwd_tail(b, s);
+  return launch_bwd_tail(b, wv_parts, s);
 }
 
 }  // namespace sa

@@ -13,12 +13,14 @@
 // operand that depends on the user (B_p with a per-user row offset) is well defined.
 //
 // Epilogues:
-//   kEpiStoreF32  out[row][n] = acc (fp32), or a split-K partial at split * split_stride
-//   kEpiAExp      out_bf16[row][n] = bf16(2^(acc - lse_scale * lse[row])) (A = softmax),
-//                 0 for columns n >= k_valid
-//   kEpiLse       dpart[row][tile] = log2 sum over the tile's columns n < k_valid of 2^acc
-//   kEpiQ         q = A[row][n] (acc - c[user][n]); out[row][n] = q (fp32) and the
-//                 row sum of q over the tile's 128 columns into dpart[row][tile]
+//   kEpiStoreF32  out[row][n] = acc (+ add_in[row][n]) in fp32, or a split-K partial at
+//                 split * split_stride
+//   kEpiAExp      a = bf16(2^(acc - lse_scale * lse[row])), 0 for columns n >= k_valid;
+//                 out_bf16[row][n] = a and, with c given, dpart[row][2 tile + h] = the
+//                 row sum of a * c[user][n] over half h (64 columns) of the tile
+//   kEpiLse       dpart[row][2 tile + h] = log2 sum of 2^acc over half h of the tile
+//                 (columns n < k_valid)
+//   kEpiDS        out_bf16[row][n] = bf16(A[row][n] (acc - c[user][n] - drow[row]))
 // Waits on mbarriers are bounded like every other kernel of the library.
 #include <cuda.h>
 
@@ -31,7 +33,7 @@ namespace {
 constexpr int kBM = 128, kBN = 128, kBK = 64;
 constexpr int kStages = 3;
 constexpr int kStageBytes = (kBM + kBN) * kBK * 2;  // 32 KB
-constexpr int kGemmThreads = 192;                   // producer, MMA, 4 epilogue warps
+constexpr int kGemmThreads = 320;                   // producer, MMA, 8 epilogue warps
 
 struct GemmParams {
   CUtensorMap ta[2], tb[2];
@@ -59,6 +61,9 @@ struct GemmParams {
   int k_pad;
   float* dpart;
   int dpart_ld;
+  const float* add_in;
+  long long ld_add;
+  const float* drow;
   long long budget;
 };
 
@@ -186,87 +191,148 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
       mbar_wait_drain(smem_u32(&bars->done), 0, p.budget);
     }
   } else {
-    // ================= epilogue: thread = output row (TMEM lane)
+    // ================= epilogue: thread = output row (TMEM lane), in 32-column chunks.
+    // Global traffic goes through a per-warp staging block in the (now idle) pipeline
+    // shared memory, so every load and store below is a full, coalesced row segment.
+    // Two warps per TMEM lane quadrant: epilogue warp e (0..7) takes rows of quadrant
+    // e & 3 and the column half e >> 2 of the tile.
     const int q = warp & 3;
+    const int half = (warp - 2) >> 2;
     const int r = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
+    float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33 + 64);  // [32][33]
+    float* cst = stg + 32 * 33;  // this warp's 64 values of c[user][n]
     const bool have = total_kt > 0 &&
                       mbar_wait_warp(smem_u32(&bars->done), 0, status, p.budget);
     if (have) {
       tc_fence_after();
       const bool valid = r < nrows;
       const long long row = (long long)row0 + r;
-      float lse2 = 0.f;
-      if (EPI == kEpiAExp && valid) lse2 = p.lse2[row] * p.lse_scale;
-      float qsum = 0.f, lmax = -INFINITY, lsum = 0.f;
+      const int wrow0 = q * 32;  // first tile row of this warp
+      float rowv = 0.f;          // per-row scalar input: lse2 or D
+      if (valid) {
+        if (EPI == kEpiAExp) rowv = p.lse2[row] * p.lse_scale;
+        if (EPI == kEpiDS) rowv = p.drow[row];
+      }
+      float csum = 0.f, lmax = -INFINITY, lsum = 0.f;
+      if ((EPI == kEpiDS || EPI == kEpiAExp) && p.c_user != nullptr) {
+        const int n = n0 + half * 64 + lane;
+        cst[lane] = n < p.k_valid ? p.c_user[(long long)user * p.k_pad + n] : 0.f;
+        cst[lane + 32] = n + 32 < p.k_valid ? p.c_user[(long long)user * p.k_pad + n + 32] : 0.f;
+        __syncwarp();
+      }
 #pragma unroll 1
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = half * 2; c < half * 2 + 2; ++c) {
         uint32_t u[32];
         tmem_ld32_raw(tmem + lane_off + c * 32, u);
         tmem_wait_tie(u);
         const int nb = n0 + c * 32;
-        if (!valid || nb >= p.N) continue;
-        if (EPI == kEpiStoreF32) {
-          float* dst = p.out_f32 + (long long)z * p.split_stride + row * p.ld_out + nb;
+        if (nb >= p.N) continue;  // warp-uniform
+        float v[32];
 #pragma unroll
-          for (int x = 0; x < 32; x += 4)
-            if (nb + x < p.N)
-              *reinterpret_cast<float4*>(dst + x) =
-                  make_float4(__uint_as_float(u[x]), __uint_as_float(u[x + 1]),
-                              __uint_as_float(u[x + 2]), __uint_as_float(u[x + 3]));
-        } else if (EPI == kEpiAExp) {
-          __nv_bfloat16* dst = p.out_bf16 + row * p.ld_out + nb;
-#pragma unroll
-          for (int x = 0; x < 32; x += 8) {
-            uint32_t w[4];
-#pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const int n = nb + x + 2 * h;
-              w[h] = cvt_bf16x2(n < p.k_valid ? ex2_approx(__uint_as_float(u[x + 2 * h]) - lse2) : 0.f,
-                                n + 1 < p.k_valid ? ex2_approx(__uint_as_float(u[x + 2 * h + 1]) - lse2) : 0.f);
-            }
-            if (nb + x < p.N) *reinterpret_cast<uint4*>(dst + x) = make_uint4(w[0], w[1], w[2], w[3]);
-          }
-        } else if (EPI == kEpiLse) {
-          // running log2-sum-exp2 over this row's columns (a fresh max per 32 columns)
+        for (int x = 0; x < 32; ++x) v[x] = __uint_as_float(u[x]);
+        if (EPI == kEpiLse) {
           float cm = -INFINITY;
 #pragma unroll
           for (int x = 0; x < 32; ++x)
-            if (nb + x < p.k_valid) cm = fmaxf(cm, __uint_as_float(u[x]));
+            if (nb + x < p.k_valid) cm = fmaxf(cm, v[x]);
           if (cm > -INFINITY) {
             float cs = 0.f;
 #pragma unroll
             for (int x = 0; x < 32; ++x)
-              if (nb + x < p.k_valid) cs += ex2_approx(__uint_as_float(u[x]) - cm);
+              if (nb + x < p.k_valid) cs += ex2_approx(v[x] - cm);
             const float nm = fmaxf(lmax, cm);
             lsum = lsum * ex2_approx(lmax - nm) + cs * ex2_approx(cm - nm);
             lmax = nm;
           }
-        } else {  // kEpiQ
-          const __nv_bfloat16* ain = p.a_in + row * p.ld_a_in + nb;
-          const float* cu = p.c_user + (long long)user * p.k_pad + nb;
-          float* dst = p.out_f32 + row * p.ld_out + nb;
+          continue;
+        }
+        // elementwise input (bf16 A for kEpiDS, fp32 addend for kEpiStoreF32), staged
+        const bool has_in = EPI == kEpiDS || (EPI == kEpiStoreF32 && p.add_in != nullptr);
+        if (has_in) {
+          __syncwarp();
+          if (EPI == kEpiDS) {  // 32 rows x 64 B: 4 lanes per row, 8 rows per instruction
 #pragma unroll
-          for (int x = 0; x < 32; x += 8) {
-            if (nb + x >= p.N) break;
-            const uint4 av = *reinterpret_cast<const uint4*>(ain + x);
-            const uint32_t aw[4] = {av.x, av.y, av.z, av.w};
-            float qv[8];
+            for (int it = 0; it < 4; ++it) {
+              const int rr = it * 8 + (lane >> 2), cc = (lane & 3) * 8;
+              uint4 w = make_uint4(0, 0, 0, 0);
+              if (wrow0 + rr < nrows && nb + cc < p.N)
+                w = *reinterpret_cast<const uint4*>(p.a_in + (row0 + wrow0 + rr) * p.ld_a_in + nb + cc);
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              const float a0 = __uint_as_float(aw[h] << 16), a1 = __uint_as_float(aw[h] & 0xFFFF0000u);
-              qv[2 * h] = a0 * (__uint_as_float(u[x + 2 * h]) - cu[x + 2 * h]);
-              qv[2 * h + 1] = a1 * (__uint_as_float(u[x + 2 * h + 1]) - cu[x + 2 * h + 1]);
+              for (int h = 0; h < 4; ++h) {
+                stg[rr * 33 + cc + 2 * h] = __uint_as_float(ww[h] << 16);
+                stg[rr * 33 + cc + 2 * h + 1] = __uint_as_float(ww[h] & 0xFFFF0000u);
+              }
             }
-            *reinterpret_cast<float4*>(dst + x) = make_float4(qv[0], qv[1], qv[2], qv[3]);
-            *reinterpret_cast<float4*>(dst + x + 4) = make_float4(qv[4], qv[5], qv[6], qv[7]);
-            qsum += ((qv[0] + qv[1]) + (qv[2] + qv[3])) + ((qv[4] + qv[5]) + (qv[6] + qv[7]));
+          } else {  // 32 rows x 128 B: 8 lanes per row, 4 rows per instruction
+#pragma unroll
+            for (int it = 0; it < 8; ++it) {
+              const int rr = it * 4 + (lane >> 3), cc = (lane & 7) * 4;
+              float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
+              if (wrow0 + rr < nrows && nb + cc < p.N)
+                w = *reinterpret_cast<const float4*>(p.add_in + (row0 + wrow0 + rr) * p.ld_add + nb + cc);
+              stg[rr * 33 + cc] = w.x;
+              stg[rr * 33 + cc + 1] = w.y;
+              stg[rr * 33 + cc + 2] = w.z;
+              stg[rr * 33 + cc + 3] = w.w;
+            }
+          }
+          __syncwarp();
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const float e = stg[lane * 33 + x];
+            if (EPI == kEpiDS) {
+              const float cu = cst[(c & 1) * 32 + x];
+              v[x] = e * (v[x] - cu - rowv);
+            } else {
+              v[x] += e;
+            }
+          }
+        }
+        if (EPI == kEpiAExp) {
+#pragma unroll
+          for (int x = 0; x < 32; ++x) {
+            const float a = nb + x < p.k_valid ? ex2_approx(v[x] - rowv) : 0.f;
+            // the value the later GEMMs see is bf16(a): sum c against that
+            const float ab = __bfloat162float(__float2bfloat16_rn(a));
+            if (p.c_user != nullptr) csum = fmaf(ab, cst[(c & 1) * 32 + x], csum);
+            v[x] = ab;
+          }
+        }
+        // stage this warp's 32 x 32 outputs, then store them row by row
+        __syncwarp();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) stg[lane * 33 + x] = v[x];
+        __syncwarp();
+        if (EPI == kEpiStoreF32) {
+          float* dst = p.out_f32 + (long long)z * p.split_stride;
+#pragma unroll
+          for (int it = 0; it < 8; ++it) {
+            const int rr = it * 4 + (lane >> 3), cc = (lane & 7) * 4;
+            if (wrow0 + rr < nrows && nb + cc < p.N)
+              *reinterpret_cast<float4*>(dst + (row0 + wrow0 + rr) * p.ld_out + nb + cc) =
+                  make_float4(stg[rr * 33 + cc], stg[rr * 33 + cc + 1], stg[rr * 33 + cc + 2],
+                              stg[rr * 33 + cc + 3]);
+          }
+        } else {  // bf16 outputs (A, dS)
+#pragma unroll
+          for (int it = 0; it < 4; ++it) {
+            const int rr = it * 8 + (lane >> 2), cc = (lane & 3) * 8;
+            if (wrow0 + rr < nrows && nb + cc < p.N) {
+              const float* sr = stg + rr * 33 + cc;
+              *reinterpret_cast<uint4*>(p.out_bf16 + (row0 + wrow0 + rr) * p.ld_out + nb + cc) =
+                  make_uint4(cvt_bf16x2(sr[0], sr[1]), cvt_bf16x2(sr[2], sr[3]),
+                             cvt_bf16x2(sr[4], sr[5]), cvt_bf16x2(sr[6], sr[7]));
+            }
           }
         }
       }
-      if (EPI == kEpiQ && valid) p.dpart[row * p.dpart_ld + blockIdx.y] = qsum;
       if (EPI == kEpiLse && valid)
-        p.dpart[row * p.dpart_ld + blockIdx.y] = lmax > -INFINITY ? lmax + lg2_approx(lsum) : -INFINITY;
+        p.dpart[row * p.dpart_ld + 2 * blockIdx.y + half] =
+            lmax > -INFINITY ? lmax + lg2_approx(lsum) : -INFINITY;
+      if (EPI == kEpiAExp && valid && p.c_user != nullptr)
+        p.dpart[row * p.dpart_ld + 2 * blockIdx.y + half] = csum;
     }
   }
   tc_fence_before();
@@ -338,13 +404,16 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.k_pad = g.k_pad;
   p.dpart = g.dpart;
   p.dpart_ld = g.dpart_ld;
+  p.add_in = g.add_in;
+  p.ld_add = g.ld_add;
+  p.drow = g.drow;
   p.budget = kDefaultWaitBudget;
   const dim3 grid((unsigned)g.m_tiles_bound, (unsigned)((g.N + kBN - 1) / kBN), (unsigned)p.splits);
   if (grid.x == 0) return cudaSuccess;
   switch (g.epi) {
     case kEpiStoreF32: return launch_t<kEpiStoreF32>(p, grid, s);
     case kEpiAExp: return launch_t<kEpiAExp>(p, grid, s);
-    case kEpiQ: return launch_t<kEpiQ>(p, grid, s);
+    case kEpiDS: return launch_t<kEpiDS>(p, grid, s);
     case kEpiLse: return launch_t<kEpiLse>(p, grid, s);
     default: return cudaErrorInvalidValue;
   }

@@ -71,8 +71,9 @@ struct Plan {
   size_t pn = 0, gt = 0, gh = 0, cj = 0, lseb = 0, db = 0, dppp = 0, dpp = 0, wvp = 0;
   // tensor-core backward (bf16)
   bool btc = false;
-  int splits = 0;
-  size_t ghb = 0, pn2 = 0, pnn = 0, ab = 0, qb = 0, dsb = 0, dpart = 0, lse2b = 0;
+  int splits = 0, wv_splits = 0;
+  size_t ghb = 0, gtb = 0, ub = 0, pn2 = 0, pnn = 0, ab = 0, dsb = 0, yb = 0, dvb = 0, dpart = 0,
+         lse2b = 0;
   size_t total = 0;
 };
 
@@ -119,21 +120,26 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
     q.btc = true;
     q.k_pad = (k + 127) / 128 * 128;
     q.splits = bwd_tc_splits(dev.sms, q.k_pad, d, n_total);
+    q.wv_splits = bwd_tc_wv_splits(dev.sms, R, q.k_pad);
     q.Gb = q.splits;
     const size_t nk = (size_t)n_total * q.k_pad;
-    q.gt = take((size_t)R * q.k_pad * d * sizeof(float));
-    q.ghb = take((size_t)R * q.k_pad * d * 2);
+    const size_t rkd = (size_t)R * q.k_pad * d;
+    q.gt = take(rkd * sizeof(float));
+    q.gtb = take(rkd * 2);
+    q.ghb = take(rkd * 2);
+    q.ub = take(rkd * 2);
     q.cj = take((size_t)R * q.k_pad * sizeof(float));
     q.pn2 = take((size_t)q.k_pad * d * 2);
     q.pnn = take((size_t)q.k_pad * d * 2);
     q.ab = take(nk * 2);
-    q.qb = take(nk * sizeof(float));
     q.dsb = take(nk * 2);
-    q.dpart = take((size_t)n_total * (q.k_pad / 128) * sizeof(float));
+    q.yb = take((size_t)n_total * d * sizeof(float));
+    q.dvb = take((size_t)n_total * sizeof(float));
+    q.dpart = take((size_t)n_total * (q.k_pad / 64) * sizeof(float));
     q.lse2b = take((size_t)n_total * sizeof(float));
     q.dppp = take((size_t)q.splits * q.k_pad * d * sizeof(float));
     q.dpp = take((size_t)q.k_pad * d * sizeof(float));
-    q.wvp = take(bwd_wv_chunks(R, k) * d * d * sizeof(float));
+    q.wvp = take((size_t)(q.wv_splits > 1 ? q.wv_splits : 1) * d * d * sizeof(float));
   } else {
     q.Gb = q.G;
     q.pn = take((size_t)q.k_pad * d * sizeof(float));
@@ -382,6 +388,7 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
   a.Pn = nullptr;
   a.Gh = nullptr;
   a.Ghb = at<__nv_bfloat16>(workspace, p.ghb);
+  a.Gtb = at<__nv_bfloat16>(workspace, p.gtb);
   a.lseb = nullptr;
   a.Db = nullptr;
   BwdTcArgs t;
@@ -390,11 +397,14 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
   t.pn2 = at<__nv_bfloat16>(workspace, p.pn2);
   t.pnn = at<__nv_bfloat16>(workspace, p.pnn);
   t.A = at<__nv_bfloat16>(workspace, p.ab);
-  t.Q = at<float>(workspace, p.qb);
   t.dS = at<__nv_bfloat16>(workspace, p.dsb);
+  t.Y = at<float>(workspace, p.yb);
+  t.D = at<float>(workspace, p.dvb);
   t.dpart = at<float>(workspace, p.dpart);
   t.lse2 = at<float>(workspace, p.lse2b);
+  t.Ub = at<__nv_bfloat16>(workspace, p.ub);
   t.splits = p.splits;
+  t.wv_splits = p.wv_splits;
   return cuda_status(launch_bwd_tc(t, s));
 }
 

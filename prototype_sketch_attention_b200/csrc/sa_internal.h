@@ -97,6 +97,7 @@ struct BwdArgs {
   float* Gt;      // [R, k_pad, d]  G / mass
   float* Gh;      // [R, k_pad, d]  (G / mass) W_v^T (nullable)
   __nv_bfloat16* Ghb;  // the same in bf16 (nullable; the tensor-core backward)
+  __nv_bfloat16* Gtb;  // Gt in bf16 (nullable; the tensor-core backward)
   float* cj;      // [R, k_pad]     (G / mass) . sketch - dmass
   float* lseb;    // [n_total]      fp32 per-token log-sum-exp (natural)
   float* Db;      // [n_total]      sum_j A_jt dA_jt
@@ -112,7 +113,8 @@ struct BwdArgs {
 size_t bwd_wv_chunks(int R, int k);
 cudaError_t launch_bwd_simt(const BwdArgs& a, cudaStream_t s);
 cudaError_t launch_bwd_prep(const BwdArgs& a, cudaStream_t s);  // Gt, Gh, c per user
-cudaError_t launch_bwd_tail(const BwdArgs& a, cudaStream_t s);  // dPn reduce, dW_v, dP, dW_k
+// dPn reduce, dW_v, dP, dW_k; wv_parts > 0: that many dW_v partials are already in wv_part
+cudaError_t launch_bwd_tail(const BwdArgs& a, int wv_parts, cudaStream_t s);
 
 // ---- tensor-core backward (bf16 inputs; sa_bwd_tc.cu)
 struct BwdTcArgs {
@@ -121,17 +123,21 @@ struct BwdTcArgs {
   __nv_bfloat16* pn2;        // [k_pad, d] P W_k^T log2(e)/sqrt(d)
   __nv_bfloat16* pnn;        // [k_pad, d] P W_k^T / sqrt(d)
   __nv_bfloat16* A;          // [n_total, k_pad]
-  float* Q;                  // [n_total, k_pad]
   __nv_bfloat16* dS;         // [n_total, k_pad]
-  float* dpart;              // [n_total, k_pad / 128]
+  float* Y;                  // [n_total, d]  A Gh_u
+  float* D;                  // [n_total]
+  float* dpart;              // [n_total, k_pad / 128] per-tile partials
   float* lse2;               // [n_total] (when lse is null)
+  __nv_bfloat16* Ub;         // [R, k_pad, d] bf16 xsketch (zero rows past k)
   int splits;                // split-K of dPn (== b.G)
+  int wv_splits;             // split-K of dW_v (partials in b.wv_part)
 };
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s);
 int bwd_tc_splits(int sms, int k_pad, int d, long long n_total);
+int bwd_tc_wv_splits(int sms, int R, int k_pad);
 
 // ---- tensor-core GEMM (backward building block, sa_gemm_sm100.cu)
-enum GemmEpi { kEpiStoreF32 = 0, kEpiAExp = 1, kEpiQ = 2, kEpiLse = 3 };
+enum GemmEpi { kEpiStoreF32 = 0, kEpiAExp = 1, kEpiDS = 2, kEpiLse = 3 };
 struct GemmOperandDesc {  // one bf16 operand, row-major in memory
   const void* base;
   uint64_t rows, cols;
@@ -164,6 +170,9 @@ struct GemmArgs {
   int k_pad;
   float* dpart;
   int dpart_ld;
+  const float* add_in;         // kEpiStoreF32: added elementwise (nullable)
+  long long ld_add;
+  const float* drow;           // kEpiDS: per-row D
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
