@@ -197,6 +197,21 @@ int sa_sketch_get_device_status(const void* workspace, void* stream);
  */
 int sa_sketch_profile_events(void* start_event, void* stop_event);
 
+/*
+ * Test hook for the tensor-core GEMM that the backward is built from (bf16 operands,
+ * fp32 accumulate, 128 x 128 tiles):  out[s][m][n] = sum over the K range of split s of
+ * A[m][k] B[n][k], for s < splits (the caller sums the split partials).
+ *   A: a_mn = 0: stored [M][K] (K contiguous); a_mn = 1: stored [K][M].
+ *   B: b_mn = 0: stored [N][K];                b_mn = 1: stored [K][N].
+ *   out: fp32 [splits][M][N], device. workspace: at least 256 bytes, 256-aligned, device
+ *   (only its status word is used). M, N, K >= 1; the contiguous dimension of A and B a
+ *   multiple of 8; N a multiple of 4; 1 <= splits <= ceil(K / 64).
+ * Returns SA_OK, SA_ERR_INVALID_ARG or SA_ERR_CUDA; device errors are latched in the
+ * workspace status word as for the forward.
+ */
+int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M, int N, int K,
+                         int splits, float* out, void* workspace, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* sa_status_string(int status);
 

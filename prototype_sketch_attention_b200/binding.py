@@ -30,7 +30,8 @@ SA_ERR_NO_DEVICE = 7
 
 EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
             "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
-            "sa_sketch_profile_events", "sa_sketch_forward_noalloc", "sa_sketch_combine")
+            "sa_sketch_profile_events", "sa_sketch_forward_noalloc", "sa_sketch_combine",
+            "sa_sketch_debug_gemm")
 
 
 class SketchAttentionError(RuntimeError):
@@ -53,6 +54,8 @@ def _load() -> ctypes.CDLL:
     lib.sa_sketch_backward.restype = i32
     lib.sa_sketch_backward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
                                        vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sa_sketch_debug_gemm.restype = i32
+    lib.sa_sketch_debug_gemm.argtypes = [vp, i32, vp, i32, i32, i32, i32, i32, vp, vp, vp]
     lib.sa_sketch_combine.restype = i32
     lib.sa_sketch_combine.argtypes = [vp, vp, i32, i32, i32, vp, i32, vp, vp]
     lib.sa_sketch_get_device_status.restype = i32
@@ -88,6 +91,10 @@ def sa_sketch_backward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass
     return int(_lib.sa_sketch_backward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass,
                                        lse, xsketch, dsketch, dmass, dX, dP, dWk, dWv, workspace,
                                        ws_bytes, stream))
+
+
+def sa_sketch_debug_gemm(A, a_mn, B, b_mn, M, N, K, splits, out, workspace, stream) -> int:
+    return int(_lib.sa_sketch_debug_gemm(A, a_mn, B, b_mn, M, N, K, splits, out, workspace, stream))
 
 
 def sa_sketch_combine(xsketch, mass, R, k, d, Wv, dt, sketch, stream) -> int:

@@ -424,6 +424,36 @@ int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int
                                     static_cast<cudaStream_t>(stream_)));
 }
 
+int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M, int N, int K,
+                         int splits, float* out, void* workspace, void* stream_) {
+  if (!A || !B || !out || !workspace || M < 1 || N < 1 || K < 1 || splits < 1 ||
+      splits > (K + 63) / 64 || (N % 4) != 0)
+    return SA_ERR_INVALID_ARG;
+  if (((a_mn ? M : K) % 8) != 0 || ((b_mn ? N : K) % 8) != 0) return SA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || !aligned16(A) || !aligned16(B) ||
+      !aligned16(out))
+    return SA_ERR_INVALID_ARG;
+  Device dev;
+  sa_status st = current_device(&dev);
+  if (st != SA_OK) return st;
+  GemmArgs g = {};
+  g.a[0] = {A, (uint64_t)(a_mn ? K : M), (uint64_t)(a_mn ? M : K), a_mn != 0};
+  g.b[0] = {B, (uint64_t)(b_mn ? K : N), (uint64_t)(b_mn ? N : K), b_mn != 0};
+  g.phases = 1;
+  g.k_tiles[0] = (K + 63) / 64;
+  g.user_mode = 0;
+  g.M = M;
+  g.N = N;
+  g.m_tiles_bound = (M + 127) / 128;
+  g.splits = splits;
+  g.epi = kEpiStoreF32;
+  g.hdr = static_cast<const WsHeader*>(workspace);
+  g.out_f32 = out;
+  g.ld_out = N;
+  g.split_stride = (long long)M * N;
+  return cuda_status(launch_gemm(g, static_cast<cudaStream_t>(stream_)));
+}
+
 int sa_sketch_get_device_status(const void* workspace, void* stream_) {
   if (!workspace) return SA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream_);
