@@ -93,10 +93,11 @@ struct FwdSmem {
 struct Bars {
   uint64_t x_full[4], x_empty[4];
   uint64_t s_full[2], s_empty[2];
-  uint64_t a_full[2], a_empty[2];
+  uint64_t a_full[2], a_empty[4];
   uint64_t u_full[2], u_empty;  // u_full[w]: segments whose last tile warpgroup w owns
   uint64_t xch[kXchSlots];
   uint64_t p_full, drain, drain2;
+  uint64_t m2iss[4];  // MMA2(i) issued, by tile mod 4 (orders MMA1 behind it)
   uint32_t tmem_base;
 };
 
@@ -111,6 +112,12 @@ constexpr int kNWG = 2;                        // softmax warpgroups (ping-pong 
 // idle (3); warps 4-11: the two softmax warpgroups
 constexpr int kThreads = 128 + 128 * kNWG;
 constexpr int kPrefetchAhead = 4;               // tiles prefetched into L2 ahead of the load
+// MMA1(i) is issued only after MMA2(i - kMma1Lead). The tensor pipe runs its queue in
+// order, and an accumulate MMA queued behind a score MMA waits for it; the accumulate MMA
+// is on the chain "A store -> MMA2 -> next A store" (one A buffer), while the score MMA of
+// tile i is needed only when its warpgroup finishes tile i - 2. With a lead of 3 the score
+// MMAs fill the gaps instead.
+constexpr int kMma1Lead = 3;
 
 // Scores of this thread's token (one TMEM lane) for the CTA's 128 prototypes.
 __device__ __forceinline__ void load_scores(uint32_t taddr, float (&v)[kProtoSlice]) {
@@ -157,6 +164,14 @@ __device__ __forceinline__ float row_max(const float (&v)[kProtoSlice]) {
     mc[j] = a;
   }
   return fmaxf(fmaxf(mc[0], mc[1]), fmaxf(mc[2], mc[3]));
+}
+
+// One 64-prototype block of token row r into the MN-major, 128B-swizzled A operand.
+__device__ __forceinline__ void store_a_block(uint8_t* arow, int r, const uint32_t (&a)[32]) {
+#pragma unroll
+  for (int ch = 0; ch < 8; ++ch)
+    *reinterpret_cast<uint4*>(arow + ((ch ^ (r & 7)) << 4)) =
+        make_uint4(a[ch * 4], a[ch * 4 + 1], a[ch * 4 + 2], a[ch * 4 + 3]);
 }
 
 // log2 of the sum of 2^x[p * 128] over the C partials of one token (C <= MAXC).
@@ -218,12 +233,14 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
       mbar_init(smem_u32(&bars->s_empty[s]), 4);
       mbar_init(smem_u32(&bars->a_full[s]), 4);
       mbar_init(smem_u32(&bars->a_empty[s]), 1);
+      mbar_init(smem_u32(&bars->a_empty[s + 2]), 1);
     }
     mbar_init(smem_u32(&bars->u_full[0]), 1);
     mbar_init(smem_u32(&bars->u_full[1]), 1);
     mbar_init(smem_u32(&bars->u_empty), 4);
     for (int s = 0; s < kXchSlots; ++s) mbar_init(smem_u32(&bars->xch[s]), 1);
     mbar_init(smem_u32(&bars->p_full), 1);
+    for (int s = 0; s < 4; ++s) mbar_init(smem_u32(&bars->m2iss[s]), 1);
     mbar_init(smem_u32(&bars->drain), 1);
     mbar_init(smem_u32(&bars->drain2), 1);
     fence_mbar_init();
@@ -310,8 +327,13 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
         const int st = (int)(i % NS);
         const int sb = (int)(i & 1);
         if (warp == 1) {
+          // m2iss[(i - kMma1Lead) mod 4]: MMA1(i - 4) already waited for MMA2(i - 4 - kMma1Lead),
+          // so only that phase or the awaited one are possible (one parity bit)
           ok = mbar_wait(smem_u32(&bars->x_full[st]), (uint32_t)((i / NS) & 1), status, budget) &&
-               mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget);
+               mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)(((i >> 1) & 1) ^ 1), status, budget) &&
+               (i < kMma1Lead ||
+                mbar_wait(smem_u32(&bars->m2iss[(i - kMma1Lead) & 3]),
+                          (uint32_t)(((i - kMma1Lead) >> 2) & 1), status, budget));
           if (!ok) break;
           tc_fence_after();
           // A = X tile, K-major, 128B swizzle: four 16-wide K steps per 64-column box
@@ -344,8 +366,10 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
             tc_mma_f16(tmem + kColU, ad0 + (uint64_t)((ks * 2048) >> 4), xd + (uint64_t)((ks * 2048) >> 4),
                        idesc2, (first && ks == 0) ? 0u : 1u);
           tc_commit(smem_u32(&bars->x_empty[st]));
-          tc_commit(smem_u32(&bars->a_empty[ab]));
+          // with one A buffer, a_empty is indexed by tile mod 4 (see the A store)
+          tc_commit(smem_u32(&bars->a_empty[NA == 2 ? ab : (i & 3)]));
           if (last) tc_commit(smem_u32(&bars->u_full[i & 1]));
+          mbar_arrive(smem_u32(&bars->m2iss[i & 3]));  // lets MMA1(i + kMma1Lead) in
         }
       }
       const uint32_t db = smem_u32(warp == 1 ? &bars->drain : &bars->drain2);
@@ -431,33 +455,37 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
       if (rank == 0 && valid && lse_out != nullptr)
         lse_out[it.t0() + r] = lse2 * 0.69314718055994530942f;
 
-      // A (bf16) into the MN-major, 128B-swizzled A operand: row = token, 64 prototypes
-      // per 128-byte row, two 16 KB blocks for prototypes [0,64) and [64,128).
+      // A = e * 2^(m - lse2) as bf16 pairs, in registers before the buffer is known free
+      // (the wait below is on the chain A store -> MMA2 -> next A store)
+      uint32_t pa0[32], pa1[32];
+      {
+        const uint64_t sc2 = f2_pack(scale, scale);
+#pragma unroll
+        for (int p = 0; p < 32; ++p) {
+          float a, b;
+          f2_unpack(f2_mul(f2_pack(v[2 * p], v[2 * p + 1]), sc2), a, b);
+          pa0[p] = cvt_bf16x2(a, b);
+          f2_unpack(f2_mul(f2_pack(v[64 + 2 * p], v[64 + 2 * p + 1]), sc2), a, b);
+          pa1[p] = cvt_bf16x2(a, b);
+        }
+      }
+      // A(i) may overwrite the buffer once MMA2 has read the one before it: with two
+      // buffers A(i - 2) (the barrier of this parity), with one A(i - 1) (barrier
+      // (i - 1) mod 4, its phase (i - 1) / 4). exp(i) has already seen MMA2(i - NS) complete
+      // (its X stage was free), so on either barrier only the awaited phase and the one
+      // before it are possible, and one parity bit tells them apart.
       const int ab = NA == 2 ? wg : 0;
-      const uint32_t epar = NA == 2 ? (uint32_t)(((i >> 1) & 1) ^ 1) : (uint32_t)((i & 1) ^ 1);
-      if (!mbar_wait_warp(smem_u32(&bars->a_empty[ab]), epar, status, budget)) {
+      const int eb = NA == 2 ? wg : ((i - 1) & 3);
+      const uint32_t epar =
+          NA == 2 ? (uint32_t)(((i >> 1) & 1) ^ 1) : (uint32_t)(((i - 1) >> 2) & 1);
+      if (!mbar_wait_warp(smem_u32(&bars->a_empty[eb]), epar, status, budget)) {
         ok = false;
         break;
       }
-      uint8_t* arow0 = smem + L::abox(ab, 0) + r * 128;
-      uint8_t* arow1 = smem + L::abox(ab, 1) + r * 128;
-      const uint64_t sc2 = f2_pack(scale, scale);
-#pragma unroll
-      for (int mb = 0; mb < 2; ++mb) {
-#pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          const int c0 = mb * 64 + ch * 8;
-          uint32_t w4[4];
-#pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            float a, b;
-            f2_unpack(f2_mul(f2_pack(v[c0 + 2 * h], v[c0 + 2 * h + 1]), sc2), a, b);
-            w4[h] = cvt_bf16x2(a, b);
-          }
-          *reinterpret_cast<uint4*>((mb ? arow1 : arow0) + ((ch ^ (r & 7)) << 4)) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-      }
+      // A (bf16) into the MN-major, 128B-swizzled A operand: row = token, 64 prototypes
+      // per 128-byte row, two 16 KB blocks for prototypes [0,64) and [64,128).
+      store_a_block(smem + L::abox(ab, 0) + r * 128, r, pa0);
+      store_a_block(smem + L::abox(ab, 1) + r * 128, r, pa1);
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->a_full[ab]));
@@ -559,21 +587,19 @@ int stages_for(int d, int C) { return d == 64 ? 4 : (C <= 8 ? 4 : 3); }
 }  // namespace
 
 size_t fwd_sm100_smem_bytes(int d, int C) {
-  const int ns = stages_for(d, C);
   if (d == 64) return FwdSmem<64, 4, 2>::bytes(C);
-  return ns == 4 ? FwdSmem<128, 4, 1>::bytes(C) : FwdSmem<128, 3, 1>::bytes(C);
+  return stages_for(d, C) == 4 ? FwdSmem<128, 4, 1>::bytes(C) : FwdSmem<128, 3, 1>::bytes(C);
 }
 
 cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
-  const int ns = stages_for(d, C);
   if (d == 64) return max_clusters_t<64, 4, 2>(C, n);
-  return ns == 4 ? max_clusters_t<128, 4, 1>(C, n) : max_clusters_t<128, 3, 1>(C, n);
+  return stages_for(d, C) == 4 ? max_clusters_t<128, 4, 1>(C, n) : max_clusters_t<128, 3, 1>(C, n);
 }
 
 cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream) {
-  const int ns = stages_for(a.d, a.C);
   if (a.d == 64) return launch_fwd_sm100_t<64, 4, 2>(a, stream);
-  return ns == 4 ? launch_fwd_sm100_t<128, 4, 1>(a, stream) : launch_fwd_sm100_t<128, 3, 1>(a, stream);
+  return stages_for(a.d, a.C) == 4 ? launch_fwd_sm100_t<128, 4, 1>(a, stream)
+                                   : launch_fwd_sm100_t<128, 3, 1>(a, stream);
 }
 
 }  // namespace sa
