@@ -403,7 +403,9 @@ def run_ours(args) -> None:
                      "peak_source": peak_src, "flop_per_launch": flop_per_launch},
         "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        "gpu_launches": 4 * args.steps,
+        # per forward: schedule, fold, the tcgen05 kernel, then the finalize (segment sums
+        # and the U Wv GEMM on the tensor cores when k is a multiple of 128, else one kernel)
+        "gpu_launches": (5 if k % 128 == 0 else 4) * args.steps,
         "clocks": clk.summary(),
     }
     if cpu is not None:

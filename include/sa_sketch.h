@@ -95,6 +95,10 @@ size_t sa_sketch_workspace_size(int R, int64_t n_total, int k, int d, sa_dtype d
  *                         Needed by the backward.
  * A user with no tokens gets sketch = 0 and mass = 0. Results are deterministic:
  * two calls on the same inputs give bitwise-equal outputs.
+ * Precision of the bf16 path: the scores use P' = P Wk^T / sqrt(d) rounded to bf16 and
+ * A is rounded to bf16 before it meets X; accumulation is fp32. When k is a multiple of
+ * 128, sketch = (U / mass) Wv runs on the tensor cores with U / mass split into two bf16
+ * parts (about 16 significant bits), else in fp32 on the CUDA cores.
  * Pointers must be 16-byte aligned.
  */
 int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
@@ -166,7 +170,7 @@ int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int
  *    (different streams, or different host threads) race and give wrong results.
  *    Serialise them, for instance on one stream.
  *  - Sizes whose plan needs more than SA_NOALLOC_SCRATCH_BYTES are rejected with
- *    SA_ERR_WORKSPACE before anything is launched (at k = 1024, d = 128 on a B200 about 48 users).
+ *    SA_ERR_WORKSPACE before anything is launched (at k = 1024, d = 128 on a B200 about 24 users).
  *  - It calls no cudaMalloc, cudaFree or allocating library routine.
  *  - device_status: nullable HOST pointer. When given, the call waits for `stream` and
  *    stores the device status word there (SA_OK, SA_ERR_BAD_OFFSETS, SA_ERR_TIMEOUT), since

@@ -69,6 +69,9 @@ struct Plan {
   int C = 0, k_pad = 0, G = 0, Gb = 0;
   size_t hdr = 0, ts = 0, pf = 0, pu = 0, pm = 0, lse2 = 0;
   size_t pn = 0, gt = 0, gh = 0, cj = 0, lseb = 0, db = 0, dppp = 0, dpp = 0, wvp = 0;
+  // tensor-core finalize (bf16 forward, k a multiple of 128): U / mass as bf16 hi + lo
+  bool ftc = false;
+  size_t ubh = 0, ubl = 0;
   // tensor-core backward (bf16)
   bool btc = false;
   int splits = 0, wv_splits = 0;
@@ -115,6 +118,11 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
     q.pu = take(segs * q.k_pad * d * sizeof(float));
     q.pm = take(segs * q.k_pad * sizeof(float));
     if (!q.tc) q.lse2 = take((size_t)n_total * sizeof(float));
+    if (q.tc && k == q.k_pad) {
+      q.ftc = true;
+      q.ubh = take((size_t)R * q.k_pad * d * 2);
+      q.ubl = take((size_t)R * q.k_pad * d * 2);
+    }
   } else if (dt == SA_BF16) {
     // tensor-core backward: token x prototype intermediates in the workspace
     q.btc = true;
@@ -316,7 +324,9 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   f.sketch = sketch;
   f.mass = mass;
   f.xsketch = xsketch;
-  return cuda_status(launch_finalize(f, s));
+  f.ubar_hi = p.ftc ? at<__nv_bfloat16>(workspace, p.ubh) : nullptr;
+  f.ubar_lo = p.ftc ? at<__nv_bfloat16>(workspace, p.ubl) : nullptr;
+  return cuda_status(p.ftc ? launch_finalize_tc(f, s) : launch_finalize(f, s));
 }
 
 int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,

@@ -35,8 +35,14 @@ struct FinalizeArgs {
   float* sketch;
   float* mass;
   float* xsketch;  // nullable
+  // tensor-core finalize (bf16, k = k_pad): U / mass as a bf16 pair hi + lo, [R, k, d] each
+  __nv_bfloat16* ubar_hi;
+  __nv_bfloat16* ubar_lo;
 };
 cudaError_t launch_finalize(const FinalizeArgs& a, cudaStream_t s);
+// Segment sums -> xsketch, mass and U / mass as hi + lo bf16; sketch = (hi + lo) Wv on the
+// tensor cores (two accumulated GEMM phases). Needs ubar_hi / ubar_lo and k == k_pad.
+cudaError_t launch_finalize_tc(const FinalizeArgs& a, cudaStream_t s);
 
 // ---- combine: sketch = (U Wv) / mass from already summed U [R, k, d] and mass [R, k]
 cudaError_t launch_combine(const float* U, const float* mass, int R, int k, int d, const void* Wv,
