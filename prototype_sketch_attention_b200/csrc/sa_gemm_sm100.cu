@@ -31,8 +31,8 @@ namespace sa {
 namespace {
 
 constexpr int kBM = 128, kBN = 128, kBK = 64;
-constexpr int kStages = 3;
 constexpr int kStageBytes = (kBM + kBN) * kBK * 2;  // 32 KB
+// pipeline stages: 3, or 2 when a CTA has at most 2 K tiles (then 3 CTAs fit per SM)
 constexpr int kGemmThreads = 320;                   // producer, MMA, 8 epilogue warps
 
 struct GemmParams {
@@ -67,8 +67,9 @@ struct GemmParams {
   long long budget;
 };
 
+template <int NST>
 struct GemmBars {
-  uint64_t full[kStages], empty[kStages], done, drain;
+  uint64_t full[NST], empty[NST], done, drain;
   uint32_t tmem_base;
 };
 
@@ -89,14 +90,15 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, in
                   : smem_desc(base + ks * 32, 16, 1024, kSwizzle128B);
 }
 
-template <int EPI>
+template <int EPI, int NST>
 __global__ void __launch_bounds__(kGemmThreads)
 sa_gemm_kernel(const __grid_constant__ GemmParams p) {
+  constexpr int kStages = NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
-  GemmBars* bars = reinterpret_cast<GemmBars*>(smem + kStages * kStageBytes);
+  GemmBars<NST>* bars = reinterpret_cast<GemmBars<NST>*>(smem + kStages * kStageBytes);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* status = const_cast<int*>(&p.hdr->status);
 
@@ -356,14 +358,21 @@ bool make_operand_map(CUtensorMap* m, const GemmOperandDesc& o) {
             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int EPI>
-cudaError_t launch_t(const GemmParams& p, dim3 grid, cudaStream_t s) {
-  const size_t smem = 1024 + kStages * kStageBytes + sizeof(GemmBars);
-  cudaError_t e = cudaFuncSetAttribute(sa_gemm_kernel<EPI>,
+template <int EPI, int NST>
+cudaError_t launch_st(const GemmParams& p, dim3 grid, cudaStream_t s) {
+  static_assert(8 * (32 * 33 + 64) * 4 <= NST * kStageBytes, "epilogue staging fits the stages");
+  const size_t smem = 1024 + NST * kStageBytes + sizeof(GemmBars<NST>);
+  cudaError_t e = cudaFuncSetAttribute(sa_gemm_kernel<EPI, NST>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  sa_gemm_kernel<EPI><<<grid, kGemmThreads, smem, s>>>(p);
+  sa_gemm_kernel<EPI, NST><<<grid, kGemmThreads, smem, s>>>(p);
   return cudaGetLastError();
+}
+
+template <int EPI>
+cudaError_t launch_t(const GemmParams& p, dim3 grid, cudaStream_t s) {
+  const int kt_max = (p.k_tiles[0] + p.splits - 1) / p.splits + (p.phases > 1 ? p.k_tiles[1] : 0);
+  return kt_max <= 2 ? launch_st<EPI, 2>(p, grid, s) : launch_st<EPI, 3>(p, grid, s);
 }
 
 }  // namespace
