@@ -224,5 +224,98 @@ def combine(xsketch: torch.Tensor, mass: torch.Tensor, Wv: torch.Tensor, *,
     return out
 
 
+def user_chunks(offsets_host: torch.Tensor, chunks: int) -> list[tuple[int, int]]:
+    """Cut users [0, R) into at most `chunks` consecutive ranges of about equal token
+    count: range c ends at the first user whose tokens reach c / chunks of the total (a
+    user is never split; a range without tokens joins the next one).
+    offsets_host: int64 [R + 1] on the host."""
+    R = offsets_host.numel() - 1
+    if R <= 0:
+        return []
+    n_total = int(offsets_host[R])
+    ends = offsets_host[1:]
+    cuts = []
+    for c in range(1, chunks):
+        u1 = int(torch.searchsorted(ends, torch.tensor(n_total * c // chunks))) + 1
+        if 0 < u1 < R and (not cuts or u1 > cuts[-1]) and int(offsets_host[u1]) > (
+                int(offsets_host[cuts[-1]]) if cuts else 0):
+            cuts.append(u1)
+    while cuts and int(offsets_host[R]) == int(offsets_host[cuts[-1]]):
+        cuts.pop()  # trailing users without tokens join the last range
+    bounds = [0] + cuts + [R]
+    return [(bounds[i], bounds[i + 1]) for i in range(len(bounds) - 1)]
+
+
+def forward_from_host(Xh: torch.Tensor, offsets_h: torch.Tensor, P: torch.Tensor,
+                      Wk: torch.Tensor, Wv: torch.Tensor, *, chunks: int = 4,
+                      state: dict | None = None) -> tuple[torch.Tensor, torch.Tensor]:
+    """Forward from host X and offsets (pinned) to host sketch and mass (pinned).
+
+    The users are cut into about `chunks` consecutive parts of equal token count. Part
+    c's X is copied to the device on a copy stream while part c - 1's forward runs on
+    the current stream, and part c's sketch and mass go back on a third stream as soon
+    as its forward is done; each part is one sa_sketch_forward call (users are
+    independent, so no combining). P, Wk, Wv live on the device. `state` (a dict the
+    caller keeps) holds the device buffers, pinned staging and streams between calls.
+    The current stream waits for the copies back before this returns, so work queued on
+    it afterwards (an event, a synchronize) sees the outputs."""
+    R = offsets_h.numel() - 1
+    n_total, d = Xh.shape
+    k = P.shape[0]
+    dev = P.device
+    if k % 4:
+        chunks = 1  # a part's mass rows must start 16-byte aligned
+    st = {} if state is None else state
+    key = (R, n_total, k, d, Xh.dtype, chunks, dev)
+    if st.get("key") != key:
+        st.clear()
+        st.update(
+            key=key,
+            Xd=torch.empty(n_total, d, dtype=Xh.dtype, device=dev),
+            offd=torch.empty(R + 2 * chunks + 2, dtype=torch.int64, device=dev),
+            offp=torch.empty(R + 2 * chunks + 2, dtype=torch.int64).pin_memory(),
+            sketch=torch.empty(R, k, d, dtype=torch.float32, device=dev),
+            mass=torch.empty(R, k, dtype=torch.float32, device=dev),
+            sk_h=torch.empty(R, k, d, dtype=torch.float32).pin_memory(),
+            ms_h=torch.empty(R, k, dtype=torch.float32).pin_memory(),
+            ws=workspace(R, n_total, k, d, Xh.dtype, False, dev),
+            s_copy=torch.cuda.Stream(dev), s_back=torch.cuda.Stream(dev), off_done=None)
+    cur = torch.cuda.current_stream(dev)
+    s_copy, s_back = st["s_copy"], st["s_back"]
+    # the pinned offsets staging is rewritten below: its previous copy must have run
+    if st["off_done"] is not None:
+        st["off_done"].synchronize()
+    parts = user_chunks(offsets_h, chunks)
+    at, spans = 0, []
+    for u0, u1 in parts:  # each part's offsets, rebased to 0, side by side in the staging
+        torch.sub(offsets_h[u0:u1 + 1], offsets_h[u0], out=st["offp"][at:at + u1 - u0 + 1])
+        spans.append((at, at + u1 - u0 + 1))
+        at += (u1 - u0 + 2) & ~1  # the next part's offsets start 16-byte aligned
+    s_copy.wait_stream(cur)
+    s_back.wait_stream(cur)
+    with torch.cuda.stream(s_copy):
+        st["offd"][:at].copy_(st["offp"][:at], non_blocking=True)
+    off_done = torch.cuda.Event()
+    off_done.record(s_copy)
+    st["off_done"] = off_done
+    for (u0, u1), (a, b) in zip(parts, spans):
+        t0, t1 = int(offsets_h[u0]), int(offsets_h[u1])
+        with torch.cuda.stream(s_copy):
+            st["Xd"][t0:t1].copy_(Xh[t0:t1], non_blocking=True)
+        landed = torch.cuda.Event()
+        landed.record(s_copy)
+        cur.wait_event(landed)
+        forward(st["Xd"][t0:t1], st["offd"][a:b], P, Wk, Wv, ws=st["ws"],
+                out={"sketch": st["sketch"][u0:u1], "mass": st["mass"][u0:u1]}, stream=cur)
+        done = torch.cuda.Event()
+        done.record(cur)
+        s_back.wait_event(done)
+        with torch.cuda.stream(s_back):
+            st["sk_h"][u0:u1].copy_(st["sketch"][u0:u1], non_blocking=True)
+            st["ms_h"][u0:u1].copy_(st["mass"][u0:u1], non_blocking=True)
+    cur.wait_stream(s_back)
+    return st["sk_h"], st["ms_h"]
+
+
 def device_status(ws: torch.Tensor, stream=None) -> int:
     return sa_sketch_get_device_status(_ptr(ws), _stream(stream))

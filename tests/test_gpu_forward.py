@@ -125,3 +125,25 @@ def test_bounded_wait_times_out_and_context_survives():
     w = inputs.make_workload([300, 40], 128, 256, "bf16", seed=8)
     _, out = gpu_forward(w)
     check_forward(w, out)
+
+
+@pytest.mark.parametrize("lengths,k", [
+    ([3000, 0, 1500, 77, 9000, 1, 4096], 1024),
+    ([700, 0, 300], 200),
+    ([500, 600], 2),
+])
+def test_forward_from_host_matches_device_forward(lengths, k):
+    # users cut into parts whose copies overlap the previous part's forward
+    from prototype_sketch_attention_b200 import binding
+    w = inputs.make_workload(lengths, 128, k, "bf16", seed=77 + k)
+    g = {n: getattr(w, n).cuda() for n in ("X", "offsets", "P", "Wk", "Wv")}
+    ref = binding.forward(g["X"], g["offsets"], g["P"], g["Wk"], g["Wv"])
+    state = {}
+    for _ in range(2):  # the second call reuses the buffers and streams
+        sk, ms = binding.forward_from_host(w.X.pin_memory(), w.offsets, g["P"], g["Wk"], g["Wv"],
+                                           chunks=4, state=state)
+        torch.cuda.synchronize()
+        exp_s, exp_m = ref["sketch"].cpu().double(), ref["mass"].cpu().double()
+        for u in range(w.R):
+            assert rel_l2(sk[u].double().numpy(), exp_s[u].numpy()) <= 1e-5
+            assert rel_l2(ms[u].double().numpy(), exp_m[u].numpy()) <= 1e-5
