@@ -147,3 +147,29 @@ def test_forward_from_host_matches_device_forward(lengths, k):
         for u in range(w.R):
             assert rel_l2(sk[u].double().numpy(), exp_s[u].numpy()) <= 1e-5
             assert rel_l2(ms[u].double().numpy(), exp_m[u].numpy()) <= 1e-5
+
+
+def test_bf16_extreme_scores_take_the_shifted_path():
+    # A few tokens point along one prototype with 10 times its norm (W_k = I): that
+    # prototype's score is ~160 in log2 units and the others stay below ~50, so
+    # sum_j 2^s overflows fp32 and each warp holding such a token redoes its 32 tokens
+    # shifted by the row max. Their softmax is one-hot by a margin that bf16 rounding of
+    # P' cannot move, so the bf16 tolerances still apply; the ordinary tokens of those
+    # warps check the shifted path's normalisation. (Their own lse is not compared: a
+    # score of 160 carries ~0.3 of bf16 rounding from P', beyond lse's 5e-2.)
+    import dataclasses
+    from parity_util import BF16_ABS
+    w = inputs.make_workload([700, 450], 128, 256, "bf16", seed=91)
+    X = w.X.float().clone()
+    gen = torch.Generator().manual_seed(5)
+    idx = torch.arange(3, int(w.offsets[-1]), 97)
+    js = torch.randint(0, w.k, (len(idx),), generator=gen)
+    X[idx] = 10.0 * w.P.float()[js]
+    w2 = dataclasses.replace(w, X=X.to(torch.bfloat16), Wk=torch.eye(w.d).to(torch.bfloat16))
+    _, out = gpu_forward(w2)
+    ref = check_forward(w2, {k: v for k, v in out.items() if k != "lse"})
+    lse = out["lse"].cpu().double().numpy()
+    normal = np.ones(len(lse), dtype=bool)
+    normal[idx.numpy()] = False
+    assert np.abs(lse[normal] - ref["lse"][normal]).max() <= BF16_ABS
+    assert np.abs(lse[~normal] - ref["lse"][~normal]).max() <= 1.0  # same dominant score
