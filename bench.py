@@ -25,6 +25,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import math
 import os
@@ -47,10 +48,15 @@ KERNEL_SOURCES = [os.path.join(ROOT, "prototype_sketch_attention_b200", "csrc", 
 
 
 def kernel_source_hash() -> str:
+    """Hash of the hot kernel's code with comments and blank space removed, so that a
+    committed profile summary stays matched across comment-only edits."""
     h = hashlib.sha256()
     for f in KERNEL_SOURCES:
-        with open(f, "rb") as fh:
-            h.update(fh.read())
+        with open(f) as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update("\n".join(ln.strip() for ln in text.splitlines() if ln.strip()).encode())
     return h.hexdigest()[:16]
 
 

@@ -55,10 +55,12 @@ constexpr uint32_t kColS0 = 0, kColS1 = 128, kColU = 256;
 // the a_s chosen so that no two stages share a slot (d = 128: a = 1, 3, 4, 5 -> slots
 // {8,9}, {4,7}, {2,6}, {0,5}; the free slots 1 and 3 hold the A tile).
 //
-// The A tile is single-buffered at d = 128 (NA = 1): it lives from the softmax's store
-// to the end of the accumulate MMA, well under one tile period, and the slots it frees
-// buy a fourth X stage, which is what bounds the tile rate (an X stage is held from its
-// load through the scores, the softmax and the accumulate MMA).
+// The A tile is single-buffered at d = 128 (NA = 1), and the slots that frees buy a
+// fourth X stage (an X stage is held from its load through the scores, the softmax and
+// the accumulate MMA). One A buffer makes "A(i) store -> MMA2(i) -> A(i+1) store" a
+// chain on every tile; the softmax computes A in registers before it waits for the
+// buffer, and score MMAs are held back so that MMA2 does not queue behind them
+// (kMma1Lead), which keeps that chain below the softmax's own per-tile time.
 template <int D, int NS, int NA>
 struct FwdSmem {
   static constexpr int kSlot = 16384;
