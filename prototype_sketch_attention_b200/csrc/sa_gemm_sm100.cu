@@ -91,7 +91,7 @@ __device__ __forceinline__ uint64_t operand_desc(uint32_t base, int mn_major, in
 }
 
 template <int EPI, int NST>
-__global__ void __launch_bounds__(kGemmThreads)
+__global__ void __launch_bounds__(kGemmThreads, (NST == 2 && EPI != kEpiStoreF32) ? 3 : 2)
 sa_gemm_kernel(const __grid_constant__ GemmParams p) {
   constexpr int kStages = NST;
   extern __shared__ uint8_t smem_raw[];
@@ -102,11 +102,15 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   int* status = const_cast<int*>(&p.hdr->status);
 
-  // ---- which output tile
+  // ---- which output tile: blockIdx.x = m_tile * n_tiles + n_tile, so the n_tiles CTAs
+  // that share one block of A rows run together and read it from DRAM once (L2 after)
+  const unsigned n_tiles = (unsigned)(p.N + kBN - 1) / kBN;
+  const int n_tile = (int)(blockIdx.x % n_tiles);
+  const long long m_tile = (long long)(blockIdx.x / n_tiles);
   int row0 = 0, nrows = 0, user = 0;
   if (p.user_mode) {
     const long long T = p.hdr->total_tiles;
-    const long long g = blockIdx.x;
+    const long long g = m_tile;
     if (g >= T || read_status(status) != 0) return;
     user = user_of_tile(p.tile_start, p.R, g);
     const long long local = g - p.tile_start[user];
@@ -114,13 +118,13 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
     const long long n = p.offsets[user + 1] - row0;
     nrows = n >= kBM ? kBM : (int)n;
   } else {
-    row0 = blockIdx.x * kBM;
+    row0 = (int)(m_tile * kBM);
     nrows = min(kBM, p.M - row0);
     if (nrows <= 0) return;
   }
-  const int n0 = blockIdx.y * kBN;
-  // K tiles of this CTA: phase 0 is split evenly across gridDim.z; phase 1 is not split
-  const int z = blockIdx.z;
+  const int n0 = n_tile * kBN;
+  // K tiles of this CTA: phase 0 is split evenly across gridDim.y; phase 1 is not split
+  const int z = blockIdx.y;
   const int kt0 = (int)((long long)p.k_tiles[0] * z / p.splits);
   const int kt1 = (int)((long long)p.k_tiles[0] * (z + 1) / p.splits);
   const int total_kt = (kt1 - kt0) + (p.phases > 1 ? p.k_tiles[1] : 0);
@@ -331,10 +335,10 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
         }
       }
       if (EPI == kEpiLse && valid)
-        p.dpart[row * p.dpart_ld + 2 * blockIdx.y + half] =
+        p.dpart[row * p.dpart_ld + 2 * n_tile + half] =
             lmax > -INFINITY ? lmax + lg2_approx(lsum) : -INFINITY;
       if (EPI == kEpiAExp && valid && p.c_user != nullptr)
-        p.dpart[row * p.dpart_ld + 2 * blockIdx.y + half] = csum;
+        p.dpart[row * p.dpart_ld + 2 * n_tile + half] = csum;
     }
   }
   tc_fence_before();
@@ -417,7 +421,9 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.ld_add = g.ld_add;
   p.drow = g.drow;
   p.budget = kDefaultWaitBudget;
-  const dim3 grid((unsigned)g.m_tiles_bound, (unsigned)((g.N + kBN - 1) / kBN), (unsigned)p.splits);
+  const long long tiles = (long long)g.m_tiles_bound * ((g.N + kBN - 1) / kBN);
+  if (tiles > 0x7FFFFFFFLL || p.splits > 65535) return cudaErrorInvalidValue;
+  const dim3 grid((unsigned)tiles, (unsigned)p.splits);
   if (grid.x == 0) return cudaSuccess;
   switch (g.epi) {
     case kEpiStoreF32: return launch_t<kEpiStoreF32>(p, grid, s);
