@@ -138,9 +138,50 @@ def _dt(x: torch.Tensor) -> int:
     raise TypeError(f"X must be bfloat16 or float32, got {x.dtype}")
 
 
-def _stream(stream) -> int:
-    s = torch.cuda.current_stream() if stream is None else stream
+def _stream(stream, device=None) -> int:
+    s = torch.cuda.current_stream(device) if stream is None else stream
     return s.cuda_stream
+
+
+def _require(cond: bool, where: str, what: str) -> None:
+    if not cond:
+        raise SketchAttentionError(SA_ERR_INVALID_ARG, f"{where}: {what}")
+
+
+def _check_tensor(where: str, name: str, t: torch.Tensor | None, shape: tuple, dtype,
+                  device=None, optional: bool = False) -> None:
+    """The C ABI sees only a pointer: shape, dtype, memory layout and device are the
+    caller's promise, so the torch conveniences check them here."""
+    if t is None:
+        _require(optional, where, f"{name} is required")
+        return
+    _require(isinstance(t, torch.Tensor), where, f"{name} must be a tensor")
+    _require(tuple(t.shape) == tuple(shape), where,
+             f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+    _require(t.dtype == dtype, where, f"{name} has dtype {t.dtype}, expected {dtype}")
+    _require(t.is_contiguous(), where, f"{name} must be contiguous")
+    if device is not None:
+        _require(t.device == device, where, f"{name} is on {t.device}, expected {device}")
+
+
+def _check_cuda(where: str, X: torch.Tensor) -> None:
+    _require(X.is_cuda, where, f"inputs are on {X.device}; the library runs on CUDA devices only")
+
+
+def _check_forward_inputs(where, X, offsets, P, Wk, Wv):
+    _require(isinstance(X, torch.Tensor) and X.dim() == 2, where, "X must be a 2-D tensor")
+    _require(isinstance(P, torch.Tensor) and P.dim() == 2, where, "P must be a 2-D tensor")
+    _require(isinstance(offsets, torch.Tensor) and offsets.dim() == 1 and offsets.numel() >= 1,
+             where, "offsets must be a 1-D tensor with R + 1 entries")
+    n_total, d = X.shape
+    k = P.shape[0]
+    _dt(X)
+    dev = X.device
+    _check_tensor(where, "X", X, (n_total, d), X.dtype, dev)
+    _check_tensor(where, "offsets", offsets, (offsets.numel(),), torch.int64, dev)
+    _check_tensor(where, "P", P, (k, d), X.dtype, dev)
+    _check_tensor(where, "Wk", Wk, (d, d), X.dtype, dev)
+    _check_tensor(where, "Wv", Wv, (d, d), X.dtype, dev)
 
 
 def workspace(R: int, n_total: int, k: int, d: int, dtype: torch.dtype, backward: bool = False,
@@ -159,8 +200,11 @@ def forward(X: torch.Tensor, offsets: torch.Tensor, P: torch.Tensor, Wk: torch.T
     """Sketch Attention forward on the GPU. Returns sketch, mass (and lse, xsketch).
 
     X [n_total, d] bf16/fp32, offsets [R+1] int64, P [k, d], Wk, Wv [d, d] (same dtype
-    as X), all contiguous on one CUDA device.
+    as X), all contiguous on one CUDA device. `out`, if given, holds fp32 sketch [R, k, d]
+    and mass [R, k], and optionally lse [n_total] and xsketch [R, k, d].
     """
+    where = "forward"
+    _check_forward_inputs(where, X, offsets, P, Wk, Wv)
     n_total, d = X.shape
     k = P.shape[0]
     R = offsets.shape[0] - 1
@@ -173,11 +217,21 @@ def forward(X: torch.Tensor, offsets: torch.Tensor, P: torch.Tensor, Wk: torch.T
             out["lse"] = torch.empty(n_total, device=dev, dtype=torch.float32)
         if want_xsketch:
             out["xsketch"] = torch.empty(R, k, d, device=dev, dtype=torch.float32)
-    if ws is None:
-        ws = workspace(R, n_total, k, d, X.dtype, False, dev)
-    st = sa_sketch_forward(_ptr(X), _ptr(offsets), R, n_total, d, _ptr(P), k, _ptr(Wk), _ptr(Wv),
-                           dt, _ptr(out["sketch"]), _ptr(out["mass"]), _ptr(out.get("lse")),
-                           _ptr(out.get("xsketch")), _ptr(ws), ws.numel(), _stream(stream))
+    f32 = torch.float32
+    _check_tensor(where, "sketch", out.get("sketch"), (R, k, d), f32, dev)
+    _check_tensor(where, "mass", out.get("mass"), (R, k), f32, dev)
+    _check_tensor(where, "lse", out.get("lse"), (n_total,), f32, dev, optional=True)
+    _check_tensor(where, "xsketch", out.get("xsketch"), (R, k, d), f32, dev, optional=True)
+    _check_cuda(where, X)
+    with torch.cuda.device(dev):
+        if ws is None:
+            ws = workspace(R, n_total, k, d, X.dtype, False, dev)
+        _require(ws.device == dev and ws.is_contiguous(), where,
+                 "ws must be contiguous on X's device")
+        st = sa_sketch_forward(_ptr(X), _ptr(offsets), R, n_total, d, _ptr(P), k, _ptr(Wk),
+                               _ptr(Wv), dt, _ptr(out["sketch"]), _ptr(out["mass"]),
+                               _ptr(out.get("lse")), _ptr(out.get("xsketch")), _ptr(ws),
+                               ws.nbytes, _stream(stream, dev))
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_sketch_forward")
     out["_ws"] = ws
@@ -186,23 +240,39 @@ def forward(X: torch.Tensor, offsets: torch.Tensor, P: torch.Tensor, Wk: torch.T
 
 def backward(X, offsets, P, Wk, Wv, fwd: dict, dsketch: torch.Tensor, dmass=None, *,
              ws: torch.Tensor | None = None, stream=None) -> dict:
-    """Gradients dX, dP, dWk, dWv given dL/dsketch (and optionally dL/dmass)."""
+    """Gradients dX, dP, dWk, dWv given dL/dsketch (and optionally dL/dmass).
+
+    `fwd` holds the forward's fp32 sketch [R, k, d], mass [R, k] and xsketch [R, k, d]
+    (lse [n_total] optional); dsketch [R, k, d] and dmass [R, k] are fp32."""
+    where = "backward"
+    _check_forward_inputs(where, X, offsets, P, Wk, Wv)
     n_total, d = X.shape
     k = P.shape[0]
     R = offsets.shape[0] - 1
     dt = _dt(X)
     dev = X.device
-    out = {"dX": torch.empty(n_total, d, device=dev, dtype=torch.float32),
-           "dP": torch.empty(k, d, device=dev, dtype=torch.float32),
-           "dWk": torch.empty(d, d, device=dev, dtype=torch.float32),
-           "dWv": torch.empty(d, d, device=dev, dtype=torch.float32)}
-    if ws is None:
-        ws = workspace(R, n_total, k, d, X.dtype, True, dev)
-    st = sa_sketch_backward(_ptr(X), _ptr(offsets), R, n_total, d, _ptr(P), k, _ptr(Wk), _ptr(Wv),
-                            dt, _ptr(fwd["sketch"]), _ptr(fwd["mass"]), _ptr(fwd.get("lse")),
-                            _ptr(fwd["xsketch"]), _ptr(dsketch), _ptr(dmass), _ptr(out["dX"]),
-                            _ptr(out["dP"]), _ptr(out["dWk"]), _ptr(out["dWv"]), _ptr(ws),
-                            ws.numel(), _stream(stream))
+    f32 = torch.float32
+    _check_tensor(where, "sketch", fwd.get("sketch"), (R, k, d), f32, dev)
+    _check_tensor(where, "mass", fwd.get("mass"), (R, k), f32, dev)
+    _check_tensor(where, "xsketch", fwd.get("xsketch"), (R, k, d), f32, dev)
+    _check_tensor(where, "lse", fwd.get("lse"), (n_total,), f32, dev, optional=True)
+    _check_tensor(where, "dsketch", dsketch, (R, k, d), f32, dev)
+    _check_tensor(where, "dmass", dmass, (R, k), f32, dev, optional=True)
+    _check_cuda(where, X)
+    out = {"dX": torch.empty(n_total, d, device=dev, dtype=f32),
+           "dP": torch.empty(k, d, device=dev, dtype=f32),
+           "dWk": torch.empty(d, d, device=dev, dtype=f32),
+           "dWv": torch.empty(d, d, device=dev, dtype=f32)}
+    with torch.cuda.device(dev):
+        if ws is None:
+            ws = workspace(R, n_total, k, d, X.dtype, True, dev)
+        _require(ws.device == dev and ws.is_contiguous(), where,
+                 "ws must be contiguous on X's device")
+        st = sa_sketch_backward(_ptr(X), _ptr(offsets), R, n_total, d, _ptr(P), k, _ptr(Wk),
+                                _ptr(Wv), dt, _ptr(fwd["sketch"]), _ptr(fwd["mass"]),
+                                _ptr(fwd.get("lse")), _ptr(fwd["xsketch"]), _ptr(dsketch),
+                                _ptr(dmass), _ptr(out["dX"]), _ptr(out["dP"]), _ptr(out["dWk"]),
+                                _ptr(out["dWv"]), _ptr(ws), ws.nbytes, _stream(stream, dev))
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_sketch_backward")
     out["_ws"] = ws
@@ -214,11 +284,24 @@ def combine(xsketch: torch.Tensor, mass: torch.Tensor, Wv: torch.Tensor, *,
     """sketch = (xsketch Wv) / mass for users whose partial xsketch and mass (from
     forward calls over parts of their tokens) have been summed. xsketch [R, k, d] and
     mass [R, k] fp32, Wv [d, d] bf16/fp32, all on one CUDA device."""
+    where = "combine"
+    _require(isinstance(xsketch, torch.Tensor) and xsketch.dim() == 3, where,
+             "xsketch must be a 3-D tensor")
     R, k, d = xsketch.shape
+    dev = xsketch.device
+    f32 = torch.float32
+    _check_tensor(where, "xsketch", xsketch, (R, k, d), f32, dev)
+    _check_tensor(where, "mass", mass, (R, k), f32, dev)
+    _require(isinstance(Wv, torch.Tensor), where, "Wv must be a tensor")
+    _check_tensor(where, "Wv", Wv, (d, d), Wv.dtype, dev)
+    dt = _dt(Wv)
     if out is None:
-        out = torch.empty(R, k, d, device=xsketch.device, dtype=torch.float32)
-    st = sa_sketch_combine(_ptr(xsketch), _ptr(mass), R, k, d, _ptr(Wv), _dt(Wv), _ptr(out),
-                           _stream(stream))
+        out = torch.empty(R, k, d, device=dev, dtype=f32)
+    _check_tensor(where, "out", out, (R, k, d), f32, dev)
+    _check_cuda(where, xsketch)
+    with torch.cuda.device(dev):
+        st = sa_sketch_combine(_ptr(xsketch), _ptr(mass), R, k, d, _ptr(Wv), dt, _ptr(out),
+                               _stream(stream, dev))
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_sketch_combine")
     return out
@@ -258,7 +341,16 @@ def forward_from_host(Xh: torch.Tensor, offsets_h: torch.Tensor, P: torch.Tensor
     independent, so no combining). P, Wk, Wv live on the device. `state` (a dict the
     caller keeps) holds the device buffers, pinned staging and streams between calls.
     The current stream waits for the copies back before this returns, so work queued on
-    it afterwards (an event, a synchronize) sees the outputs."""
+    it afterwards (an event, a synchronize) sees the outputs. The returned host tensors
+    are the state's staging: the next call with the same `state` overwrites them."""
+    where = "forward_from_host"
+    _require(isinstance(Xh, torch.Tensor) and Xh.dim() == 2 and Xh.device.type == "cpu"
+             and Xh.is_contiguous(), where, "Xh must be a contiguous 2-D host tensor")
+    _require(isinstance(offsets_h, torch.Tensor) and offsets_h.dim() == 1
+             and offsets_h.numel() >= 1 and offsets_h.dtype == torch.int64
+             and offsets_h.device.type == "cpu", where, "offsets_h must be host int64 [R + 1]")
+    _require(isinstance(P, torch.Tensor) and P.is_cuda, where, "P, Wk, Wv must be on the GPU")
+    _require(int(chunks) >= 1, where, "chunks must be at least 1")
     R = offsets_h.numel() - 1
     n_total, d = Xh.shape
     k = P.shape[0]
