@@ -11,6 +11,12 @@ mean). Sources: the "100,000 videos in your pocket" blog, section "1. Sketch
 Attention compresses the history"; the evolve.pub review of arXiv 2609.08443,
 "Summary" and the FAQ on how Sketch Attention differs from standard attention.
 
+``stca_forward`` / ``stca_backward`` (``stca_oracle.cpp``) are the candidate-to-sketch
+cross attention that reads the sketch (the sketch branch of STCA, one sketch read per
+user for all of its candidates): blog sections "2. STCA reasons at two time scales" and
+"3. The system makes it cheap enough to matter". They are pinned by
+``tests/test_oracle_stca_pins.py``.
+
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, invariants, brute force at 50 digits, autograd and finite
 differences for the backward). The paper's analytic FLOP ratios (49.9x, 63.9x)
@@ -28,19 +34,28 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "sa_oracle.cpp")
 _LIB = os.path.join(_HERE, "libsa_oracle.so")
+_STCA_SRC = os.path.join(_HERE, "stca_oracle.cpp")
+_STCA_LIB = os.path.join(_HERE, "libstca_oracle.so")
 _lock = threading.Lock()
 _lib = None
+_stca_lib = None
+
+
+def _build_one(src: str, lib: str, force: bool) -> str:
+    if not force and os.path.exists(lib) and os.path.getmtime(lib) >= os.path.getmtime(src):
+        return lib
+    tmp = lib + f".tmp{os.getpid()}"
+    cmd = ["g++", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c++17", "-o", tmp, src]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, lib)
+    return lib
 
 
 def build(force: bool = False) -> str:
-    """Compile the oracle with g++ (OpenMP). Returns the path of the shared object."""
-    if not force and os.path.exists(_LIB) and os.path.getmtime(_LIB) >= os.path.getmtime(_SRC):
-        return _LIB
-    tmp = _LIB + f".tmp{os.getpid()}"
-    cmd = ["g++", "-O3", "-fopenmp", "-fPIC", "-shared", "-std=c++17", "-o", tmp, _SRC]
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, _LIB)
-    return _LIB
+    """Compile the oracles with g++ (OpenMP). Returns the path of the Sketch Attention
+    oracle's shared object (the cross-attention oracle is built beside it)."""
+    _build_one(_STCA_SRC, _STCA_LIB, force)
+    return _build_one(_SRC, _LIB, force)
 
 
 def _load():
@@ -60,6 +75,26 @@ def _load():
                                                dp, dp, dp, dp, ctypes.c_int]
             _lib = lib
     return _lib
+
+
+def _load_stca():
+    global _stca_lib
+    with _lock:
+        if _stca_lib is None:
+            # STCA_ORACLE_LIB lets the mutation test load a deliberately broken build.
+            path = os.environ.get("STCA_ORACLE_LIB") or _build_one(_STCA_SRC, _STCA_LIB, False)
+            lib = ctypes.CDLL(path)
+            dp = ctypes.POINTER(ctypes.c_double)
+            ip = ctypes.POINTER(ctypes.c_int64)
+            i32, i64 = ctypes.c_int, ctypes.c_int64
+            lib.stca_oracle_forward.restype = i32
+            lib.stca_oracle_forward.argtypes = [dp, ip, i32, i64, i32, dp, i32, dp, dp, dp,
+                                                dp, dp, i32]
+            lib.stca_oracle_backward.restype = i32
+            lib.stca_oracle_backward.argtypes = [dp, ip, i32, i64, i32, dp, i32, dp, dp, dp,
+                                                 dp, dp, dp, dp, dp, dp, i32]
+            _stca_lib = lib
+    return _stca_lib
 
 
 def _f64(a) -> np.ndarray:
@@ -129,3 +164,49 @@ def backward(X, offsets, P, Wk, Wv, dsketch, dmass=None, nthreads: int = 0) -> d
                                     _ptr(dWk), _ptr(dWv), int(nthreads))
     _check_rc(rc)
     return {"dX": dX, "dP": dP, "dWk": dWk, "dWv": dWv}
+
+
+def _stca_args(Q, cand_offsets, S, Wq, WK, WV):
+    Q, S = _f64(Q), _f64(S)
+    Wq, WK, WV = _f64(Wq), _f64(WK), _f64(WV)
+    off = np.ascontiguousarray(np.asarray(cand_offsets, dtype=np.int64))
+    n_cand, d = Q.shape
+    R = off.shape[0] - 1
+    assert S.ndim == 3 and S.shape[0] == R and S.shape[2] == d
+    assert Wq.shape == (d, d) and WK.shape == (d, d) and WV.shape == (d, d)
+    return Q, off, S, Wq, WK, WV, n_cand, d, R, S.shape[1]
+
+
+def stca_forward(Q, cand_offsets, S, Wq, WK, WV, nthreads: int = 0) -> dict:
+    """Candidate-to-sketch cross attention in fp64.
+
+    Q [n_cand, d] candidates (users' groups concatenated), cand_offsets [R+1] (int64),
+    S [R, k, d] the users' sketches, Wq, WK, WV [d, d]. Returns out [n_cand, d] and
+    lse [n_cand] (the log-sum-exp of each candidate's scores over the k rows).
+    """
+    Q, off, S, Wq, WK, WV, n_cand, d, R, k = _stca_args(Q, cand_offsets, S, Wq, WK, WV)
+    out = np.zeros((n_cand, d))
+    lse = np.zeros(n_cand)
+    rc = _load_stca().stca_oracle_forward(_ptr(Q), _ptr(off, ctypes.c_int64), R, n_cand, d,
+                                          _ptr(S), k, _ptr(Wq), _ptr(WK), _ptr(WV), _ptr(out),
+                                          _ptr(lse), int(nthreads))
+    _check_rc(rc)
+    return {"out": out, "lse": lse}
+
+
+def stca_backward(Q, cand_offsets, S, Wq, WK, WV, dout, nthreads: int = 0) -> dict:
+    """Gradients given dL/dout [n_cand, d]: dQ [n_cand, d], dS [R, k, d] (what flows into
+    each user's sketch, i.e. Sketch Attention's dL/dsketch) and dWq, dWK, dWV [d, d]
+    summed over users."""
+    Q, off, S, Wq, WK, WV, n_cand, d, R, k = _stca_args(Q, cand_offsets, S, Wq, WK, WV)
+    G = _f64(dout)
+    assert G.shape == (n_cand, d)
+    dQ = np.zeros((n_cand, d))
+    dS = np.zeros((R, k, d))
+    dWq, dWK, dWV = np.zeros((d, d)), np.zeros((d, d)), np.zeros((d, d))
+    rc = _load_stca().stca_oracle_backward(_ptr(Q), _ptr(off, ctypes.c_int64), R, n_cand, d,
+                                           _ptr(S), k, _ptr(Wq), _ptr(WK), _ptr(WV), _ptr(G),
+                                           _ptr(dQ), _ptr(dS), _ptr(dWq), _ptr(dWK), _ptr(dWV),
+                                           int(nthreads))
+    _check_rc(rc)
+    return {"dQ": dQ, "dS": dS, "dWq": dWq, "dWK": dWK, "dWV": dWV}
