@@ -19,6 +19,8 @@ The JSON line also carries:
                 with the per-step H2D of X and offsets and the D2H of sketch and mass
   cpu_baseline  the fp64 oracle on the host cores, on a bounded sample (rank 0, N=1)
   clocks        SM clock median and throttle reasons sampled during the timed region
+  other_workloads  (one GPU) the forward on one 100K-token user and on 40 users of 100K
+                tokens each: step and kernel times, kernel fraction of the bf16 peak
 `--impl reference` times the oracle (the reference arm here) on the same config.
 """
 from __future__ import annotations
@@ -202,6 +204,64 @@ def oracle_sample_rate(w, target_s: float, max_tokens: int = 2_000_000):
     return S / t, S, t, used, users
 
 
+# ------------------------------------------------------------------ other workloads
+OTHER_WORKLOADS = (
+    (2, "1 user, n=100,000, d=128, k=1024, bf16 in / fp32 accumulate, forward"),
+    (5, "R=40 users x n=100,000, d=128, k=1024, bf16 in / fp32 accumulate, forward"),
+)
+
+
+def time_other_workloads(binding, inputs, dev, steps: int, peak: float) -> list:
+    """The single user of 100K tokens and the 40 x 100K batch, each timed like the main
+    workload (kernel events from the library, step events around each call) with a
+    256 MB L2 flush between steps outside the timed events. Reported beside the
+    headline; a failure here is reported, not raised."""
+    import torch
+    out = []
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    for idx, desc in OTHER_WORKLOADS:
+        try:
+            w = inputs.make_config(idx, with_grad=False)
+            X, off = w.X.to(dev), w.offsets.to(dev)
+            P, Wk, Wv = w.P.to(dev), w.Wk.to(dev), w.Wv.to(dev)
+            o = binding.forward(X, off, P, Wk, Wv, want_lse=False, want_xsketch=False)
+            for _ in range(3):
+                binding.forward(X, off, P, Wk, Wv, ws=o["_ws"], out=o)
+            torch.cuda.synchronize()
+            stream = torch.cuda.current_stream()
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(steps)]
+            for e4 in ev:  # materialise the CUDA events before the library records them
+                for e in e4:
+                    e.record(stream)
+            torch.cuda.synchronize()
+            for e4 in ev:
+                flush.zero_()
+                e4[0].record(stream)
+                binding.sa_sketch_profile_events(e4[2].cuda_event, e4[3].cuda_event)
+                binding.forward(X, off, P, Wk, Wv, ws=o["_ws"], out=o)
+                e4[1].record(stream)
+            torch.cuda.synchronize()
+            binding.sa_sketch_profile_events(None, None)
+            st = binding.device_status(o["_ws"])
+            if st != 0:
+                raise RuntimeError(binding.sa_status_string(st))
+            step_ms = sum(e4[0].elapsed_time(e4[1]) for e4 in ev) / steps
+            kern_ms = sum(event_ms(e4[2], e4[3]) for e4 in ev) / steps
+            n = w.n_total
+            achieved = 4.0 * w.k * w.d * n / (kern_ms / 1e3) / 1e12
+            out.append({"workload": desc, "n_total": n, "steps": steps,
+                        "ms_per_step": step_ms, "tokens_per_s": n / (step_ms / 1e3),
+                        "kernel_ms": kern_ms, "kernel_tflops": achieved,
+                        "kernel_frac": achieved / peak, "l2": "256 MB flush between steps"})
+            del X, off, P, Wk, Wv, o
+        except Exception as e:  # reported beside the headline, never fatal to it
+            binding.sa_sketch_profile_events(None, None)
+            out.append({"workload": desc, "error": repr(e)[:300]})
+    del flush
+    torch.cuda.synchronize()
+    return out
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
@@ -377,6 +437,10 @@ def run_ours(args) -> None:
     h2d = X.numel() * X.element_size() + off.numel() * 8
     d2h = R * k * d * 4 + R * k * 4  # sketch and mass back to the host
 
+    others = None
+    if world == 1 and not args.no_other_workloads:
+        others = time_other_workloads(binding, inputs, dev, max(3, min(args.steps, 50)), peak)
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         rate, S, secs, used, users = oracle_sample_rate(w, args.cpu_seconds)
@@ -413,6 +477,8 @@ def run_ours(args) -> None:
         line["cpu_baseline"] = cpu
     if bwd is not None and world == 1:
         line["backward"] = bwd
+    if others is not None:
+        line["other_workloads"] = others
     print(json.dumps(line), flush=True)
 
 
@@ -424,6 +490,8 @@ def main(argv=None) -> int:
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
+    ap.add_argument("--no-other-workloads", action="store_true",
+                    help="skip the 1 x 100K and 40 x 100K forward timings")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
