@@ -192,3 +192,47 @@ def test_sharded_backward_feeds_cut_users_whole_statistics():
     # the parts' own xsketch add up to the user's
     tot = sum(o["part_xsketch"][o["part_users"] == 2].sum(0) for o in outs)
     np.testing.assert_allclose(tot, ref["xsketch"][2], rtol=1e-12, atol=1e-12)
+
+
+# ---------------------------------------------------------------- failure detection
+def _absent_rank_worker(rank, world, port, outdir):
+    """Rank 1 fails before the forward (it never joins the cut user's all-reduce); rank 0
+    must leave the collective with an error once the process group's timeout runs out,
+    instead of waiting for ever. Rank 1 stays alive (holding its connection) until rank 0
+    has reported, so the error rank 0 sees is the timeout, not a closed socket."""
+    import datetime
+    import time
+    dist.init_process_group("gloo", init_method=f"tcp://127.0.0.1:{port}", rank=rank,
+                            world_size=world, timeout=datetime.timedelta(seconds=3))
+    flag = os.path.join(outdir, "rank0_done")
+    try:
+        if rank == 1:
+            deadline = time.monotonic() + 60.0
+            while not os.path.exists(flag) and time.monotonic() < deadline:
+                time.sleep(0.05)
+            return
+        w, f = _workload(CUT)
+        plan = plan_shards(CUT[0], world, CUT[3])
+        t = {n: torch.from_numpy(np.ascontiguousarray(f[n])) for n in ("X", "P", "Wk", "Wv")}
+        Xl = t["X"][torch.from_numpy(plan.local_rows(rank))].contiguous()
+        t0 = time.monotonic()
+        try:
+            sharded_forward(plan, rank, Xl, t["P"], t["Wk"], t["Wv"],
+                            forward_fn=_oracle_forward, combine_fn=_combine)
+            status = "no error"
+        except RuntimeError as e:
+            status = "error: " + str(e)[:200]
+        with open(os.path.join(outdir, "rank0.txt"), "w") as fh:
+            fh.write(f"{time.monotonic() - t0:.3f}\n{status}\n")
+        open(flag, "w").close()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_absent_rank_ends_the_collective_with_an_error():
+    assert plan_shards(CUT[0], 2, CUT[3]).split_users(), "the case must need an all-reduce"
+    with tempfile.TemporaryDirectory() as outdir:
+        mp.spawn(_absent_rank_worker, args=(2, _free_port(), outdir), nprocs=2, join=True)
+        secs, status = open(os.path.join(outdir, "rank0.txt")).read().splitlines()[:2]
+    assert status.startswith("error"), status
+    assert float(secs) < 30.0, secs
