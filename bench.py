@@ -184,24 +184,46 @@ def oracle_sample(w, S: int):
             w.Wv.double().numpy())
 
 
-def oracle_sample_rate(w, target_s: float, max_tokens: int = 2_000_000):
+def oracle_sample_rate(w, target_s: float, max_tokens: int = 2_000_000, keep: dict | None = None):
     """Times the fp64 oracle on the first S tokens of the batch (S sized for ~target_s of
-    wall time). Returns (tokens/s, tokens, seconds, threads, users)."""
+    wall time). Returns (tokens/s, tokens, seconds, threads, users); `keep`, if given,
+    receives the timed run's outputs and sample offsets."""
     import oracle
     threads = os.cpu_count() or 1
 
     def run(S):
         X, off, P, Wk, Wv = oracle_sample(w, S)
         t0 = time.perf_counter()
-        oracle.forward(X, off, P, Wk, Wv, nthreads=threads)
-        return time.perf_counter() - t0, len(off) - 1
+        res = oracle.forward(X, off, P, Wk, Wv, nthreads=threads)
+        return time.perf_counter() - t0, len(off) - 1, res, off
 
     probe = 8192
-    tp, _ = run(probe)
+    tp = run(probe)[0]
     S = int(min(w.n_total, max_tokens, max(probe, probe * target_s / max(tp, 1e-6))))
-    t, users = run(S)
+    t, users, res, off = run(S)
+    if keep is not None:
+        keep.update(res=res, off=off)
     used = min(threads, math.ceil(S / 1024))  # the oracle parallelises over 1024-token chunks
     return S / t, S, t, used, users
+
+
+def sampled_parity(w, gpu_out: dict, keep: dict) -> dict:
+    """The GPU forward's sketch and mass against the oracle's, on the users that lie
+    wholly inside the oracle's timed sample (relative L2 and max |error| per user)."""
+    import numpy as np
+    off = w.offsets.numpy()
+    whole = [u for u in range(len(keep["off"]) - 1) if off[u + 1] <= keep["off"][-1]]
+    if not whole:
+        return {"users": []}
+    sk = gpu_out["sketch"][whole].double().cpu().numpy()
+    ms = gpu_out["mass"][whole].double().cpu().numpy()
+    rs, rm = keep["res"]["sketch"][whole], keep["res"]["mass"][whole]
+    rel = lambda a, b: float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+    return {"users": whole,
+            "sketch_rel_l2_max": max(rel(sk[i], rs[i]) for i in range(len(whole))),
+            "sketch_max_abs": float(np.abs(sk - rs).max()),
+            "mass_rel_l2_max": max(rel(ms[i], rm[i]) for i in range(len(whole))),
+            "tolerance": {"rel_l2": 1e-2, "max_abs": 5e-2}}
 
 
 # ------------------------------------------------------------------ other workloads
@@ -443,10 +465,15 @@ def run_ours(args) -> None:
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, S, secs, used, users = oracle_sample_rate(w, args.cpu_seconds)
+        keep = {}
+        rate, S, secs, used, users = oracle_sample_rate(w, args.cpu_seconds, keep=keep)
         cpu = {"value": rate, "unit": UNIT, "cores": used, "kind": "oracle",
                "sample": f"first {S} tokens of config 3 ({users} users; k=1024, d=128), "
                          f"fp64 oracle, {secs:.1f} s wall"}
+        try:  # the same oracle run checks the timed forward's output on those users
+            cpu["parity_sampled"] = sampled_parity(w, out, keep)
+        except Exception as e:
+            cpu["parity_sampled"] = {"error": repr(e)[:300]}
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
