@@ -72,6 +72,18 @@ def measured_peak():
         return FALLBACK_PEAK_TFLOPS, "fallback (1.59 PFLOP/s, profiling recipe)"
 
 
+DATASHEET_BF16_TFLOPS = 2250.0  # B200 dense bf16, for context beside the measured peak
+
+
+def sustained_peak():
+    """The measured bf16 GEMM rate held for seconds under the power cap (None if absent)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops_sustained"])
+    except Exception:
+        return None
+
+
 def profiled_traffic():
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current kernel source (null otherwise)."""
@@ -492,7 +504,10 @@ def run_ours(args) -> None:
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(),
                      "kernel": "sa_fwd_sm100_kernel<128>", "kernel_ms": kern_ms,
-                     "peak_source": peak_src, "flop_per_launch": flop_per_launch},
+                     "peak_source": peak_src, "flop_per_launch": flop_per_launch,
+                     "frac_of_sustained": (achieved / sustained_peak()
+                                           if sustained_peak() else None),
+                     "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
         "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
         # per forward: schedule, fold, the tcgen05 kernel, then the finalize (segment sums
