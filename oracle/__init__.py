@@ -93,6 +93,12 @@ def _load_stca():
             lib.stca_oracle_backward.restype = i32
             lib.stca_oracle_backward.argtypes = [dp, ip, i32, i64, i32, dp, i32, dp, dp, dp,
                                                  dp, dp, dp, dp, dp, dp, i32]
+            lib.stca_oracle_forward_keys.restype = i32
+            lib.stca_oracle_forward_keys.argtypes = [dp, ip, i32, i64, i32, dp, ip, i64, dp, dp,
+                                                     dp, dp, dp, i32]
+            lib.stca_oracle_backward_keys.restype = i32
+            lib.stca_oracle_backward_keys.argtypes = [dp, ip, i32, i64, i32, dp, ip, i64, dp, dp,
+                                                      dp, dp, dp, dp, dp, dp, dp, i32]
             _stca_lib = lib
     return _stca_lib
 
@@ -210,3 +216,62 @@ def stca_backward(Q, cand_offsets, S, Wq, WK, WV, dout, nthreads: int = 0) -> di
                                            int(nthreads))
     _check_rc(rc)
     return {"dQ": dQ, "dS": dS, "dWq": dWq, "dWK": dWK, "dWV": dWV}
+
+
+def _keys_args(Q, cand_offsets, Kx, key_offsets, Wq, WK, WV):
+    Q, Kx = _f64(Q), _f64(Kx)
+    Wq, WK, WV = _f64(Wq), _f64(WK), _f64(WV)
+    coff = np.ascontiguousarray(np.asarray(cand_offsets, dtype=np.int64))
+    koff = np.ascontiguousarray(np.asarray(key_offsets, dtype=np.int64))
+    n_cand, d = Q.shape
+    R = coff.shape[0] - 1
+    assert koff.shape == (R + 1,) and Kx.ndim == 2 and Kx.shape[1] == d
+    assert Wq.shape == (d, d) and WK.shape == (d, d) and WV.shape == (d, d)
+    return Q, coff, Kx, koff, Wq, WK, WV, n_cand, d, R
+
+
+def stca_forward_keys(Q, cand_offsets, Kx, key_offsets, Wq, WK, WV, nthreads: int = 0) -> dict:
+    """Cross attention with ragged key rows: user u's candidates attend over
+    Kx[key_offsets[u]:key_offsets[u+1]]. A user with candidates but no key rows gets
+    out = 0 and lse = -inf."""
+    Q, coff, Kx, koff, Wq, WK, WV, n_cand, d, R = _keys_args(Q, cand_offsets, Kx, key_offsets,
+                                                             Wq, WK, WV)
+    out = np.zeros((n_cand, d))
+    lse = np.zeros(n_cand)
+    rc = _load_stca().stca_oracle_forward_keys(
+        _ptr(Q), _ptr(coff, ctypes.c_int64), R, n_cand, d, _ptr(Kx), _ptr(koff, ctypes.c_int64),
+        Kx.shape[0], _ptr(Wq), _ptr(WK), _ptr(WV), _ptr(out), _ptr(lse), int(nthreads))
+    _check_rc(rc)
+    return {"out": out, "lse": lse}
+
+
+def stca_backward_keys(Q, cand_offsets, Kx, key_offsets, Wq, WK, WV, dout,
+                       nthreads: int = 0) -> dict:
+    """Gradients of stca_forward_keys given dL/dout: dQ, dKx [n_keys, d], dWq, dWK, dWV."""
+    Q, coff, Kx, koff, Wq, WK, WV, n_cand, d, R = _keys_args(Q, cand_offsets, Kx, key_offsets,
+                                                             Wq, WK, WV)
+    G = _f64(dout)
+    assert G.shape == (n_cand, d)
+    dQ = np.zeros((n_cand, d))
+    dK = np.zeros(Kx.shape)
+    dWq, dWK, dWV = np.zeros((d, d)), np.zeros((d, d)), np.zeros((d, d))
+    rc = _load_stca().stca_oracle_backward_keys(
+        _ptr(Q), _ptr(coff, ctypes.c_int64), R, n_cand, d, _ptr(Kx), _ptr(koff, ctypes.c_int64),
+        Kx.shape[0], _ptr(Wq), _ptr(WK), _ptr(WV), _ptr(G), _ptr(dQ), _ptr(dK), _ptr(dWq),
+        _ptr(dWK), _ptr(dWV), int(nthreads))
+    _check_rc(rc)
+    return {"dQ": dQ, "dKx": dK, "dWq": dWq, "dWK": dWK, "dWV": dWV}
+
+
+def recent_suffix(X, offsets, L: int):
+    """The recent branch's key rows: the last min(n_u, L) tokens of every user's history,
+    concatenated, with their offsets (row selection only)."""
+    X = np.asarray(X)
+    off = np.asarray(offsets, dtype=np.int64)
+    rows, koff = [], [0]
+    for u in range(len(off) - 1):
+        a, b = int(off[u]), int(off[u + 1])
+        rows.append(np.arange(max(a, b - L), b, dtype=np.int64))
+        koff.append(koff[-1] + len(rows[-1]))
+    idx = np.concatenate(rows) if rows else np.zeros(0, dtype=np.int64)
+    return X[idx], np.asarray(koff, dtype=np.int64)

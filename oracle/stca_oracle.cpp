@@ -1,4 +1,4 @@
-// Candidate-to-sketch cross attention (the sketch branch of STCA), fp64 CPU oracle.
+// Candidate-to-history cross attention (the two branches of STCA), fp64 CPU oracle.
 //
 // TEST INFRASTRUCTURE ONLY, like sa_oracle.cpp: only tests/, __graft_entry__.smoke() and
 // bench.py's cpu_baseline leg may load it. It shares no code with the CUDA library.
@@ -11,13 +11,17 @@
 //   z_cj = (q_c . K_j) / sqrt(d)                            (the candidate scores every row)
 //   a_cj = exp(z_cj) / sum_i exp(z_ci)                      (softmax over the k sketch rows)
 //   O_c  = sum_j a_cj V_j,   lse_c = log sum_j exp(z_cj)
+// The *_keys entry points take each user's key rows as a ragged list instead (k_u rows
+// for user u), which covers the other branch: the candidate attending over the user's
+// most recent tokens (the last min(n_u, L) rows of the history).
 // Sources: "100,000 videos in your pocket" blog (danielsamfdo.github.io), section
 // "2. STCA reasons at two time scales" (the sketch branch: the candidate attends over
-// the fixed-size sketch) and section "3. The system makes it cheap enough to matter"
-// (multi-request user-level batching: a user's candidates share one sketch read). The
-// pages give no equations for STCA; single-head scaled dot-product attention with
-// square, bias-free projections W_q, W_K, W_V, one layer (stacking repeats it), no
-// mask, is the plainest reading and is what this file computes.
+// the fixed-size sketch; the recent branch: over the recent 10K suffix) and section
+// "3. The system makes it cheap enough to matter" (multi-request user-level batching: a
+// user's candidates share one sketch read). The pages give no equations for STCA;
+// single-head scaled dot-product attention with square, bias-free projections W_q,
+// W_K, W_V, one layer (stacking repeats it), no mask, is the plainest reading and is
+// what this file computes for both branches.
 //
 // Candidate sums over a user's candidates (dK, dV and the weight gradients of the
 // backward) are taken over fixed chunks of candidates whose partials are added in
@@ -98,24 +102,31 @@ double candidate_forward(const double* q, const double* K, const double* V, int 
 
 extern "C" {
 
-// Forward over a ragged batch of users.
+// Forward over a ragged batch of users whose key rows are ragged too.
 //   Q     [n_cand, d]   candidate embeddings, users' groups concatenated
 //   coff  [R+1]         coff[0] = 0, non-decreasing, coff[R] = n_cand
-//   S     [R, k, d]     each user's sketch
+//   Kx    [n_keys, d]   the rows each user's candidates attend over, users concatenated
+//                       (a sketch: k rows per user; the recent suffix: the last tokens)
+//   koff  [R+1]         koff[0] = 0, non-decreasing, koff[R] = n_keys
 //   Wq, WK, WV [d, d]
-// Outputs: O [n_cand, d]; lse [n_cand] (may be null).
+// Outputs: O [n_cand, d]; lse [n_cand] (may be null). A user with candidates but no key
+// rows gives O = 0 and lse = -inf (the attention has nothing to read).
 // Returns 0 on success, 1 on bad sizes, 2 on bad offsets.
-int stca_oracle_forward(const double* Q, const int64_t* coff, int R, int64_t n_cand, int d,
-                        const double* S, int k, const double* Wq, const double* WK,
-                        const double* WV, double* O, double* lse, int nthreads) {
-  if (int rc = check_args(coff, R, n_cand, d, k)) return rc;
+int stca_oracle_forward_keys(const double* Q, const int64_t* coff, int R, int64_t n_cand, int d,
+                             const double* Kx, const int64_t* koff, int64_t n_keys,
+                             const double* Wq, const double* WK, const double* WV, double* O,
+                             double* lse, int nthreads) {
+  if (int rc = check_args(coff, R, n_cand, d, 1)) return rc;
+  if (int rc = check_args(koff, R, n_keys, d, 1)) return rc;
   const int nt = threads_or_default(nthreads);
-  const int64_t kd = (int64_t)k * d;
-  std::vector<double> K(kd), V(kd);
+  std::vector<double> K, V;
   for (int u = 0; u < R; ++u) {
     const int64_t c0 = coff[u], c1 = coff[u + 1];
     if (c1 == c0) continue;
-    project_rows(S + (int64_t)u * kd, k, d, WK, WV, K.data(), V.data());
+    const int k = (int)(koff[u + 1] - koff[u]);
+    K.assign((size_t)k * d, 0.0);
+    V.assign((size_t)k * d, 0.0);
+    project_rows(Kx + koff[u] * d, k, d, WK, WV, K.data(), V.data());
 #pragma omp parallel for schedule(dynamic, 16) num_threads(nt)
     for (int64_t c = c0; c < c1; ++c) {
       std::vector<double> q(d), a(k);
@@ -127,9 +138,20 @@ int stca_oracle_forward(const double* Q, const int64_t* coff, int R, int64_t n_c
   return 0;
 }
 
+// The sketch case: every user has k key rows, S [R, k, d].
+int stca_oracle_forward(const double* Q, const int64_t* coff, int R, int64_t n_cand, int d,
+                        const double* S, int k, const double* Wq, const double* WK,
+                        const double* WV, double* O, double* lse, int nthreads) {
+  if (R < 0 || k <= 0) return 1;
+  std::vector<int64_t> koff((size_t)R + 1);
+  for (int u = 0; u <= R; ++u) koff[u] = (int64_t)u * k;
+  return stca_oracle_forward_keys(Q, coff, R, n_cand, d, S, koff.data(), (int64_t)R * k, Wq, WK,
+                                  WV, O, lse, nthreads);
+}
+
 // Backward: gradients of a loss L given dO = dL/dO [n_cand, d].
-// Outputs: dQ [n_cand, d]; dS [R, k, d] (per user: the gradient that flows into the
-// sketch, and from there into Sketch Attention's backward); dWq, dWK, dWV [d, d] summed
+// Outputs: dQ [n_cand, d]; dS [n_keys, d] (per user: the gradient that flows into its
+// key rows; for a sketch, into Sketch Attention's backward); dWq, dWK, dWV [d, d] summed
 // over users (all overwritten, not accumulated into).
 //
 // Derivation (per user, chain rule through the forward above):
@@ -139,24 +161,30 @@ int stca_oracle_forward(const double* Q, const int64_t* coff, int R, int64_t n_c
 //   dQ_c  = dq_c W_q^T,   dS_uj = dK_j W_K^T + dV_j W_V^T
 //   dW_q += sum_c Q_c^T dq_c,   dW_K += sum_j S_uj^T dK_j,   dW_V += sum_j S_uj^T dV_j
 // A user without candidates gets dS = 0. Returns 0 / 1 / 2 as the forward.
-int stca_oracle_backward(const double* Q, const int64_t* coff, int R, int64_t n_cand, int d,
-                         const double* S, int k, const double* Wq, const double* WK,
-                         const double* WV, const double* dO, double* dQ, double* dS,
-                         double* dWq, double* dWK, double* dWV, int nthreads) {
-  if (int rc = check_args(coff, R, n_cand, d, k)) return rc;
+int stca_oracle_backward_keys(const double* Q, const int64_t* coff, int R, int64_t n_cand, int d,
+                              const double* Kx, const int64_t* koff, int64_t n_keys,
+                              const double* Wq, const double* WK, const double* WV,
+                              const double* dO, double* dQ, double* dS, double* dWq,
+                              double* dWK, double* dWV, int nthreads) {
+  if (int rc = check_args(coff, R, n_cand, d, 1)) return rc;
+  if (int rc = check_args(koff, R, n_keys, d, 1)) return rc;
   const int nt = threads_or_default(nthreads);
-  const int64_t kd = (int64_t)k * d, dd = (int64_t)d * d;
+  const int64_t dd = (int64_t)d * d;
   const double inv_sqrt_d = 1.0 / std::sqrt((double)d);
-  std::memset(dS, 0, sizeof(double) * (size_t)R * kd);
+  std::memset(dS, 0, sizeof(double) * (size_t)n_keys * d);
   std::memset(dWq, 0, sizeof(double) * dd);
   std::memset(dWK, 0, sizeof(double) * dd);
   std::memset(dWV, 0, sizeof(double) * dd);
-  std::vector<double> K(kd), V(kd);
-  const int64_t acc_len = 2 * kd + dd;  // [dK | dV | dWq] per chunk of candidates
+  std::vector<double> K, V;
   for (int u = 0; u < R; ++u) {
     const int64_t c0 = coff[u], c1 = coff[u + 1];
     if (c1 == c0) continue;
-    const double* Su = S + (int64_t)u * kd;
+    const int k = (int)(koff[u + 1] - koff[u]);
+    const int64_t kd = (int64_t)k * d;
+    const int64_t acc_len = 2 * kd + dd;  // [dK | dV | dWq] per chunk of candidates
+    const double* Su = Kx + koff[u] * d;
+    K.assign((size_t)kd, 0.0);
+    V.assign((size_t)kd, 0.0);
     project_rows(Su, k, d, WK, WV, K.data(), V.data());
     const int64_t nchunks = (c1 - c0 + kCandChunk - 1) / kCandChunk;
     std::vector<double> part(nchunks * acc_len, 0.0);
@@ -209,7 +237,7 @@ int stca_oracle_backward(const double* Q, const int64_t* coff, int R, int64_t n_
       for (int64_t i = 0; i < kd; ++i) { dK[i] += p[i]; dV[i] += p[kd + i]; }
       for (int64_t i = 0; i < dd; ++i) dWq[i] += p[2 * kd + i];
     }
-    double* dSu = dS + (int64_t)u * kd;
+    double* dSu = dS + koff[u] * d;
     for (int j = 0; j < k; ++j) {
       const double* dkj = dK.data() + (int64_t)j * d;
       const double* dvj = dV.data() + (int64_t)j * d;
@@ -227,6 +255,18 @@ int stca_oracle_backward(const double* Q, const int64_t* coff, int R, int64_t n_
     }
   }
   return 0;
+}
+
+// The sketch case: every user has k key rows, S and dS [R, k, d].
+int stca_oracle_backward(const double* Q, const int64_t* coff, int R, int64_t n_cand, int d,
+                         const double* S, int k, const double* Wq, const double* WK,
+                         const double* WV, const double* dO, double* dQ, double* dS,
+                         double* dWq, double* dWK, double* dWV, int nthreads) {
+  if (R < 0 || k <= 0) return 1;
+  std::vector<int64_t> koff((size_t)R + 1);
+  for (int u = 0; u <= R; ++u) koff[u] = (int64_t)u * k;
+  return stca_oracle_backward_keys(Q, coff, R, n_cand, d, S, koff.data(), (int64_t)R * k, Wq,
+                                   WK, WV, dO, dQ, dS, dWq, dWK, dWV, nthreads);
 }
 
 }  // extern "C"

@@ -287,3 +287,97 @@ def test_composes_with_sketch_attention_backward():
     loss.backward()
     for key, ref in (("dX", Xt.grad), ("dP", Pt.grad), ("dWk", Wkt.grad), ("dWv", Wvt.grad)):
         np.testing.assert_allclose(got[key], ref.numpy(), rtol=1e-9, atol=1e-11, err_msg=key)
+
+
+# --------------------------------------------------------------------------- ragged key rows
+def _ragged_case(key_counts=(9, 1, 0, 30), groups=(4, 2, 3, 50), d=8, seed=30):
+    g = np.random.default_rng(seed)
+    coff = np.concatenate([[0], np.cumsum(groups)]).astype(np.int64)
+    koff = np.concatenate([[0], np.cumsum(key_counts)]).astype(np.int64)
+    Q = g.standard_normal((int(coff[-1]), d))
+    Kx = g.standard_normal((int(koff[-1]), d))
+    Wq, WK, WV = (g.standard_normal((d, d)) / math.sqrt(d) for _ in range(3))
+    return Q, coff, Kx, koff, Wq, WK, WV
+
+
+def test_ragged_keys_match_torch_sdpa_per_user():
+    """Each user attends over its own number of key rows (1, 9, 30, and none: out = 0,
+    lse = -inf)."""
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    Q, coff, Kx, koff, Wq, WK, WV = _ragged_case()
+    got = oracle.stca_forward_keys(Q, coff, Kx, koff, Wq, WK, WV)
+    t = lambda a: torch.tensor(a, dtype=torch.float64)
+    for u in range(4):
+        a, b = int(coff[u]), int(coff[u + 1])
+        ka, kb = int(koff[u]), int(koff[u + 1])
+        if ka == kb:
+            assert not got["out"][a:b].any() and np.isneginf(got["lse"][a:b]).all()
+            continue
+        q, K, V = t(Q[a:b]) @ t(Wq), t(Kx[ka:kb]) @ t(WK), t(Kx[ka:kb]) @ t(WV)
+        ref = F.scaled_dot_product_attention(q[None], K[None], V[None])[0]
+        np.testing.assert_allclose(got["out"][a:b], ref.numpy(), rtol=1e-12, atol=1e-13)
+        lse = torch.logsumexp(q @ K.T / math.sqrt(Q.shape[1]), dim=1)
+        np.testing.assert_allclose(got["lse"][a:b], lse.numpy(), rtol=1e-13)
+
+
+def test_equal_key_counts_reduce_to_the_sketch_case():
+    Q, off, S, Wq, WK, WV = rand_case(groups=(5, 0, 9), k=6, d=8, seed=31)
+    a = oracle.stca_forward(Q, off, S, Wq, WK, WV)
+    b = oracle.stca_forward_keys(Q, off, S.reshape(-1, 8), np.arange(4) * 6, Wq, WK, WV)
+    assert np.array_equal(a["out"], b["out"]) and np.array_equal(a["lse"], b["lse"])
+
+
+def test_recent_suffix_is_the_last_tokens_of_each_history():
+    """The recent branch reads the last min(n_u, L) tokens: with L = 4, a user of 10
+    tokens contributes rows 6..9, a user of 3 all three, an empty user none."""
+    X = np.arange(17 * 2, dtype=float).reshape(17, 2)
+    off = np.array([0, 10, 13, 13, 17])
+    Kx, koff = oracle.recent_suffix(X, off, 4)
+    assert koff.tolist() == [0, 4, 7, 7, 11]
+    np.testing.assert_array_equal(Kx, X[[6, 7, 8, 9, 10, 11, 12, 13, 14, 15, 16]])
+
+
+def test_recent_branch_matches_sdpa_on_the_suffix():
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    g = np.random.default_rng(32)
+    d, L = 8, 25
+    off = np.array([0, 100, 110, 110, 160])
+    X = g.standard_normal((160, d))
+    coff = np.array([0, 3, 5, 6, 9])
+    Q = g.standard_normal((9, d))
+    Wq, WK, WV = (g.standard_normal((d, d)) / math.sqrt(d) for _ in range(3))
+    Kx, koff = oracle.recent_suffix(X, off, L)
+    got = oracle.stca_forward_keys(Q, coff, Kx, koff, Wq, WK, WV)
+    t = lambda a: torch.tensor(a, dtype=torch.float64)
+    for u in (0, 1, 3):
+        a, b = int(coff[u]), int(coff[u + 1])
+        rows = X[max(off[u], off[u + 1] - L):off[u + 1]]
+        ref = F.scaled_dot_product_attention((t(Q[a:b]) @ t(Wq))[None], (t(rows) @ t(WK))[None],
+                                             (t(rows) @ t(WV))[None])[0]
+        np.testing.assert_allclose(got["out"][a:b], ref.numpy(), rtol=1e-12, atol=1e-13)
+    assert not got["out"][5].any()  # user 2 has no history
+
+
+def test_ragged_backward_matches_torch_autograd():
+    torch = pytest.importorskip("torch")
+    F = torch.nn.functional
+    Q, coff, Kx, koff, Wq, WK, WV = _ragged_case(seed=33)
+    G = np.random.default_rng(34).standard_normal(Q.shape)
+    got = oracle.stca_backward_keys(Q, coff, Kx, koff, Wq, WK, WV, G)
+    tt = lambda a: torch.tensor(a, dtype=torch.float64, requires_grad=True)
+    Qt, Kt, Wqt, WKt, WVt = tt(Q), tt(Kx), tt(Wq), tt(WK), tt(WV)
+    loss = torch.zeros((), dtype=torch.float64)
+    for u in range(4):
+        a, b = int(coff[u]), int(coff[u + 1])
+        ka, kb = int(koff[u]), int(koff[u + 1])
+        if a == b or ka == kb:
+            continue
+        o = F.scaled_dot_product_attention((Qt[a:b] @ Wqt)[None], (Kt[ka:kb] @ WKt)[None],
+                                           (Kt[ka:kb] @ WVt)[None])[0]
+        loss = loss + (torch.tensor(G[a:b]) * o).sum()
+    loss.backward()
+    ref = {"dQ": Qt.grad, "dKx": Kt.grad, "dWq": Wqt.grad, "dWK": WKt.grad, "dWV": WVt.grad}
+    for key, r in ref.items():
+        np.testing.assert_allclose(got[key], r.numpy(), rtol=1e-10, atol=1e-11, err_msg=key)
