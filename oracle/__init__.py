@@ -17,6 +17,10 @@ user for all of its candidates): blog sections "2. STCA reasons at two time scal
 "3. The system makes it cheap enough to matter". They are pinned by
 ``tests/test_oracle_stca_pins.py``.
 
+``codec`` (``codec.py``, numpy) is the sketch cache codec: bf16, and FP8 E4M3 with one
+scale per row, built from the formats' definitions; pinned bit for bit against torch's
+conversions by ``tests/test_oracle_codec_pins.py``.
+
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (closed forms, invariants, brute force at 50 digits, autograd and finite
 differences for the backward). The paper's analytic FLOP ratios (49.9x, 63.9x)
