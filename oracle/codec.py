@@ -13,6 +13,10 @@ readings, taken here, are:
         S_je / s_j rounded to the nearest FP8 E4M3 value (ties to even; the OCP "fn"
         variant: finite only, largest magnitude 448); decode = code * s_j.
 
+The scale and the quotient S_je / s_j are computed in fp32 (IEEE division, rounded to
+nearest), since the quotient decides an integer code and a GPU encoder takes that
+decision in fp32; decode's product is rounded to fp32 once. Zeros are written as +0.
+
 E4M3 here is built from its definition (1 sign bit, 4 exponent bits with bias 7,
 3 mantissa bits; exponent field 0 holds the subnormals k * 2^-9), not from a library,
 so that a library's conversion can serve as an independent check.
@@ -85,8 +89,8 @@ def fp8_encode(S) -> tuple[np.ndarray, np.ndarray]:
     S = np.asarray(S, dtype=np.float32)
     amax = np.abs(S).max(axis=-1)
     scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
-    y = S.astype(np.float64) / scale[..., None].astype(np.float64)
-    return e4m3_bits(np.clip(y, -E4M3_MAX, E4M3_MAX)), scale
+    y = (S / scale[..., None]).astype(np.float32)  # fp32 IEEE division
+    return e4m3_bits(np.clip(y.astype(np.float64), -E4M3_MAX, E4M3_MAX)), scale
 
 
 def fp8_decode(codes, scales) -> np.ndarray:
