@@ -19,8 +19,9 @@ The JSON line also carries:
                 with the per-step H2D of X and offsets and the D2H of sketch and mass
   cpu_baseline  the fp64 oracle on the host cores, on a bounded sample (rank 0, N=1)
   clocks        SM clock median and throttle reasons sampled during the timed region
-  other_workloads  (one GPU) the forward on one 100K-token user and on 40 users of 100K
-                tokens each: step and kernel times, kernel fraction of the bf16 peak
+  other_workloads  (one GPU) the forward on one 100K-token user, on 40 users of 100K
+                tokens each and on the 300-user serving batch at k = 256 ... 2048: step
+                and kernel times, kernel fraction of the bf16 peak
 `--impl reference` times the oracle (the reference arm here) on the same config.
 """
 from __future__ import annotations
@@ -240,22 +241,24 @@ def sampled_parity(w, gpu_out: dict, keep: dict) -> dict:
 
 # ------------------------------------------------------------------ other workloads
 OTHER_WORKLOADS = (
-    (2, "1 user, n=100,000, d=128, k=1024, bf16 in / fp32 accumulate, forward"),
-    (5, "R=40 users x n=100,000, d=128, k=1024, bf16 in / fp32 accumulate, forward"),
-)
+    (2, None, "1 user, n=100,000, d=128, k=1024, bf16 in / fp32 accumulate, forward"),
+    (5, None, "R=40 users x n=100,000, d=128, k=1024, bf16 in / fp32 accumulate, forward"),
+) + tuple(
+    (4, kk, f"serving batch: R=300 users, n~logU[1000,100000], d=128, k={kk}, bf16 in / "
+            "fp32 accumulate, forward") for kk in (256, 512, 1024, 2048))
 
 
 def time_other_workloads(binding, inputs, dev, steps: int, peak: float) -> list:
-    """The single user of 100K tokens and the 40 x 100K batch, each timed like the main
-    workload (kernel events from the library, step events around each call) with a
-    256 MB L2 flush between steps outside the timed events. Reported beside the
-    headline; a failure here is reported, not raised."""
+    """The single user of 100K tokens, the 40 x 100K batch and the 300-user serving
+    batch at each k, each timed like the main workload (kernel events from the library,
+    step events around each call) with a 256 MB L2 flush between steps outside the timed
+    events. Reported beside the headline; a failure here is reported, not raised."""
     import torch
     out = []
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    for idx, desc in OTHER_WORKLOADS:
+    for idx, kk, desc in OTHER_WORKLOADS:
         try:
-            w = inputs.make_config(idx, with_grad=False)
+            w = inputs.make_config(idx, k=kk, with_grad=False)
             X, off = w.X.to(dev), w.offsets.to(dev)
             P, Wk, Wv = w.P.to(dev), w.Wk.to(dev), w.Wv.to(dev)
             o = binding.forward(X, off, P, Wk, Wv, want_lse=False, want_xsketch=False)
@@ -533,7 +536,7 @@ def main(argv=None) -> int:
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-backward", action="store_true", help="skip the backward timing")
     ap.add_argument("--no-other-workloads", action="store_true",
-                    help="skip the 1 x 100K and 40 x 100K forward timings")
+                    help="skip the 1 x 100K, 40 x 100K and serving-batch forward timings")
     ap.add_argument("--cpu-seconds", type=float, default=15.0)
     args = ap.parse_args(argv)
     if args.warmup < 3:
