@@ -216,6 +216,34 @@ int sa_sketch_profile_events(void* start_event, void* stop_event);
 int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M, int N, int K,
                          int splits, float* out, void* workspace, void* stream);
 
+/*
+ * Candidate-to-sketch cross attention: the sketch branch of STCA, with every candidate
+ * of a user reading that user's one sketch ("100,000 videos in your pocket" blog,
+ * sections "2. STCA reasons at two time scales" and "3. The system makes it cheap
+ * enough to matter", multi-request user-level batching). For user u and each candidate
+ * c in [cand_offsets[u], cand_offsets[u+1]):
+ *   q = Q_c Wq,  K_j = S_uj WK,  V_j = S_uj WV            (j < k, the sketch rows)
+ *   out_c = sum_j softmax_j(q . K_j / sqrt(d)) V_j,  lse_c = log sum_j exp(q . K_j / sqrt(d))
+ *
+ *   Q            [n_cand, d]  bf16, device   candidates, users' groups concatenated
+ *   cand_offsets [R + 1]      int64, device  0 = c_0 <= c_1 <= ... <= c_R = n_cand
+ *   S            [R, k, d]    fp32, device   the users' sketches (sa_sketch_forward output)
+ *   Wq, WK, WV   [d, d]       bf16, device   row-major, x W for a row vector x
+ *   out          [n_cand, d]  fp32, device   output (overwritten)
+ *   lse          [n_cand]     fp32, device   output, nullable
+ * d in {64, 128}; 1 <= k <= SA_MAX_K; n_cand <= INT32_MAX; pointers 16-byte aligned.
+ * A user without candidates reads nothing. Precision: Q Wq WK^T, the attention weights
+ * and the sketch enter the tensor cores as bf16, with fp32 accumulation.
+ * The workspace (sa_stca_workspace_size bytes, 256-aligned, caller-owned) holds the
+ * bf16 sketch and the candidates' bf16 weights over the k rows (2 k bytes each); errors
+ * follow sa_sketch_forward's conventions, and the device status word in the workspace
+ * is read with sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
+ */
+size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d);
+int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
+                    const float* S, int k, const void* Wq, const void* WK, const void* WV,
+                    float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* sa_status_string(int status);
 

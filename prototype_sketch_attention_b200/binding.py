@@ -31,7 +31,7 @@ SA_ERR_NO_DEVICE = 7
 EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
             "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
             "sa_sketch_profile_events", "sa_sketch_forward_noalloc", "sa_sketch_combine",
-            "sa_sketch_debug_gemm")
+            "sa_sketch_debug_gemm", "sa_stca_workspace_size", "sa_stca_forward")
 
 
 class SketchAttentionError(RuntimeError):
@@ -69,6 +69,10 @@ def _load() -> ctypes.CDLL:
     lib.sa_sketch_forward_noalloc.restype = i32
     lib.sa_sketch_forward_noalloc.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
                                               vp, vp, vp, vp, vp, vp]
+    lib.sa_stca_workspace_size.restype = sz
+    lib.sa_stca_workspace_size.argtypes = [i32, i64, i32, i32]
+    lib.sa_stca_forward.restype = i32
+    lib.sa_stca_forward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     return lib
 
 
@@ -99,6 +103,16 @@ def sa_sketch_debug_gemm(A, a_mn, B, b_mn, M, N, K, splits, out, workspace, stre
 
 def sa_sketch_combine(xsketch, mass, R, k, d, Wv, dt, sketch, stream) -> int:
     return int(_lib.sa_sketch_combine(xsketch, mass, R, k, d, Wv, dt, sketch, stream))
+
+
+def sa_stca_workspace_size(R: int, n_cand: int, k: int, d: int) -> int:
+    return int(_lib.sa_stca_workspace_size(R, n_cand, k, d))
+
+
+def sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse, workspace,
+                    ws_bytes, stream) -> int:
+    return int(_lib.sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse,
+                                    workspace, ws_bytes, stream))
 
 
 def sa_sketch_get_device_status(workspace, stream) -> int:
@@ -304,6 +318,46 @@ def combine(xsketch: torch.Tensor, mass: torch.Tensor, Wv: torch.Tensor, *,
                                _stream(stream, dev))
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_sketch_combine")
+    return out
+
+
+def stca_forward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, Wq: torch.Tensor,
+                 WK: torch.Tensor, WV: torch.Tensor, *, want_lse: bool = True,
+                 ws: torch.Tensor | None = None, stream=None) -> dict:
+    """Candidate-to-sketch cross attention on the GPU: every candidate of user u attends
+    over the k rows of u's sketch. Q [n_cand, d] bf16, cand_offsets [R+1] int64,
+    S [R, k, d] fp32 (the forward's sketch), Wq, WK, WV [d, d] bf16, all contiguous on one
+    CUDA device. Returns out [n_cand, d] fp32 (and lse [n_cand])."""
+    where = "stca_forward"
+    _require(isinstance(Q, torch.Tensor) and Q.dim() == 2, where, "Q must be a 2-D tensor")
+    _require(isinstance(S, torch.Tensor) and S.dim() == 3, where, "S must be a 3-D tensor")
+    _require(isinstance(cand_offsets, torch.Tensor) and cand_offsets.dim() == 1
+             and cand_offsets.numel() >= 1, where, "cand_offsets must be a 1-D tensor with R + 1 entries")
+    n_cand, d = Q.shape
+    R, k = cand_offsets.numel() - 1, S.shape[1]
+    dev = Q.device
+    bf = torch.bfloat16
+    _check_tensor(where, "Q", Q, (n_cand, d), bf, dev)
+    _check_tensor(where, "cand_offsets", cand_offsets, (R + 1,), torch.int64, dev)
+    _check_tensor(where, "S", S, (R, k, d), torch.float32, dev)
+    for name, W in (("Wq", Wq), ("WK", WK), ("WV", WV)):
+        _check_tensor(where, name, W, (d, d), bf, dev)
+    _check_cuda(where, Q)
+    out = {"out": torch.empty(n_cand, d, device=dev, dtype=torch.float32)}
+    if want_lse:
+        out["lse"] = torch.empty(n_cand, device=dev, dtype=torch.float32)
+    with torch.cuda.device(dev):
+        if ws is None:
+            nb = sa_stca_workspace_size(R, n_cand, k, d)
+            if nb == 0:
+                raise SketchAttentionError(SA_ERR_UNSUPPORTED, "sa_stca_workspace_size")
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        st = sa_stca_forward(_ptr(Q), _ptr(cand_offsets), R, n_cand, d, _ptr(S), k, _ptr(Wq),
+                             _ptr(WK), _ptr(WV), _ptr(out["out"]), _ptr(out.get("lse")),
+                             _ptr(ws), ws.nbytes, _stream(stream, dev))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_stca_forward")
+    out["_ws"] = ws
     return out
 
 

@@ -329,6 +329,47 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   return cuda_status(p.ftc ? launch_finalize_tc(f, s) : launch_finalize(f, s));
 }
 
+size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d) {
+  if (R < 0 || R > SA_MAX_USERS || n_cand < 0 || n_cand > INT32_MAX) return 0;
+  if ((d != 64 && d != 128) || k < 1 || k > SA_MAX_K) return 0;
+  StcaPlan p;
+  return stca_plan(R, n_cand, k, d, &p);
+}
+
+int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
+                    const float* S, int k, const void* Wq, const void* WK, const void* WV,
+                    float* out, float* lse, void* workspace, size_t ws_bytes, void* stream_) {
+  if (R < 0 || R > SA_MAX_USERS || n_cand < 0 || n_cand > INT32_MAX) return SA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || k < 1 || k > SA_MAX_K) return SA_ERR_UNSUPPORTED;
+  if (!cand_offsets || !Wq || !WK || !WV || (n_cand > 0 && (!Q || !out)) || (R > 0 && !S))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(cand_offsets) || !aligned16(S) || !aligned16(Wq) ||
+      !aligned16(WK) || !aligned16(WV) || !aligned16(out) || !aligned16(lse))
+    return SA_ERR_INVALID_ARG;
+  Device dev;
+  sa_status st;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  StcaArgs a;
+  stca_plan(R, n_cand, k, d, &a.plan);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      ws_bytes < a.plan.total)
+    return SA_ERR_WORKSPACE;
+  a.Q = Q;
+  a.coff = cand_offsets;
+  a.R = R;
+  a.k = k;
+  a.d = d;
+  a.n_cand = n_cand;
+  a.S = S;
+  a.Wq = Wq;
+  a.WK = WK;
+  a.WV = WV;
+  a.out = out;
+  a.lse = lse;
+  a.workspace = workspace;
+  return cuda_status(launch_stca_forward(a, static_cast<cudaStream_t>(stream_)));
+}
+
 int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
                        const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,
                        const float* sketch, const float* mass, const float* lse,

@@ -182,6 +182,29 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
+// ---- candidate-to-sketch cross attention (sa_stca.cu)
+struct StcaPlan {  // workspace layout (byte offsets, 256-aligned)
+  int k_pad = 0, nparts = 0;
+  size_t hdr = 0, ts = 0, sb = 0, mt = 0, qp = 0, dpart = 0, lse2 = 0, ab = 0, o = 0, ohi = 0,
+         olo = 0, total = 0;
+};
+size_t stca_plan(int R, long long n_cand, int k, int d, StcaPlan* p);
+struct StcaArgs {
+  const void* Q;         // bf16 [n_cand, d]
+  const int64_t* coff;   // [R + 1]
+  int R, k, d;
+  long long n_cand;
+  const float* S;        // [R, k, d]
+  const void* Wq;        // bf16 [d, d]
+  const void* WK;
+  const void* WV;
+  float* out;            // [n_cand, d]
+  float* lse;            // [n_cand] natural log, nullable
+  void* workspace;
+  StcaPlan plan;
+};
+cudaError_t launch_stca_forward(const StcaArgs& a, cudaStream_t s);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();
 
