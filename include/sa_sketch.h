@@ -239,10 +239,30 @@ int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M
  * follow sa_sketch_forward's conventions, and the device status word in the workspace
  * is read with sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
  */
-size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d);
+size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d, int backward);
 int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
                     const float* S, int k, const void* Wq, const void* WK, const void* WV,
                     float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Gradients of the cross attention above, given dout = dL/dout [n_cand, d] (fp32,
+ * device):
+ *   dQ  [n_cand, d]  fp32, device   dL/dQ
+ *   dS  [R, k, d]    fp32, device   dL/dS, the gradient that flows into each user's
+ *                                   sketch (Sketch Attention's dsketch); zero for users
+ *                                   without candidates
+ *   dWq, dWK, dWV [d, d] fp32, device, summed over users
+ * All outputs are overwritten. cand_offsets_host is a HOST copy of cand_offsets (the
+ * per-user gradient of the sketch is one GEMM per user, sized on the host); it is
+ * checked before anything is launched (SA_ERR_BAD_OFFSETS). The forward is recomputed
+ * inside. Workspace: sa_stca_workspace_size(..., backward = 1) bytes. Other arguments,
+ * precision and conventions as for sa_stca_forward.
+ */
+int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* cand_offsets_host,
+                     int R, int64_t n_cand, int d, const float* S, int k, const void* Wq,
+                     const void* WK, const void* WV, const float* dout, float* dQ, float* dS,
+                     float* dWq, float* dWK, float* dWV, void* workspace, size_t ws_bytes,
+                     void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* sa_status_string(int status);

@@ -184,11 +184,14 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
 // ---- candidate-to-sketch cross attention (sa_stca.cu)
 struct StcaPlan {  // workspace layout (byte offsets, 256-aligned)
-  int k_pad = 0, nparts = 0;
+  int k_pad = 0, nparts = 0, splits = 0;
   size_t hdr = 0, ts = 0, sb = 0, mt = 0, qp = 0, dpart = 0, lse2 = 0, ab = 0, o = 0, ohi = 0,
          olo = 0, total = 0;
+  // backward only
+  size_t mts = 0, qn = 0, do_f = 0, do_b = 0, dd = 0, czero = 0, dz = 0, g1 = 0, g1hi = 0,
+         g1lo = 0, gb = 0, ob = 0, ghi = 0, glo = 0, part = 0, dm = 0;
 };
-size_t stca_plan(int R, long long n_cand, int k, int d, StcaPlan* p);
+size_t stca_plan(int R, long long n_cand, int k, int d, bool backward, int sms, StcaPlan* p);
 struct StcaArgs {
   const void* Q;         // bf16 [n_cand, d]
   const int64_t* coff;   // [R + 1]
@@ -204,6 +207,14 @@ struct StcaArgs {
   StcaPlan plan;
 };
 cudaError_t launch_stca_forward(const StcaArgs& a, cudaStream_t s);
+struct StcaGrads {
+  const float* dout;          // [n_cand, d]
+  const int64_t* coff_host;   // [R + 1], host copy of the candidate offsets
+  float* dQ;                  // [n_cand, d]
+  float* dS;                  // [R, k, d]
+  float *dWq, *dWK, *dWV;     // [d, d]
+};
+cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& g, cudaStream_t s);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();

@@ -76,3 +76,55 @@ def test_cross_attention_without_candidates():
     cw = inputs.make_cross_workload([0, 0], 256, 128, seed=45)
     got, lse = _run(cw)
     assert got.shape == (0, 128) and lse.shape == (0,)
+
+
+def _check_grads(got, ref):
+    for key, r in ref.items():
+        g = got[key]
+        e = rel_l2(g, r)
+        assert e <= BF16_REL, (key, e)
+        assert np.abs(g - r).max() <= BF16_ABS * max(np.abs(r).max(), 1e-30), (key, "max-abs")
+
+
+@pytest.mark.parametrize("counts,k,d", [([300, 0, 1, 129], 1024, 128), ([5, 77], 200, 64),
+                                        ([1, 2, 3, 255, 256, 257], 2048, 128)])
+def test_cross_attention_backward_small_full_compare(counts, k, d):
+    from prototype_sketch_attention_b200 import binding
+    cw = inputs.make_cross_workload(counts, k, d, seed=700 + k + d)
+    G = torch.randn(int(cw.cand_offsets[-1]), d, generator=torch.Generator().manual_seed(701))
+    dev = torch.device("cuda")
+    out = binding.stca_backward(cw.Q.to(dev), cw.cand_offsets.to(dev), cw.S.to(dev),
+                                cw.Wq.to(dev), cw.WK.to(dev), cw.WV.to(dev), G.to(dev))
+    assert binding.device_status(out["_ws"]) == 0
+    got = {key: out[key].cpu().double().numpy() for key in ("dQ", "dS", "dWq", "dWK", "dWV")}
+    f = cw.to_f64()
+    ref = oracle.stca_backward(f["Q"], f["cand_offsets"], f["S"], f["Wq"], f["WK"], f["WV"],
+                               G.double().numpy(), nthreads=nthreads())
+    _check_grads(got, ref)
+    assert not got["dS"][[i for i, c in enumerate(counts) if c == 0]].any()
+
+
+def test_history_to_candidates_chain_gradient():
+    """Sketch Attention, then the cross attention over its sketch: the cross attention's
+    dS fed to sa_sketch_backward as dL/dsketch gives the chain's gradient w.r.t. the
+    history, checked against the two oracles chained the same way."""
+    from prototype_sketch_attention_b200 import binding
+    w = inputs.make_workload([2000, 700, 1500], 128, 256, "bf16", seed=71)
+    g, fwd = gpu_forward(w)
+    cw = inputs.make_cross_workload([40, 9, 120], 256, 128, seed=72, S=fwd["sketch"].cpu())
+    G = torch.randn(169, 128, generator=torch.Generator().manual_seed(73))
+    dev = torch.device("cuda")
+    cb = binding.stca_backward(cw.Q.to(dev), cw.cand_offsets.to(dev), fwd["sketch"],
+                               cw.Wq.to(dev), cw.WK.to(dev), cw.WV.to(dev), G.to(dev))
+    sb = binding.backward(g["X"], g["offsets"], g["P"], g["Wk"], g["Wv"], fwd, cb["dS"])
+    assert binding.device_status(sb["_ws"]) == 0
+    sub = w.to_f64()
+    ref_f = oracle.forward(sub["X"], sub["offsets"], sub["P"], sub["Wk"], sub["Wv"],
+                           nthreads=nthreads())
+    f = cw.to_f64()
+    ref_c = oracle.stca_backward(f["Q"], f["cand_offsets"], ref_f["sketch"], f["Wq"], f["WK"],
+                                 f["WV"], G.double().numpy(), nthreads=nthreads())
+    ref = oracle.backward(sub["X"], sub["offsets"], sub["P"], sub["Wk"], sub["Wv"], ref_c["dS"],
+                          nthreads=nthreads())
+    got = {key: sb[key].cpu().double().numpy() for key in ("dX", "dP", "dWk", "dWv")}
+    _check_grads(got, ref)
