@@ -264,6 +264,27 @@ int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* 
                      float* dWq, float* dWK, float* dWV, void* workspace, size_t ws_bytes,
                      void* stream);
 
+/*
+ * Sketch cache codec. The sketch is user-only and reused across candidates and
+ * requests ("100,000 videos in your pocket" blog, section "3. The system makes it cheap
+ * enough to matter", low-rank caching), so it is kept packed between requests:
+ *   SA_CODEC_BF16: codes [rows, d] bf16, each value rounded to nearest (ties to even);
+ *   SA_CODEC_FP8:  codes [rows, d] FP8 E4M3 (finite-only, saturating at 448) of
+ *                  x / s_row, with s_row = max |row| / 448 (1 for an all-zero row) in
+ *                  scales [rows] fp32; scale and quotient in fp32 IEEE arithmetic;
+ *                  zeros are stored as +0. Unpack: code * s_row, rounded to fp32.
+ *   sketch [rows, d] fp32, device (rows = R k for R users' sketches); d in {64, 128};
+ *   pointers 16-byte aligned; scales may be null for SA_CODEC_BF16.
+ * Allocates nothing, enqueues one kernel on `stream`, never synchronises. Returns SA_OK,
+ * SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED or SA_ERR_CUDA.
+ */
+#define SA_CODEC_BF16 0
+#define SA_CODEC_FP8 1
+int sa_sketch_pack(const float* sketch, int64_t rows, int d, int format, void* codes,
+                   float* scales, void* stream);
+int sa_sketch_unpack(const void* codes, const float* scales, int64_t rows, int d, int format,
+                     float* sketch, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* sa_status_string(int status);
 

@@ -32,7 +32,9 @@ EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward
             "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
             "sa_sketch_profile_events", "sa_sketch_forward_noalloc", "sa_sketch_combine",
             "sa_sketch_debug_gemm", "sa_stca_workspace_size", "sa_stca_forward",
-            "sa_stca_backward")
+            "sa_stca_backward", "sa_sketch_pack", "sa_sketch_unpack")
+SA_CODEC_BF16 = 0
+SA_CODEC_FP8 = 1
 
 
 class SketchAttentionError(RuntimeError):
@@ -72,6 +74,10 @@ def _load() -> ctypes.CDLL:
                                               vp, vp, vp, vp, vp, vp]
     lib.sa_stca_workspace_size.restype = sz
     lib.sa_stca_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+    lib.sa_sketch_pack.restype = i32
+    lib.sa_sketch_pack.argtypes = [vp, i64, i32, i32, vp, vp, vp]
+    lib.sa_sketch_unpack.restype = i32
+    lib.sa_sketch_unpack.argtypes = [vp, vp, i64, i32, i32, vp, vp]
     lib.sa_stca_backward.restype = i32
     lib.sa_stca_backward.argtypes = [vp, vp, vp, i32, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp,
                                      vp, vp, vp, vp, sz, vp]
@@ -123,6 +129,48 @@ def sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse, w
                     ws_bytes, stream) -> int:
     return int(_lib.sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse,
                                     workspace, ws_bytes, stream))
+
+
+def sa_sketch_pack(sketch, rows, d, fmt, codes, scales, stream) -> int:
+    return int(_lib.sa_sketch_pack(sketch, rows, d, fmt, codes, scales, stream))
+
+
+def sa_sketch_unpack(codes, scales, rows, d, fmt, sketch, stream) -> int:
+    return int(_lib.sa_sketch_unpack(codes, scales, rows, d, fmt, sketch, stream))
+
+
+def sketch_pack(S: torch.Tensor, fmt: int = SA_CODEC_FP8, stream=None) -> dict:
+    """Packs fp32 sketches [..., d] (contiguous, CUDA) for the cache: codes (uint8 for
+    fp8, bfloat16 for bf16) and, for fp8, one fp32 scale per row."""
+    where = "sketch_pack"
+    _require(isinstance(S, torch.Tensor) and S.dim() >= 2, where, "S must be [..., d]")
+    d = S.shape[-1]
+    rows = S.numel() // d if d else 0
+    _check_tensor(where, "S", S, tuple(S.shape), torch.float32, S.device)
+    _check_cuda(where, S)
+    dt = torch.uint8 if fmt == SA_CODEC_FP8 else torch.bfloat16
+    out = {"codes": torch.empty(S.shape, dtype=dt, device=S.device),
+           "scales": (torch.empty(S.shape[:-1], dtype=torch.float32, device=S.device)
+                      if fmt == SA_CODEC_FP8 else None), "format": fmt}
+    with torch.cuda.device(S.device):
+        st = sa_sketch_pack(_ptr(S), rows, d, fmt, _ptr(out["codes"]), _ptr(out["scales"]),
+                            _stream(stream, S.device))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_pack")
+    return out
+
+
+def sketch_unpack(packed: dict, stream=None) -> torch.Tensor:
+    """The fp32 sketches back from sketch_pack's output."""
+    codes, fmt = packed["codes"], packed["format"]
+    d = codes.shape[-1]
+    S = torch.empty(codes.shape, dtype=torch.float32, device=codes.device)
+    with torch.cuda.device(codes.device):
+        st = sa_sketch_unpack(_ptr(codes), _ptr(packed.get("scales")), codes.numel() // d, d, fmt,
+                              _ptr(S), _stream(stream, codes.device))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_unpack")
+    return S
 
 
 def sa_sketch_get_device_status(workspace, stream) -> int:

@@ -422,6 +422,28 @@ int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* 
   return cuda_status(launch_stca_backward(a, g, static_cast<cudaStream_t>(stream_)));
 }
 
+int sa_sketch_pack(const float* sketch, int64_t rows, int d, int format, void* codes,
+                   float* scales, void* stream) {
+  if (rows < 0 || (format != SA_CODEC_BF16 && format != SA_CODEC_FP8)) return SA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+  if (rows > 0 && (!sketch || !codes || (format == SA_CODEC_FP8 && !scales)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(sketch) || !aligned16(codes) || !aligned16(scales)) return SA_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_sketch_pack(sketch, rows, d, format, codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
+int sa_sketch_unpack(const void* codes, const float* scales, int64_t rows, int d, int format,
+                     float* sketch, void* stream) {
+  if (rows < 0 || (format != SA_CODEC_BF16 && format != SA_CODEC_FP8)) return SA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+  if (rows > 0 && (!sketch || !codes || (format == SA_CODEC_FP8 && !scales)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(sketch) || !aligned16(codes) || !aligned16(scales)) return SA_ERR_INVALID_ARG;
+  return cuda_status(launch_sketch_unpack(codes, scales, rows, d, format, sketch,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
                        const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,
                        const float* sketch, const float* mass, const float* lse,

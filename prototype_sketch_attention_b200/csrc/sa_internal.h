@@ -216,6 +216,12 @@ struct StcaGrads {
 };
 cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& g, cudaStream_t s);
 
+// ---- sketch cache codec (sa_codec.cu): format 0 = bf16, 1 = fp8 E4M3 with row scales
+cudaError_t launch_sketch_pack(const float* S, long long rows, int d, int format, void* codes,
+                               float* scales, cudaStream_t s);
+cudaError_t launch_sketch_unpack(const void* codes, const float* scales, long long rows, int d,
+                                 int format, float* S, cudaStream_t s);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();
 
