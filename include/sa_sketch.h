@@ -216,6 +216,75 @@ int sa_sketch_profile_events(void* start_event, void* stop_event);
 int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M, int N, int K,
                          int splits, float* out, void* workspace, void* stream);
 
+/*
+ * Candidate-to-sketch cross attention: the sketch branch of STCA, with every candidate
+ * of a user reading that user's one sketch ("100,000 videos in your pocket" blog,
+ * sections "2. STCA reasons at two time scales" and "3. The system makes it cheap
+ * enough to matter", multi-request user-level batching). For user u and each candidate
+ * c in [cand_offsets[u], cand_offsets[u+1]):
+ *   q = Q_c Wq,  K_j = S_uj WK,  V_j = S_uj WV            (j < k, the sketch rows)
+ *   out_c = sum_j softmax_j(q . K_j / sqrt(d)) V_j,  lse_c = log sum_j exp(q . K_j / sqrt(d))
+ *
+ *   Q            [n_cand, d]  bf16, device   candidates, users' groups concatenated
+ *   cand_offsets [R + 1]      int64, device  0 = c_0 <= c_1 <= ... <= c_R = n_cand
+ *   S            [R, k, d]    fp32, device   the users' sketches (sa_sketch_forward output)
+ *   Wq, WK, WV   [d, d]       bf16, device   row-major, x W for a row vector x
+ *   out          [n_cand, d]  fp32, device   output (overwritten)
+ *   lse          [n_cand]     fp32, device   output, nullable
+ * d in {64, 128}; 1 <= k <= SA_MAX_K; n_cand <= INT32_MAX; pointers 16-byte aligned.
+ * A user without candidates reads nothing. Precision: Q Wq WK^T, the attention weights
+ * and the sketch enter the tensor cores as bf16, with fp32 accumulation.
+ * The workspace (sa_stca_workspace_size bytes, 256-aligned, caller-owned) holds the
+ * bf16 sketch and the candidates' bf16 weights over the k rows (2 k bytes each); errors
+ * follow sa_sketch_forward's conventions, and the device status word in the workspace
+ * is read with sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
+ */
+size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d, int backward);
+int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
+                    const float* S, int k, const void* Wq, const void* WK, const void* WV,
+                    float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Gradients of the cross attention above, given dout = dL/dout [n_cand, d] (fp32,
+ * device):
+ *   dQ  [n_cand, d]  fp32, device   dL/dQ
+ *   dS  [R, k, d]    fp32, device   dL/dS, the gradient that flows into each user's
+ *                                   sketch (Sketch Attention's dsketch); zero for users
+ *                                   without candidates
+ *   dWq, dWK, dWV [d, d] fp32, device, summed over users
+ * All outputs are overwritten. cand_offsets_host is a HOST copy of cand_offsets (the
+ * per-user gradient of the sketch is one GEMM per user, sized on the host); it is
+ * checked before anything is launched (SA_ERR_BAD_OFFSETS). The forward is recomputed
+ * inside. Workspace: sa_stca_workspace_size(..., backward = 1) bytes. Other arguments,
+ * precision and conventions as for sa_stca_forward.
+ */
+int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* cand_offsets_host,
+                     int R, int64_t n_cand, int d, const float* S, int k, const void* Wq,
+                     const void* WK, const void* WV, const float* dout, float* dQ, float* dS,
+                     float* dWq, float* dWK, float* dWV, void* workspace, size_t ws_bytes,
+                     void* stream);
+
+/*
+ * Sketch cache codec. The sketch is user-only and reused across candidates and
+ * requests ("100,000 videos in your pocket" blog, section "3. The system makes it cheap
+ * enough to matter", low-rank caching), so it is kept packed between requests:
+ *   SA_CODEC_BF16: codes [rows, d] bf16, each value rounded to nearest (ties to even);
+ *   SA_CODEC_FP8:  codes [rows, d] FP8 E4M3 (finite-only, saturating at 448) of
+ *                  x / s_row, with s_row = max |row| / 448 (1 for an all-zero row) in
+ *                  scales [rows] fp32; scale and quotient in fp32 IEEE arithmetic;
+ *                  zeros are stored as +0. Unpack: code * s_row, rounded to fp32.
+ *   sketch [rows, d] fp32, device (rows = R k for R users' sketches); d in {64, 128};
+ *   pointers 16-byte aligned; scales may be null for SA_CODEC_BF16.
+ * Allocates nothing, enqueues one kernel on `stream`, never synchronises. Returns SA_OK,
+ * SA_ERR_INVALID_ARG, SA_ERR_UNSUPPORTED or SA_ERR_CUDA.
+ */
+#define SA_CODEC_BF16 0
+#define SA_CODEC_FP8 1
+int sa_sketch_pack(const float* sketch, int64_t rows, int d, int format, void* codes,
+                   float* scales, void* stream);
+int sa_sketch_unpack(const void* codes, const float* scales, int64_t rows, int d, int format,
+                     float* sketch, void* stream);
+
 /* Static, human-readable name of a status code. */
 const char* sa_status_string(int status);
 

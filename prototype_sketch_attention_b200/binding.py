@@ -31,7 +31,10 @@ SA_ERR_NO_DEVICE = 7
 EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward",
             "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
             "sa_sketch_profile_events", "sa_sketch_forward_noalloc", "sa_sketch_combine",
-            "sa_sketch_debug_gemm")
+            "sa_sketch_debug_gemm", "sa_stca_workspace_size", "sa_stca_forward",
+            "sa_stca_backward", "sa_sketch_pack", "sa_sketch_unpack")
+SA_CODEC_BF16 = 0
+SA_CODEC_FP8 = 1
 
 
 class SketchAttentionError(RuntimeError):
@@ -69,6 +72,17 @@ def _load() -> ctypes.CDLL:
     lib.sa_sketch_forward_noalloc.restype = i32
     lib.sa_sketch_forward_noalloc.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32,
                                               vp, vp, vp, vp, vp, vp]
+    lib.sa_stca_workspace_size.restype = sz
+    lib.sa_stca_workspace_size.argtypes = [i32, i64, i32, i32, i32]
+    lib.sa_sketch_pack.restype = i32
+    lib.sa_sketch_pack.argtypes = [vp, i64, i32, i32, vp, vp, vp]
+    lib.sa_sketch_unpack.restype = i32
+    lib.sa_sketch_unpack.argtypes = [vp, vp, i64, i32, i32, vp, vp]
+    lib.sa_stca_backward.restype = i32
+    lib.sa_stca_backward.argtypes = [vp, vp, vp, i32, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp,
+                                     vp, vp, vp, vp, sz, vp]
+    lib.sa_stca_forward.restype = i32
+    lib.sa_stca_forward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
     return lib
 
 
@@ -99,6 +113,64 @@ def sa_sketch_debug_gemm(A, a_mn, B, b_mn, M, N, K, splits, out, workspace, stre
 
 def sa_sketch_combine(xsketch, mass, R, k, d, Wv, dt, sketch, stream) -> int:
     return int(_lib.sa_sketch_combine(xsketch, mass, R, k, d, Wv, dt, sketch, stream))
+
+
+def sa_stca_workspace_size(R: int, n_cand: int, k: int, d: int, backward: int = 0) -> int:
+    return int(_lib.sa_stca_workspace_size(R, n_cand, k, d, backward))
+
+
+def sa_stca_backward(Q, cand_offsets, cand_offsets_host, R, n_cand, d, S, k, Wq, WK, WV, dout, dQ,
+                     dS, dWq, dWK, dWV, workspace, ws_bytes, stream) -> int:
+    return int(_lib.sa_stca_backward(Q, cand_offsets, cand_offsets_host, R, n_cand, d, S, k, Wq, WK,
+                                     WV, dout, dQ, dS, dWq, dWK, dWV, workspace, ws_bytes, stream))
+
+
+def sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse, workspace,
+                    ws_bytes, stream) -> int:
+    return int(_lib.sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse,
+                                    workspace, ws_bytes, stream))
+
+
+def sa_sketch_pack(sketch, rows, d, fmt, codes, scales, stream) -> int:
+    return int(_lib.sa_sketch_pack(sketch, rows, d, fmt, codes, scales, stream))
+
+
+def sa_sketch_unpack(codes, scales, rows, d, fmt, sketch, stream) -> int:
+    return int(_lib.sa_sketch_unpack(codes, scales, rows, d, fmt, sketch, stream))
+
+
+def sketch_pack(S: torch.Tensor, fmt: int = SA_CODEC_FP8, stream=None) -> dict:
+    """Packs fp32 sketches [..., d] (contiguous, CUDA) for the cache: codes (uint8 for
+    fp8, bfloat16 for bf16) and, for fp8, one fp32 scale per row."""
+    where = "sketch_pack"
+    _require(isinstance(S, torch.Tensor) and S.dim() >= 2, where, "S must be [..., d]")
+    d = S.shape[-1]
+    rows = S.numel() // d if d else 0
+    _check_tensor(where, "S", S, tuple(S.shape), torch.float32, S.device)
+    _check_cuda(where, S)
+    dt = torch.uint8 if fmt == SA_CODEC_FP8 else torch.bfloat16
+    out = {"codes": torch.empty(S.shape, dtype=dt, device=S.device),
+           "scales": (torch.empty(S.shape[:-1], dtype=torch.float32, device=S.device)
+                      if fmt == SA_CODEC_FP8 else None), "format": fmt}
+    with torch.cuda.device(S.device):
+        st = sa_sketch_pack(_ptr(S), rows, d, fmt, _ptr(out["codes"]), _ptr(out["scales"]),
+                            _stream(stream, S.device))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_pack")
+    return out
+
+
+def sketch_unpack(packed: dict, stream=None) -> torch.Tensor:
+    """The fp32 sketches back from sketch_pack's output."""
+    codes, fmt = packed["codes"], packed["format"]
+    d = codes.shape[-1]
+    S = torch.empty(codes.shape, dtype=torch.float32, device=codes.device)
+    with torch.cuda.device(codes.device):
+        st = sa_sketch_unpack(_ptr(codes), _ptr(packed.get("scales")), codes.numel() // d, d, fmt,
+                              _ptr(S), _stream(stream, codes.device))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_unpack")
+    return S
 
 
 def sa_sketch_get_device_status(workspace, stream) -> int:
@@ -304,6 +376,89 @@ def combine(xsketch: torch.Tensor, mass: torch.Tensor, Wv: torch.Tensor, *,
                                _stream(stream, dev))
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_sketch_combine")
+    return out
+
+
+def stca_forward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, Wq: torch.Tensor,
+                 WK: torch.Tensor, WV: torch.Tensor, *, want_lse: bool = True,
+                 ws: torch.Tensor | None = None, stream=None) -> dict:
+    """Candidate-to-sketch cross attention on the GPU: every candidate of user u attends
+    over the k rows of u's sketch. Q [n_cand, d] bf16, cand_offsets [R+1] int64,
+    S [R, k, d] fp32 (the forward's sketch), Wq, WK, WV [d, d] bf16, all contiguous on one
+    CUDA device. Returns out [n_cand, d] fp32 (and lse [n_cand])."""
+    where = "stca_forward"
+    _require(isinstance(Q, torch.Tensor) and Q.dim() == 2, where, "Q must be a 2-D tensor")
+    _require(isinstance(S, torch.Tensor) and S.dim() == 3, where, "S must be a 3-D tensor")
+    _require(isinstance(cand_offsets, torch.Tensor) and cand_offsets.dim() == 1
+             and cand_offsets.numel() >= 1, where, "cand_offsets must be a 1-D tensor with R + 1 entries")
+    n_cand, d = Q.shape
+    R, k = cand_offsets.numel() - 1, S.shape[1]
+    dev = Q.device
+    bf = torch.bfloat16
+    _check_tensor(where, "Q", Q, (n_cand, d), bf, dev)
+    _check_tensor(where, "cand_offsets", cand_offsets, (R + 1,), torch.int64, dev)
+    _check_tensor(where, "S", S, (R, k, d), torch.float32, dev)
+    for name, W in (("Wq", Wq), ("WK", WK), ("WV", WV)):
+        _check_tensor(where, name, W, (d, d), bf, dev)
+    _check_cuda(where, Q)
+    out = {"out": torch.empty(n_cand, d, device=dev, dtype=torch.float32)}
+    if want_lse:
+        out["lse"] = torch.empty(n_cand, device=dev, dtype=torch.float32)
+    with torch.cuda.device(dev):
+        if ws is None:
+            nb = sa_stca_workspace_size(R, n_cand, k, d, 0)
+            if nb == 0:
+                raise SketchAttentionError(SA_ERR_UNSUPPORTED, "sa_stca_workspace_size")
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        st = sa_stca_forward(_ptr(Q), _ptr(cand_offsets), R, n_cand, d, _ptr(S), k, _ptr(Wq),
+                             _ptr(WK), _ptr(WV), _ptr(out["out"]), _ptr(out.get("lse")),
+                             _ptr(ws), ws.nbytes, _stream(stream, dev))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_stca_forward")
+    out["_ws"] = ws
+    return out
+
+
+def stca_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, Wq: torch.Tensor,
+                  WK: torch.Tensor, WV: torch.Tensor, dout: torch.Tensor, *,
+                  ws: torch.Tensor | None = None, stream=None) -> dict:
+    """Gradients of stca_forward given dL/dout [n_cand, d] fp32: dQ, dS (into each
+    user's sketch), dWq, dWK, dWV. Inputs as for stca_forward."""
+    where = "stca_backward"
+    _require(isinstance(Q, torch.Tensor) and Q.dim() == 2, where, "Q must be a 2-D tensor")
+    _require(isinstance(S, torch.Tensor) and S.dim() == 3, where, "S must be a 3-D tensor")
+    _require(isinstance(cand_offsets, torch.Tensor) and cand_offsets.dim() == 1
+             and cand_offsets.numel() >= 1, where, "cand_offsets must be a 1-D tensor with R + 1 entries")
+    n_cand, d = Q.shape
+    R, k = cand_offsets.numel() - 1, S.shape[1]
+    dev = Q.device
+    bf, f32 = torch.bfloat16, torch.float32
+    _check_tensor(where, "Q", Q, (n_cand, d), bf, dev)
+    _check_tensor(where, "cand_offsets", cand_offsets, (R + 1,), torch.int64, dev)
+    _check_tensor(where, "S", S, (R, k, d), f32, dev)
+    for name, W in (("Wq", Wq), ("WK", WK), ("WV", WV)):
+        _check_tensor(where, name, W, (d, d), bf, dev)
+    _check_tensor(where, "dout", dout, (n_cand, d), f32, dev)
+    _check_cuda(where, Q)
+    coff_h = cand_offsets.cpu().contiguous()
+    out = {"dQ": torch.empty(n_cand, d, device=dev, dtype=f32),
+           "dS": torch.empty(R, k, d, device=dev, dtype=f32),
+           "dWq": torch.empty(d, d, device=dev, dtype=f32),
+           "dWK": torch.empty(d, d, device=dev, dtype=f32),
+           "dWV": torch.empty(d, d, device=dev, dtype=f32)}
+    with torch.cuda.device(dev):
+        if ws is None:
+            nb = sa_stca_workspace_size(R, n_cand, k, d, 1)
+            if nb == 0:
+                raise SketchAttentionError(SA_ERR_UNSUPPORTED, "sa_stca_workspace_size")
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        st = sa_stca_backward(_ptr(Q), _ptr(cand_offsets), _ptr(coff_h), R, n_cand, d, _ptr(S), k,
+                              _ptr(Wq), _ptr(WK), _ptr(WV), _ptr(dout), _ptr(out["dQ"]),
+                              _ptr(out["dS"]), _ptr(out["dWq"]), _ptr(out["dWK"]),
+                              _ptr(out["dWV"]), _ptr(ws), ws.nbytes, _stream(stream, dev))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_stca_backward")
+    out["_ws"] = ws
     return out
 
 

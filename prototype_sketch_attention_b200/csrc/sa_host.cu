@@ -329,6 +329,121 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   return cuda_status(p.ftc ? launch_finalize_tc(f, s) : launch_finalize(f, s));
 }
 
+size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d, int backward) {
+  if (R < 0 || R > SA_MAX_USERS || n_cand < 0 || n_cand > INT32_MAX) return 0;
+  if ((d != 64 && d != 128) || k < 1 || k > SA_MAX_K) return 0;
+  Device dev;
+  if (backward && current_device(&dev) != SA_OK) return 0;
+  StcaPlan p;
+  return stca_plan(R, n_cand, k, d, backward != 0, backward ? dev.sms : 0, &p);
+}
+
+int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
+                    const float* S, int k, const void* Wq, const void* WK, const void* WV,
+                    float* out, float* lse, void* workspace, size_t ws_bytes, void* stream_) {
+  if (R < 0 || R > SA_MAX_USERS || n_cand < 0 || n_cand > INT32_MAX) return SA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || k < 1 || k > SA_MAX_K) return SA_ERR_UNSUPPORTED;
+  if (!cand_offsets || !Wq || !WK || !WV || (n_cand > 0 && (!Q || !out)) || (R > 0 && !S))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(cand_offsets) || !aligned16(S) || !aligned16(Wq) ||
+      !aligned16(WK) || !aligned16(WV) || !aligned16(out) || !aligned16(lse))
+    return SA_ERR_INVALID_ARG;
+  Device dev;
+  sa_status st;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  StcaArgs a;
+  stca_plan(R, n_cand, k, d, false, 0, &a.plan);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      ws_bytes < a.plan.total)
+    return SA_ERR_WORKSPACE;
+  a.Q = Q;
+  a.coff = cand_offsets;
+  a.R = R;
+  a.k = k;
+  a.d = d;
+  a.n_cand = n_cand;
+  a.S = S;
+  a.Wq = Wq;
+  a.WK = WK;
+  a.WV = WV;
+  a.out = out;
+  a.lse = lse;
+  a.workspace = workspace;
+  return cuda_status(launch_stca_forward(a, static_cast<cudaStream_t>(stream_)));
+}
+
+int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* cand_offsets_host,
+                     int R, int64_t n_cand, int d, const float* S, int k, const void* Wq,
+                     const void* WK, const void* WV, const float* dout, float* dQ, float* dS,
+                     float* dWq, float* dWK, float* dWV, void* workspace, size_t ws_bytes,
+                     void* stream_) {
+  if (R < 0 || R > SA_MAX_USERS || n_cand < 0 || n_cand > INT32_MAX) return SA_ERR_INVALID_ARG;
+  if ((d != 64 && d != 128) || k < 1 || k > SA_MAX_K) return SA_ERR_UNSUPPORTED;
+  if (!cand_offsets || !cand_offsets_host || !Wq || !WK || !WV || !dWq || !dWK || !dWV ||
+      (n_cand > 0 && (!Q || !dout || !dQ)) || (R > 0 && (!S || !dS)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(cand_offsets) || !aligned16(S) || !aligned16(Wq) ||
+      !aligned16(WK) || !aligned16(WV) || !aligned16(dout) || !aligned16(dQ) || !aligned16(dS) ||
+      !aligned16(dWq) || !aligned16(dWK) || !aligned16(dWV))
+    return SA_ERR_INVALID_ARG;
+  // the host offsets decide the per-user GEMMs: check them before anything is launched
+  if (cand_offsets_host[0] != 0 || cand_offsets_host[R] != n_cand) return SA_ERR_BAD_OFFSETS;
+  for (int u = 0; u < R; ++u)
+    if (cand_offsets_host[u + 1] < cand_offsets_host[u]) return SA_ERR_BAD_OFFSETS;
+  Device dev;
+  sa_status st;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  StcaArgs a;
+  stca_plan(R, n_cand, k, d, true, dev.sms, &a.plan);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      ws_bytes < a.plan.total)
+    return SA_ERR_WORKSPACE;
+  a.Q = Q;
+  a.coff = cand_offsets;
+  a.R = R;
+  a.k = k;
+  a.d = d;
+  a.n_cand = n_cand;
+  a.S = S;
+  a.Wq = Wq;
+  a.WK = WK;
+  a.WV = WV;
+  a.out = nullptr;
+  a.lse = nullptr;
+  a.workspace = workspace;
+  StcaGrads g;
+  g.dout = dout;
+  g.coff_host = cand_offsets_host;
+  g.dQ = dQ;
+  g.dS = dS;
+  g.dWq = dWq;
+  g.dWK = dWK;
+  g.dWV = dWV;
+  return cuda_status(launch_stca_backward(a, g, static_cast<cudaStream_t>(stream_)));
+}
+
+int sa_sketch_pack(const float* sketch, int64_t rows, int d, int format, void* codes,
+                   float* scales, void* stream) {
+  if (rows < 0 || (format != SA_CODEC_BF16 && format != SA_CODEC_FP8)) return SA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+  if (rows > 0 && (!sketch || !codes || (format == SA_CODEC_FP8 && !scales)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(sketch) || !aligned16(codes) || !aligned16(scales)) return SA_ERR_INVALID_ARG;
+  return cuda_status(
+      launch_sketch_pack(sketch, rows, d, format, codes, scales, static_cast<cudaStream_t>(stream)));
+}
+
+int sa_sketch_unpack(const void* codes, const float* scales, int64_t rows, int d, int format,
+                     float* sketch, void* stream) {
+  if (rows < 0 || (format != SA_CODEC_BF16 && format != SA_CODEC_FP8)) return SA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+  if (rows > 0 && (!sketch || !codes || (format == SA_CODEC_FP8 && !scales)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(sketch) || !aligned16(codes) || !aligned16(scales)) return SA_ERR_INVALID_ARG;
+  return cuda_status(launch_sketch_unpack(codes, scales, rows, d, format, sketch,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
 int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_total, int d,
                        const void* P, int k, const void* Wk, const void* Wv, sa_dtype dt,
                        const float* sketch, const float* mass, const float* lse,

@@ -182,6 +182,46 @@ struct GemmArgs {
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
+// ---- candidate-to-sketch cross attention (sa_stca.cu)
+struct StcaPlan {  // workspace layout (byte offsets, 256-aligned)
+  int k_pad = 0, nparts = 0, splits = 0;
+  size_t hdr = 0, ts = 0, sb = 0, mt = 0, qp = 0, dpart = 0, lse2 = 0, ab = 0, o = 0, ohi = 0,
+         olo = 0, total = 0;
+  // backward only
+  size_t mts = 0, qn = 0, do_f = 0, do_b = 0, dd = 0, czero = 0, dz = 0, g1 = 0, g1hi = 0,
+         g1lo = 0, gb = 0, ob = 0, ghi = 0, glo = 0, part = 0, dm = 0;
+};
+size_t stca_plan(int R, long long n_cand, int k, int d, bool backward, int sms, StcaPlan* p);
+struct StcaArgs {
+  const void* Q;         // bf16 [n_cand, d]
+  const int64_t* coff;   // [R + 1]
+  int R, k, d;
+  long long n_cand;
+  const float* S;        // [R, k, d]
+  const void* Wq;        // bf16 [d, d]
+  const void* WK;
+  const void* WV;
+  float* out;            // [n_cand, d]
+  float* lse;            // [n_cand] natural log, nullable
+  void* workspace;
+  StcaPlan plan;
+};
+cudaError_t launch_stca_forward(const StcaArgs& a, cudaStream_t s);
+struct StcaGrads {
+  const float* dout;          // [n_cand, d]
+  const int64_t* coff_host;   // [R + 1], host copy of the candidate offsets
+  float* dQ;                  // [n_cand, d]
+  float* dS;                  // [R, k, d]
+  float *dWq, *dWK, *dWV;     // [d, d]
+};
+cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& g, cudaStream_t s);
+
+// ---- sketch cache codec (sa_codec.cu): format 0 = bf16, 1 = fp8 E4M3 with row scales
+cudaError_t launch_sketch_pack(const float* S, long long rows, int d, int format, void* codes,
+                               float* scales, cudaStream_t s);
+cudaError_t launch_sketch_unpack(const void* codes, const float* scales, long long rows, int d,
+                                 int format, float* S, cudaStream_t s);
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();
 

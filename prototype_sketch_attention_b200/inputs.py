@@ -127,3 +127,41 @@ def make_config(idx: int, k: int | None = None, with_grad: bool | None = None) -
                       name=name, gen=gen)
     w.meta["desc"] = c["desc"]
     return w
+
+
+@dataclass
+class CrossWorkload:
+    """Inputs of the candidate-to-sketch cross attention (CPU tensors)."""
+    R: int
+    k: int
+    d: int
+    counts: np.ndarray          # candidates per user
+    cand_offsets: torch.Tensor  # int64 [R+1]
+    Q: torch.Tensor             # bf16 [n_cand, d]
+    S: torch.Tensor             # fp32 [R, k, d]
+    Wq: torch.Tensor            # bf16 [d, d]
+    WK: torch.Tensor
+    WV: torch.Tensor
+
+    def to_f64(self) -> dict:
+        return dict(Q=self.Q.double().numpy(), cand_offsets=self.cand_offsets.numpy(),
+                    S=self.S.double().numpy(), Wq=self.Wq.double().numpy(),
+                    WK=self.WK.double().numpy(), WV=self.WV.double().numpy())
+
+
+def make_cross_workload(counts, k: int, d: int, seed: int, s_std: float = 1.0,
+                        S: torch.Tensor | None = None) -> CrossWorkload:
+    """Draw candidates Q ~ N(0, 1) (bf16), weights ~ N(0, 1/d) (bf16) and, unless given,
+    sketches S ~ N(0, s_std^2) (fp32) for the given candidate counts per user."""
+    gen = torch.Generator().manual_seed(seed)
+    counts = np.asarray(counts, dtype=np.int64)
+    R = len(counts)
+    off = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int64))
+    n = int(off[-1])
+    Q = torch.randn(n, d, generator=gen).to(torch.bfloat16)
+    Wq, WK, WV = ((torch.randn(d, d, generator=gen) / math.sqrt(d)).to(torch.bfloat16)
+                  for _ in range(3))
+    if S is None:
+        S = torch.randn(R, k, d, generator=gen) * s_std
+    return CrossWorkload(R=R, k=k, d=d, counts=counts, cand_offsets=off, Q=Q, S=S.float(),
+                         Wq=Wq, WK=WK, WV=WV)

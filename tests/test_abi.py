@@ -94,3 +94,16 @@ def test_combine_rejects_bad_arguments_on_host(lib):
     assert f(None, None, 1, 8, 100, None, 0, None, None) == 2   # d not in {64, 128}
     assert f(None, None, 1, 8, 64, None, 0, None, None) == 1    # null pointers
     assert f(None, None, 0, 8, 64, None, 0, None, None) == 0    # no users: nothing to do
+
+
+def test_codec_rejects_bad_arguments_on_host(lib):
+    vp, i32, i64 = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64
+    f = lib.sa_sketch_pack
+    f.restype = i32
+    f.argtypes = [vp, i64, i32, i32, vp, vp, vp]
+    assert f(16, 4, 128, 7, 16, 16, None) == 1     # unknown format
+    assert f(16, -1, 128, 1, 16, 16, None) == 1    # rows < 0
+    assert f(16, 4, 96, 1, 16, 16, None) == 2      # d not in {64, 128}
+    assert f(16, 4, 128, 1, 16, None, None) == 1   # fp8 needs scales
+    assert f(18, 4, 128, 0, 16, None, None) == 1   # misaligned
+    assert f(None, 0, 128, 1, None, None, None) == 0  # nothing to do

@@ -1,0 +1,162 @@
+"""CPU model of the launch sequence in csrc/sa_stca.cu, checked against the oracle.
+
+Each step below restates what one launch computes, from the contracts in
+csrc/sa_internal.h (launch_fold: Pf = scale * P Wk^T, rounded to bf16 when asked; the
+GEMM's kEpiLse / kEpiAExp / kEpiStoreF32 epilogues) and the kernels of sa_stca.cu,
+including every rounding to bf16. If the composition's algebra were wrong (a fold with
+its operands swapped, a missing log2(e), the sketch used untransposed, W_V applied on
+the wrong side), this model would miss the oracle by far more than the bf16 tolerance.
+It needs no GPU and shares nothing with the oracle.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from prototype_sketch_attention_b200 import inputs
+
+
+def bf16(a):
+    return torch.from_numpy(np.asarray(a, dtype=np.float32)).bfloat16().float().numpy().astype(np.float64)
+
+
+def fold(P, Wk, scale, to_bf16):
+    out = scale * (np.asarray(P, np.float64) @ np.asarray(Wk, np.float64).T)
+    return bf16(out) if to_bf16 else out.astype(np.float32).astype(np.float64)
+
+
+def model_forward(cw):
+    Q = cw.Q.float().numpy().astype(np.float64)
+    S = cw.S.numpy().astype(np.float64)
+    Wq, WK, WV = (t.float().numpy().astype(np.float64) for t in (cw.Wq, cw.WK, cw.WV))
+    R, k, d = S.shape
+    k_pad = (k + 127) // 128 * 128
+    coff = cw.cand_offsets.numpy()
+    Sb = np.zeros((R, k_pad, d))
+    Sb[:, :k] = bf16(S)                                        # stca_sketch_bf16_kernel
+    Mt = fold(WK, Wq, 1.0, True)                               # M^T = W_K W_q^T
+    Qp = fold(Q, Mt, math.log2(math.e) / math.sqrt(d), True)   # Q' = Q M log2(e) / sqrt(d)
+    out = np.zeros((Q.shape[0], d))
+    lse = np.zeros(Q.shape[0])
+    for u in range(R):
+        a, b = int(coff[u]), int(coff[u + 1])
+        if a == b:
+            continue
+        z = Qp[a:b] @ Sb[u].T                                  # scores, log2 units
+        z[:, k:] = -np.inf                                     # columns >= k_valid
+        m = z.max(axis=1, keepdims=True)
+        lse2 = (m + np.log2(np.exp2(z - m).sum(axis=1, keepdims=True)))[:, 0]
+        A = bf16(np.exp2(z - lse2[:, None]))                   # kEpiAExp
+        O = (A @ Sb[u]).astype(np.float32).astype(np.float64)  # kEpiStoreF32
+        hi = bf16(O)
+        lo = bf16(O - hi)
+        out[a:b] = hi @ bf16(WV) + lo @ bf16(WV)               # two GEMM phases
+        lse[a:b] = lse2 * math.log(2.0)
+    return out, lse
+
+
+@pytest.mark.parametrize("counts,k,d", [([300, 0, 1, 129], 1024, 128), ([5, 77], 200, 64),
+                                        ([40], 384, 64)])
+def test_composition_model_meets_the_oracle_within_bf16_tolerance(counts, k, d):
+    cw = inputs.make_cross_workload(counts, k, d, seed=500 + k + d + len(counts))
+    got, lse = model_forward(cw)
+    f = cw.to_f64()
+    ref = oracle.stca_forward(f["Q"], f["cand_offsets"], f["S"], f["Wq"], f["WK"], f["WV"])
+    off = f["cand_offsets"]
+    for u in range(cw.R):
+        a, b = int(off[u]), int(off[u + 1])
+        if a == b:
+            continue
+        num = np.linalg.norm(got[a:b] - ref["out"][a:b])
+        den = np.linalg.norm(ref["out"][a:b])
+        assert num / den <= 1e-2, (u, num / den)
+        assert np.abs(got[a:b] - ref["out"][a:b]).max() <= 5e-2
+    assert np.abs(lse - ref["lse"]).max() <= 5e-2
+
+
+def test_composition_model_catches_a_swapped_fold():
+    """The check above has teeth: folding W_q W_K^T the other way round fails it."""
+    cw = inputs.make_cross_workload([64, 30], 256, 64, seed=7)
+    f = cw.to_f64()
+    ref = oracle.stca_forward(f["Q"], f["cand_offsets"], f["S"], f["Wq"], f["WK"], f["WV"])
+    global fold
+    orig = fold
+    try:
+        fold = lambda P, Wk, scale, to_bf16: orig(Wk, P, scale, to_bf16) if P.shape == Wk.shape \
+            else orig(P, Wk, scale, to_bf16)
+        got, _ = model_forward(cw)
+    finally:
+        fold = orig
+    err = np.linalg.norm(got - ref["out"]) / np.linalg.norm(ref["out"])
+    assert err > 5e-2, err
+
+
+def model_backward(cw, G):
+    """The backward's launch sequence in sa_stca.cu, step by step, with its roundings."""
+    Q = cw.Q.float().numpy().astype(np.float64)
+    S = cw.S.numpy().astype(np.float64)
+    Wq, WK, WV = (t.float().numpy().astype(np.float64) for t in (cw.Wq, cw.WK, cw.WV))
+    R, k, d = S.shape
+    k_pad = (k + 127) // 128 * 128
+    coff = cw.cand_offsets.numpy()
+    n = Q.shape[0]
+    isd = 1.0 / math.sqrt(d)
+    Sb = np.zeros((R, k_pad, d))
+    Sb[:, :k] = bf16(S)
+    Mt = fold(WK, Wq, 1.0, True)
+    Qp = fold(Q, Mt, math.log2(math.e) * isd, True)
+    A = np.zeros((n, k_pad))
+    O = np.zeros((n, d))
+    for u in range(R):
+        a, b = int(coff[u]), int(coff[u + 1])
+        if a == b:
+            continue
+        z = Qp[a:b] @ Sb[u].T
+        z[:, k:] = -np.inf
+        m = z.max(axis=1, keepdims=True)
+        lse2 = m + np.log2(np.exp2(z - m).sum(axis=1, keepdims=True))
+        A[a:b] = bf16(np.exp2(z - lse2))
+        O[a:b] = (A[a:b] @ Sb[u]).astype(np.float32)
+    Gh, Gl = bf16(G), bf16(G - bf16(G))
+    dO = (Gh @ bf16(WV).T + Gl @ bf16(WV).T).astype(np.float32).astype(np.float64)
+    dWV = bf16(O).T @ bf16(G)
+    D = (dO * O).sum(axis=1)
+    dOb = bf16(dO)
+    dZ = np.zeros((n, k_pad))
+    G1 = np.zeros((n, d))
+    for u in range(R):
+        a, b = int(coff[u]), int(coff[u + 1])
+        if a == b:
+            continue
+        dZ[a:b] = bf16(A[a:b] * (dOb[a:b] @ Sb[u].T - D[a:b, None]))
+        G1[a:b] = (dZ[a:b] @ Sb[u]).astype(np.float32)
+    Mts = fold(WK, Wq, isd, True)
+    G1h, G1l = bf16(G1), bf16(G1 - bf16(G1))
+    dQ = G1h @ Mts + G1l @ Mts
+    dM = isd * (Q.T @ bf16(G1))
+    dWq = dM @ WK
+    dWK = dM.T @ Wq
+    Qn = fold(Q, Mt, isd, True)
+    dS = np.zeros((R, k, d))
+    for u in range(R):
+        a, b = int(coff[u]), int(coff[u + 1])
+        if a == b:
+            continue
+        dS[u] = (dZ[a:b].T @ Qn[a:b] + A[a:b].T @ dOb[a:b])[:k]
+    return {"dQ": dQ, "dS": dS, "dWq": dWq, "dWK": dWK, "dWV": dWV}
+
+
+@pytest.mark.parametrize("counts,k,d", [([300, 0, 1, 129], 1024, 128), ([5, 77], 200, 64)])
+def test_backward_composition_model_meets_the_oracle(counts, k, d):
+    cw = inputs.make_cross_workload(counts, k, d, seed=600 + k + d)
+    G = np.random.default_rng(601).standard_normal((int(cw.cand_offsets[-1]), d))
+    got = model_backward(cw, G)
+    f = cw.to_f64()
+    ref = oracle.stca_backward(f["Q"], f["cand_offsets"], f["S"], f["Wq"], f["WK"], f["WV"], G)
+    for key in ref:
+        r = ref[key]
+        e = np.linalg.norm(got[key] - r) / max(np.linalg.norm(r), 1e-30)
+        assert e <= 1e-2, (key, e)
+        assert np.abs(got[key] - r).max() <= 5e-2 * max(np.abs(r).max(), 1e-30), (key, "max-abs")
