@@ -162,8 +162,12 @@ int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int
  * pages describe no such interface; it has no counterpart in the paper.
  *
  * Same arguments, results and conventions as sa_sketch_forward, minus the workspace.
- * The scratch space is one device array of SA_NOALLOC_SCRATCH_BYTES per GPU, reserved
- * when this entry point is first used on that GPU and held until the process exits.
+ * The scratch space is one device array of SA_NOALLOC_SCRATCH_BYTES per GPU, held until
+ * the process exits. It is reserved when the CUDA module that holds it loads on that GPU:
+ * at the first use of the library's kernels under lazy module loading (the default), but
+ * already when the context is created under CUDA_MODULE_LOADING=EAGER, in which case every
+ * process that loads this library holds it on every GPU it uses, whether or not it calls
+ * this entry point.
  *  - The first call on each device looks up the array's device address (set-up, with
  *    that device current). Make that first call before any stream capture begins.
  *  - Every call on a device shares the one array: calls whose work overlaps on the GPU
@@ -174,7 +178,11 @@ int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int
  *  - It calls no cudaMalloc, cudaFree or allocating library routine.
  *  - device_status: nullable HOST pointer. When given, the call waits for `stream` and
  *    stores the device status word there (SA_OK, SA_ERR_BAD_OFFSETS, SA_ERR_TIMEOUT), since
- *    the caller cannot name the scratch array in sa_sketch_get_device_status.
+ *    the caller cannot name the scratch array in sa_sketch_get_device_status. If that read
+ *    fails (for example a stream in capture, or an earlier asynchronous CUDA error), the
+ *    call returns SA_ERR_CUDA and leaves *device_status unchanged. Pass NULL while a stream
+ *    capture is active.
+ *  - Argument errors give the same codes as sa_sketch_forward.
  */
 #define SA_NOALLOC_SCRATCH_BYTES (32u << 20)
 int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, int R, int64_t n_total,

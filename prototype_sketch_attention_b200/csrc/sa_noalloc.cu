@@ -56,7 +56,11 @@ extern "C" int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, 
                                          float* sketch, float* mass, float* lse,
                                          float* xsketch, int* device_status, void* stream) {
   const size_t need = sa_sketch_workspace_size(R, n_total, k, d, dt, 0);
-  if (need == 0) return SA_ERR_UNSUPPORTED;
+  // No plan for these arguments: the regular forward fails the same checks before any
+  // launch (it never reads a workspace it was not given) and returns their exact code.
+  if (need == 0)
+    return sa_sketch_forward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass, lse,
+                             xsketch, nullptr, 0, stream);
   if (need > (size_t)SA_NOALLOC_SCRATCH_BYTES) return SA_ERR_WORKSPACE;
   void* scratch = nullptr;
   int st = scratch_for_current_device(&scratch);
@@ -64,6 +68,8 @@ extern "C" int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, 
   st = sa_sketch_forward(X, offsets, R, n_total, d, P, k, Wk, Wv, dt, sketch, mass, lse, xsketch,
                          scratch, (size_t)SA_NOALLOC_SCRATCH_BYTES, stream);
   if (st != SA_OK || device_status == nullptr) return st;
-  *device_status = sa_sketch_get_device_status(scratch, stream);
+  const int dev_st = sa_sketch_get_device_status(scratch, stream);
+  if (dev_st == SA_ERR_CUDA) return SA_ERR_CUDA;  // the status read itself failed
+  *device_status = dev_st;
   return SA_OK;
 }

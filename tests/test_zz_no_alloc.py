@@ -52,6 +52,40 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
         assert np.abs(lse_got - ref["lse"].cpu().double().numpy()).max() <= BF16_ABS, call
 
 
+def test_noalloc_matches_the_oracle():
+    """One case checked against the fp64 oracle directly, so this file stands alone."""
+    from parity_util import check_forward
+    w = inputs.make_workload([2100, 0, 130, 700], 128, 512, "bf16", seed=4343)
+    g = {n: getattr(w, n).cuda() for n in ("X", "offsets", "P", "Wk", "Wv")}
+    R, n_total, d, k = w.R, w.n_total, w.d, w.k
+    for call in range(2):
+        out = {"sketch": torch.full((R, k, d), float("nan"), device="cuda"),
+               "mass": torch.full((R, k), float("nan"), device="cuda"),
+               "lse": torch.full((n_total,), float("nan"), device="cuda"),
+               "xsketch": torch.full((R, k, d), float("nan"), device="cuda")}
+        rc, st = _noalloc(g, R, n_total, d, k, out)
+        assert rc == binding.SA_OK and st == binding.SA_OK, (call, rc, st)
+        check_forward(w, out)
+
+
+def test_noalloc_argument_errors_match_the_forward():
+    w = inputs.make_workload([300], 128, 256, "bf16", seed=5)
+    g = {n: getattr(w, n).cuda() for n in ("X", "offsets", "P", "Wk", "Wv")}
+    out = {"sketch": torch.empty((1, 256, 128), device="cuda"),
+           "mass": torch.empty((1, 256), device="cuda"),
+           "lse": torch.empty((300,), device="cuda"),
+           "xsketch": torch.empty((1, 256, 128), device="cuda")}
+    rc, _ = _noalloc(g, 1, 300, 96, 256, out)
+    assert rc == binding.SA_ERR_UNSUPPORTED
+    st = ctypes.c_int(-1)
+    rc = binding.sa_sketch_forward_noalloc(
+        g["X"].data_ptr(), g["offsets"].data_ptr(), 1, 300, 128, g["P"].data_ptr(), 256,
+        g["Wk"].data_ptr(), g["Wv"].data_ptr(), 9, out["sketch"].data_ptr(),
+        out["mass"].data_ptr(), None, None, ctypes.addressof(st),
+        torch.cuda.current_stream().cuda_stream)
+    assert rc == binding.SA_ERR_INVALID_ARG and st.value == -1
+
+
 def test_noalloc_rejects_sizes_beyond_its_scratch():
     # 200 users at k = 2048 need far more than the fixed scratch: rejected before launch
     R, n_total, d, k = 200, 200 * 128, 128, 2048
