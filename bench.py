@@ -405,11 +405,11 @@ def run_ours(args) -> None:
     if st != 0:
         raise SystemExit(f"forward failed on device: {binding.sa_status_string(st)}")
 
-    # ---- e2e through the public API: pinned host inputs -> device -> forward -> host.
-    # binding.forward_from_host cuts the users into parts, so each part's host-to-device
-    # copy overlaps the previous part's forward (one sa_sketch_forward call per part).
+    # ---- e2e through the C ABI with HOST buffers: sa_sketch_forward_host takes pinned
+    # host X and offsets and writes pinned host sketch and mass; it cuts the users into
+    # parts, so each part's host-to-device copy overlaps the previous part's forward.
     Xh = w.X.pin_memory()
-    offh = w.offsets.clone()
+    offh = w.offsets.pin_memory()
     e2e_state = {}
     e2e_steps = max(3, min(args.steps, 20))
 

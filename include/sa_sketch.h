@@ -136,6 +136,66 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
                        void* workspace, size_t ws_bytes, void* stream);
 
 /*
+ * Forward from HOST inputs to HOST outputs, with the copies overlapped with the compute.
+ * Same computation as sa_sketch_forward (blog "1. Sketch Attention compresses the
+ * history"); users are independent, and the batch is ragged (blog "3. The system makes it
+ * cheap enough to matter": multi-request user-level batching), so the call cuts the users
+ * into at most `parts` consecutive parts of about equal token count
+ * (sa_sketch_host_parts) and pipelines them: part p's X is copied to the device on
+ * `h2d_stream` while part p - 1's forward runs on `stream`, and part p's sketch and mass
+ * are copied back on `d2h_stream` as soon as its forward has finished.
+ *
+ *   X_host       [n_total, d] dt, HOST       history tokens of all users
+ *   offsets_host [R + 1] int64, HOST         offsets[0] = 0, non-decreasing,
+ *                                            offsets[R] = n_total (checked on the host)
+ *   P, Wk, Wv    dt, DEVICE                  as for sa_sketch_forward
+ *   sketch_host  [R, k, d] fp32, HOST        output (overwritten)
+ *   mass_host    [R, k] fp32, HOST           output (overwritten)
+ *   device_buffer, device_bytes              DEVICE scratch of at least
+ *                sa_sketch_forward_host_buffer_size(...) bytes, 256-byte aligned: the
+ *                device copy of X and offsets, the device sketch and mass, and the
+ *                forward's workspace. Not shared with another call in flight.
+ *   parts        1..64 (use 1 when k is not a multiple of 4)
+ *   stream, h2d_stream, d2h_stream           three cudaStream_t (as void*); the two copy
+ *                streams should be distinct from `stream` and from each other for the
+ *                copies to overlap (the default stream serialises everything)
+ * The call only enqueues work. The outputs are complete once `stream` has reached the end
+ * of this call's work (synchronise it, or record an event on it). X_host and offsets_host
+ * must stay unchanged until then. For the copies to run asynchronously the four host
+ * buffers must be page-locked (cudaHostAlloc or cudaHostRegister); pageable buffers give
+ * correct results but serialise the copies with the host. It creates and releases a few
+ * CUDA events per call and allocates no memory. Returns SA_OK, the argument codes of
+ * sa_sketch_forward, SA_ERR_BAD_OFFSETS (offsets_host invalid), SA_ERR_WORKSPACE or
+ * SA_ERR_CUDA. Device-side errors are latched in the workspace inside device_buffer, at
+ * offset 0 of the workspace region; read them with sa_sketch_forward_host_status.
+ */
+size_t sa_sketch_forward_host_buffer_size(int R, int64_t n_total, int k, int d, sa_dtype dt,
+                                          int parts);
+int sa_sketch_forward_host(const void* X_host, const int64_t* offsets_host, int R,
+                           int64_t n_total, int d, const void* P, int k, const void* Wk,
+                           const void* Wv, sa_dtype dt, float* sketch_host, float* mass_host,
+                           void* device_buffer, size_t device_bytes, int parts, void* stream,
+                           void* h2d_stream, void* d2h_stream);
+
+/*
+ * Device status word of the last sa_sketch_forward_host call that used `device_buffer`
+ * with these sizes (synchronises `stream`); the same codes as sa_sketch_get_device_status.
+ */
+int sa_sketch_forward_host_status(const void* device_buffer, int R, int64_t n_total, int k,
+                                  int d, sa_dtype dt, int parts, void* stream);
+
+/*
+ * The cut that sa_sketch_forward_host uses: users [0, R) into at most `parts` consecutive
+ * parts of about equal token count. Cut c ends a part at the first user whose tokens
+ * reach c / parts of the total; a cut that would leave a part without tokens is dropped,
+ * and users without tokens at the end join the last part, so every part but a lone one
+ * holds tokens and no user is split. Writes the part boundaries to bounds[0..np] (HOST,
+ * room for parts + 1 ints; bounds[0] = 0, bounds[np] = R) and returns np (0 when R = 0),
+ * or -SA_ERR_INVALID_ARG if the offsets are not a valid ragged partition. Host only.
+ */
+int sa_sketch_host_parts(const int64_t* offsets_host, int R, int parts, int* bounds);
+
+/*
  * Epilogue for a user whose tokens were split across calls (for example across GPUs,
  * one part per rank). The forward's accumulation is a plain sum over tokens, so the
  * parts' xsketch and mass outputs add up to the whole user's (the sketch's definition
@@ -189,6 +249,16 @@ int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, int R, int6
                               int d, const void* P, int k, const void* Wk, const void* Wv,
                               sa_dtype dt, float* sketch, float* mass, float* lse,
                               float* xsketch, int* device_status, void* stream);
+
+/*
+ * Launch shape of the bf16 forward on the current device: the persistent grid holds
+ * *clusters clusters of *cluster_size CTAs (one CTA per 128 prototypes), and cluster g
+ * walks tiles [g T / clusters, (g + 1) T / clusters) of the T 128-token tiles of the
+ * batch (users' tiles concatenated). A user whose tiles straddle one of those bounds is
+ * accumulated by two clusters and summed in the finalize. For fp32 inputs (CUDA-core
+ * path) both are set to 0. Returns SA_OK, or the argument codes of sa_sketch_forward.
+ */
+int sa_sketch_forward_grid(int k, int d, sa_dtype dt, int* clusters, int* cluster_size);
 
 /*
  * Reads the device status word that the last call using `workspace` left behind.

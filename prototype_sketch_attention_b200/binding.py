@@ -32,7 +32,9 @@ EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward
             "sa_sketch_get_device_status", "sa_status_string", "sa_sketch_debug_wait_timeout",
             "sa_sketch_profile_events", "sa_sketch_forward_noalloc", "sa_sketch_combine",
             "sa_sketch_debug_gemm", "sa_stca_workspace_size", "sa_stca_forward",
-            "sa_stca_backward", "sa_sketch_pack", "sa_sketch_unpack")
+            "sa_stca_backward", "sa_sketch_pack", "sa_sketch_unpack",
+            "sa_sketch_forward_host_buffer_size", "sa_sketch_forward_host",
+            "sa_sketch_forward_host_status", "sa_sketch_host_parts", "sa_sketch_forward_grid")
 SA_CODEC_BF16 = 0
 SA_CODEC_FP8 = 1
 
@@ -83,6 +85,17 @@ def _load() -> ctypes.CDLL:
                                      vp, vp, vp, vp, sz, vp]
     lib.sa_stca_forward.restype = i32
     lib.sa_stca_forward.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sa_sketch_forward_host_buffer_size.restype = sz
+    lib.sa_sketch_forward_host_buffer_size.argtypes = [i32, i64, i32, i32, i32, i32]
+    lib.sa_sketch_forward_host.restype = i32
+    lib.sa_sketch_forward_host.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32, vp, vp,
+                                           vp, sz, i32, vp, vp, vp]
+    lib.sa_sketch_forward_host_status.restype = i32
+    lib.sa_sketch_forward_host_status.argtypes = [vp, i32, i64, i32, i32, i32, i32, vp]
+    lib.sa_sketch_forward_grid.restype = i32
+    lib.sa_sketch_forward_grid.argtypes = [i32, i32, i32, vp, vp]
+    lib.sa_sketch_host_parts.restype = i32
+    lib.sa_sketch_host_parts.argtypes = [vp, i32, i32, vp]
     return lib
 
 
@@ -129,6 +142,41 @@ def sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse, w
                     ws_bytes, stream) -> int:
     return int(_lib.sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse,
                                     workspace, ws_bytes, stream))
+
+
+def sa_sketch_forward_host_buffer_size(R, n_total, k, d, dt, parts) -> int:
+    return int(_lib.sa_sketch_forward_host_buffer_size(R, n_total, k, d, dt, parts))
+
+
+def sa_sketch_forward_host(X_host, offsets_host, R, n_total, d, P, k, Wk, Wv, dt, sketch_host,
+                           mass_host, device_buffer, device_bytes, parts, stream, h2d_stream,
+                           d2h_stream) -> int:
+    return int(_lib.sa_sketch_forward_host(X_host, offsets_host, R, n_total, d, P, k, Wk, Wv, dt,
+                                           sketch_host, mass_host, device_buffer, device_bytes,
+                                           parts, stream, h2d_stream, d2h_stream))
+
+
+def sa_sketch_forward_host_status(device_buffer, R, n_total, k, d, dt, parts, stream) -> int:
+    return int(_lib.sa_sketch_forward_host_status(device_buffer, R, n_total, k, d, dt, parts,
+                                                  stream))
+
+
+def sa_sketch_forward_grid(k, d, dt, clusters, cluster_size) -> int:
+    return int(_lib.sa_sketch_forward_grid(k, d, dt, clusters, cluster_size))
+
+
+def forward_grid(k: int, d: int, dtype=torch.bfloat16) -> tuple[int, int]:
+    """(clusters, cluster_size) of the bf16 forward's persistent grid on the current device."""
+    c, s = ctypes.c_int(0), ctypes.c_int(0)
+    st = sa_sketch_forward_grid(k, d, SA_BF16 if dtype == torch.bfloat16 else SA_F32,
+                                ctypes.addressof(c), ctypes.addressof(s))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_sketch_forward_grid")
+    return c.value, s.value
+
+
+def sa_sketch_host_parts(offsets_host, R, parts, bounds) -> int:
+    return int(_lib.sa_sketch_host_parts(offsets_host, R, parts, bounds))
 
 
 def sa_sketch_pack(sketch, rows, d, fmt, codes, scales, stream) -> int:
@@ -463,41 +511,31 @@ def stca_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, 
 
 
 def user_chunks(offsets_host: torch.Tensor, chunks: int) -> list[tuple[int, int]]:
-    """Cut users [0, R) into at most `chunks` consecutive ranges of about equal token
-    count: range c ends at the first user whose tokens reach c / chunks of the total (a
-    user is never split; a range without tokens joins the next one).
-    offsets_host: int64 [R + 1] on the host."""
-    R = offsets_host.numel() - 1
-    if R <= 0:
-        return []
-    n_total = int(offsets_host[R])
-    ends = offsets_host[1:]
-    cuts = []
-    for c in range(1, chunks):
-        u1 = int(torch.searchsorted(ends, torch.tensor(n_total * c // chunks))) + 1
-        if 0 < u1 < R and (not cuts or u1 > cuts[-1]) and int(offsets_host[u1]) > (
-                int(offsets_host[cuts[-1]]) if cuts else 0):
-            cuts.append(u1)
-    while cuts and int(offsets_host[R]) == int(offsets_host[cuts[-1]]):
-        cuts.pop()  # trailing users without tokens join the last range
-    bounds = [0] + cuts + [R]
-    return [(bounds[i], bounds[i + 1]) for i in range(len(bounds) - 1)]
+    """The library's cut of users [0, R) into at most `chunks` consecutive parts of about
+    equal token count (sa_sketch_host_parts). offsets_host: int64 [R + 1] on the host."""
+    _require(isinstance(offsets_host, torch.Tensor) and offsets_host.dtype == torch.int64
+             and offsets_host.device.type == "cpu" and offsets_host.dim() == 1,
+             "user_chunks", "offsets_host must be a host int64 [R + 1] tensor")
+    off = offsets_host.contiguous()
+    R = off.numel() - 1
+    bounds = (ctypes.c_int * (max(int(chunks), 1) + 1))()
+    np_ = sa_sketch_host_parts(off.data_ptr(), R, int(chunks), ctypes.addressof(bounds))
+    if np_ < 0:
+        raise SketchAttentionError(-np_, "sa_sketch_host_parts")
+    return [(bounds[i], bounds[i + 1]) for i in range(np_)]
 
 
 def forward_from_host(Xh: torch.Tensor, offsets_h: torch.Tensor, P: torch.Tensor,
                       Wk: torch.Tensor, Wv: torch.Tensor, *, chunks: int = 4,
                       state: dict | None = None) -> tuple[torch.Tensor, torch.Tensor]:
-    """Forward from host X and offsets (pinned) to host sketch and mass (pinned).
-
-    The users are cut into about `chunks` consecutive parts of equal token count. Part
-    c's X is copied to the device on a copy stream while part c - 1's forward runs on
-    the current stream, and part c's sketch and mass go back on a third stream as soon
-    as its forward is done; each part is one sa_sketch_forward call (users are
-    independent, so no combining). P, Wk, Wv live on the device. `state` (a dict the
-    caller keeps) holds the device buffers, pinned staging and streams between calls.
-    The current stream waits for the copies back before this returns, so work queued on
-    it afterwards (an event, a synchronize) sees the outputs. The returned host tensors
-    are the state's staging: the next call with the same `state` overwrites them."""
+    """Forward from host X and offsets to host sketch and mass through
+    sa_sketch_forward_host, which cuts the users into `chunks` parts and overlaps each
+    part's copy to the device with the previous part's forward (the library owns the
+    pipeline; this function only marshals). Xh and offsets_h should be pinned. P, Wk, Wv
+    live on the device. `state` (a dict the caller keeps) holds the device buffer, the
+    pinned outputs and the two copy streams between calls. The outputs are complete once
+    the current stream reaches the end of this call's work; the returned host tensors are
+    the state's staging, which the next call with the same `state` overwrites."""
     where = "forward_from_host"
     _require(isinstance(Xh, torch.Tensor) and Xh.dim() == 2 and Xh.device.type == "cpu"
              and Xh.is_contiguous(), where, "Xh must be a contiguous 2-D host tensor")
@@ -510,58 +548,41 @@ def forward_from_host(Xh: torch.Tensor, offsets_h: torch.Tensor, P: torch.Tensor
     n_total, d = Xh.shape
     k = P.shape[0]
     dev = P.device
-    if k % 4:
-        chunks = 1  # a part's mass rows must start 16-byte aligned
+    dt = _dt(Xh)
+    _check_tensor(where, "P", P, (k, d), Xh.dtype, dev)
+    _check_tensor(where, "Wk", Wk, (d, d), Xh.dtype, dev)
+    _check_tensor(where, "Wv", Wv, (d, d), Xh.dtype, dev)
     st = {} if state is None else state
-    key = (R, n_total, k, d, Xh.dtype, chunks, dev)
+    key = (R, n_total, k, d, Xh.dtype, int(chunks), dev)
     if st.get("key") != key:
         st.clear()
-        st.update(
-            key=key,
-            Xd=torch.empty(n_total, d, dtype=Xh.dtype, device=dev),
-            offd=torch.empty(R + 2 * chunks + 2, dtype=torch.int64, device=dev),
-            offp=torch.empty(R + 2 * chunks + 2, dtype=torch.int64).pin_memory(),
-            sketch=torch.empty(R, k, d, dtype=torch.float32, device=dev),
-            mass=torch.empty(R, k, dtype=torch.float32, device=dev),
-            sk_h=torch.empty(R, k, d, dtype=torch.float32).pin_memory(),
-            ms_h=torch.empty(R, k, dtype=torch.float32).pin_memory(),
-            ws=workspace(R, n_total, k, d, Xh.dtype, False, dev),
-            s_copy=torch.cuda.Stream(dev), s_back=torch.cuda.Stream(dev), off_done=None)
+        with torch.cuda.device(dev):
+            nb = sa_sketch_forward_host_buffer_size(R, n_total, k, d, dt, int(chunks))
+            if nb == 0:
+                raise SketchAttentionError(SA_ERR_UNSUPPORTED, "sa_sketch_forward_host_buffer_size")
+            st.update(key=key, buf=torch.empty(nb, dtype=torch.uint8, device=dev),
+                      sk_h=torch.empty(R, k, d, dtype=torch.float32).pin_memory(),
+                      ms_h=torch.empty(R, k, dtype=torch.float32).pin_memory(),
+                      s_h2d=torch.cuda.Stream(dev), s_d2h=torch.cuda.Stream(dev))
+    off = offsets_h.contiguous()
     cur = torch.cuda.current_stream(dev)
-    s_copy, s_back = st["s_copy"], st["s_back"]
-    # the pinned offsets staging is rewritten below: its previous copy must have run
-    if st["off_done"] is not None:
-        st["off_done"].synchronize()
-    parts = user_chunks(offsets_h, chunks)
-    at, spans = 0, []
-    for u0, u1 in parts:  # each part's offsets, rebased to 0, side by side in the staging
-        torch.sub(offsets_h[u0:u1 + 1], offsets_h[u0], out=st["offp"][at:at + u1 - u0 + 1])
-        spans.append((at, at + u1 - u0 + 1))
-        at += (u1 - u0 + 2) & ~1  # the next part's offsets start 16-byte aligned
-    s_copy.wait_stream(cur)
-    s_back.wait_stream(cur)
-    with torch.cuda.stream(s_copy):
-        st["offd"][:at].copy_(st["offp"][:at], non_blocking=True)
-    off_done = torch.cuda.Event()
-    off_done.record(s_copy)
-    st["off_done"] = off_done
-    for (u0, u1), (a, b) in zip(parts, spans):
-        t0, t1 = int(offsets_h[u0]), int(offsets_h[u1])
-        with torch.cuda.stream(s_copy):
-            st["Xd"][t0:t1].copy_(Xh[t0:t1], non_blocking=True)
-        landed = torch.cuda.Event()
-        landed.record(s_copy)
-        cur.wait_event(landed)
-        forward(st["Xd"][t0:t1], st["offd"][a:b], P, Wk, Wv, ws=st["ws"],
-                out={"sketch": st["sketch"][u0:u1], "mass": st["mass"][u0:u1]}, stream=cur)
-        done = torch.cuda.Event()
-        done.record(cur)
-        s_back.wait_event(done)
-        with torch.cuda.stream(s_back):
-            st["sk_h"][u0:u1].copy_(st["sketch"][u0:u1], non_blocking=True)
-            st["ms_h"][u0:u1].copy_(st["mass"][u0:u1], non_blocking=True)
-    cur.wait_stream(s_back)
+    with torch.cuda.device(dev):
+        rc = sa_sketch_forward_host(_ptr(Xh), off.data_ptr(), R, n_total, d, _ptr(P), k, _ptr(Wk),
+                                    _ptr(Wv), dt, _ptr(st["sk_h"]), _ptr(st["ms_h"]),
+                                    _ptr(st["buf"]), st["buf"].nbytes, int(chunks),
+                                    cur.cuda_stream, st["s_h2d"].cuda_stream,
+                                    st["s_d2h"].cuda_stream)
+    if rc != SA_OK:
+        raise SketchAttentionError(rc, "sa_sketch_forward_host")
     return st["sk_h"], st["ms_h"]
+
+
+def forward_from_host_status(state: dict, stream=None) -> int:
+    """Device status of the last forward_from_host call made with `state` (synchronises)."""
+    R, n_total, k, d, dtype, chunks, dev = state["key"]
+    return sa_sketch_forward_host_status(_ptr(state["buf"]), R, n_total, k, d,
+                                         SA_BF16 if dtype == torch.bfloat16 else SA_F32, chunks,
+                                         _stream(stream, dev))
 
 
 def device_status(ws: torch.Tensor, stream=None) -> int:

@@ -579,6 +579,19 @@ int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M
   return cuda_status(launch_gemm(g, static_cast<cudaStream_t>(stream_)));
 }
 
+int sa_sketch_forward_grid(int k, int d, sa_dtype dt, int* clusters, int* cluster_size) {
+  if (!clusters || !cluster_size) return SA_ERR_INVALID_ARG;
+  sa_status st = check_sizes(0, 0, k, d, dt);
+  if (st != SA_OK) return st;
+  Device dev;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  Plan p;
+  if ((st = make_plan(dev, 0, 0, k, d, dt, false, &p)) != SA_OK) return st;
+  *clusters = p.tc ? p.G : 0;
+  *cluster_size = p.tc ? p.C : 0;
+  return SA_OK;
+}
+
 int sa_sketch_get_device_status(const void* workspace, void* stream_) {
   if (!workspace) return SA_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream_);

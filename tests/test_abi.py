@@ -107,3 +107,38 @@ def test_codec_rejects_bad_arguments_on_host(lib):
     assert f(16, 4, 128, 1, 16, None, None) == 1   # fp8 needs scales
     assert f(18, 4, 128, 0, 16, None, None) == 1   # misaligned
     assert f(None, 0, 128, 1, None, None, None) == 0  # nothing to do
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), 2), (dict(k=0), 2), (dict(dt=7), 1), (dict(R=-1), 1), (dict(n_total=-5), 1),
+])
+def test_noalloc_returns_the_forwards_argument_codes(lib, kw, code):
+    """The forward without a workspace rejects bad arguments with the same codes as
+    sa_sketch_forward, before any CUDA call (these run without a GPU)."""
+    vp, i64, i32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    f = lib.sa_sketch_forward_noalloc
+    f.restype = i32
+    f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32, vp, vp, vp, vp, vp, vp]
+    a = dict(R=1, n_total=10, d=128, k=1024, dt=1)
+    a.update(kw)
+    got = f(16, 16, a["R"], a["n_total"], a["d"], 16, a["k"], 16, 16, a["dt"], 16, 16, None, None,
+            None, None)
+    assert got == code == _fwd(lib, **kw)
+
+
+def test_forward_host_rejects_bad_host_offsets(lib):
+    """The host-to-host forward checks the host offsets before any CUDA call."""
+    import numpy as np
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    f = lib.sa_sketch_forward_host
+    f.restype = i32
+    f.argtypes = [vp, vp, i32, i64, i32, vp, i32, vp, vp, i32, vp, vp, vp, sz, i32, vp, vp, vp]
+    X = np.zeros((10, 128), dtype=np.uint16)
+    out = np.zeros((2, 1024, 128), dtype=np.float32)
+    m = np.zeros((2, 1024), dtype=np.float32)
+    for off, code in (([0, 6, 4], 6), ([1, 4, 10], 6), ([0, 4, 9], 6), ([0, 4, 10], 3)):
+        o = np.asarray(off, dtype=np.int64)
+        rc = f(X.ctypes.data, o.ctypes.data, 2, 10, 128, 16, 1024, 16, 16, 1, out.ctypes.data,
+               m.ctypes.data, None, 0, 4, None, None, None)
+        # valid offsets without a device fail on the plan (no device) or the buffer
+        assert rc == code or (code == 3 and rc == 7), (off, rc)

@@ -62,21 +62,45 @@ def _unit_mass_all_users(w, out):
     np.testing.assert_allclose(mass, n, rtol=2e-3)
 
 
+def _boundary_users(w, k, d):
+    """Users whose tiles straddle a bound between two clusters' tile ranges of the
+    persistent forward grid: two clusters accumulate parts of them, which the finalize
+    sums. Longest first."""
+    from prototype_sketch_attention_b200 import binding
+    G, _ = binding.forward_grid(k, d)
+    tiles = (np.diff(w.offsets.numpy()) + 127) // 128
+    ts = np.concatenate([[0], np.cumsum(tiles)])
+    T = int(ts[-1])
+    bounds = [g * T // G for g in range(1, G)]
+    users = {int(np.searchsorted(ts, b, side="right") - 1) for b in bounds}
+    users = [u for u in users if any(ts[u] < b < ts[u + 1] for b in bounds)]
+    return sorted(users, key=lambda u: -int(tiles[u]))
+
+
 def test_config3_sampled_users():
+    """Shortest, median and longest user, and the longest user cut between clusters."""
     w = inputs.make_config(3)
     _, out = gpu_forward(w)
     _unit_mass_all_users(w, out)
     order = np.argsort(w.lengths)
-    check_forward(w, out, users=[int(order[0]), int(order[len(order) // 2])])
+    cut = _boundary_users(w, w.k, w.d)
+    assert cut, "the batch spans several clusters"
+    users = {int(order[0]), int(order[len(order) // 2]), int(order[-1]), cut[0]}
+    check_forward(w, out, users=sorted(users))
 
 
 @pytest.mark.parametrize("k", [256, 512, 1024, 2048])
 def test_config4_sampled_users(k):
+    """The two shortest users, the median, the longest, and the longest user cut between
+    clusters."""
     w = inputs.make_config(4, k=k)
     _, out = gpu_forward(w)
     _unit_mass_all_users(w, out)
     order = np.argsort(w.lengths)
-    check_forward(w, out, users=[int(order[0]), int(order[1]), int(order[150])])
+    cut = _boundary_users(w, k, w.d)
+    assert cut, "the batch spans several clusters"
+    users = {int(order[0]), int(order[1]), int(order[150]), int(order[-1]), cut[0]}
+    check_forward(w, out, users=sorted(users))
 
 
 def test_deterministic_bitwise():
@@ -133,20 +157,25 @@ def test_bounded_wait_times_out_and_context_survives():
     ([500, 600], 2),
 ])
 def test_forward_from_host_matches_device_forward(lengths, k):
-    # users cut into parts whose copies overlap the previous part's forward
+    # sa_sketch_forward_host: users cut into parts whose copies overlap the previous
+    # part's forward, host buffers in and out; against the device forward and the oracle
     from prototype_sketch_attention_b200 import binding
     w = inputs.make_workload(lengths, 128, k, "bf16", seed=77 + k)
     g = {n: getattr(w, n).cuda() for n in ("X", "offsets", "P", "Wk", "Wv")}
     ref = binding.forward(g["X"], g["offsets"], g["P"], g["Wk"], g["Wv"])
     state = {}
-    for _ in range(2):  # the second call reuses the buffers and streams
-        sk, ms = binding.forward_from_host(w.X.pin_memory(), w.offsets, g["P"], g["Wk"], g["Wv"],
-                                           chunks=4, state=state)
-        torch.cuda.synchronize()
+    Xh, offh = w.X.pin_memory(), w.offsets.pin_memory()
+    for call in range(2):  # the second call reuses the buffers and streams
+        sk, ms = binding.forward_from_host(Xh, offh, g["P"], g["Wk"], g["Wv"], chunks=4,
+                                           state=state)
+        torch.cuda.current_stream().synchronize()
+        assert binding.forward_from_host_status(state) == 0
         exp_s, exp_m = ref["sketch"].cpu().double(), ref["mass"].cpu().double()
         for u in range(w.R):
             assert rel_l2(sk[u].double().numpy(), exp_s[u].numpy()) <= 1e-5
             assert rel_l2(ms[u].double().numpy(), exp_m[u].numpy()) <= 1e-5
+        if call == 0:
+            check_forward(w, {"sketch": sk.clone(), "mass": ms.clone()})
 
 
 def test_bf16_extreme_scores_take_the_shifted_path():
