@@ -35,7 +35,7 @@ def test_backward_small_full_compare(lengths, k, d, dtype, with_gm):
     sub = w.to_f64()
     ref = oracle.backward(sub["X"], sub["offsets"], sub["P"], sub["Wk"], sub["Wv"], G, Gm,
                           nthreads=nthreads())
-    check_grads(got, ref, fp32=(dtype == "f32"))
+    check_grads(got, ref, fp32=(dtype == "f32"), offsets=sub["offsets"])
 
 
 def test_config5_full_size_one_user_gradient():
@@ -55,7 +55,8 @@ def test_config5_full_size_one_user_gradient():
     dX_u = got["dX"][off[u]:off[u + 1]]
     rest = np.concatenate([got["dX"][:off[u]], got["dX"][off[u + 1]:]])
     assert not rest.any()
-    check_grads({"dX": dX_u, "dP": got["dP"], "dWk": got["dWk"], "dWv": got["dWv"]}, ref, fp32=False)
+    check_grads({"dX": dX_u, "dP": got["dP"], "dWk": got["dWk"], "dWv": got["dWv"]}, ref, fp32=False,
+                offsets=sub["offsets"])
 
 
 @pytest.mark.parametrize("lengths,k,d", [([300, 0, 1037], 256, 128), ([129, 5], 384, 64)])
@@ -71,8 +72,8 @@ def test_backward_recomputes_lse_when_not_given(lengths, k, d):
     sub = w.to_f64()
     ref = oracle.backward(sub["X"], sub["offsets"], sub["P"], sub["Wk"], sub["Wv"], G,
                           nthreads=nthreads())
-    check_grads(with_lse, ref, fp32=False)
-    check_grads(without, ref, fp32=False)
+    check_grads(with_lse, ref, fp32=False, offsets=sub["offsets"])
+    check_grads(without, ref, fp32=False, offsets=sub["offsets"])
     for key in ("dX", "dP", "dWk", "dWv"):
         assert rel_l2(without[key], with_lse[key]) <= 2e-3, key
 
@@ -86,4 +87,4 @@ def test_backward_bf16_k_not_multiple_of_128():
     sub = w.to_f64()
     ref = oracle.backward(sub["X"], sub["offsets"], sub["P"], sub["Wk"], sub["Wv"], G,
                           nthreads=nthreads())
-    check_grads(got, ref, fp32=False)
+    check_grads(got, ref, fp32=False, offsets=sub["offsets"])
