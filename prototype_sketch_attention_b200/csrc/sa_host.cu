@@ -45,16 +45,19 @@ sa_status current_device(Device* dev) {
   return SA_OK;
 }
 
-// Co-resident clusters of the tcgen05 forward, cached per (device, d, C).
-sa_status tc_clusters(const Device& dev, int d, int C, int* G) {
+// Co-resident clusters of the tcgen05 forward (which = 0) or of the single-pass backward
+// (which = 1), cached per (device, kernel, d, C).
+sa_status tc_clusters(const Device& dev, int d, int C, int* G, int which = 0) {
   static std::mutex mu;
-  static std::map<std::tuple<int, int, int>, int> cache;
+  static std::map<std::tuple<int, int, int, int>, int> cache;
   std::lock_guard<std::mutex> lock(mu);
-  const auto key = std::make_tuple(dev.id, d, C);
+  const auto key = std::make_tuple(dev.id, which, d, C);
   auto it = cache.find(key);
   if (it == cache.end()) {
     int n = 0;
-    if (fwd_sm100_max_clusters(d, C, &n) != cudaSuccess) {
+    const cudaError_t e =
+        which == 0 ? fwd_sm100_max_clusters(d, C, &n) : bwd_fused_max_clusters(d, C, &n);
+    if (e != cudaSuccess) {
       cudaGetLastError();
       return SA_ERR_CUDA;
     }
@@ -72,11 +75,10 @@ struct Plan {
   // tensor-core finalize (bf16 forward, k a multiple of 128): U / mass as bf16 hi + lo
   bool ftc = false;
   size_t ubh = 0, ubl = 0;
-  // tensor-core backward (bf16)
+  // tensor-core backward (bf16): the single-pass kernel's clusters in C and G
   bool btc = false;
-  int splits = 0, wv_splits = 0;
-  size_t ghb = 0, gtb = 0, ub = 0, pn2 = 0, pnn = 0, ab = 0, dsb = 0, yb = 0, dvb = 0, dpart = 0,
-         lse2b = 0;
+  int wv_splits = 0;
+  size_t ghb = 0, gtb = 0, ub = 0, pn2 = 0, pnn = 0, dpart = 0, lse2b = 0;
   size_t total = 0;
 };
 
@@ -124,13 +126,14 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
       q.ubl = take((size_t)R * q.k_pad * d * 2);
     }
   } else if (dt == SA_BF16) {
-    // tensor-core backward: token x prototype intermediates in the workspace
+    // tensor-core backward: the single-pass kernel keeps every token x prototype value
+    // on chip; per-user Gh, Gt, c, per-cluster dPn partials, and the lse-recompute buffers
     q.btc = true;
-    q.k_pad = (k + 127) / 128 * 128;
-    q.splits = bwd_tc_splits(dev.sms, q.k_pad, d, n_total);
+    q.C = (k + 127) / 128;
+    q.k_pad = q.C * 128;
+    if ((st = tc_clusters(dev, d, q.C, &q.G, 1)) != SA_OK) return st;
     q.wv_splits = bwd_tc_wv_splits(dev.sms, R, q.k_pad);
-    q.Gb = q.splits;
-    const size_t nk = (size_t)n_total * q.k_pad;
+    q.Gb = q.G;
     const size_t rkd = (size_t)R * q.k_pad * d;
     q.gt = take(rkd * sizeof(float));
     q.gtb = take(rkd * 2);
@@ -139,13 +142,9 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
     q.cj = take((size_t)R * q.k_pad * sizeof(float));
     q.pn2 = take((size_t)q.k_pad * d * 2);
     q.pnn = take((size_t)q.k_pad * d * 2);
-    q.ab = take(nk * 2);
-    q.dsb = take(nk * 2);
-    q.yb = take((size_t)n_total * d * sizeof(float));
-    q.dvb = take((size_t)n_total * sizeof(float));
     q.dpart = take((size_t)n_total * (q.k_pad / 64) * sizeof(float));
     q.lse2b = take((size_t)n_total * sizeof(float));
-    q.dppp = take((size_t)q.splits * q.k_pad * d * sizeof(float));
+    q.dppp = take((size_t)q.G * q.k_pad * d * sizeof(float));
     q.dpp = take((size_t)q.k_pad * d * sizeof(float));
     q.wvp = take((size_t)(q.wv_splits > 1 ? q.wv_splits : 1) * d * d * sizeof(float));
   } else {
@@ -521,14 +520,11 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
   t.lse = lse;
   t.pn2 = at<__nv_bfloat16>(workspace, p.pn2);
   t.pnn = at<__nv_bfloat16>(workspace, p.pnn);
-  t.A = at<__nv_bfloat16>(workspace, p.ab);
-  t.dS = at<__nv_bfloat16>(workspace, p.dsb);
-  t.Y = at<float>(workspace, p.yb);
-  t.D = at<float>(workspace, p.dvb);
   t.dpart = at<float>(workspace, p.dpart);
   t.lse2 = at<float>(workspace, p.lse2b);
   t.Ub = at<__nv_bfloat16>(workspace, p.ub);
-  t.splits = p.splits;
+  t.C = p.C;
+  t.G = p.G;
   t.wv_splits = p.wv_splits;
   return cuda_status(launch_bwd_tc(t, s));
 }

@@ -122,24 +122,39 @@ cudaError_t launch_bwd_prep(const BwdArgs& a, cudaStream_t s);  // Gt, Gh, c per
 // dPn reduce, dW_v, dP, dW_k; wv_parts > 0: that many dW_v partials are already in wv_part
 cudaError_t launch_bwd_tail(const BwdArgs& a, int wv_parts, cudaStream_t s);
 
+// ---- single-pass backward kernel (sa_bwd_fused.cu)
+struct BwdFusedArgs {
+  const void* X;               // bf16 [n_total, d]
+  const int64_t* offsets;
+  int R, k_valid, C, k_pad, d, G;
+  int64_t n_total;
+  const WsHeader* hdr;
+  const long long* tile_start;
+  const __nv_bfloat16* pn;     // [k_pad, d] P W_k^T / sqrt(d)
+  const __nv_bfloat16* gh;     // [R, k_pad, d] (G / mass) W_v^T
+  const float* cj;             // [R, k_pad]
+  const float* lse;            // [n_total] per-token log-sum-exp
+  float lse_scale;             // lse2 = lse_scale * lse[t] (log2 units)
+  float* dX;                   // [n_total, d], zeroed by the caller; partials are added
+  float* dpp_part;             // [G, k_pad, d] per-cluster partials of dPn
+  long long budget;
+};
+cudaError_t bwd_fused_max_clusters(int d, int C, int* n);
+cudaError_t launch_bwd_fused(const BwdFusedArgs& a, cudaStream_t s);
+
 // ---- tensor-core backward (bf16 inputs; sa_bwd_tc.cu)
 struct BwdTcArgs {
   BwdArgs b;                 // shared inputs, outputs and SIMT-stage workspace
   const float* lse;          // forward's lse (natural log); null: recomputed here
-  __nv_bfloat16* pn2;        // [k_pad, d] P W_k^T log2(e)/sqrt(d)
+  __nv_bfloat16* pn2;        // [k_pad, d] P W_k^T log2(e)/sqrt(d) (lse recompute only)
   __nv_bfloat16* pnn;        // [k_pad, d] P W_k^T / sqrt(d)
-  __nv_bfloat16* A;          // [n_total, k_pad]
-  __nv_bfloat16* dS;         // [n_total, k_pad]
-  float* Y;                  // [n_total, d]  A Gh_u
-  float* D;                  // [n_total]
-  float* dpart;              // [n_total, k_pad / 128] per-tile partials
+  float* dpart;              // [n_total, k_pad / 64] per-tile partials (lse recompute)
   float* lse2;               // [n_total] (when lse is null)
   __nv_bfloat16* Ub;         // [R, k_pad, d] bf16 xsketch (zero rows past k)
-  int splits;                // split-K of dPn (== b.G)
+  int C, G;                  // cluster size and co-resident clusters of the fused kernel
   int wv_splits;             // split-K of dW_v (partials in b.wv_part)
 };
 cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s);
-int bwd_tc_splits(int sms, int k_pad, int d, long long n_total);
 int bwd_tc_wv_splits(int sms, int R, int k_pad);
 
 // ---- tensor-core GEMM (backward building block, sa_gemm_sm100.cu)
