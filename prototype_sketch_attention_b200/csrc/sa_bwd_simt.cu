@@ -31,7 +31,8 @@ __device__ __forceinline__ float ldf<__nv_bfloat16>(const __nv_bfloat16* p, size
   return __bfloat162float(p[i]);
 }
 
-// ---- per-user prep: Gt, Gh, c.   grid (R, k_pad/32), 256 threads
+// ---- per-user prep: Gt, c, and Gh unless a GEMM computes it (Gtlo given: then Gt's bf16
+// hi and lo parts).   grid (R, k_pad/32), 256 threads
 template <typename TIn>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a, const TIn* __restrict__ Wv) {
   extern __shared__ float sm[];
@@ -39,7 +40,8 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a, const TIn* __r
   float* wv = sm;              // [d][d+1]  wv[c][e] = Wv[c][e]
   float* gt = wv + d * ld;     // [32][d]
   const int u = blockIdx.x, j0 = blockIdx.y * kCP;
-  for (int i = threadIdx.x; i < d * d; i += blockDim.x) wv[(i / d) * ld + (i % d)] = ldf(Wv, i);
+  if (!a.Gtlo)  // W_v is needed here only when this kernel computes Gh itself
+    for (int i = threadIdx.x; i < d * d; i += blockDim.x) wv[(i / d) * ld + (i % d)] = ldf(Wv, i);
   for (int i = threadIdx.x; i < kCP * d; i += blockDim.x) {
     const int jj = i / d, e = i % d, j = j0 + jj;
     float v = 0.f;
@@ -49,10 +51,14 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a, const TIn* __r
     }
     gt[i] = v;
     a.Gt[((size_t)u * a.k_pad + j) * d + e] = v;
-    if (a.Gtb) a.Gtb[((size_t)u * a.k_pad + j) * d + e] = __float2bfloat16_rn(v);
+    if (a.Gtb) {
+      const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+      a.Gtb[((size_t)u * a.k_pad + j) * d + e] = hi;
+      if (a.Gtlo) a.Gtlo[((size_t)u * a.k_pad + j) * d + e] = __float2bfloat16_rn(v - __bfloat162float(hi));
+    }
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < kCP * d; i += blockDim.x) {
+  for (int i = threadIdx.x; i < (a.Gtlo ? 0 : kCP * d); i += blockDim.x) {  // else a GEMM
     const int jj = i / d, c = i % d;
     float acc = 0.f;
     for (int e = 0; e < d; ++e) acc = fmaf(gt[jj * d + e], wv[c * ld + e], acc);

@@ -10,7 +10,8 @@
 // then dP = dPn W_k / sqrt(d), dW_k = dPn^T P / sqrt(d), dW_v = sum_u U_u^T Gt_u.
 //
 // Launch sequence (bf16):
-//   prep (CUDA cores)   Gt (fp32, bf16), bf16 Gh, c per user
+//   prep (CUDA cores)   Gt (fp32, and bf16 hi + lo parts), c per user
+//   GEMM                bf16 Gh = (Gt_hi + Gt_lo) W_v^T for every user (two phases)
 //   fold                pnn = bf16(Pn)  [and pn2 = bf16(Pn log2 e) when the lse is recomputed]
 //   GEMM (split-K)      partials of dW_v = U^T Gt over (user, prototype) rows (bf16 U)
 //   [lse not given]     GEMM S2 = X pn2^T -> per-tile log2-sum-exp -> lse2 per token
@@ -81,6 +82,25 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
   const long long n = b.n_total;
   const int nparts = 2 * (k_pad / 128);  // per-row lse partials: two column halves per tile
   if ((e = launch_bwd_prep(b, s)) != cudaSuccess) return e;
+  if (R > 0) {  // Gh = Gt W_v^T for every user: (Gt_hi + Gt_lo) W_v^T, two accumulated phases
+    GemmArgs t = {};
+    t.hdr = b.hdr;
+    t.phases = 2;
+    t.a[0] = op(b.Gtb, (uint64_t)R * k_pad, (uint64_t)d, false);
+    t.b[0] = op(b.Wv, (uint64_t)d, (uint64_t)d, false);
+    t.a[1] = op(b.Gtlo, (uint64_t)R * k_pad, (uint64_t)d, false);
+    t.b[1] = op(b.Wv, (uint64_t)d, (uint64_t)d, false);
+    t.k_tiles[0] = t.k_tiles[1] = (d + 63) / 64;
+    t.user_mode = 0;
+    t.M = R * k_pad;
+    t.N = d;
+    t.m_tiles_bound = (R * k_pad + 127) / 128;
+    t.splits = 1;
+    t.epi = kEpiStoreBf16;
+    t.out_bf16 = b.Ghb;
+    t.ld_out = d;
+    if ((e = launch_gemm(t, s)) != cudaSuccess) return e;
+  }
   const float isd = 1.0f / std::sqrt((float)d);
   if ((e = launch_fold(b.P, b.Wk, SA_BF16, k, k_pad, d, isd, a.pnn, true, s)) != cudaSuccess)
     return e;

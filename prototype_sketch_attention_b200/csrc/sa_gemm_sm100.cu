@@ -21,6 +21,7 @@
 //   kEpiLse       dpart[row][2 tile + h] = log2 sum of 2^acc over half h of the tile
 //                 (columns n < k_valid)
 //   kEpiDS        out_bf16[row][n] = bf16(A[row][n] (acc - c[user][n] - drow[row]))
+//   kEpiStoreBf16 out_bf16[row][n] = bf16(acc)
 // Waits on mbarriers are bounded like every other kernel of the library.
 #include <cuda.h>
 
@@ -430,6 +431,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     case kEpiAExp: return launch_t<kEpiAExp>(p, grid, s);
     case kEpiDS: return launch_t<kEpiDS>(p, grid, s);
     case kEpiLse: return launch_t<kEpiLse>(p, grid, s);
+    case kEpiStoreBf16: return launch_t<kEpiStoreBf16>(p, grid, s);
     default: return cudaErrorInvalidValue;
   }
 }

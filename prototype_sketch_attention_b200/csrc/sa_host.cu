@@ -78,7 +78,7 @@ struct Plan {
   // tensor-core backward (bf16): the single-pass kernel's clusters in C and G
   bool btc = false;
   int wv_splits = 0;
-  size_t ghb = 0, gtb = 0, ub = 0, pn2 = 0, pnn = 0, dpart = 0, lse2b = 0;
+  size_t ghb = 0, gtb = 0, gtlo = 0, ub = 0, pn2 = 0, pnn = 0, dpart = 0, lse2b = 0;
   size_t total = 0;
 };
 
@@ -137,6 +137,7 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
     const size_t rkd = (size_t)R * q.k_pad * d;
     q.gt = take(rkd * sizeof(float));
     q.gtb = take(rkd * 2);
+    q.gtlo = take(rkd * 2);
     q.ghb = take(rkd * 2);
     q.ub = take(rkd * 2);
     q.cj = take((size_t)R * q.k_pad * sizeof(float));
@@ -513,6 +514,7 @@ int sa_sketch_backward(const void* X, const int64_t* offsets, int R, int64_t n_t
   a.Gh = nullptr;
   a.Ghb = at<__nv_bfloat16>(workspace, p.ghb);
   a.Gtb = at<__nv_bfloat16>(workspace, p.gtb);
+  a.Gtlo = at<__nv_bfloat16>(workspace, p.gtlo);
   a.lseb = nullptr;
   a.Db = nullptr;
   BwdTcArgs t;

@@ -104,6 +104,7 @@ struct BwdArgs {
   float* Gh;      // [R, k_pad, d]  (G / mass) W_v^T (nullable)
   __nv_bfloat16* Ghb;  // the same in bf16 (nullable; the tensor-core backward)
   __nv_bfloat16* Gtb;  // Gt in bf16 (nullable; the tensor-core backward)
+  __nv_bfloat16* Gtlo; // bf16(Gt - bf16(Gt)) (nullable): Gh then comes from a tensor-core GEMM
   float* cj;      // [R, k_pad]     (G / mass) . sketch - dmass
   float* lseb;    // [n_total]      fp32 per-token log-sum-exp (natural)
   float* Db;      // [n_total]      sum_j A_jt dA_jt
@@ -158,7 +159,7 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s);
 int bwd_tc_wv_splits(int sms, int R, int k_pad);
 
 // ---- tensor-core GEMM (backward building block, sa_gemm_sm100.cu)
-enum GemmEpi { kEpiStoreF32 = 0, kEpiAExp = 1, kEpiDS = 2, kEpiLse = 3 };
+enum GemmEpi { kEpiStoreF32 = 0, kEpiAExp = 1, kEpiDS = 2, kEpiLse = 3, kEpiStoreBf16 = 4 };
 struct GemmOperandDesc {  // one bf16 operand, row-major in memory
   const void* base;
   uint64_t rows, cols;
