@@ -272,7 +272,8 @@ int sa_sketch_get_device_status(const void* workspace, void* stream);
  * Measurement hook. When both handles are non-null, every later sa_sketch_forward
  * call made by this host thread records `start_event` on its stream just before the
  * main forward kernel (the tcgen05 kernel for bf16, the SIMT kernels for fp32) and
- * `stop_event` just after it. The caller then reads that kernel's own duration with
+ * `stop_event` just after it; sa_stca_keys_forward calls likewise around their flash
+ * kernel. The caller then reads that kernel's own duration with
  * cudaEventElapsedTime. Both handles are cudaEvent_t passed as void*; the caller owns
  * them. Passing two nulls turns the hook off. Returns SA_OK, or SA_ERR_INVALID_ARG if
  * exactly one handle is null.
@@ -341,6 +342,72 @@ int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* 
                      const void* WK, const void* WV, const float* dout, float* dQ, float* dS,
                      float* dWq, float* dWK, float* dWV, void* workspace, size_t ws_bytes,
                      void* stream);
+
+/*
+ * Cross attention from each user's candidates to a ragged range of that user's key rows:
+ * the recent branch of STCA, whose keys are the user's last 10K raw history tokens ("100,000
+ * videos in your pocket" blog, section "2. STCA reasons at two time scales", recent branch).
+ * For user u and each candidate c in [cand_offsets[u], cand_offsets[u+1]):
+ *   q = Q_c Wq,  K_j = Kx_j WK,  V_j = Kx_j WV      (j in [key_begin[u], key_end[u]))
+ *   out_c = sum_j softmax_j(q . K_j / sqrt(d)) V_j,  lse_c = log sum_j exp(q . K_j / sqrt(d))
+ * A user whose range is empty gets out = 0 and lse = -inf.
+ *
+ *   Q            [n_cand, d]  bf16, device   candidates, users' groups concatenated
+ *   cand_offsets [R + 1]      int64, device  0 = c_0 <= c_1 <= ... <= c_R = n_cand
+ *   Kx           [n_keys, d]  bf16, device   key rows; for the recent branch the history X
+ *                                            itself (sa_sketch_forward's input), read in place
+ *   key_begin, key_end [R]    int64, device  user u's rows are Kx[key_begin[u] : key_end[u]];
+ *                                            0 <= key_begin[u] <= key_end[u] <= n_keys, else
+ *                                            SA_ERR_BAD_OFFSETS in the device status word.
+ *                                            Ranges of different users may overlap.
+ *   Wq, WK, WV   [d, d]       bf16, device   row-major, x W for a row vector x
+ *   out          [n_cand, d]  fp32, device   output (overwritten)
+ *   lse          [n_cand]     fp32, device   output, nullable
+ * d in {64, 128}; n_cand, n_keys <= INT32_MAX; R <= SA_MAX_USERS; Q, Kx, weights and outputs
+ * 16-byte aligned, key_begin / key_end 8-byte aligned. Precision: Q Wq WK^T / sqrt(d) is
+ * formed in fp32 and enters the tensor cores as a bf16 pair hi + lo (about 16 significant
+ * bits); the key rows and the attention weights enter as bf16; accumulation is fp32 and the
+ * softmax runs in fp32 along each candidate's row with a running maximum (a flash-style
+ * kernel: the scores of a candidate never leave the chip).
+ * The workspace (sa_stca_keys_workspace_size bytes, 256-aligned, caller-owned) holds the
+ * schedule, Q Wq WK^T and the unprojected output (about 16 d bytes per candidate); errors
+ * follow sa_sketch_forward's conventions, and the device status word in the workspace is
+ * read with sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
+ */
+size_t sa_stca_keys_workspace_size(int R, int64_t n_cand, int d, int backward);
+int sa_stca_keys_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
+                         const void* Kx, int64_t n_keys, const int64_t* key_begin,
+                         const int64_t* key_end, const void* Wq, const void* WK, const void* WV,
+                         float* out, float* lse, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * Gradients of sa_stca_keys_forward given dout = dL/dout [n_cand, d] (fp32, device):
+ *   dQ  [n_cand, d]  fp32, device   dL/dQ
+ *   dKx [n_keys, d]  fp32, device   dL/dKx: for the recent branch the gradient that flows
+ *                                   into the history rows; 0 on rows no range covers, a
+ *                                   sum over users on rows several ranges cover
+ *   dWq, dWK, dWV [d, d] fp32, device, summed over users
+ * All outputs are overwritten. The forward is recomputed inside. Workspace:
+ * sa_stca_keys_workspace_size(..., backward = 1) bytes. Other arguments, precision and
+ * conventions as for sa_stca_keys_forward.
+ */
+int sa_stca_keys_backward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand,
+                          int d, const void* Kx, int64_t n_keys, const int64_t* key_begin,
+                          const int64_t* key_end, const void* Wq, const void* WK, const void* WV,
+                          const float* dout, float* dQ, float* dKx, float* dWq, float* dWK,
+                          float* dWV, void* workspace, size_t ws_bytes, void* stream);
+
+/*
+ * The recent branch's key ranges over a history X laid out as for sa_sketch_forward: user
+ * u's last min(n_u, L) tokens, key_begin[u] = max(offsets[u], offsets[u+1] - L) and
+ * key_end[u] = offsets[u+1] ("100,000 videos in your pocket" blog, section "2. STCA
+ * reasons at two time scales": the recent 10K, L = 10000). offsets [R + 1] int64, device;
+ * key_begin, key_end [R] int64, device (written). L >= 0. Enqueues one kernel on `stream`;
+ * offsets are not validated here (sa_stca_keys_forward checks the ranges it receives).
+ * Returns SA_OK, SA_ERR_INVALID_ARG, SA_ERR_NO_DEVICE or SA_ERR_CUDA.
+ */
+int sa_stca_recent_ranges(const int64_t* offsets, int R, int64_t L, int64_t* key_begin,
+                          int64_t* key_end, void* stream);
 
 /*
  * Sketch cache codec. The sketch is user-only and reused across candidates and

@@ -34,7 +34,9 @@ EXPORTED = ("sa_sketch_workspace_size", "sa_sketch_forward", "sa_sketch_backward
             "sa_sketch_debug_gemm", "sa_stca_workspace_size", "sa_stca_forward",
             "sa_stca_backward", "sa_sketch_pack", "sa_sketch_unpack",
             "sa_sketch_forward_host_buffer_size", "sa_sketch_forward_host",
-            "sa_sketch_forward_host_status", "sa_sketch_host_parts", "sa_sketch_forward_grid")
+            "sa_sketch_forward_host_status", "sa_sketch_host_parts", "sa_sketch_forward_grid",
+            "sa_stca_keys_workspace_size", "sa_stca_keys_forward", "sa_stca_keys_backward",
+            "sa_stca_recent_ranges")
 SA_CODEC_BF16 = 0
 SA_CODEC_FP8 = 1
 
@@ -96,6 +98,16 @@ def _load() -> ctypes.CDLL:
     lib.sa_sketch_forward_grid.argtypes = [i32, i32, i32, vp, vp]
     lib.sa_sketch_host_parts.restype = i32
     lib.sa_sketch_host_parts.argtypes = [vp, i32, i32, vp]
+    lib.sa_stca_keys_workspace_size.restype = sz
+    lib.sa_stca_keys_workspace_size.argtypes = [i32, i64, i32, i32]
+    lib.sa_stca_keys_forward.restype = i32
+    lib.sa_stca_keys_forward.argtypes = [vp, vp, i32, i64, i32, vp, i64, vp, vp, vp, vp, vp, vp,
+                                         vp, vp, sz, vp]
+    lib.sa_stca_keys_backward.restype = i32
+    lib.sa_stca_keys_backward.argtypes = [vp, vp, i32, i64, i32, vp, i64, vp, vp, vp, vp, vp, vp,
+                                          vp, vp, vp, vp, vp, vp, sz, vp]
+    lib.sa_stca_recent_ranges.restype = i32
+    lib.sa_stca_recent_ranges.argtypes = [vp, i32, i64, vp, vp, vp]
     return lib
 
 
@@ -142,6 +154,28 @@ def sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse, w
                     ws_bytes, stream) -> int:
     return int(_lib.sa_stca_forward(Q, cand_offsets, R, n_cand, d, S, k, Wq, WK, WV, out, lse,
                                     workspace, ws_bytes, stream))
+
+
+def sa_stca_keys_workspace_size(R: int, n_cand: int, d: int, backward: int = 0) -> int:
+    return int(_lib.sa_stca_keys_workspace_size(R, n_cand, d, backward))
+
+
+def sa_stca_keys_forward(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin, key_end, Wq, WK,
+                         WV, out, lse, workspace, ws_bytes, stream) -> int:
+    return int(_lib.sa_stca_keys_forward(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin,
+                                         key_end, Wq, WK, WV, out, lse, workspace, ws_bytes,
+                                         stream))
+
+
+def sa_stca_keys_backward(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin, key_end, Wq, WK,
+                          WV, dout, dQ, dKx, dWq, dWK, dWV, workspace, ws_bytes, stream) -> int:
+    return int(_lib.sa_stca_keys_backward(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin,
+                                          key_end, Wq, WK, WV, dout, dQ, dKx, dWq, dWK, dWV,
+                                          workspace, ws_bytes, stream))
+
+
+def sa_stca_recent_ranges(offsets, R, L, key_begin, key_end, stream) -> int:
+    return int(_lib.sa_stca_recent_ranges(offsets, R, L, key_begin, key_end, stream))
 
 
 def sa_sketch_forward_host_buffer_size(R, n_total, k, d, dt, parts) -> int:
@@ -506,6 +540,110 @@ def stca_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, 
                               _ptr(out["dWV"]), _ptr(ws), ws.nbytes, _stream(stream, dev))
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_stca_backward")
+    out["_ws"] = ws
+    return out
+
+
+def recent_ranges(offsets: torch.Tensor, L: int, *, stream=None) -> tuple[torch.Tensor, torch.Tensor]:
+    """The recent branch's key ranges over a history laid out by `offsets` [R+1] (int64,
+    CUDA): each user's last min(n_u, L) rows. Returns (key_begin, key_end), int64 [R]."""
+    where = "recent_ranges"
+    _require(isinstance(offsets, torch.Tensor) and offsets.dim() == 1 and offsets.numel() >= 1,
+             where, "offsets must be a 1-D tensor with R + 1 entries")
+    R = offsets.numel() - 1
+    dev = offsets.device
+    _check_tensor(where, "offsets", offsets, (R + 1,), torch.int64, dev)
+    _check_cuda(where, offsets)
+    kb = torch.empty(R, dtype=torch.int64, device=dev)
+    ke = torch.empty(R, dtype=torch.int64, device=dev)
+    with torch.cuda.device(dev):
+        st = sa_stca_recent_ranges(_ptr(offsets), R, int(L), _ptr(kb), _ptr(ke),
+                                   _stream(stream, dev))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_stca_recent_ranges")
+    return kb, ke
+
+
+def _check_keys_inputs(where, Q, cand_offsets, Kx, key_begin, key_end, Wq, WK, WV):
+    _require(isinstance(Q, torch.Tensor) and Q.dim() == 2, where, "Q must be a 2-D tensor")
+    _require(isinstance(Kx, torch.Tensor) and Kx.dim() == 2, where, "Kx must be a 2-D tensor")
+    _require(isinstance(cand_offsets, torch.Tensor) and cand_offsets.dim() == 1
+             and cand_offsets.numel() >= 1, where, "cand_offsets must be a 1-D tensor with R + 1 entries")
+    n_cand, d = Q.shape
+    R = cand_offsets.numel() - 1
+    dev = Q.device
+    bf = torch.bfloat16
+    _check_tensor(where, "Q", Q, (n_cand, d), bf, dev)
+    _check_tensor(where, "Kx", Kx, (Kx.shape[0], d), bf, dev)
+    _check_tensor(where, "cand_offsets", cand_offsets, (R + 1,), torch.int64, dev)
+    _check_tensor(where, "key_begin", key_begin, (R,), torch.int64, dev)
+    _check_tensor(where, "key_end", key_end, (R,), torch.int64, dev)
+    for name, W in (("Wq", Wq), ("WK", WK), ("WV", WV)):
+        _check_tensor(where, name, W, (d, d), bf, dev)
+    _check_cuda(where, Q)
+    return n_cand, d, R, Kx.shape[0], dev
+
+
+def stca_keys_forward(Q: torch.Tensor, cand_offsets: torch.Tensor, Kx: torch.Tensor,
+                      key_begin: torch.Tensor, key_end: torch.Tensor, Wq: torch.Tensor,
+                      WK: torch.Tensor, WV: torch.Tensor, *, want_lse: bool = True,
+                      ws: torch.Tensor | None = None, stream=None) -> dict:
+    """Cross attention from user u's candidates to the key rows Kx[key_begin[u]:key_end[u]]
+    (the recent branch: Kx = the history X, ranges from recent_ranges). Q [n_cand, d] bf16,
+    cand_offsets [R+1] int64, Kx [n_keys, d] bf16, key_begin / key_end [R] int64,
+    Wq, WK, WV [d, d] bf16, all on one CUDA device. Returns out [n_cand, d] fp32 (and
+    lse [n_cand])."""
+    where = "stca_keys_forward"
+    n_cand, d, R, n_keys, dev = _check_keys_inputs(where, Q, cand_offsets, Kx, key_begin, key_end,
+                                                   Wq, WK, WV)
+    out = {"out": torch.empty(n_cand, d, device=dev, dtype=torch.float32)}
+    if want_lse:
+        out["lse"] = torch.empty(n_cand, device=dev, dtype=torch.float32)
+    with torch.cuda.device(dev):
+        if ws is None:
+            nb = sa_stca_keys_workspace_size(R, n_cand, d, 0)
+            if nb == 0:
+                raise SketchAttentionError(SA_ERR_UNSUPPORTED, "sa_stca_keys_workspace_size")
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        st = sa_stca_keys_forward(_ptr(Q), _ptr(cand_offsets), R, n_cand, d, _ptr(Kx), n_keys,
+                                  _ptr(key_begin), _ptr(key_end), _ptr(Wq), _ptr(WK), _ptr(WV),
+                                  _ptr(out["out"]), _ptr(out.get("lse")), _ptr(ws), ws.nbytes,
+                                  _stream(stream, dev))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_stca_keys_forward")
+    out["_ws"] = ws
+    return out
+
+
+def stca_keys_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, Kx: torch.Tensor,
+                       key_begin: torch.Tensor, key_end: torch.Tensor, Wq: torch.Tensor,
+                       WK: torch.Tensor, WV: torch.Tensor, dout: torch.Tensor, *,
+                       ws: torch.Tensor | None = None, stream=None) -> dict:
+    """Gradients of stca_keys_forward given dL/dout [n_cand, d] fp32: dQ, dKx [n_keys, d]
+    (into the key rows), dWq, dWK, dWV. Inputs as for stca_keys_forward."""
+    where = "stca_keys_backward"
+    n_cand, d, R, n_keys, dev = _check_keys_inputs(where, Q, cand_offsets, Kx, key_begin, key_end,
+                                                   Wq, WK, WV)
+    f32 = torch.float32
+    _check_tensor(where, "dout", dout, (n_cand, d), f32, dev)
+    out = {"dQ": torch.empty(n_cand, d, device=dev, dtype=f32),
+           "dKx": torch.empty(n_keys, d, device=dev, dtype=f32),
+           "dWq": torch.empty(d, d, device=dev, dtype=f32),
+           "dWK": torch.empty(d, d, device=dev, dtype=f32),
+           "dWV": torch.empty(d, d, device=dev, dtype=f32)}
+    with torch.cuda.device(dev):
+        if ws is None:
+            nb = sa_stca_keys_workspace_size(R, n_cand, d, 1)
+            if nb == 0:
+                raise SketchAttentionError(SA_ERR_UNSUPPORTED, "sa_stca_keys_workspace_size")
+            ws = torch.empty(nb, dtype=torch.uint8, device=dev)
+        st = sa_stca_keys_backward(_ptr(Q), _ptr(cand_offsets), R, n_cand, d, _ptr(Kx), n_keys,
+                                   _ptr(key_begin), _ptr(key_end), _ptr(Wq), _ptr(WK), _ptr(WV),
+                                   _ptr(dout), _ptr(out["dQ"]), _ptr(out["dKx"]),
+                                   _ptr(out["dWq"]), _ptr(out["dWK"]), _ptr(out["dWV"]),
+                                   _ptr(ws), ws.nbytes, _stream(stream, dev))
+    if st != SA_OK:
+        raise SketchAttentionError(st, "sa_stca_keys_backward")
     out["_ws"] = ws
     return out
 

@@ -189,9 +189,6 @@ T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
 }
 
-thread_local cudaEvent_t g_prof_start = nullptr;
-thread_local cudaEvent_t g_prof_stop = nullptr;
-
 cudaError_t prof_mark(cudaEvent_t ev, cudaStream_t s) {
   return ev ? cudaEventRecord(ev, s) : cudaSuccess;
 }
@@ -206,6 +203,16 @@ sa_status cuda_status(cudaError_t e) {
 }  // namespace sa
 
 namespace sa {
+thread_local cudaEvent_t g_prof_start = nullptr;
+thread_local cudaEvent_t g_prof_stop = nullptr;
+
+cudaError_t prof_mark_start(cudaStream_t s) {
+  return g_prof_start ? cudaEventRecord(g_prof_start, s) : cudaSuccess;
+}
+cudaError_t prof_mark_stop(cudaStream_t s) {
+  return g_prof_stop ? cudaEventRecord(g_prof_stop, s) : cudaSuccess;
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda needed).
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -420,6 +427,125 @@ int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* 
   g.dWK = dWK;
   g.dWV = dWV;
   return cuda_status(launch_stca_backward(a, g, static_cast<cudaStream_t>(stream_)));
+}
+
+namespace {
+
+// Arguments shared by the ragged-key forward and backward (SA_OK or an argument code).
+int check_keys_args(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
+                    const void* Kx, int64_t n_keys, const int64_t* key_begin,
+                    const int64_t* key_end, const void* Wq, const void* WK, const void* WV) {
+  if (R < 0 || R > SA_MAX_USERS || n_cand < 0 || n_cand > INT32_MAX || n_keys < 0 ||
+      n_keys > INT32_MAX)
+    return SA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return SA_ERR_UNSUPPORTED;
+  if (!cand_offsets || !Wq || !WK || !WV || (n_cand > 0 && !Q) || (n_keys > 0 && !Kx) ||
+      (R > 0 && (!key_begin || !key_end)))
+    return SA_ERR_INVALID_ARG;
+  if (!aligned16(Q) || !aligned16(cand_offsets) || !aligned16(Kx) || !aligned16(Wq) ||
+      !aligned16(WK) || !aligned16(WV) || (reinterpret_cast<uintptr_t>(key_begin) & 7u) ||
+      (reinterpret_cast<uintptr_t>(key_end) & 7u))
+    return SA_ERR_INVALID_ARG;
+  return SA_OK;
+}
+
+}  // namespace
+
+size_t sa_stca_keys_workspace_size(int R, int64_t n_cand, int d, int backward) {
+  if (R < 0 || R > SA_MAX_USERS || n_cand < 0 || n_cand > INT32_MAX) return 0;
+  if (d != 64 && d != 128) return 0;
+  Device dev;
+  if (backward && current_device(&dev) != SA_OK) return 0;
+  StcaKeysPlan p;
+  return stca_keys_plan(R, n_cand, d, backward != 0, backward ? dev.sms : 0, &p);
+}
+
+int sa_stca_keys_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
+                         const void* Kx, int64_t n_keys, const int64_t* key_begin,
+                         const int64_t* key_end, const void* Wq, const void* WK, const void* WV,
+                         float* out, float* lse, void* workspace, size_t ws_bytes, void* stream_) {
+  int st = check_keys_args(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin, key_end, Wq, WK,
+                           WV);
+  if (st != SA_OK) return st;
+  if ((n_cand > 0 && !out) || !aligned16(out) || !aligned16(lse)) return SA_ERR_INVALID_ARG;
+  Device dev;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  StcaKeysArgs a;
+  stca_keys_plan(R, n_cand, d, false, 0, &a.plan);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      ws_bytes < a.plan.total)
+    return SA_ERR_WORKSPACE;
+  a.Q = Q;
+  a.coff = cand_offsets;
+  a.R = R;
+  a.d = d;
+  a.n_cand = n_cand;
+  a.Kx = Kx;
+  a.n_keys = n_keys;
+  a.kb = key_begin;
+  a.ke = key_end;
+  a.Wq = Wq;
+  a.WK = WK;
+  a.WV = WV;
+  a.out = out;
+  a.lse = lse;
+  a.workspace = workspace;
+  return cuda_status(launch_stca_keys_forward(a, static_cast<cudaStream_t>(stream_)));
+}
+
+int sa_stca_keys_backward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand,
+                          int d, const void* Kx, int64_t n_keys, const int64_t* key_begin,
+                          const int64_t* key_end, const void* Wq, const void* WK, const void* WV,
+                          const float* dout, float* dQ, float* dKx, float* dWq, float* dWK,
+                          float* dWV, void* workspace, size_t ws_bytes, void* stream_) {
+  int st = check_keys_args(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin, key_end, Wq, WK,
+                           WV);
+  if (st != SA_OK) return st;
+  if (!dWq || !dWK || !dWV || (n_cand > 0 && (!dout || !dQ)) || (n_keys > 0 && !dKx) ||
+      !aligned16(dout) || !aligned16(dQ) || !aligned16(dKx) || !aligned16(dWq) ||
+      !aligned16(dWK) || !aligned16(dWV))
+    return SA_ERR_INVALID_ARG;
+  Device dev;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  StcaKeysArgs a;
+  stca_keys_plan(R, n_cand, d, true, dev.sms, &a.plan);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 ||
+      ws_bytes < a.plan.total)
+    return SA_ERR_WORKSPACE;
+  a.Q = Q;
+  a.coff = cand_offsets;
+  a.R = R;
+  a.d = d;
+  a.n_cand = n_cand;
+  a.Kx = Kx;
+  a.n_keys = n_keys;
+  a.kb = key_begin;
+  a.ke = key_end;
+  a.Wq = Wq;
+  a.WK = WK;
+  a.WV = WV;
+  a.out = nullptr;
+  a.lse = nullptr;
+  a.workspace = workspace;
+  StcaKeysGrads g;
+  g.dout = dout;
+  g.dQ = dQ;
+  g.dKx = dKx;
+  g.dWq = dWq;
+  g.dWK = dWK;
+  g.dWV = dWV;
+  return cuda_status(launch_stca_keys_backward(a, g, static_cast<cudaStream_t>(stream_)));
+}
+
+int sa_stca_recent_ranges(const int64_t* offsets, int R, int64_t L, int64_t* key_begin,
+                          int64_t* key_end, void* stream_) {
+  if (R < 0 || R > SA_MAX_USERS || L < 0) return SA_ERR_INVALID_ARG;
+  if (R > 0 && (!offsets || !key_begin || !key_end)) return SA_ERR_INVALID_ARG;
+  Device dev;
+  int st;
+  if ((st = current_device(&dev)) != SA_OK) return st;
+  return cuda_status(launch_recent_ranges(offsets, R, L, key_begin, key_end,
+                                          static_cast<cudaStream_t>(stream_)));
 }
 
 int sa_sketch_pack(const float* sketch, int64_t rows, int d, int format, void* codes,

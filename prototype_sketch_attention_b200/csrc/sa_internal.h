@@ -232,11 +232,70 @@ struct StcaGrads {
 };
 cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& g, cudaStream_t s);
 
+// shared pieces of the cross attention (sa_stca.cu)
+cudaError_t stca_split_hilo(const float* x, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                            cudaStream_t s);
+cudaError_t stca_to_bf16(const float* x, long long n, __nv_bfloat16* y, cudaStream_t s);
+cudaError_t stca_rowdot(const float* a, const float* b, long long n, int d, float* D,
+                        cudaStream_t s);
+cudaError_t stca_weight_grads(const float* dM, const void* Wq, const void* WK, int d, float* dWq,
+                              float* dWK, cudaStream_t s);
+cudaError_t gemm_hilo(const WsHeader* hdr, const __nv_bfloat16* hi, const __nv_bfloat16* lo,
+                      long long n, int d, GemmOperandDesc bop, float* out, cudaStream_t s);
+cudaError_t gemm_tn_sum(const WsHeader* hdr, const __nv_bfloat16* A, const __nv_bfloat16* B,
+                        long long n, int d, int splits, float* part, float scale, float* out,
+                        cudaStream_t s);
+
+// ---- cross attention over ragged key rows (sa_stca_keys.cu)
+struct StcaKeysPlan {  // workspace layout (byte offsets, 256-aligned)
+  int splits = 0;
+  size_t hdr = 0, ts = 0, mt = 0, qh = 0, ql = 0, o = 0, lse2 = 0, ohi = 0, olo = 0, total = 0;
+  // backward only
+  size_t mts = 0, ghi = 0, glo = 0, gb = 0, do_f = 0, ob = 0, dd = 0, g1 = 0, g1hi = 0,
+         g1lo = 0, part = 0, dm = 0, kpre = 0;
+};
+size_t stca_keys_plan(int R, long long n_cand, int d, bool backward, int sms, StcaKeysPlan* p);
+struct StcaKeysArgs {
+  const void* Q;          // bf16 [n_cand, d]
+  const int64_t* coff;    // [R + 1]
+  int R, d;
+  long long n_cand;
+  const void* Kx;         // bf16 [n_keys, d]
+  long long n_keys;
+  const int64_t* kb;      // [R] first key row of each user
+  const int64_t* ke;      // [R] one past its last key row
+  const void* Wq;         // bf16 [d, d]
+  const void* WK;
+  const void* WV;
+  float* out;             // [n_cand, d]
+  float* lse;             // [n_cand] natural log, nullable
+  void* workspace;
+  StcaKeysPlan plan;
+};
+struct StcaKeysGrads {
+  const float* dout;      // [n_cand, d]
+  float* dQ;              // [n_cand, d]
+  float* dKx;             // [n_keys, d]
+  float *dWq, *dWK, *dWV; // [d, d]
+};
+cudaError_t launch_stca_keys_forward(const StcaKeysArgs& a, cudaStream_t s);
+cudaError_t launch_stca_keys_backward(const StcaKeysArgs& a, const StcaKeysGrads& g,
+                                      cudaStream_t s);
+// key range of every user = its last min(n_u, L) history rows
+cudaError_t launch_recent_ranges(const int64_t* offsets, int R, int64_t L, int64_t* kb,
+                                 int64_t* ke, cudaStream_t s);
+
 // ---- sketch cache codec (sa_codec.cu): format 0 = bf16, 1 = fp8 E4M3 with row scales
 cudaError_t launch_sketch_pack(const float* S, long long rows, int d, int format, void* codes,
                                float* scales, cudaStream_t s);
 cudaError_t launch_sketch_unpack(const void* codes, const float* scales, long long rows, int d,
                                  int format, float* S, cudaStream_t s);
+
+// the measurement hook's events (sa_sketch_profile_events) recorded around a main kernel
+extern thread_local cudaEvent_t g_prof_start;
+extern thread_local cudaEvent_t g_prof_stop;
+cudaError_t prof_mark_start(cudaStream_t s);
+cudaError_t prof_mark_stop(cudaStream_t s);
 
 // cuTensorMapEncodeTiled through the runtime's driver entry point (null if unavailable)
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn();

@@ -285,6 +285,32 @@ cudaError_t forward_core(const StcaArgs& a, const Bufs& b, cudaStream_t s) {
   return cudaSuccess;
 }
 
+}  // namespace
+
+cudaError_t stca_split_hilo(const float* x, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
+                            cudaStream_t s) {
+  stca_split_kernel<<<1024, 256, 0, s>>>(x, n, hi, lo);
+  return cudaGetLastError();
+}
+
+cudaError_t stca_to_bf16(const float* x, long long n, __nv_bfloat16* y, cudaStream_t s) {
+  stca_to_bf16_kernel<<<1024, 256, 0, s>>>(x, n, y);
+  return cudaGetLastError();
+}
+
+cudaError_t stca_rowdot(const float* a, const float* b, long long n, int d, float* D,
+                        cudaStream_t s) {
+  stca_rowdot_kernel<<<1024, 256, 0, s>>>(a, b, n, d, D);
+  return cudaGetLastError();
+}
+
+cudaError_t stca_weight_grads(const float* dM, const void* Wq, const void* WK, int d, float* dWq,
+                              float* dWK, cudaStream_t s) {
+  stca_weight_grads_kernel<<<d, 128, 0, s>>>(dM, static_cast<const __nv_bfloat16*>(Wq),
+                                             static_cast<const __nv_bfloat16*>(WK), d, dWq, dWK);
+  return cudaGetLastError();
+}
+
 // out[n, N] = (hi + lo) B with B given as an operand descriptor (two accumulated phases).
 cudaError_t gemm_hilo(const WsHeader* hdr, const __nv_bfloat16* hi, const __nv_bfloat16* lo,
                       long long n, int d, GemmOperandDesc bop, float* out, cudaStream_t s) {
@@ -333,8 +359,6 @@ cudaError_t gemm_tn_sum(const WsHeader* hdr, const __nv_bfloat16* A, const __nv_
                                                             out);
   return cudaGetLastError();
 }
-
-}  // namespace
 
 cudaError_t launch_stca_forward(const StcaArgs& a, cudaStream_t s) {
   const Bufs b = bufs(a.plan, a.workspace);

@@ -1,0 +1,803 @@
+// Cross attention from each user's candidates to a ragged set of that user's key rows, on
+// tcgen05 (sm_100a): the recent branch of STCA, whose keys are the user's most recent
+// raw history tokens ("100,000 videos in your pocket" blog, section "2. STCA reasons at
+// two time scales", recent branch: the candidate attends over the last 10K tokens).
+//
+// User u's candidates c in [coff[u], coff[u+1]) attend over the key rows
+// Kx[kb[u] : ke[u]] (for the recent branch, Kx is the history X itself and the range is
+// the last min(n_u, L) tokens, so nothing is copied). With the same refold as the sketch
+// branch, Q' = Q W_q W_K^T log2(e) / sqrt(d) (computed before this kernel):
+//   z_cj = Q'_c . Kx_j (log2 units),  a_cj = 2^(z_cj - lse2_c),  O'_c = sum_j a_cj Kx_j,
+// and out = O' W_V afterwards. Keys and values are the same rows, so one TMA tile of 128
+// key rows is the B operand of both MMAs: K-major for Z = Q' Kx^T, MN-major for
+// O' += P Kx. Q' is formed in fp32 and enters the score MMA as a bf16 pair hi + lo (two
+// accumulated MMAs, about 16 significant bits): with scores of tens of units a single bf16
+// rounding of Q' would move the weights by several percent.
+//
+// One CTA per (user, 128-candidate tile). The softmax runs along each candidate's row of
+// Z in TMEM, one thread per candidate, with a running maximum that is raised only when a
+// tile's maximum exceeds it by more than 8 (in log2 units): then O' (in TMEM) and the
+// running sum are rescaled once; otherwise the exponentials stay below 2^8 and nothing is
+// rescaled. P = 2^(z - m) goes to shared memory as bf16 (the K-major A operand of the
+// second MMA), O' accumulates in TMEM, and at the end O' / l and lse2 = m + log2 l leave.
+// Roles: warp 0 TMA, warp 1 TMEM allocation and the MMAs, warps 4-7 the softmax
+// (thread = candidate = TMEM lane). Every mbarrier wait is bounded.
+#include <cuda.h>
+
+#include <algorithm>
+#include <cmath>
+
+#include "sa_common.cuh"
+#include "sa_internal.h"
+
+namespace sa {
+namespace {
+
+constexpr int kBox = 16384;   // 128 rows x 128 bytes, 128B swizzle
+constexpr int kNKMax = 3;     // key stages (fewer at d = 128, where Q' takes two tiles)
+constexpr int kThreads = 256;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColZ0 = 0, kColZ1 = 128, kColO = 256;
+constexpr float kRescale = 8.f;  // raise the running max only when a tile exceeds it by this
+constexpr float kLn2 = 0.6931471805599453f;
+constexpr float kLog2e = 1.4426950408889634f;
+
+template <int D>
+struct KSmem {
+  static constexpr int kBoxes = D / 64;
+  static constexpr int kTile = kBoxes * kBox;
+  static constexpr int kNK = D == 128 ? 2 : 3;
+  static constexpr int oQ = 0;                 // Q' as bf16 hi, then lo
+  static constexpr int oK = oQ + 2 * kTile;
+  static constexpr int oP = oK + kNK * kTile;  // 2 buffers x two 64-key blocks
+  static constexpr int oBars = oP + 4 * kBox;
+};
+
+struct KBars {
+  uint64_t q_full, k_full[kNKMax], k_empty[kNKMax];
+  uint64_t z_full[2], z_empty[2], p_full[2], p_empty[2];
+  uint64_t drain;
+  uint32_t tmem_base;
+};
+
+__device__ __forceinline__ void tmem_ld16k(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
+      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void tmem_wait16k(uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.wait::ld.sync.aligned;"
+      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
+        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
+        "+r"(r[14]), "+r"(r[15])
+      :
+      : "memory");
+}
+__device__ __forceinline__ void tmem_st16k(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
+        "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
+        "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
+                     const __grid_constant__ CUtensorMap tmap_ql,
+                     const __grid_constant__ CUtensorMap tmap_k,
+                     const int64_t* __restrict__ coff, const int64_t* __restrict__ kb,
+                     const int64_t* __restrict__ ke, int R, const WsHeader* hdr_c,
+                     const long long* __restrict__ tile_start, float* __restrict__ O,
+                     float* __restrict__ lse2_out, float* __restrict__ lse_out, long long budget) {
+  using L = KSmem<D>;
+  constexpr int KS_D = D / 16;
+  constexpr int kNK = L::kNK;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  KBars* bars = reinterpret_cast<KBars*>(smem + L::oBars);
+  WsHeader* hdr = const_cast<WsHeader*>(hdr_c);
+  int* status = &hdr->status;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // this CTA's candidate tile: a user's tile of up to 128 candidates
+  const long long g = blockIdx.x;
+  if (__syncthreads_or(read_status(status) != 0) || g >= hdr->total_tiles) return;
+  const int u = user_of_tile(tile_start, R, g);
+  const long long c0 = coff[u] + (g - tile_start[u]) * 128;
+  const int nv = (int)min(128LL, coff[u + 1] - c0);
+  const long long k0 = kb[u], k1 = ke[u];
+  const int nkt = (int)((k1 - k0 + 127) / 128);  // key tiles (0 for a user without keys)
+
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bars->q_full), 1);
+    for (int s = 0; s < kNK; ++s) {
+      mbar_init(smem_u32(&bars->k_full[s]), 1);
+      mbar_init(smem_u32(&bars->k_empty[s]), 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(smem_u32(&bars->z_full[b]), 1);
+      mbar_init(smem_u32(&bars->z_empty[b]), 4);
+      mbar_init(smem_u32(&bars->p_full[b]), 4);
+      mbar_init(smem_u32(&bars->p_empty[b]), 1);
+    }
+    mbar_init(smem_u32(&bars->drain), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  if (warp == 0) {
+    // ================= TMA: the candidate tile of Q' once, then the user's key tiles
+    if (lane == 0 && nkt > 0) {
+      tma_prefetch_desc(&tmap_qh);
+      tma_prefetch_desc(&tmap_ql);
+      tma_prefetch_desc(&tmap_k);
+      const uint32_t qf = smem_u32(&bars->q_full);
+      mbar_arrive_expect_tx(qf, 2 * L::kTile);
+      for (int b = 0; b < L::kBoxes; ++b) {
+        tma_load_2d(sbase + L::oQ + b * kBox, &tmap_qh, b * 64, (int)c0, qf);
+        tma_load_2d(sbase + L::oQ + L::kTile + b * kBox, &tmap_ql, b * 64, (int)c0, qf);
+      }
+      int j = 0;
+      for (; j < nkt; ++j) {
+        const int st = j % kNK;
+        if (!mbar_wait(smem_u32(&bars->k_empty[st]), (uint32_t)(((j / kNK) & 1) ^ 1), status, budget)) break;
+        const uint32_t fb = smem_u32(&bars->k_full[st]);
+        mbar_arrive_expect_tx(fb, L::kTile);
+        for (int b = 0; b < L::kBoxes; ++b)
+          tma_load_2d(sbase + L::oK + st * L::kTile + b * kBox, &tmap_k, b * 64, (int)(k0 + 128LL * j), fb);
+      }
+      for (int i = (j > kNK ? j - kNK : 0); i < j; ++i)
+        mbar_wait_drain(smem_u32(&bars->k_full[i % kNK]), (uint32_t)((i / kNK) & 1), budget);
+      mbar_wait_drain(qf, 0, budget);
+    }
+  } else if (warp == 1) {
+    // ================= MMAs: Z(j) = Q' Kx_j^T, then O' += P(j) Kx_j once P(j) is stored;
+    // Z(j + 1) is issued before O'(j) so the softmax of tile j + 1 can start early
+    if (lane == 0 && nkt > 0) {
+      const uint32_t id_z = idesc_bf16_f32(128, 128, 0, 0);  // Q' (K) x Kx (K)
+      const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);    // P (K) x Kx (MN)
+      const uint64_t dqh = smem_desc(sbase + L::oQ, 16, 1024, kSwizzle128B);
+      const uint64_t dql = smem_desc(sbase + L::oQ + L::kTile, 16, 1024, kSwizzle128B);
+      bool ok = mbar_wait(smem_u32(&bars->q_full), 0, status, budget);
+      auto issue_z = [&](int j) {
+        const int st = j % kNK, zb = j & 1;
+        ok = ok && mbar_wait(smem_u32(&bars->k_full[st]), (uint32_t)((j / kNK) & 1), status, budget) &&
+             mbar_wait(smem_u32(&bars->z_empty[zb]), (uint32_t)(((j >> 1) & 1) ^ 1), status, budget);
+        if (!ok) return;
+        tc_fence_after();
+        const uint64_t dk = smem_desc(sbase + L::oK + st * L::kTile, 16, 1024, kSwizzle128B);
+        // Z = (Q'_hi + Q'_lo) Kx^T: Q' enters at about 16 significant bits
+#pragma unroll
+        for (int ks = 0; ks < KS_D; ++ks) {
+          const uint64_t koff = (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4);
+          tc_mma_f16(tmem + (zb ? kColZ1 : kColZ0), dqh + koff, dk + koff, id_z, ks > 0 ? 1u : 0u);
+        }
+#pragma unroll
+        for (int ks = 0; ks < KS_D; ++ks) {
+          const uint64_t koff = (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4);
+          tc_mma_f16(tmem + (zb ? kColZ1 : kColZ0), dql + koff, dk + koff, id_z, 1u);
+        }
+        tc_commit(smem_u32(&bars->z_full[zb]));
+      };
+      issue_z(0);
+      for (int j = 0; ok && j < nkt; ++j) {
+        if (j + 1 < nkt) issue_z(j + 1);
+        const int st = j % kNK, pb = j & 1;
+        ok = ok && mbar_wait(smem_u32(&bars->p_full[pb]), (uint32_t)((j >> 1) & 1), status, budget);
+        if (!ok) break;
+        tc_fence_after();
+        const uint64_t dp = smem_desc(sbase + L::oP + pb * 2 * kBox, 16, 1024, kSwizzle128B);
+        const uint64_t dk = smem_desc(sbase + L::oK + st * L::kTile, kBox, 1024, kSwizzle128B);
+#pragma unroll
+        for (int ks = 0; ks < 8; ++ks)
+          tc_mma_f16(tmem + kColO, dp + (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4),
+                     dk + (uint64_t)((ks * 2048) >> 4), id_o, (j > 0 || ks > 0) ? 1u : 0u);
+        tc_commit(smem_u32(&bars->k_empty[st]));
+        tc_commit(smem_u32(&bars->p_empty[pb]));  // P(j) read, and O' holds tiles 0..j
+      }
+      tc_commit(smem_u32(&bars->drain));
+      mbar_wait_drain(smem_u32(&bars->drain), 0, budget);
+    }
+  } else if (warp >= 4) {
+    // ================= softmax: thread = candidate row = TMEM lane
+    const int q4 = warp & 3;
+    const int r = q4 * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; ok && j < nkt; ++j) {
+      const int zb = j & 1, pb = j & 1;
+      const int nk = (int)min(128LL, k1 - k0 - 128LL * j);  // valid keys of this tile
+      if (!mbar_wait_warp(smem_u32(&bars->z_full[zb]), (uint32_t)((j >> 1) & 1), status, budget)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t zt = tmem + lane_off + (zb ? kColZ1 : kColZ0);
+      // this tile's row maximum over the valid keys
+      float mt = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t z[16];
+        tmem_ld16k(zt + c * 16, z);
+        tmem_wait16k(z);
+#pragma unroll
+        for (int x = 0; x < 16; ++x)
+          if (c * 16 + x < nk) mt = fmaxf(mt, __uint_as_float(z[x]));
+      }
+      // P(j - 2) has been read: its buffer is free (and O' holds every tile before j - 1)
+      if (!mbar_wait_warp(smem_u32(&bars->p_empty[pb]), (uint32_t)(((j >> 1) & 1) ^ 1), status, budget)) {
+        ok = false;
+        break;
+      }
+      // raise the running max only past the margin; O' and l then shrink by 2^(m - mt)
+      const bool raise = mt > m + kRescale;
+      if (__any_sync(0xffffffffu, raise)) {
+        if (j > 0) {  // O' must hold tiles 0..j - 1: the release of P(j - 1)
+          if (!mbar_wait_warp(smem_u32(&bars->p_empty[(j - 1) & 1]), (uint32_t)(((j - 1) >> 1) & 1),
+                              status, budget)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const float f = raise ? ex2_approx(m - mt) : 1.f;
+#pragma unroll
+          for (int c = 0; c < D / 16; ++c) {
+            uint32_t o[16];
+            tmem_ld16k(tmem + lane_off + kColO + c * 16, o);
+            tmem_wait16k(o);
+#pragma unroll
+            for (int x = 0; x < 16; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
+            tmem_st16k(tmem + lane_off + kColO + c * 16, o);
+          }
+          asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+          l *= f;
+        }
+        if (raise) m = mt;
+      }
+      // P = 2^(z - m) (0 for keys past the range) as bf16 into the K-major P tile
+      uint8_t* prow0 = smem + L::oP + pb * 2 * kBox + r * 128;
+      float ls = 0.f;
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint32_t z[16], pk[8];
+        tmem_ld16k(zt + c * 16, z);
+        tmem_wait16k(z);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const float e0 = c * 16 + 2 * x < nk ? ex2_approx(__uint_as_float(z[2 * x]) - m) : 0.f;
+          const float e1 = c * 16 + 2 * x + 1 < nk ? ex2_approx(__uint_as_float(z[2 * x + 1]) - m) : 0.f;
+          ls += e0 + e1;
+          pk[x] = cvt_bf16x2(e0, e1);
+        }
+        uint8_t* prow = prow0 + (c >> 2) * kBox;
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int ch = (c & 3) * 2 + h;
+          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) =
+              make_uint4(pk[4 * h], pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
+        }
+      }
+      l += ls;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->z_empty[zb]));
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[pb]));
+    }
+    // ---- O' / l and lse2 for the valid candidate rows (a user without keys: 0 and -inf)
+    const bool have = ok && nkt > 0 &&
+                      mbar_wait_warp(smem_u32(&bars->p_empty[(nkt - 1) & 1]),
+                                     (uint32_t)(((nkt - 1) >> 1) & 1), status, budget);
+    if (have) tc_fence_after();
+    const float inv = l > 0.f ? 1.f / l : 0.f;
+    float* orow = O + (c0 + r) * D;
+#pragma unroll
+    for (int c = 0; c < D / 16; ++c) {
+      uint32_t o[16];
+      if (have) {
+        tmem_ld16k(tmem + lane_off + kColO + c * 16, o);
+        tmem_wait16k(o);
+      } else {
+#pragma unroll
+        for (int x = 0; x < 16; ++x) o[x] = 0u;
+      }
+      if (r < nv) {
+#pragma unroll
+        for (int x = 0; x < 16; x += 4)
+          *reinterpret_cast<float4*>(orow + c * 16 + x) =
+              make_float4(__uint_as_float(o[x]) * inv, __uint_as_float(o[x + 1]) * inv,
+                          __uint_as_float(o[x + 2]) * inv, __uint_as_float(o[x + 3]) * inv);
+      }
+    }
+    if (r < nv) {
+      const float l2 = (have && l > 0.f) ? m + lg2_approx(l) : -INFINITY;
+      lse2_out[c0 + r] = l2;
+      if (lse_out) lse_out[c0 + r] = l2 * kLn2;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+
+// Output of users whose candidates see no key rows, when there are no key rows at all:
+// O' = 0 and lse = -inf.
+__global__ void keys_empty_kernel(long long n, int d, float* __restrict__ O, float* __restrict__ lse2,
+                                  float* __restrict__ lse) {
+  for (long long i = blockIdx.x * (long long)blockDim.x + threadIdx.x; i < n * d;
+       i += (long long)gridDim.x * blockDim.x) {
+    O[i] = 0.f;
+    if (i % d == 0) {
+      lse2[i / d] = -INFINITY;
+      if (lse) lse[i / d] = -INFINITY;
+    }
+  }
+}
+
+// M[f][e] = sum_g W_q[f][g] W_K[e][g] in fp32 (block f, thread e).
+__global__ void keys_mfold_kernel(const __nv_bfloat16* __restrict__ Wq,
+                                  const __nv_bfloat16* __restrict__ WK, int d, float* __restrict__ M) {
+  const int f = blockIdx.x, e = threadIdx.x;
+  float acc = 0.f;
+  for (int g = 0; g < d; ++g)
+    acc = fmaf(__bfloat162float(Wq[f * d + g]), __bfloat162float(WK[e * d + g]), acc);
+  M[f * d + e] = acc;
+}
+
+// Q'_c = scale Q_c M in fp32, stored as hi = bf16(Q'_c) and lo = bf16(Q'_c - hi) (block per
+// candidate, thread e).
+__global__ void keys_qfold_kernel(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ M,
+                                  long long n, int d, float scale, __nv_bfloat16* __restrict__ hi,
+                                  __nv_bfloat16* __restrict__ lo) {
+  const int e = threadIdx.x;
+  for (long long c = blockIdx.x; c < n; c += gridDim.x) {
+    float acc = 0.f;
+    for (int f = 0; f < d; ++f) acc = fmaf(__bfloat162float(Q[c * d + f]), M[f * d + e], acc);
+    const float v = acc * scale;
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    hi[c * d + e] = h;
+    lo[c * d + e] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
+}
+
+// Validates the key ranges: 0 <= kb[u] <= ke[u] <= n_keys (else SA_ERR_BAD_OFFSETS).
+__global__ void check_ranges_kernel(const int64_t* __restrict__ kb, const int64_t* __restrict__ ke,
+                                    int R, long long n_keys, WsHeader* hdr) {
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < R; u += gridDim.x * blockDim.x)
+    if (kb[u] < 0 || ke[u] < kb[u] || ke[u] > n_keys) latch_status(&hdr->status, SA_ERR_BAD_OFFSETS);
+}
+
+// The recent branch's keys: user u's last min(n_u, L) history rows.
+__global__ void recent_ranges_kernel(const int64_t* __restrict__ off, int R, long long L,
+                                     int64_t* __restrict__ kb, int64_t* __restrict__ ke) {
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < R; u += gridDim.x * blockDim.x) {
+    const long long a = off[u], b = off[u + 1];
+    kb[u] = b - a > L ? b - L : a;
+    ke[u] = b;
+  }
+}
+
+// kpre[u] = sum over users before u of their key counts (kpre[R] = all pairs): one block,
+// each thread scans a contiguous chunk of users.
+__global__ void __launch_bounds__(1024) key_prefix_kernel(const int64_t* __restrict__ kb,
+                                                          const int64_t* __restrict__ ke, int R,
+                                                          long long* __restrict__ kpre) {
+  __shared__ long long part[1024];
+  const int t = threadIdx.x;
+  const int chunk = (R + 1023) / 1024;
+  const int a = min(R, t * chunk), b = min(R, a + chunk);
+  long long sum = 0;
+  for (int u = a; u < b; ++u) sum += max(ke[u] - kb[u], (int64_t)0);
+  part[t] = sum;
+  __syncthreads();
+  for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan over the 1024 chunk sums
+    const long long v = t >= o ? part[t - o] : 0;
+    __syncthreads();
+    part[t] += v;
+    __syncthreads();
+  }
+  long long run = part[t] - sum;
+  for (int u = a; u < b; ++u) {
+    kpre[u] = run;
+    run += max(ke[u] - kb[u], (int64_t)0);
+  }
+  if (t == 1023) kpre[R] = part[1023];
+}
+
+// largest u with pre[u] <= x, for a non-decreasing pre[0..R] with pre[0] <= x < pre[R]
+__device__ __forceinline__ int segment_of(const long long* pre, int R, long long x) {
+  int lo = 0, hi = R;
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (pre[mid] <= x) lo = mid; else hi = mid;
+  }
+  return lo;
+}
+
+template <int E>
+__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const uint2 w = *reinterpret_cast<const uint2*>(p);
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&w.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w.y);
+    v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
+  } else {
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(p);
+    v[0] = __low2float(a); v[1] = __high2float(a);
+  }
+}
+
+// Q' = hi + lo
+template <int E>
+__device__ __forceinline__ void load_q(const __nv_bfloat16* hi, const __nv_bfloat16* lo,
+                                       long long i, float (&v)[E]) {
+  float a[E], b[E];
+  load_bf16<E>(hi + i, a);
+  load_bf16<E>(lo + i, b);
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = a[e] + b[e];
+}
+
+template <int E>
+__device__ __forceinline__ void load_f32(const float* p, float (&v)[E]) {
+  if constexpr (E == 4) {
+    const float4 w = *reinterpret_cast<const float4*>(p);
+    v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
+  } else {
+    const float2 w = *reinterpret_cast<const float2*>(p);
+    v[0] = w.x; v[1] = w.y;
+  }
+}
+
+// Sums two per-lane partial dot products over the warp (every lane gets both totals).
+__device__ __forceinline__ void warp_sum2(float& x, float& y) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    x += __shfl_xor_sync(0xffffffffu, x, o);
+    y += __shfl_xor_sync(0xffffffffu, y, o);
+  }
+}
+
+// Backward, candidate side (CUDA cores, one warp per candidate c of user u):
+//   a_cj = 2^(Q'_c . Kx_j - lse2_c),  dz_cj = a_cj (dO_c . Kx_j - D_c),  G1_c = sum_j dz_cj Kx_j
+// over the user's key rows j; lane l holds elements [l E, l E + E) of each row.
+template <int D>
+__global__ void keys_bwd_g1_kernel(const __nv_bfloat16* __restrict__ Qh,
+                                   const __nv_bfloat16* __restrict__ Ql, const float* __restrict__ dO,
+                                   const float* __restrict__ lse2, const float* __restrict__ Dd,
+                                   const int64_t* __restrict__ coff, int R,
+                                   const __nv_bfloat16* __restrict__ Kx, const int64_t* __restrict__ kb,
+                                   const int64_t* __restrict__ ke, long long n_cand,
+                                   float* __restrict__ G1, const WsHeader* hdr) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  if (__any_sync(0xffffffffu, read_status(&hdr->status) != 0)) return;
+  const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long c = w0; c < n_cand; c += nw) {
+    const int u = segment_of(reinterpret_cast<const long long*>(coff), R, c);
+    const long long j0 = kb[u], j1 = ke[u];
+    float q[E], o[E], g[E];
+    load_q<E>(Qh, Ql, c * D + lane * E, q);
+    load_f32<E>(dO + c * D + lane * E, o);
+    const float l2 = lse2[c], dc = Dd[c];
+#pragma unroll
+    for (int e = 0; e < E; ++e) g[e] = 0.f;
+    for (long long j = j0; j < j1; ++j) {
+      float k[E];
+      load_bf16<E>(Kx + j * D + lane * E, k);
+      float z = 0.f, p = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        z = fmaf(q[e], k[e], z);
+        p = fmaf(o[e], k[e], p);
+      }
+      warp_sum2(z, p);
+      const float dz = ex2_approx(z - l2) * (p - dc);
+#pragma unroll
+      for (int e = 0; e < E; ++e) g[e] = fmaf(dz, k[e], g[e]);
+    }
+    float* gp = G1 + c * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) gp[e] = g[e];
+  }
+}
+
+// Backward, key side (CUDA cores, one warp per (user, key row) pair):
+//   dKx_j += sum over the user's candidates c of dz_cj Qn_c + a_cj dO_c,  Qn = Q' ln 2,
+// added into dKx (zeroed before), so rows shared by several users' ranges sum.
+template <int D>
+__global__ void keys_bwd_dk_kernel(const __nv_bfloat16* __restrict__ Qh,
+                                   const __nv_bfloat16* __restrict__ Ql, const float* __restrict__ dO,
+                                   const float* __restrict__ lse2, const float* __restrict__ Dd,
+                                   const int64_t* __restrict__ coff, int R,
+                                   const __nv_bfloat16* __restrict__ Kx, const int64_t* __restrict__ kb,
+                                   const long long* __restrict__ kpre, float* __restrict__ dKx,
+                                   const WsHeader* hdr) {
+  constexpr int E = D / 32;
+  const int lane = threadIdx.x & 31;
+  if (__any_sync(0xffffffffu, read_status(&hdr->status) != 0)) return;
+  const long long total = kpre[R];
+  const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long v = w0; v < total; v += nw) {
+    const int u = segment_of(kpre, R, v);
+    const long long j = kb[u] + (v - kpre[u]);
+    float k[E], acc[E];
+    load_bf16<E>(Kx + j * D + lane * E, k);
+#pragma unroll
+    for (int e = 0; e < E; ++e) acc[e] = 0.f;
+    for (long long c = coff[u]; c < coff[u + 1]; ++c) {
+      float q[E], o[E];
+      load_q<E>(Qh, Ql, c * D + lane * E, q);
+      load_f32<E>(dO + c * D + lane * E, o);
+      float z = 0.f, p = 0.f;
+#pragma unroll
+      for (int e = 0; e < E; ++e) {
+        z = fmaf(q[e], k[e], z);
+        p = fmaf(o[e], k[e], p);
+      }
+      warp_sum2(z, p);
+      const float a = ex2_approx(z - lse2[c]);
+      const float dzl = a * (p - Dd[c]) * kLn2;
+#pragma unroll
+      for (int e = 0; e < E; ++e) acc[e] = fmaf(dzl, q[e], fmaf(a, o[e], acc[e]));
+    }
+    float* dp = dKx + j * D + lane * E;
+#pragma unroll
+    for (int e = 0; e < E; ++e) atomicAdd(dp + e, acc[e]);
+  }
+}
+
+bool map_rows_bf16(CUtensorMap* m, const void* base, uint64_t rows, int cols) {
+  auto fn = tmap_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+GemmOperandDesc opk(const void* base, uint64_t rows, uint64_t cols, bool mn_major) {
+  GemmOperandDesc o;
+  o.base = base;
+  o.rows = rows;
+  o.cols = cols;
+  o.mn_major = mn_major;
+  return o;
+}
+
+template <typename T>
+T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+// Steps shared by the forward and the backward: schedule, range check, Q', and the flash
+// kernel (O' [n_cand, d] fp32 and lse2 into the workspace; lse if asked).
+cudaError_t keys_core(const StcaKeysArgs& a, float* lse, bool fwd_call, cudaStream_t s) {
+  const StcaKeysPlan& p = a.plan;
+  WsHeader* hdr = at<WsHeader>(a.workspace, p.hdr);
+  long long* ts = at<long long>(a.workspace, p.ts);
+  cudaError_t e;
+  if ((e = launch_schedule(a.coff, a.R, a.n_cand, hdr, ts, s)) != cudaSuccess) return e;
+  if (a.R > 0) {
+    check_ranges_kernel<<<(a.R + 255) / 256, 256, 0, s>>>(a.kb, a.ke, a.R, a.n_keys, hdr);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  const long long n = a.n_cand;
+  const int d = a.d;
+  if (n == 0) return cudaSuccess;
+  float* O = at<float>(a.workspace, p.o);
+  float* lse2 = at<float>(a.workspace, p.lse2);
+  if (a.n_keys == 0) {
+    keys_empty_kernel<<<1024, 256, 0, s>>>(n, d, O, lse2, lse);
+    return cudaGetLastError();
+  }
+  // M = W_q W_K^T (fp32), then Q' = Q M log2(e) / sqrt(d) in fp32, stored as bf16 hi + lo
+  float* M = at<float>(a.workspace, p.mt);
+  __nv_bfloat16* Qh = at<__nv_bfloat16>(a.workspace, p.qh);
+  __nv_bfloat16* Ql = at<__nv_bfloat16>(a.workspace, p.ql);
+  keys_mfold_kernel<<<d, d, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wq),
+                                    static_cast<const __nv_bfloat16*>(a.WK), d, M);
+  keys_qfold_kernel<<<(unsigned)std::min<long long>(n, 148LL * 32), d, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(a.Q), M, n, d, kLog2e / std::sqrt((float)d), Qh, Ql);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  CUtensorMap tqh, tql, tk;
+  if (!map_rows_bf16(&tqh, Qh, (uint64_t)n, d) || !map_rows_bf16(&tql, Ql, (uint64_t)n, d) ||
+      !map_rows_bf16(&tk, a.Kx, (uint64_t)a.n_keys, d))
+    return cudaErrorInvalidValue;
+  const long long grid = n / 128 + a.R + 1;  // bounds the candidate tiles; the rest exit
+  if (fwd_call && (e = prof_mark_start(s)) != cudaSuccess) return e;
+  if (d == 64) {
+    const size_t smem = 1024 + KSmem<64>::oBars + sizeof(KBars);
+    if ((e = cudaFuncSetAttribute(stca_keys_fwd_kernel<64>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    stca_keys_fwd_kernel<64><<<(unsigned)grid, kThreads, smem, s>>>(
+        tqh, tql, tk, a.coff, a.kb, a.ke, a.R, hdr, ts, O, lse2, lse, kDefaultWaitBudget);
+  } else {
+    const size_t smem = 1024 + KSmem<128>::oBars + sizeof(KBars);
+    if ((e = cudaFuncSetAttribute(stca_keys_fwd_kernel<128>,
+                                  cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem)) != cudaSuccess)
+      return e;
+    stca_keys_fwd_kernel<128><<<(unsigned)grid, kThreads, smem, s>>>(
+        tqh, tql, tk, a.coff, a.kb, a.ke, a.R, hdr, ts, O, lse2, lse, kDefaultWaitBudget);
+  }
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  return fwd_call ? prof_mark_stop(s) : cudaSuccess;
+}
+
+}  // namespace
+
+size_t stca_keys_plan(int R, long long n_cand, int d, bool backward, int sms, StcaKeysPlan* p) {
+  StcaKeysPlan q;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at_ = o;
+    o = (o + bytes + 255) / 256 * 256;
+    return at_;
+  };
+  const size_t n = (size_t)n_cand, nd = n * d;
+  q.hdr = take(sizeof(WsHeader));
+  q.ts = take((size_t)(R + 1) * sizeof(long long));
+  q.mt = take((size_t)d * d * sizeof(float));
+  q.qh = take(nd * 2);
+  q.ql = take(nd * 2);
+  q.o = take(nd * sizeof(float));
+  q.lse2 = take(n * sizeof(float));
+  q.ohi = take(nd * 2);
+  q.olo = take(nd * 2);
+  if (backward) {
+    const long long kt = ((long long)n + 63) / 64;
+    long long sp = 2LL * (sms > 0 ? sms : 148);
+    if (sp > kt) sp = kt;
+    q.splits = (int)(sp < 1 ? 1 : sp);
+    q.mts = take((size_t)d * d * 2);
+    q.ghi = take(nd * 2);
+    q.glo = take(nd * 2);
+    q.gb = take(nd * 2);
+    q.do_f = take(nd * sizeof(float));
+    q.ob = take(nd * 2);
+    q.dd = take(n * sizeof(float));
+    q.g1 = take(nd * sizeof(float));
+    q.g1hi = take(nd * 2);
+    q.g1lo = take(nd * 2);
+    q.part = take((size_t)q.splits * d * d * sizeof(float));
+    q.dm = take((size_t)d * d * sizeof(float));
+    q.kpre = take((size_t)(R + 1) * sizeof(long long));
+  }
+  q.total = o;
+  *p = q;
+  return o;
+}
+
+cudaError_t launch_stca_keys_forward(const StcaKeysArgs& a, cudaStream_t s) {
+  const StcaKeysPlan& p = a.plan;
+  cudaError_t e;
+  if ((e = keys_core(a, a.lse, true, s)) != cudaSuccess) return e;
+  const long long n = a.n_cand;
+  if (n == 0) return cudaSuccess;
+  const int d = a.d;
+  const WsHeader* hdr = at<WsHeader>(a.workspace, p.hdr);
+  __nv_bfloat16* hi = at<__nv_bfloat16>(a.workspace, p.ohi);
+  __nv_bfloat16* lo = at<__nv_bfloat16>(a.workspace, p.olo);
+  if ((e = stca_split_hilo(at<float>(a.workspace, p.o), n * d, hi, lo, s)) != cudaSuccess) return e;
+  // out = (hi + lo) W_V, W_V[f][e]: rows = K, cols = N
+  return gemm_hilo(hdr, hi, lo, n, d, opk(a.WV, (uint64_t)d, (uint64_t)d, true), a.out, s);
+}
+
+cudaError_t launch_stca_keys_backward(const StcaKeysArgs& a, const StcaKeysGrads& gr,
+                                      cudaStream_t s) {
+  const StcaKeysPlan& p = a.plan;
+  void* ws = a.workspace;
+  auto bf = [&](size_t off) { return at<__nv_bfloat16>(ws, off); };
+  auto f32 = [&](size_t off) { return at<float>(ws, off); };
+  const WsHeader* hdr = at<WsHeader>(ws, p.hdr);
+  const int R = a.R, d = a.d;
+  const long long n = a.n_cand;
+  const float isd = 1.0f / std::sqrt((float)d);
+  cudaError_t e;
+  if ((e = keys_core(a, nullptr, false, s)) != cudaSuccess) return e;
+  if (a.n_keys > 0 &&
+      (e = cudaMemsetAsync(gr.dKx, 0, (size_t)a.n_keys * d * sizeof(float), s)) != cudaSuccess)
+    return e;
+  if (n == 0) {
+    for (float* g : {gr.dWq, gr.dWK, gr.dWV})
+      if ((e = cudaMemsetAsync(g, 0, (size_t)d * d * sizeof(float), s)) != cudaSuccess) return e;
+    return cudaSuccess;
+  }
+  const float* O = f32(p.o);
+  // G = dL/dout as hi + lo (for dO') and bf16 (for dW_V); O' as bf16 (for dW_V)
+  if ((e = stca_split_hilo(gr.dout, n * d, bf(p.ghi), bf(p.glo), s)) != cudaSuccess) return e;
+  if ((e = stca_to_bf16(gr.dout, n * d, bf(p.gb), s)) != cudaSuccess) return e;
+  if ((e = stca_to_bf16(O, n * d, bf(p.ob), s)) != cudaSuccess) return e;
+  // dO' = G W_V^T: B[n = f][k = e] = W_V[f][e], K-major
+  if ((e = gemm_hilo(hdr, bf(p.ghi), bf(p.glo), n, d, opk(a.WV, (uint64_t)d, (uint64_t)d, false),
+                     f32(p.do_f), s)) != cudaSuccess)
+    return e;
+  // dW_V = O'^T G
+  if ((e = gemm_tn_sum(hdr, bf(p.ob), bf(p.gb), n, d, p.splits, f32(p.part), 1.0f, gr.dWV, s)) !=
+      cudaSuccess)
+    return e;
+  // D_c = dO'_c . O'_c
+  if ((e = stca_rowdot(f32(p.do_f), O, n, d, f32(p.dd), s)) != cudaSuccess) return e;
+  const __nv_bfloat16* Qh = bf(p.qh);
+  const __nv_bfloat16* Ql = bf(p.ql);
+  const __nv_bfloat16* Kx = static_cast<const __nv_bfloat16*>(a.Kx);
+  if (a.n_keys > 0) {
+    if (R > 0) {
+      key_prefix_kernel<<<1, 1024, 0, s>>>(a.kb, a.ke, R, at<long long>(ws, p.kpre));
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    const unsigned gq = (unsigned)std::min<long long>((n + 7) / 8, 148LL * 64);
+    const unsigned gk = (unsigned)std::min<long long>((a.n_keys + 7) / 8, 148LL * 64);
+    if (d == 64) {
+      keys_bwd_g1_kernel<64><<<gq, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd), a.coff, R,
+                                                Kx, a.kb, a.ke, n, f32(p.g1), hdr);
+      if (R > 0)
+        keys_bwd_dk_kernel<64><<<gk, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd), a.coff,
+                                                  R, Kx, a.kb, at<long long>(ws, p.kpre), gr.dKx,
+                                                  hdr);
+    } else {
+      keys_bwd_g1_kernel<128><<<gq, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd), a.coff,
+                                                 R, Kx, a.kb, a.ke, n, f32(p.g1), hdr);
+      if (R > 0)
+        keys_bwd_dk_kernel<128><<<gk, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd),
+                                                   a.coff, R, Kx, a.kb, at<long long>(ws, p.kpre),
+                                                   gr.dKx, hdr);
+    }
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  } else if ((e = cudaMemsetAsync(f32(p.g1), 0, (size_t)n * d * sizeof(float), s)) != cudaSuccess) {
+    return e;
+  }
+  // dQ = G1 M^T / sqrt(d) (Mts = M^T / sqrt(d) stored [f][r]: B MN-major, rows = K = f)
+  if ((e = stca_split_hilo(f32(p.g1), n * d, bf(p.g1hi), bf(p.g1lo), s)) != cudaSuccess) return e;
+  if ((e = launch_fold(a.WK, a.Wq, SA_BF16, d, d, d, isd, bf(p.mts), true, s)) != cudaSuccess)
+    return e;
+  if ((e = gemm_hilo(hdr, bf(p.g1hi), bf(p.g1lo), n, d, opk(bf(p.mts), (uint64_t)d, (uint64_t)d, true),
+                     gr.dQ, s)) != cudaSuccess)
+    return e;
+  // dM = Q^T G1 / sqrt(d), then dW_q = dM W_K and dW_K = dM^T W_q
+  if ((e = stca_to_bf16(f32(p.g1), n * d, bf(p.gb), s)) != cudaSuccess) return e;
+  if ((e = gemm_tn_sum(hdr, static_cast<const __nv_bfloat16*>(a.Q), bf(p.gb), n, d, p.splits,
+                       f32(p.part), isd, f32(p.dm), s)) != cudaSuccess)
+    return e;
+  return stca_weight_grads(f32(p.dm), a.Wq, a.WK, d, gr.dWq, gr.dWK, s);
+}
+
+cudaError_t launch_recent_ranges(const int64_t* offsets, int R, int64_t L, int64_t* kb,
+                                 int64_t* ke, cudaStream_t s) {
+  if (R == 0) return cudaSuccess;
+  recent_ranges_kernel<<<(R + 255) / 256, 256, 0, s>>>(offsets, R, L, kb, ke);
+  return cudaGetLastError();
+}
+
+}  // namespace sa

@@ -165,3 +165,46 @@ def make_cross_workload(counts, k: int, d: int, seed: int, s_std: float = 1.0,
         S = torch.randn(R, k, d, generator=gen) * s_std
     return CrossWorkload(R=R, k=k, d=d, counts=counts, cand_offsets=off, Q=Q, S=S.float(),
                          Wq=Wq, WK=WK, WV=WV)
+
+
+@dataclass
+class RecentWorkload:
+    """Inputs of the recent branch: candidates attending over each user's last L history
+    rows (CPU tensors)."""
+    R: int
+    d: int
+    L: int
+    lengths: np.ndarray         # history rows per user
+    offsets: torch.Tensor       # int64 [R+1], the history layout
+    X: torch.Tensor             # bf16 [n_total, d], the history (the keys, read in place)
+    counts: np.ndarray          # candidates per user
+    cand_offsets: torch.Tensor  # int64 [R+1]
+    Q: torch.Tensor             # bf16 [n_cand, d]
+    Wq: torch.Tensor            # bf16 [d, d]
+    WK: torch.Tensor
+    WV: torch.Tensor
+
+    def suffix_rows(self) -> np.ndarray:
+        """History row indices of every user's last min(n_u, L) rows, users in order."""
+        off = self.offsets.numpy()
+        rows = [np.arange(max(off[u], off[u + 1] - self.L), off[u + 1]) for u in range(self.R)]
+        return np.concatenate(rows).astype(np.int64) if rows else np.zeros(0, dtype=np.int64)
+
+
+def make_recent_workload(lengths, counts, d: int, L: int, seed: int,
+                         q_std: float = 1.0) -> RecentWorkload:
+    """Draw the history X ~ N(0, 1), candidates Q ~ N(0, q_std^2) and Wq, WK, WV ~ N(0, 1/d),
+    all bf16, in that order, for the given history lengths and candidate counts per user."""
+    gen = torch.Generator().manual_seed(seed)
+    lengths = np.asarray(lengths, dtype=np.int64)
+    counts = np.asarray(counts, dtype=np.int64)
+    assert len(lengths) == len(counts)
+    R = len(lengths)
+    off = torch.from_numpy(np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64))
+    coff = torch.from_numpy(np.concatenate([[0], np.cumsum(counts)]).astype(np.int64))
+    X = torch.randn(int(off[-1]), d, generator=gen).to(torch.bfloat16)
+    Q = (torch.randn(int(coff[-1]), d, generator=gen) * q_std).to(torch.bfloat16)
+    Wq, WK, WV = ((torch.randn(d, d, generator=gen) / math.sqrt(d)).to(torch.bfloat16)
+                  for _ in range(3))
+    return RecentWorkload(R=R, d=d, L=int(L), lengths=lengths, offsets=off, X=X, counts=counts,
+                          cand_offsets=coff, Q=Q, Wq=Wq, WK=WK, WV=WV)

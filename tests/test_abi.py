@@ -142,3 +142,40 @@ def test_forward_host_rejects_bad_host_offsets(lib):
                m.ctypes.data, None, 0, 4, None, None, None)
         # valid offsets without a device fail on the plan (no device) or the buffer
         assert rc == code or (code == 3 and rc == 7), (off, rc)
+
+
+def test_ragged_key_attention_rejects_bad_arguments_on_host(lib):
+    """The ragged-key cross attention checks sizes, pointers and alignment before any
+    CUDA call (these run without a GPU)."""
+    vp, i64, i32, sz = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_size_t
+    f = lib.sa_stca_keys_forward
+    f.restype = i32
+    f.argtypes = [vp, vp, i32, i64, i32, vp, i64, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]
+
+    def call(**kw):
+        a = dict(Q=16, coff=16, R=1, n=4, d=128, Kx=16, nk=10, kb=8, ke=8, out=16)
+        a.update(kw)
+        return f(a["Q"], a["coff"], a["R"], a["n"], a["d"], a["Kx"], a["nk"], a["kb"], a["ke"],
+                 16, 16, 16, a["out"], None, 256, 1 << 30, None)
+
+    assert call(d=96) == 2                 # d not in {64, 128}
+    assert call(R=-1) == 1
+    assert call(n=-1) == 1
+    assert call(nk=-1) == 1
+    assert call(nk=1 << 31) == 1           # key rows past the 32-bit TMA coordinate
+    assert call(Kx=None) == 1              # keys announced but no pointer
+    assert call(kb=None) == 1
+    assert call(kb=12) == 1                # ranges not 8-byte aligned
+    assert call(Q=24) == 1                 # Q not 16-byte aligned
+    assert call(out=None) == 1
+    g = lib.sa_stca_recent_ranges
+    g.restype = i32
+    g.argtypes = [vp, i32, i64, vp, vp, vp]
+    assert g(16, 1, -1, 8, 8, None) == 1   # L < 0
+    assert g(None, 2, 10, 8, 8, None) == 1
+    h = lib.sa_stca_keys_workspace_size
+    h.restype = sz
+    h.argtypes = [i32, i64, i32, i32]
+    assert h(1, 10, 96, 0) == 0
+    assert h(-1, 10, 128, 0) == 0
+    assert h(2, 10, 128, 0) > 0
