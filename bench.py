@@ -88,6 +88,15 @@ def sustained_peak():
         return None
 
 
+def measured_hbm() -> float:
+    """The measured copy bandwidth in GB/s (the profiling recipe's 6.65 TB/s if absent)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"])
+    except Exception:
+        return 6650.0
+
+
 def profiled_traffic():
     """DRAM bytes per launch from the committed ncu summary, if it was taken on the
     current kernel source (null otherwise)."""
@@ -380,6 +389,82 @@ def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> di
         return {"error": repr(e)[:300]}
 
 
+def time_sketch_branch(binding, dev, sketch, peak: float, hbm_gbs: float, steps: int = 20) -> dict:
+    """The sketch branch of STCA with MRLB on the headline batch's sketches (40 users,
+    k = 1024, d = 128): every user's 300 candidates read that user's one sketch
+    (sa_stca_forward, sa_stca_backward), and the sketch cache codec packing and unpacking
+    those 40 sketches (FP8 E4M3 with row scales). A 256 MB L2 flush precedes every timed
+    call, outside its events. Reported beside the headline; a failure here is reported,
+    not raised."""
+    import torch
+    out = {}
+    try:
+        gen = torch.Generator().manual_seed(78)
+        R, k, d = sketch.shape
+        n_cand = R * RECENT_CANDIDATES
+        coff = torch.arange(0, n_cand + 1, RECENT_CANDIDATES, dtype=torch.int64).to(dev)
+        Q = torch.randn(n_cand, d, generator=gen).to(torch.bfloat16).to(dev)
+        Wq, WK, WV = ((torch.randn(d, d, generator=gen) / d ** 0.5).to(torch.bfloat16).to(dev)
+                      for _ in range(3))
+        G = torch.randn(n_cand, d, generator=gen).to(dev)
+        flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+        stream = torch.cuda.current_stream()
+
+        def timed(fn, n):
+            for _ in range(3):
+                fn()
+            ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                  for _ in range(n)]
+            torch.cuda.synchronize()
+            for a, b in ev:
+                flush.zero_()
+                a.record(stream)
+                fn()
+                b.record(stream)
+            torch.cuda.synchronize()
+            return sum(a.elapsed_time(b) for a, b in ev) / n
+
+        o = binding.stca_forward(Q, coff, sketch, Wq, WK, WV)
+        g = binding.stca_backward(Q, coff, sketch, Wq, WK, WV, G)
+        fwd_ms = timed(lambda: binding.stca_forward(Q, coff, sketch, Wq, WK, WV, ws=o["_ws"]), steps)
+        bwd_ms = timed(lambda: binding.stca_backward(Q, coff, sketch, Wq, WK, WV, G, ws=g["_ws"]), 5)
+        for ws in (o["_ws"], g["_ws"]):
+            st = binding.device_status(ws)
+            if st != 0:
+                raise RuntimeError(binding.sa_status_string(st))
+        flop = 4.0 * k * d * n_cand  # scores and weighted sum over the k rows, per candidate
+        out["stca_sketch"] = {
+            "workload": f"{R} users x {RECENT_CANDIDATES} candidates over each user's k={k} x "
+                        f"d={d} sketch",
+            "forward_ms": fwd_ms, "forward_tflops": flop / (fwd_ms / 1e3) / 1e12,
+            "forward_frac": flop / (fwd_ms / 1e3) / 1e12 / peak,
+            "backward_ms": bwd_ms,
+            "note": "composed from the tcgen05 GEMM: Q' fold, lse, weights, O = A S, O W_V; "
+                    "4kd FLOP per candidate; one sketch read per user",
+            "l2": "256 MB flush before every timed call"}
+    except Exception as e:
+        out["stca_sketch"] = {"error": repr(e)[:300]}
+    try:
+        rows = sketch.numel() // sketch.shape[-1]
+        pk = binding.sketch_pack(sketch)
+        pack_ms = timed(lambda: binding.sketch_pack(sketch), steps)
+        unpack_ms = timed(lambda: binding.sketch_unpack(pk), steps)
+        d = sketch.shape[-1]
+        pack_bytes = rows * d * 4 + rows * d + rows * 4      # fp32 in; codes and scales out
+        out["codec"] = {
+            "workload": f"FP8 E4M3 with row scales, {rows} rows x d={d} (the 40 sketches)",
+            "pack_ms": pack_ms, "unpack_ms": unpack_ms,
+            "pack_gbs": pack_bytes / (pack_ms / 1e3) / 1e9,
+            "unpack_gbs": pack_bytes / (unpack_ms / 1e3) / 1e9,
+            "pack_frac_of_hbm": pack_bytes / (pack_ms / 1e3) / 1e9 / hbm_gbs,
+            "bytes_per_call": pack_bytes,
+            "note": "one kernel each; 21 MB moved, so launch latency is a visible share",
+            "l2": "256 MB flush before every timed call"}
+    except Exception as e:
+        out["codec"] = {"error": repr(e)[:300]}
+    return out
+
+
 # ------------------------------------------------------------------ reference arm
 def run_reference(args) -> None:
     rank = int(os.environ.get("RANK", "0"))
@@ -568,9 +653,10 @@ def run_ours(args) -> None:
     if world == 1 and not args.no_other_workloads:
         others = time_other_workloads(binding, inputs, dev, max(3, min(args.steps, 50)), peak)
 
-    recent = None
+    recent = sketch_branch = None
     if world == 1 and not args.no_other_workloads:
         recent = time_recent_branch(binding, dev, X, off, peak)
+        sketch_branch = time_sketch_branch(binding, dev, out["sketch"], peak, measured_hbm())
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -620,6 +706,8 @@ def run_ours(args) -> None:
         line["other_workloads"] = others
     if recent is not None:
         line["stca_recent"] = recent
+    if sketch_branch is not None:
+        line.update(sketch_branch)
     print(json.dumps(line), flush=True)
 
 

@@ -311,12 +311,17 @@ int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M
  *   out          [n_cand, d]  fp32, device   output (overwritten)
  *   lse          [n_cand]     fp32, device   output, nullable
  * d in {64, 128}; 1 <= k <= SA_MAX_K; n_cand <= INT32_MAX; pointers 16-byte aligned.
- * A user without candidates reads nothing. Precision: Q Wq WK^T, the attention weights
- * and the sketch enter the tensor cores as bf16, with fp32 accumulation.
- * The workspace (sa_stca_workspace_size bytes, 256-aligned, caller-owned) holds the
- * bf16 sketch and the candidates' bf16 weights over the k rows (2 k bytes each); errors
- * follow sa_sketch_forward's conventions, and the device status word in the workspace
- * is read with sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
+ * A user without candidates reads nothing. R k_pad <= INT32_MAX (k_pad = k rounded up to
+ * a multiple of 128). The forward runs sa_stca_keys_forward's flash kernel with the
+ * bf16 sketch as the key rows. Precision: Q Wq WK^T / sqrt(d) is formed in fp32 and
+ * enters the tensor cores as a bf16 pair hi + lo; the sketch and the attention weights
+ * enter as bf16; accumulation is fp32. The backward (below) computes with Q Wq WK^T in
+ * bf16 and forms the weights over the k rows in bf16 (2 k bytes per candidate).
+ * The workspace (sa_stca_workspace_size bytes, 256-aligned, caller-owned) holds the bf16
+ * sketch and, per candidate, Q Wq WK^T and the unprojected output (forward) or the
+ * weights and their gradients (backward); errors follow sa_sketch_forward's
+ * conventions, and the device status word in the workspace is read with
+ * sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
  */
 size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d, int backward);
 int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,

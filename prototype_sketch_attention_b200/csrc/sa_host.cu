@@ -352,6 +352,7 @@ int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n
   if ((d != 64 && d != 128) || k < 1 || k > SA_MAX_K) return SA_ERR_UNSUPPORTED;
   if (!cand_offsets || !Wq || !WK || !WV || (n_cand > 0 && (!Q || !out)) || (R > 0 && !S))
     return SA_ERR_INVALID_ARG;
+  if ((long long)R * ((k + 127) / 128 * 128) > INT32_MAX) return SA_ERR_INVALID_ARG;
   if (!aligned16(Q) || !aligned16(cand_offsets) || !aligned16(S) || !aligned16(Wq) ||
       !aligned16(WK) || !aligned16(WV) || !aligned16(out) || !aligned16(lse))
     return SA_ERR_INVALID_ARG;

@@ -203,6 +203,9 @@ struct StcaPlan {  // workspace layout (byte offsets, 256-aligned)
   int k_pad = 0, nparts = 0, splits = 0;
   size_t hdr = 0, ts = 0, sb = 0, mt = 0, qp = 0, dpart = 0, lse2 = 0, ab = 0, o = 0, ohi = 0,
          olo = 0, total = 0;
+  // forward: the ragged-key attention's workspace first (its header is the status word),
+  // then the bf16 sketch and every user's row range within it
+  size_t kb = 0, ke = 0;
   // backward only
   size_t mts = 0, qn = 0, do_f = 0, do_b = 0, dd = 0, czero = 0, dz = 0, g1 = 0, g1hi = 0,
          g1lo = 0, gb = 0, ob = 0, ghi = 0, glo = 0, part = 0, dm = 0;

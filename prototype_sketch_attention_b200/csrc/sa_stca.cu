@@ -7,13 +7,16 @@
 // the sketch branch, and "3. The system makes it cheap enough to matter", multi-request
 // user-level batching). Refold: with Q' = Q (W_q W_K^T) log2(e) / sqrt(d) the scores are
 // Q' S_u^T in log2 units, keys and values are the same matrix S_u, and W_V is applied
-// once per candidate after the weighted sum. Steps, all on one stream:
+// once per candidate after the weighted sum.
+// The forward is the flash kernel of the ragged-key attention (sa_stca_keys.cu) with the
+// bf16 sketch as the key rows: S -> bf16 [R, k_pad, d], user u's keys the rows
+// [u k_pad, u k_pad + k). The backward is composed from the tcgen05 GEMM, all on one
+// stream:
 //   1. schedule over the candidate offsets (128-candidate tiles that never span users)
 //   2. S -> bf16 [R, k_pad, d] (zero rows past k); M^T = W_K W_q^T; Q' = Q M
 //   3. per-candidate log2-sum-exp2 of Q' S_u^T: GEMM (kEpiLse partials) + combine
 //   4. A = 2^(Q' S_u^T - lse2) in bf16 (GEMM, kEpiAExp), then O = A S_u in fp32
-//   5. out = O W_V, with O entering as bf16 hi + lo (two accumulated GEMM phases)
-// The backward recomputes steps 1-4 and then, with G = dL/dout and natural-log units
+// and then, with G = dL/dout and natural-log units
 // (z = Q M S_u^T / sqrt(d), M = W_q W_K^T):
 //   dO = G W_V^T,  dW_V = O^T G,  D_c = dO_c . O_c,  dZ = A (dO S_u^T - D)
 //   G1 = dZ S_u,  dQ = G1 M^T / sqrt(d),  dM = Q^T G1 / sqrt(d)
@@ -38,6 +41,15 @@ __global__ void stca_sketch_bf16_kernel(const float* __restrict__ S, int R, int 
        i += (long long)gridDim.x * blockDim.x) {
     const long long e = i % d, rj = i / d, j = rj % k_pad, u = rj / k_pad;
     Sb[i] = __float2bfloat16_rn(j < k ? S[(u * k + j) * d + e] : 0.f);
+  }
+}
+
+// User u's sketch rows within the bf16 sketch: [u k_pad, u k_pad + k).
+__global__ void stca_sketch_ranges_kernel(int R, int k, int k_pad, int64_t* __restrict__ kb,
+                                          int64_t* __restrict__ ke) {
+  for (int u = blockIdx.x * blockDim.x + threadIdx.x; u < R; u += gridDim.x * blockDim.x) {
+    kb[u] = (int64_t)u * k_pad;
+    ke[u] = (int64_t)u * k_pad + k;
   }
 }
 
@@ -143,6 +155,17 @@ size_t stca_plan(int R, long long n_cand, int k, int d, bool backward, int sms, 
     o = (o + bytes + 255) / 256 * 256;
     return at;
   };
+  if (!backward) {  // the flash kernel over each user's sketch rows
+    StcaKeysPlan kp;
+    o = stca_keys_plan(R, n_cand, d, false, 0, &kp);
+    q.hdr = kp.hdr;
+    q.sb = take((size_t)R * q.k_pad * d * 2);
+    q.kb = take((size_t)R * sizeof(int64_t));
+    q.ke = take((size_t)R * sizeof(int64_t));
+    q.total = o;
+    *p = q;
+    return o;
+  }
   const size_t n = (size_t)n_cand;
   const size_t nd = n * d;
   q.hdr = take(sizeof(WsHeader));
@@ -360,18 +383,38 @@ cudaError_t gemm_tn_sum(const WsHeader* hdr, const __nv_bfloat16* A, const __nv_
   return cudaGetLastError();
 }
 
+// The forward is the ragged-key attention (sa_stca_keys.cu) over each user's sketch rows:
+// the sketch in bf16 [R, k_pad, d], user u's keys the rows [u k_pad, u k_pad + k).
 cudaError_t launch_stca_forward(const StcaArgs& a, cudaStream_t s) {
-  const Bufs b = bufs(a.plan, a.workspace);
-  const long long n = a.n_cand;
-  const int d = a.d;
+  const StcaPlan& p = a.plan;
+  uint8_t* ws = static_cast<uint8_t*>(a.workspace);
+  __nv_bfloat16* Sb = reinterpret_cast<__nv_bfloat16*>(ws + p.sb);
+  int64_t* kb = reinterpret_cast<int64_t*>(ws + p.kb);
+  int64_t* ke = reinterpret_cast<int64_t*>(ws + p.ke);
   cudaError_t e;
-  if ((e = launch_schedule(a.coff, a.R, n, b.hdr, b.ts, s)) != cudaSuccess) return e;
-  if (n == 0) return cudaSuccess;
-  if ((e = forward_core(a, b, s)) != cudaSuccess) return e;
-  stca_split_kernel<<<1024, 256, 0, s>>>(b.O, n * d, b.Ohi, b.Olo);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  // out = (hi + lo) W_V, W_V[f][e]: rows = K, cols = N
-  return gemm_hilo(b.hdr, b.Ohi, b.Olo, n, d, opd(a.WV, (uint64_t)d, (uint64_t)d, true), a.out, s);
+  if (a.R > 0) {
+    stca_sketch_bf16_kernel<<<1024, 256, 0, s>>>(a.S, a.R, a.k, p.k_pad, a.d, Sb);
+    stca_sketch_ranges_kernel<<<(a.R + 255) / 256, 256, 0, s>>>(a.R, a.k, p.k_pad, kb, ke);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  StcaKeysArgs k;
+  k.Q = a.Q;
+  k.coff = a.coff;
+  k.R = a.R;
+  k.d = a.d;
+  k.n_cand = a.n_cand;
+  k.Kx = Sb;
+  k.n_keys = (long long)a.R * p.k_pad;
+  k.kb = kb;
+  k.ke = ke;
+  k.Wq = a.Wq;
+  k.WK = a.WK;
+  k.WV = a.WV;
+  k.out = a.out;
+  k.lse = a.lse;
+  k.workspace = a.workspace;
+  stca_keys_plan(a.R, a.n_cand, a.d, false, 0, &k.plan);
+  return launch_stca_keys_forward(k, s);
 }
 
 cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& gr, cudaStream_t s) {

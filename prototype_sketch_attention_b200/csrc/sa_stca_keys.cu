@@ -14,14 +14,18 @@
 // accumulated MMAs, about 16 significant bits): with scores of tens of units a single bf16
 // rounding of Q' would move the weights by several percent.
 //
-// One CTA per (user, 128-candidate tile). The softmax runs along each candidate's row of
-// Z in TMEM, one thread per candidate, with a running maximum that is raised only when a
-// tile's maximum exceeds it by more than 8 (in log2 units): then O' (in TMEM) and the
-// running sum are rescaled once; otherwise the exponentials stay below 2^8 and nothing is
-// rescaled. P = 2^(z - m) goes to shared memory as bf16 (the K-major A operand of the
-// second MMA), O' accumulates in TMEM, and at the end O' / l and lse2 = m + log2 l leave.
-// Roles: warp 0 TMA, warp 1 TMEM allocation and the MMAs, warps 4-7 the softmax
-// (thread = candidate = TMEM lane). Every mbarrier wait is bounded.
+// One CTA per (user, 128-candidate tile). Two softmax warpgroups take alternate key tiles
+// (warpgroup w the tiles j with j mod 2 = w), each with its own score buffer Z_w, P
+// buffer and accumulator O'_w in TMEM, and its own running maximum m_w and sum l_w along
+// each candidate's row (one thread per candidate = TMEM lane). The running maximum is
+// raised only when a tile's maximum exceeds it by more than 8 (in log2 units): then O'_w
+// and l_w are rescaled once; otherwise the exponentials stay below 2^8. P = 2^(z - m_w)
+// goes to shared memory as bf16 (the K-major A operand of O'_w += P Kx). At the end the
+// two halves merge: m = max(m_0, m_1), O' = (O'_0 2^(m_0 - m) + O'_1 2^(m_1 - m)) / l and
+// lse2 = m + log2 l with l = l_0 2^(m_0 - m) + l_1 2^(m_1 - m).
+// Roles: warp 0 TMA, warp 1 TMEM allocation and the MMAs, warps 4-7 and 8-11 the softmax
+// warpgroups (warpgroup 0 also merges and writes the output). Every mbarrier wait is
+// bounded.
 #include <cuda.h>
 
 #include <algorithm>
@@ -34,10 +38,13 @@ namespace sa {
 namespace {
 
 constexpr int kBox = 16384;   // 128 rows x 128 bytes, 128B swizzle
-constexpr int kNKMax = 3;     // key stages (fewer at d = 128, where Q' takes two tiles)
-constexpr int kThreads = 256;
+constexpr int kNKMax = 3;     // key stages
+constexpr int kThreads = 384;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColZ0 = 0, kColZ1 = 128, kColO = 256;
+// TMEM columns: score buffers Z_0 at 0 and Z_1 at 128, accumulators O'_0 at 256 and O'_1
+// at 384 (d <= 128 columns each)
+__host__ __device__ constexpr uint32_t col_z(int w) { return w ? 128u : 0u; }
+__host__ __device__ constexpr uint32_t col_o(int w) { return w ? 384u : 256u; }
 constexpr float kRescale = 8.f;  // raise the running max only when a tile exceeds it by this
 constexpr float kLn2 = 0.6931471805599453f;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -46,47 +53,65 @@ template <int D>
 struct KSmem {
   static constexpr int kBoxes = D / 64;
   static constexpr int kTile = kBoxes * kBox;
-  static constexpr int kNK = D == 128 ? 2 : 3;
+  static constexpr int kNK = 3;  // at d = 128: 7 x 32 KB + 1 KB + barriers, within 227 KB
   static constexpr int oQ = 0;                 // Q' as bf16 hi, then lo
   static constexpr int oK = oQ + 2 * kTile;
   static constexpr int oP = oK + kNK * kTile;  // 2 buffers x two 64-key blocks
-  static constexpr int oBars = oP + 4 * kBox;
+  static constexpr int oML = oP + 4 * kBox;    // warpgroup 1's m and l per row (merge)
+  static constexpr int oBars = oML + 2 * 128 * 4;
 };
 
 struct KBars {
   uint64_t q_full, k_full[kNKMax], k_empty[kNKMax];
   uint64_t z_full[2], z_empty[2], p_full[2], p_empty[2];
-  uint64_t drain;
+  uint64_t merge, drain;
   uint32_t tmem_base;
 };
 
-__device__ __forceinline__ void tmem_ld16k(uint32_t taddr, uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x16.b32"
-      " {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
-      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
-        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
-        "=r"(r[14]), "=r"(r[15])
-      : "r"(taddr)
-      : "memory");
+// Empty asm that carries the registers through: uses after it cannot move above it.
+__device__ __forceinline__ void tie32(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31]));
 }
-__device__ __forceinline__ void tmem_wait16k(uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.wait::ld.sync.aligned;"
-      : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]),
-        "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]),
-        "+r"(r[14]), "+r"(r[15])
-      :
-      : "memory");
+
+// 64 consecutive TMEM columns of this warp's 32 lanes: two loads, one wait.
+__device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
+  tmem_ld32_raw(taddr, a);
+  tmem_ld32_raw(taddr + 32, b);
+  tmem_wait_tie(a);
+  tie32(b);
 }
-__device__ __forceinline__ void tmem_st16k(uint32_t taddr, const uint32_t (&r)[16]) {
+
+__device__ __forceinline__ void tmem_st32k(uint32_t taddr, const uint32_t (&r)[32]) {
   asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0],"
-      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};"
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0],"
+      " {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16,"
+      " %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};"
       ::"r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]),
         "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]),
-        "r"(r[14]), "r"(r[15])
+        "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]),
+        "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]),
+        "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
+}
+
+// 2^(z - m) of 16 scores as 8 bf16 pairs (0 for columns at or past nk), and their sum.
+__device__ __forceinline__ float exp_pack16(const uint32_t* z, int col0, int nk, float m,
+                                            uint32_t (&pk)[8]) {
+  float s = 0.f;
+#pragma unroll
+  for (int x = 0; x < 8; ++x) {
+    const float e0 = col0 + 2 * x < nk ? ex2_approx(__uint_as_float(z[2 * x]) - m) : 0.f;
+    const float e1 = col0 + 2 * x + 1 < nk ? ex2_approx(__uint_as_float(z[2 * x + 1]) - m) : 0.f;
+    s += e0 + e1;
+    pk[x] = cvt_bf16x2(e0, e1);
+  }
+  return s;
 }
 
 template <int D>
@@ -131,6 +156,7 @@ stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
       mbar_init(smem_u32(&bars->p_full[b]), 4);
       mbar_init(smem_u32(&bars->p_empty[b]), 1);
     }
+    mbar_init(smem_u32(&bars->merge), 4);
     mbar_init(smem_u32(&bars->drain), 1);
     fence_mbar_init();
   }
@@ -144,7 +170,7 @@ stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
   const uint32_t tmem = bars->tmem_base;
 
   if (warp == 0) {
-    // ================= TMA: the candidate tile of Q' once, then the user's key tiles
+    // ================= TMA: the candidate tile of Q' (hi, lo) once, then the key tiles
     if (lane == 0 && nkt > 0) {
       tma_prefetch_desc(&tmap_qh);
       tma_prefetch_desc(&tmap_ql);
@@ -169,8 +195,9 @@ stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
       mbar_wait_drain(qf, 0, budget);
     }
   } else if (warp == 1) {
-    // ================= MMAs: Z(j) = Q' Kx_j^T, then O' += P(j) Kx_j once P(j) is stored;
-    // Z(j + 1) is issued before O'(j) so the softmax of tile j + 1 can start early
+    // ================= MMAs: Z(j) = Q' Kx_j^T into Z_(j mod 2), then O'_(j mod 2) += P(j) Kx_j
+    // once P(j) is stored; Z(j + 1) is issued before O'(j) so that the other warpgroup's
+    // softmax of tile j + 1 runs while this one's P(j) is produced
     if (lane == 0 && nkt > 0) {
       const uint32_t id_z = idesc_bf16_f32(128, 128, 0, 0);  // Q' (K) x Kx (K)
       const uint32_t id_o = idesc_bf16_f32(128, D, 0, 1);    // P (K) x Kx (MN)
@@ -188,12 +215,12 @@ stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
 #pragma unroll
         for (int ks = 0; ks < KS_D; ++ks) {
           const uint64_t koff = (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4);
-          tc_mma_f16(tmem + (zb ? kColZ1 : kColZ0), dqh + koff, dk + koff, id_z, ks > 0 ? 1u : 0u);
+          tc_mma_f16(tmem + col_z(zb), dqh + koff, dk + koff, id_z, ks > 0 ? 1u : 0u);
         }
 #pragma unroll
         for (int ks = 0; ks < KS_D; ++ks) {
           const uint64_t koff = (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4);
-          tc_mma_f16(tmem + (zb ? kColZ1 : kColZ0), dql + koff, dk + koff, id_z, 1u);
+          tc_mma_f16(tmem + col_z(zb), dql + koff, dk + koff, id_z, 1u);
         }
         tc_commit(smem_u32(&bars->z_full[zb]));
       };
@@ -208,65 +235,66 @@ stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
         const uint64_t dk = smem_desc(sbase + L::oK + st * L::kTile, kBox, 1024, kSwizzle128B);
 #pragma unroll
         for (int ks = 0; ks < 8; ++ks)
-          tc_mma_f16(tmem + kColO, dp + (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4),
-                     dk + (uint64_t)((ks * 2048) >> 4), id_o, (j > 0 || ks > 0) ? 1u : 0u);
+          tc_mma_f16(tmem + col_o(pb), dp + (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4),
+                     dk + (uint64_t)((ks * 2048) >> 4), id_o, (j >= 2 || ks > 0) ? 1u : 0u);
         tc_commit(smem_u32(&bars->k_empty[st]));
-        tc_commit(smem_u32(&bars->p_empty[pb]));  // P(j) read, and O' holds tiles 0..j
+        tc_commit(smem_u32(&bars->p_empty[pb]));  // P(j) read, and O'_(j mod 2) holds tile j
       }
       tc_commit(smem_u32(&bars->drain));
       mbar_wait_drain(smem_u32(&bars->drain), 0, budget);
     }
   } else if (warp >= 4) {
-    // ================= softmax: thread = candidate row = TMEM lane
+    // ================= softmax warpgroup w: key tiles j = w, w + 2, ...; thread = candidate
+    const int w = (warp - 4) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
+    const uint32_t zt = tmem + lane_off + col_z(w);
+    const uint32_t ot = tmem + lane_off + col_o(w);
+    uint8_t* prow0 = smem + L::oP + w * 2 * kBox + r * 128;
     float m = -INFINITY, l = 0.f;
     bool ok = true;
-    for (int j = 0; ok && j < nkt; ++j) {
-      const int zb = j & 1, pb = j & 1;
+    int last = -1;
+    for (int j = w; ok && j < nkt; j += 2) {
       const int nk = (int)min(128LL, k1 - k0 - 128LL * j);  // valid keys of this tile
-      if (!mbar_wait_warp(smem_u32(&bars->z_full[zb]), (uint32_t)((j >> 1) & 1), status, budget)) {
+      if (!mbar_wait_warp(smem_u32(&bars->z_full[w]), (uint32_t)((j >> 1) & 1), status, budget)) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const uint32_t zt = tmem + lane_off + (zb ? kColZ1 : kColZ0);
-      // this tile's row maximum over the valid keys
-      float mt = -INFINITY;
+      float mt = -INFINITY;  // this tile's row maximum over the valid keys
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t za[32], zb[32];
+        tmem_ld64(zt + h * 64, za, zb);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t z[16];
-        tmem_ld16k(zt + c * 16, z);
-        tmem_wait16k(z);
-#pragma unroll
-        for (int x = 0; x < 16; ++x)
-          if (c * 16 + x < nk) mt = fmaxf(mt, __uint_as_float(z[x]));
+        for (int x = 0; x < 32; ++x) {
+          if (h * 64 + x < nk) mt = fmaxf(mt, __uint_as_float(za[x]));
+          if (h * 64 + 32 + x < nk) mt = fmaxf(mt, __uint_as_float(zb[x]));
+        }
       }
-      // P(j - 2) has been read: its buffer is free (and O' holds every tile before j - 1)
-      if (!mbar_wait_warp(smem_u32(&bars->p_empty[pb]), (uint32_t)(((j >> 1) & 1) ^ 1), status, budget)) {
+      // P(j - 2) has been read, and O'_w holds every earlier tile of this warpgroup
+      if (!mbar_wait_warp(smem_u32(&bars->p_empty[w]), (uint32_t)(((j >> 1) & 1) ^ 1), status, budget)) {
         ok = false;
         break;
       }
-      // raise the running max only past the margin; O' and l then shrink by 2^(m - mt)
+      // raise the running max only past the margin; O'_w and l shrink by 2^(m - mt)
       const bool raise = mt > m + kRescale;
       if (__any_sync(0xffffffffu, raise)) {
-        if (j > 0) {  // O' must hold tiles 0..j - 1: the release of P(j - 1)
-          if (!mbar_wait_warp(smem_u32(&bars->p_empty[(j - 1) & 1]), (uint32_t)(((j - 1) >> 1) & 1),
-                              status, budget)) {
-            ok = false;
-            break;
-          }
+        if (j >= 2) {
           tc_fence_after();
           const float f = raise ? ex2_approx(m - mt) : 1.f;
+#pragma unroll 1
+          for (int c = 0; c < D / 64; ++c) {
+            uint32_t oa[32], ob[32];
+            tmem_ld64(ot + c * 64, oa, ob);
 #pragma unroll
-          for (int c = 0; c < D / 16; ++c) {
-            uint32_t o[16];
-            tmem_ld16k(tmem + lane_off + kColO + c * 16, o);
-            tmem_wait16k(o);
-#pragma unroll
-            for (int x = 0; x < 16; ++x) o[x] = __float_as_uint(__uint_as_float(o[x]) * f);
-            tmem_st16k(tmem + lane_off + kColO + c * 16, o);
+            for (int x = 0; x < 32; ++x) {
+              oa[x] = __float_as_uint(__uint_as_float(oa[x]) * f);
+              ob[x] = __float_as_uint(__uint_as_float(ob[x]) * f);
+            }
+            tmem_st32k(ot + c * 64, oa);
+            tmem_st32k(ot + c * 64 + 32, ob);
           }
           asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
           l *= f;
@@ -274,65 +302,84 @@ stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
         if (raise) m = mt;
       }
       // P = 2^(z - m) (0 for keys past the range) as bf16 into the K-major P tile
-      uint8_t* prow0 = smem + L::oP + pb * 2 * kBox + r * 128;
       float ls = 0.f;
+#pragma unroll 1
+      for (int h = 0; h < 2; ++h) {
+        uint32_t za[32], zb[32];
+        tmem_ld64(zt + h * 64, za, zb);
+        uint8_t* prow = prow0 + h * kBox;  // keys [64h, 64h + 64): one 128-byte row
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint32_t z[16], pk[8];
-        tmem_ld16k(zt + c * 16, z);
-        tmem_wait16k(z);
+        for (int q = 0; q < 4; ++q) {
+          uint32_t pk[8];
+          ls += exp_pack16((q < 2 ? za : zb) + (q & 1) * 16, h * 64 + q * 16, nk, m, pk);
 #pragma unroll
-        for (int x = 0; x < 8; ++x) {
-          const float e0 = c * 16 + 2 * x < nk ? ex2_approx(__uint_as_float(z[2 * x]) - m) : 0.f;
-          const float e1 = c * 16 + 2 * x + 1 < nk ? ex2_approx(__uint_as_float(z[2 * x + 1]) - m) : 0.f;
-          ls += e0 + e1;
-          pk[x] = cvt_bf16x2(e0, e1);
-        }
-        uint8_t* prow = prow0 + (c >> 2) * kBox;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const int ch = (c & 3) * 2 + h;
-          *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) =
-              make_uint4(pk[4 * h], pk[4 * h + 1], pk[4 * h + 2], pk[4 * h + 3]);
+          for (int hh = 0; hh < 2; ++hh) {
+            const int ch = q * 2 + hh;
+            *reinterpret_cast<uint4*>(prow + ((ch ^ (r & 7)) << 4)) =
+                make_uint4(pk[4 * hh], pk[4 * hh + 1], pk[4 * hh + 2], pk[4 * hh + 3]);
+          }
         }
       }
       l += ls;
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->z_empty[zb]));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->z_empty[w]));
       fence_proxy_async_smem();
       __syncwarp();
-      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[pb]));
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_full[w]));
+      last = j;
     }
-    // ---- O' / l and lse2 for the valid candidate rows (a user without keys: 0 and -inf)
-    const bool have = ok && nkt > 0 &&
-                      mbar_wait_warp(smem_u32(&bars->p_empty[(nkt - 1) & 1]),
-                                     (uint32_t)(((nkt - 1) >> 1) & 1), status, budget);
-    if (have) tc_fence_after();
-    const float inv = l > 0.f ? 1.f / l : 0.f;
-    float* orow = O + (c0 + r) * D;
+    // ---- this warpgroup's accumulator is complete once its last O' MMA is
+    if (ok && last >= 0)
+      ok = mbar_wait_warp(smem_u32(&bars->p_empty[w]), (uint32_t)((last >> 1) & 1), status, budget);
+    float* ml = reinterpret_cast<float*>(smem + L::oML);
+    if (w == 1) {  // hand m_1 and l_1 to warpgroup 0
+      ml[r] = m;
+      ml[128 + r] = ok ? l : 0.f;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->merge));
+    } else {
+      const bool merged = mbar_wait_warp(smem_u32(&bars->merge), 0, status, budget);
+      const float m1 = ml[r], l1 = merged ? ml[128 + r] : 0.f;
+      const float l0 = ok ? l : 0.f;
+      const float mm = fmaxf(m, m1);
+      const float f0 = l0 > 0.f ? ex2_approx(m - mm) : 0.f;
+      const float f1 = l1 > 0.f ? ex2_approx(m1 - mm) : 0.f;
+      const float lt = l0 * f0 + l1 * f1;
+      const float inv = lt > 0.f ? 1.f / lt : 0.f;
+      const float g0 = f0 * inv, g1 = f1 * inv;
+      if (nkt > 0) tc_fence_after();
+      float* orow = O + (c0 + r) * D;
+#pragma unroll 1
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t oa[32], ob[32];
+        if (nkt > 0) {  // O'_0 (every user with keys has tile 0)
+          tmem_ld32_raw(tmem + lane_off + col_o(0) + c * 32, oa);
+          tmem_wait_tie(oa);
+        }
+        if (nkt > 1) {  // O'_1 only if warpgroup 1 had a tile
+          tmem_ld32_raw(tmem + lane_off + col_o(1) + c * 32, ob);
+          tmem_wait_tie(ob);
+        }
+        if (r < nv) {
 #pragma unroll
-    for (int c = 0; c < D / 16; ++c) {
-      uint32_t o[16];
-      if (have) {
-        tmem_ld16k(tmem + lane_off + kColO + c * 16, o);
-        tmem_wait16k(o);
-      } else {
+          for (int x = 0; x < 32; x += 4) {
+            float v[4];
 #pragma unroll
-        for (int x = 0; x < 16; ++x) o[x] = 0u;
+            for (int y = 0; y < 4; ++y) {
+              const float a0 = nkt > 0 ? __uint_as_float(oa[x + y]) * g0 : 0.f;
+              v[y] = nkt > 1 ? fmaf(__uint_as_float(ob[x + y]), g1, a0) : a0;
+            }
+            *reinterpret_cast<float4*>(orow + c * 32 + x) = make_float4(v[0], v[1], v[2], v[3]);
+          }
+        }
       }
       if (r < nv) {
-#pragma unroll
-        for (int x = 0; x < 16; x += 4)
-          *reinterpret_cast<float4*>(orow + c * 16 + x) =
-              make_float4(__uint_as_float(o[x]) * inv, __uint_as_float(o[x + 1]) * inv,
-                          __uint_as_float(o[x + 2]) * inv, __uint_as_float(o[x + 3]) * inv);
+        const float l2 = lt > 0.f ? mm + lg2_approx(lt) : -INFINITY;
+        lse2_out[c0 + r] = l2;
+        if (lse_out) lse_out[c0 + r] = l2 * kLn2;
       }
-    }
-    if (r < nv) {
-      const float l2 = (have && l > 0.f) ? m + lg2_approx(l) : -INFINITY;
-      lse2_out[c0 + r] = l2;
-      if (lse_out) lse_out[c0 + r] = l2 * kLn2;
     }
   }
 
@@ -343,7 +390,6 @@ stca_keys_fwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
     tmem_dealloc(tmem, kTmemCols);
   }
 }
-
 
 // Output of users whose candidates see no key rows, when there are no key rows at all:
 // O' = 0 and lse = -inf.

@@ -1,12 +1,12 @@
-"""CPU model of the launch sequence in csrc/sa_stca.cu, checked against the oracle.
+"""CPU model of the launch sequences in csrc/sa_stca.cu, checked against the oracle.
 
 Each step below restates what one launch computes, from the contracts in
 csrc/sa_internal.h (launch_fold: Pf = scale * P Wk^T, rounded to bf16 when asked; the
-GEMM's kEpiLse / kEpiAExp / kEpiStoreF32 epilogues) and the kernels of sa_stca.cu,
-including every rounding to bf16. If the composition's algebra were wrong (a fold with
-its operands swapped, a missing log2(e), the sketch used untransposed, W_V applied on
-the wrong side), this model would miss the oracle by far more than the bf16 tolerance.
-It needs no GPU and shares nothing with the oracle.
+GEMM's kEpiLse / kEpiAExp / kEpiStoreF32 epilogues) and the kernels of sa_stca.cu and
+sa_stca_keys.cu, including every rounding to bf16. If the composition's algebra were
+wrong (a fold with its operands swapped, a missing log2(e), the sketch used
+untransposed, W_V applied on the wrong side), this model would miss the oracle by far
+more than the bf16 tolerance. It needs no GPU and shares nothing with the oracle.
 """
 import math
 
@@ -28,32 +28,34 @@ def fold(P, Wk, scale, to_bf16):
 
 
 def model_forward(cw):
+    """The forward: the flash kernel of sa_stca_keys.cu over the bf16 sketch rows. The
+    kernel's running maximum stays within 8 (log2 units) of the row maximum and only
+    scales the bf16 weights' exponent, so the model uses the row maximum."""
     Q = cw.Q.float().numpy().astype(np.float64)
     S = cw.S.numpy().astype(np.float64)
     Wq, WK, WV = (t.float().numpy().astype(np.float64) for t in (cw.Wq, cw.WK, cw.WV))
     R, k, d = S.shape
-    k_pad = (k + 127) // 128 * 128
     coff = cw.cand_offsets.numpy()
-    Sb = np.zeros((R, k_pad, d))
-    Sb[:, :k] = bf16(S)                                        # stca_sketch_bf16_kernel
-    Mt = fold(WK, Wq, 1.0, True)                               # M^T = W_K W_q^T
-    Qp = fold(Q, Mt, math.log2(math.e) / math.sqrt(d), True)   # Q' = Q M log2(e) / sqrt(d)
+    Sb = bf16(S)                                               # stca_sketch_bf16_kernel
+    M = fold(Wq, WK, 1.0, False)                               # keys_mfold: W_q W_K^T, fp32
+    Qp = fold(Q, M.T, math.log2(math.e) / math.sqrt(d), False)  # keys_qfold: Q M ..., fp32
+    hi_q = bf16(Qp)
+    lo_q = bf16(Qp - hi_q)
     out = np.zeros((Q.shape[0], d))
     lse = np.zeros(Q.shape[0])
     for u in range(R):
         a, b = int(coff[u]), int(coff[u + 1])
         if a == b:
             continue
-        z = Qp[a:b] @ Sb[u].T                                  # scores, log2 units
-        z[:, k:] = -np.inf                                     # columns >= k_valid
+        z = (hi_q[a:b] + lo_q[a:b]) @ Sb[u].T                  # two score MMAs, log2 units
         m = z.max(axis=1, keepdims=True)
-        lse2 = (m + np.log2(np.exp2(z - m).sum(axis=1, keepdims=True)))[:, 0]
-        A = bf16(np.exp2(z - lse2[:, None]))                   # kEpiAExp
-        O = (A @ Sb[u]).astype(np.float32).astype(np.float64)  # kEpiStoreF32
+        e = np.exp2(z - m)
+        l = e.sum(axis=1, keepdims=True)
+        O = (bf16(e) @ Sb[u] / l).astype(np.float32).astype(np.float64)  # bf16 P, fp32 O'
         hi = bf16(O)
         lo = bf16(O - hi)
         out[a:b] = hi @ bf16(WV) + lo @ bf16(WV)               # two GEMM phases
-        lse[a:b] = lse2 * math.log(2.0)
+        lse[a:b] = (m[:, 0] + np.log2(l[:, 0])) * math.log(2.0)
     return out, lse
 
 
