@@ -89,6 +89,18 @@ def test_config3_sampled_users():
     check_forward(w, out, users=sorted(users))
 
 
+def test_config5_forward_sampled_users():
+    """The benchmark's headline batch, 40 users x 100K tokens, in the benchmark's launch:
+    the first, a middle and the last user and two users cut between clusters, against
+    the oracle; unit mass for every user."""
+    w = inputs.make_config(5, with_grad=False)
+    _, out = gpu_forward(w)
+    _unit_mass_all_users(w, out)
+    cut = _boundary_users(w, w.k, w.d)
+    assert len(cut) >= 2, "the batch spans several clusters"
+    check_forward(w, out, users=sorted({0, 19, 39, cut[0], cut[-1]}))
+
+
 @pytest.mark.parametrize("k", [256, 512, 1024, 2048])
 def test_config4_sampled_users(k):
     """The two shortest users, the median, the longest, and the longest user cut between
