@@ -26,7 +26,7 @@ LIB = os.path.join(PKG, "libsa_sketch.so")
 SOURCES = ["sa_host.cu", "sa_prep.cu", "sa_fwd_sm100.cu", "sa_fwd_simt.cu", "sa_bwd_simt.cu",
            "sa_gemm_sm100.cu", "sa_bwd_tc.cu",
            "sa_noalloc.cu", "sa_stca.cu", "sa_codec.cu", "sa_forward_host.cu", "sa_bwd_fused.cu",
-           "sa_stca_keys.cu"]
+           "sa_stca_keys.cu", "sa_stca_keys_bwd.cu"]
 HEADERS = ["sa_common.cuh", "sa_internal.h"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

@@ -255,6 +255,18 @@ __device__ __forceinline__ void tmem_wait_tie(uint32_t (&r)[32]) {
       : "memory");
 }
 
+// Empty asm that carries 32 registers through: a use after it cannot be scheduled before
+// it (pairs with tmem_wait_tie when two tcgen05.ld share one wait).
+__device__ __forceinline__ void tie32(uint32_t (&r)[32]) {
+  asm volatile(""
+               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
+                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
+                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
+                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
+                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
+                 "+r"(r[30]), "+r"(r[31]));
+}
+
 // Shared-memory matrix descriptor for tcgen05 (start, leading and stride byte
 // offsets in 16-byte units; version 1; swizzle mode in bits 61..63).
 enum : uint32_t { kSwizzleNone = 0, kSwizzle128B = 2, kSwizzle32B = 6 };

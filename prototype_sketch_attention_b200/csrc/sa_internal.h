@@ -239,8 +239,6 @@ cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& g, cudaStre
 cudaError_t stca_split_hilo(const float* x, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,
                             cudaStream_t s);
 cudaError_t stca_to_bf16(const float* x, long long n, __nv_bfloat16* y, cudaStream_t s);
-cudaError_t stca_rowdot(const float* a, const float* b, long long n, int d, float* D,
-                        cudaStream_t s);
 cudaError_t stca_weight_grads(const float* dM, const void* Wq, const void* WK, int d, float* dWq,
                               float* dWK, cudaStream_t s);
 cudaError_t gemm_hilo(const WsHeader* hdr, const __nv_bfloat16* hi, const __nv_bfloat16* lo,
@@ -254,8 +252,8 @@ struct StcaKeysPlan {  // workspace layout (byte offsets, 256-aligned)
   int splits = 0;
   size_t hdr = 0, ts = 0, mt = 0, qh = 0, ql = 0, o = 0, lse2 = 0, ohi = 0, olo = 0, total = 0;
   // backward only
-  size_t mts = 0, ghi = 0, glo = 0, gb = 0, do_f = 0, ob = 0, dd = 0, g1 = 0, g1hi = 0,
-         g1lo = 0, part = 0, dm = 0, kpre = 0;
+  size_t mts = 0, ghi = 0, glo = 0, gb = 0, do_f = 0, do_b = 0, ob = 0, dd = 0, g1 = 0,
+         g1hi = 0, g1lo = 0, part = 0, dm = 0;
 };
 size_t stca_keys_plan(int R, long long n_cand, int d, bool backward, int sms, StcaKeysPlan* p);
 struct StcaKeysArgs {
@@ -284,6 +282,28 @@ struct StcaKeysGrads {
 cudaError_t launch_stca_keys_forward(const StcaKeysArgs& a, cudaStream_t s);
 cudaError_t launch_stca_keys_backward(const StcaKeysArgs& a, const StcaKeysGrads& g,
                                       cudaStream_t s);
+// the backward's tcgen05 kernel (sa_stca_keys_bwd.cu): G1 = sum_j dz_cj Kx_j per candidate
+// (written) and dKx += ln 2 (dz^T Q' + (a log2 e)^T dO') per key row (added)
+struct StcaKeysBwdArgs {
+  const __nv_bfloat16* Qh;   // [n_cand, d] Q' hi
+  const __nv_bfloat16* Ql;   // [n_cand, d] Q' lo
+  const __nv_bfloat16* dOb;  // [n_cand, d] dL/dO' in bf16
+  const void* Kx;            // bf16 [n_keys, d]
+  long long n_keys, n_cand;
+  const int64_t* coff;
+  const int64_t* kb;
+  const int64_t* ke;
+  int R, d;
+  const WsHeader* hdr;
+  const long long* tile_start;  // the forward's candidate-tile schedule
+  const float* lse2;         // [n_cand] log2 units
+  const float* Dd;           // [n_cand] dO'_c . O'_c
+  float* G1;                 // [n_cand, d] written
+  float* dKx;                // [n_keys, d] added to (zeroed by the caller)
+};
+cudaError_t launch_stca_keys_bwd_kernel(const StcaKeysBwdArgs& a, cudaStream_t s);
+// 2-D tensor map over bf16 rows [rows, cols]: boxes of 64 columns x 128 rows, 128B swizzle
+bool tmap_rows_bf16(CUtensorMap* m, const void* base, uint64_t rows, int cols);
 // key range of every user = its last min(n_u, L) history rows
 cudaError_t launch_recent_ranges(const int64_t* offsets, int R, int64_t L, int64_t* kb,
                                  int64_t* ke, cudaStream_t s);

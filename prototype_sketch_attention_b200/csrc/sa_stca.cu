@@ -321,12 +321,6 @@ cudaError_t stca_to_bf16(const float* x, long long n, __nv_bfloat16* y, cudaStre
   return cudaGetLastError();
 }
 
-cudaError_t stca_rowdot(const float* a, const float* b, long long n, int d, float* D,
-                        cudaStream_t s) {
-  stca_rowdot_kernel<<<1024, 256, 0, s>>>(a, b, n, d, D);
-  return cudaGetLastError();
-}
-
 cudaError_t stca_weight_grads(const float* dM, const void* Wq, const void* WK, int d, float* dWq,
                               float* dWK, cudaStream_t s) {
   stca_weight_grads_kernel<<<d, 128, 0, s>>>(dM, static_cast<const __nv_bfloat16*>(Wq),

@@ -26,6 +26,10 @@
 // Roles: warp 0 TMA, warp 1 TMEM allocation and the MMAs, warps 4-7 and 8-11 the softmax
 // warpgroups (warpgroup 0 also merges and writes the output). Every mbarrier wait is
 // bounded.
+//
+// The backward (launch_stca_keys_backward) recomputes this forward, forms dO' = G W_V^T and
+// dW_V = O'^T G on the tcgen05 GEMM, then runs its own tcgen05 kernel (sa_stca_keys_bwd.cu)
+// for G1 = dL/dQn and dKx, and finishes dQ, dW_q and dW_K with GEMMs.
 #include <cuda.h>
 
 #include <algorithm>
@@ -67,17 +71,6 @@ struct KBars {
   uint64_t merge, drain;
   uint32_t tmem_base;
 };
-
-// Empty asm that carries the registers through: uses after it cannot move above it.
-__device__ __forceinline__ void tie32(uint32_t (&r)[32]) {
-  asm volatile(""
-               : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]),
-                 "+r"(r[6]), "+r"(r[7]), "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]),
-                 "+r"(r[12]), "+r"(r[13]), "+r"(r[14]), "+r"(r[15]), "+r"(r[16]), "+r"(r[17]),
-                 "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]), "+r"(r[22]), "+r"(r[23]),
-                 "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]), "+r"(r[29]),
-                 "+r"(r[30]), "+r"(r[31]));
-}
 
 // 64 consecutive TMEM columns of this warp's 32 lanes: two loads, one wait.
 __device__ __forceinline__ void tmem_ld64(uint32_t taddr, uint32_t (&a)[32], uint32_t (&b)[32]) {
@@ -431,6 +424,21 @@ __global__ void keys_qfold_kernel(const __nv_bfloat16* __restrict__ Q, const flo
   }
 }
 
+// D_c = sum_e bf16(dO'_ce) O'_ce, one warp per candidate.
+__global__ void keys_rowdot_kernel(const __nv_bfloat16* __restrict__ dOb, const float* __restrict__ O,
+                                   long long n, int d, float* __restrict__ D) {
+  const int lane = threadIdx.x & 31;
+  const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
+  for (long long c = w0; c < n; c += nw) {
+    float acc = 0.f;
+    for (int e = lane; e < d; e += 32) acc = fmaf(__bfloat162float(dOb[c * d + e]), O[c * d + e], acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) D[c] = acc;
+  }
+}
+
 // Validates the key ranges: 0 <= kb[u] <= ke[u] <= n_keys (else SA_ERR_BAD_OFFSETS).
 __global__ void check_ranges_kernel(const int64_t* __restrict__ kb, const int64_t* __restrict__ ke,
                                     int R, long long n_keys, WsHeader* hdr) {
@@ -448,189 +456,6 @@ __global__ void recent_ranges_kernel(const int64_t* __restrict__ off, int R, lon
   }
 }
 
-// kpre[u] = sum over users before u of their key counts (kpre[R] = all pairs): one block,
-// each thread scans a contiguous chunk of users.
-__global__ void __launch_bounds__(1024) key_prefix_kernel(const int64_t* __restrict__ kb,
-                                                          const int64_t* __restrict__ ke, int R,
-                                                          long long* __restrict__ kpre) {
-  __shared__ long long part[1024];
-  const int t = threadIdx.x;
-  const int chunk = (R + 1023) / 1024;
-  const int a = min(R, t * chunk), b = min(R, a + chunk);
-  long long sum = 0;
-  for (int u = a; u < b; ++u) sum += max(ke[u] - kb[u], (int64_t)0);
-  part[t] = sum;
-  __syncthreads();
-  for (int o = 1; o < 1024; o <<= 1) {  // inclusive scan over the 1024 chunk sums
-    const long long v = t >= o ? part[t - o] : 0;
-    __syncthreads();
-    part[t] += v;
-    __syncthreads();
-  }
-  long long run = part[t] - sum;
-  for (int u = a; u < b; ++u) {
-    kpre[u] = run;
-    run += max(ke[u] - kb[u], (int64_t)0);
-  }
-  if (t == 1023) kpre[R] = part[1023];
-}
-
-// largest u with pre[u] <= x, for a non-decreasing pre[0..R] with pre[0] <= x < pre[R]
-__device__ __forceinline__ int segment_of(const long long* pre, int R, long long x) {
-  int lo = 0, hi = R;
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pre[mid] <= x) lo = mid; else hi = mid;
-  }
-  return lo;
-}
-
-template <int E>
-__device__ __forceinline__ void load_bf16(const __nv_bfloat16* p, float (&v)[E]) {
-  if constexpr (E == 4) {
-    const uint2 w = *reinterpret_cast<const uint2*>(p);
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&w.x);
-    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&w.y);
-    v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
-  } else {
-    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(p);
-    v[0] = __low2float(a); v[1] = __high2float(a);
-  }
-}
-
-// Q' = hi + lo
-template <int E>
-__device__ __forceinline__ void load_q(const __nv_bfloat16* hi, const __nv_bfloat16* lo,
-                                       long long i, float (&v)[E]) {
-  float a[E], b[E];
-  load_bf16<E>(hi + i, a);
-  load_bf16<E>(lo + i, b);
-#pragma unroll
-  for (int e = 0; e < E; ++e) v[e] = a[e] + b[e];
-}
-
-template <int E>
-__device__ __forceinline__ void load_f32(const float* p, float (&v)[E]) {
-  if constexpr (E == 4) {
-    const float4 w = *reinterpret_cast<const float4*>(p);
-    v[0] = w.x; v[1] = w.y; v[2] = w.z; v[3] = w.w;
-  } else {
-    const float2 w = *reinterpret_cast<const float2*>(p);
-    v[0] = w.x; v[1] = w.y;
-  }
-}
-
-// Sums two per-lane partial dot products over the warp (every lane gets both totals).
-__device__ __forceinline__ void warp_sum2(float& x, float& y) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) {
-    x += __shfl_xor_sync(0xffffffffu, x, o);
-    y += __shfl_xor_sync(0xffffffffu, y, o);
-  }
-}
-
-// Backward, candidate side (CUDA cores, one warp per candidate c of user u):
-//   a_cj = 2^(Q'_c . Kx_j - lse2_c),  dz_cj = a_cj (dO_c . Kx_j - D_c),  G1_c = sum_j dz_cj Kx_j
-// over the user's key rows j; lane l holds elements [l E, l E + E) of each row.
-template <int D>
-__global__ void keys_bwd_g1_kernel(const __nv_bfloat16* __restrict__ Qh,
-                                   const __nv_bfloat16* __restrict__ Ql, const float* __restrict__ dO,
-                                   const float* __restrict__ lse2, const float* __restrict__ Dd,
-                                   const int64_t* __restrict__ coff, int R,
-                                   const __nv_bfloat16* __restrict__ Kx, const int64_t* __restrict__ kb,
-                                   const int64_t* __restrict__ ke, long long n_cand,
-                                   float* __restrict__ G1, const WsHeader* hdr) {
-  constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  if (__any_sync(0xffffffffu, read_status(&hdr->status) != 0)) return;
-  const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long c = w0; c < n_cand; c += nw) {
-    const int u = segment_of(reinterpret_cast<const long long*>(coff), R, c);
-    const long long j0 = kb[u], j1 = ke[u];
-    float q[E], o[E], g[E];
-    load_q<E>(Qh, Ql, c * D + lane * E, q);
-    load_f32<E>(dO + c * D + lane * E, o);
-    const float l2 = lse2[c], dc = Dd[c];
-#pragma unroll
-    for (int e = 0; e < E; ++e) g[e] = 0.f;
-    for (long long j = j0; j < j1; ++j) {
-      float k[E];
-      load_bf16<E>(Kx + j * D + lane * E, k);
-      float z = 0.f, p = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        z = fmaf(q[e], k[e], z);
-        p = fmaf(o[e], k[e], p);
-      }
-      warp_sum2(z, p);
-      const float dz = ex2_approx(z - l2) * (p - dc);
-#pragma unroll
-      for (int e = 0; e < E; ++e) g[e] = fmaf(dz, k[e], g[e]);
-    }
-    float* gp = G1 + c * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) gp[e] = g[e];
-  }
-}
-
-// Backward, key side (CUDA cores, one warp per (user, key row) pair):
-//   dKx_j += sum over the user's candidates c of dz_cj Qn_c + a_cj dO_c,  Qn = Q' ln 2,
-// added into dKx (zeroed before), so rows shared by several users' ranges sum.
-template <int D>
-__global__ void keys_bwd_dk_kernel(const __nv_bfloat16* __restrict__ Qh,
-                                   const __nv_bfloat16* __restrict__ Ql, const float* __restrict__ dO,
-                                   const float* __restrict__ lse2, const float* __restrict__ Dd,
-                                   const int64_t* __restrict__ coff, int R,
-                                   const __nv_bfloat16* __restrict__ Kx, const int64_t* __restrict__ kb,
-                                   const long long* __restrict__ kpre, float* __restrict__ dKx,
-                                   const WsHeader* hdr) {
-  constexpr int E = D / 32;
-  const int lane = threadIdx.x & 31;
-  if (__any_sync(0xffffffffu, read_status(&hdr->status) != 0)) return;
-  const long long total = kpre[R];
-  const long long w0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const long long nw = ((long long)gridDim.x * blockDim.x) >> 5;
-  for (long long v = w0; v < total; v += nw) {
-    const int u = segment_of(kpre, R, v);
-    const long long j = kb[u] + (v - kpre[u]);
-    float k[E], acc[E];
-    load_bf16<E>(Kx + j * D + lane * E, k);
-#pragma unroll
-    for (int e = 0; e < E; ++e) acc[e] = 0.f;
-    for (long long c = coff[u]; c < coff[u + 1]; ++c) {
-      float q[E], o[E];
-      load_q<E>(Qh, Ql, c * D + lane * E, q);
-      load_f32<E>(dO + c * D + lane * E, o);
-      float z = 0.f, p = 0.f;
-#pragma unroll
-      for (int e = 0; e < E; ++e) {
-        z = fmaf(q[e], k[e], z);
-        p = fmaf(o[e], k[e], p);
-      }
-      warp_sum2(z, p);
-      const float a = ex2_approx(z - lse2[c]);
-      const float dzl = a * (p - Dd[c]) * kLn2;
-#pragma unroll
-      for (int e = 0; e < E; ++e) acc[e] = fmaf(dzl, q[e], fmaf(a, o[e], acc[e]));
-    }
-    float* dp = dKx + j * D + lane * E;
-#pragma unroll
-    for (int e = 0; e < E; ++e) atomicAdd(dp + e, acc[e]);
-  }
-}
-
-bool map_rows_bf16(CUtensorMap* m, const void* base, uint64_t rows, int cols) {
-  auto fn = tmap_encode_fn();
-  if (!fn) return false;
-  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
-  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
-  const cuuint32_t box[2] = {64, 128};
-  const cuuint32_t estr[2] = {1, 1};
-  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
-            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
 
 GemmOperandDesc opk(const void* base, uint64_t rows, uint64_t cols, bool mn_major) {
   GemmOperandDesc o;
@@ -677,8 +502,8 @@ cudaError_t keys_core(const StcaKeysArgs& a, float* lse, bool fwd_call, cudaStre
       static_cast<const __nv_bfloat16*>(a.Q), M, n, d, kLog2e / std::sqrt((float)d), Qh, Ql);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   CUtensorMap tqh, tql, tk;
-  if (!map_rows_bf16(&tqh, Qh, (uint64_t)n, d) || !map_rows_bf16(&tql, Ql, (uint64_t)n, d) ||
-      !map_rows_bf16(&tk, a.Kx, (uint64_t)a.n_keys, d))
+  if (!tmap_rows_bf16(&tqh, Qh, (uint64_t)n, d) || !tmap_rows_bf16(&tql, Ql, (uint64_t)n, d) ||
+      !tmap_rows_bf16(&tk, a.Kx, (uint64_t)a.n_keys, d))
     return cudaErrorInvalidValue;
   const long long grid = n / 128 + a.R + 1;  // bounds the candidate tiles; the rest exit
   if (fwd_call && (e = prof_mark_start(s)) != cudaSuccess) return e;
@@ -702,6 +527,19 @@ cudaError_t keys_core(const StcaKeysArgs& a, float* lse, bool fwd_call, cudaStre
 }
 
 }  // namespace
+
+// 2-D tensor map over bf16 rows [rows, cols]: boxes of 64 columns x 128 rows, 128B swizzle.
+bool tmap_rows_bf16(CUtensorMap* m, const void* base, uint64_t rows, int cols) {
+  auto fn = tmap_encode_fn();
+  if (!fn) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)cols * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box,
+            estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
 
 size_t stca_keys_plan(int R, long long n_cand, int d, bool backward, int sms, StcaKeysPlan* p) {
   StcaKeysPlan q;
@@ -731,6 +569,7 @@ size_t stca_keys_plan(int R, long long n_cand, int d, bool backward, int sms, St
     q.glo = take(nd * 2);
     q.gb = take(nd * 2);
     q.do_f = take(nd * sizeof(float));
+    q.do_b = take(nd * 2);
     q.ob = take(nd * 2);
     q.dd = take(n * sizeof(float));
     q.g1 = take(nd * sizeof(float));
@@ -738,7 +577,6 @@ size_t stca_keys_plan(int R, long long n_cand, int d, bool backward, int sms, St
     q.g1lo = take(nd * 2);
     q.part = take((size_t)q.splits * d * d * sizeof(float));
     q.dm = take((size_t)d * d * sizeof(float));
-    q.kpre = take((size_t)(R + 1) * sizeof(long long));
   }
   q.total = o;
   *p = q;
@@ -793,34 +631,30 @@ cudaError_t launch_stca_keys_backward(const StcaKeysArgs& a, const StcaKeysGrads
   if ((e = gemm_tn_sum(hdr, bf(p.ob), bf(p.gb), n, d, p.splits, f32(p.part), 1.0f, gr.dWV, s)) !=
       cudaSuccess)
     return e;
-  // D_c = dO'_c . O'_c
-  if ((e = stca_rowdot(f32(p.do_f), O, n, d, f32(p.dd), s)) != cudaSuccess) return e;
-  const __nv_bfloat16* Qh = bf(p.qh);
-  const __nv_bfloat16* Ql = bf(p.ql);
-  const __nv_bfloat16* Kx = static_cast<const __nv_bfloat16*>(a.Kx);
-  if (a.n_keys > 0) {
-    if (R > 0) {
-      key_prefix_kernel<<<1, 1024, 0, s>>>(a.kb, a.ke, R, at<long long>(ws, p.kpre));
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-    const unsigned gq = (unsigned)std::min<long long>((n + 7) / 8, 148LL * 64);
-    const unsigned gk = (unsigned)std::min<long long>((a.n_keys + 7) / 8, 148LL * 64);
-    if (d == 64) {
-      keys_bwd_g1_kernel<64><<<gq, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd), a.coff, R,
-                                                Kx, a.kb, a.ke, n, f32(p.g1), hdr);
-      if (R > 0)
-        keys_bwd_dk_kernel<64><<<gk, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd), a.coff,
-                                                  R, Kx, a.kb, at<long long>(ws, p.kpre), gr.dKx,
-                                                  hdr);
-    } else {
-      keys_bwd_g1_kernel<128><<<gq, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd), a.coff,
-                                                 R, Kx, a.kb, a.ke, n, f32(p.g1), hdr);
-      if (R > 0)
-        keys_bwd_dk_kernel<128><<<gk, 256, 0, s>>>(Qh, Ql, f32(p.do_f), f32(p.lse2), f32(p.dd),
-                                                   a.coff, R, Kx, a.kb, at<long long>(ws, p.kpre),
-                                                   gr.dKx, hdr);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // dO' in bf16 (the MMAs' operand) and D_c = bf16(dO'_c) . O'_c, consistent with it
+  if ((e = stca_to_bf16(f32(p.do_f), n * d, bf(p.do_b), s)) != cudaSuccess) return e;
+  keys_rowdot_kernel<<<1024, 256, 0, s>>>(bf(p.do_b), O, n, d, f32(p.dd));
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (a.n_keys > 0) {  // G1 and dKx on the tensor cores
+    StcaKeysBwdArgs k;
+    k.Qh = bf(p.qh);
+    k.Ql = bf(p.ql);
+    k.dOb = bf(p.do_b);
+    k.Kx = a.Kx;
+    k.n_keys = a.n_keys;
+    k.n_cand = n;
+    k.coff = a.coff;
+    k.kb = a.kb;
+    k.ke = a.ke;
+    k.R = R;
+    k.d = d;
+    k.hdr = hdr;
+    k.tile_start = at<long long>(ws, p.ts);
+    k.lse2 = f32(p.lse2);
+    k.Dd = f32(p.dd);
+    k.G1 = f32(p.g1);
+    k.dKx = gr.dKx;
+    if ((e = launch_stca_keys_bwd_kernel(k, s)) != cudaSuccess) return e;
   } else if ((e = cudaMemsetAsync(f32(p.g1), 0, (size_t)n * d * sizeof(float), s)) != cudaSuccess) {
     return e;
   }
