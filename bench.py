@@ -358,21 +358,30 @@ def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> di
             raise RuntimeError(binding.sa_status_string(st))
         fwd_ms = sum(e4[0].elapsed_time(e4[1]) for e4 in ev) / steps
         kern_ms = sum(event_ms(e4[2], e4[3]) for e4 in ev) / steps
-        nb = 3
-        b0, b1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        nb = 5
+        bev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
+        for e4 in bev:
+            for e in e4:
+                e.record(stream)
         binding.stca_keys_backward(Q, coff, X, kb, ke, Wq, WK, WV, G, ws=g["_ws"])
         torch.cuda.synchronize()
-        b0.record(stream)
-        for _ in range(nb):
+        for e4 in bev:
+            flush.zero_()
+            e4[0].record(stream)
+            binding.sa_sketch_profile_events(e4[2].cuda_event, e4[3].cuda_event)
             binding.stca_keys_backward(Q, coff, X, kb, ke, Wq, WK, WV, G, ws=g["_ws"])
-        b1.record(stream)
+            e4[1].record(stream)
         torch.cuda.synchronize()
+        binding.sa_sketch_profile_events(None, None)
         st = binding.device_status(g["_ws"])
         if st != 0:
             raise RuntimeError(binding.sa_status_string(st))
-        bwd_ms = b0.elapsed_time(b1) / nb
+        bwd_ms = sum(e4[0].elapsed_time(e4[1]) for e4 in bev) / nb
+        bwd_kern_ms = sum(event_ms(e4[2], e4[3]) for e4 in bev) / nb
         flop = 4.0 * d * pairs  # scores and weighted sum, per (candidate, key) pair
         achieved = flop / (kern_ms / 1e3) / 1e12
+        bflop = 10.0 * d * pairs  # scores, dP, G1 and dKx (two terms), per pair
+        bachieved = bflop / (bwd_kern_ms / 1e3) / 1e12
         return {"workload": f"{R} users x {RECENT_CANDIDATES} candidates over the last "
                             f"{RECENT_L} of {X.shape[0] // R} history rows each, d={d}",
                 "pairs": pairs, "forward_ms": fwd_ms, "pairs_per_s": pairs / (fwd_ms / 1e3),
@@ -380,10 +389,13 @@ def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> di
                 "kernel_tflops": achieved, "kernel_frac": achieved / peak,
                 "flop_per_pair": 4 * d,
                 "tensor_flop_per_pair": 6 * d,  # the score MMA runs twice (Q' hi and lo)
-                "backward_ms": bwd_ms,
-                "note": "forward: M and Q' folds, flash kernel, O' split, O' W_V GEMM; "
-                        "the backward recomputes the forward, score gradients on CUDA cores",
-                "l2": "256 MB flush between forward steps"}
+                "backward_ms": bwd_ms, "backward_kernel": "stca_keys_bwd_kernel<128>",
+                "backward_kernel_ms": bwd_kern_ms, "backward_kernel_tflops": bachieved,
+                "backward_kernel_frac": bachieved / peak, "backward_flop_per_pair": 10 * d,
+                "note": "forward: M and Q' folds, flash kernel, O' split, O' W_V GEMM; the "
+                        "backward recomputes the forward, then dO' and dW_V GEMMs, the tcgen05 "
+                        "kernel (G1, dKx), dQ and the weight gradients",
+                "l2": "256 MB flush between steps"}
     except Exception as e:  # reported beside the headline, never fatal to it
         binding.sa_sketch_profile_events(None, None)
         return {"error": repr(e)[:300]}
@@ -439,7 +451,7 @@ def time_sketch_branch(binding, dev, sketch, peak: float, hbm_gbs: float, steps:
             "forward_ms": fwd_ms, "forward_tflops": flop / (fwd_ms / 1e3) / 1e12,
             "forward_frac": flop / (fwd_ms / 1e3) / 1e12 / peak,
             "backward_ms": bwd_ms,
-            "note": "composed from the tcgen05 GEMM: Q' fold, lse, weights, O = A S, O W_V; "
+            "note": "the recent branch's kernels with the bf16 sketch rows as the keys; "
                     "4kd FLOP per candidate; one sketch read per user",
             "l2": "256 MB flush before every timed call"}
     except Exception as e:

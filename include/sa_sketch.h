@@ -272,8 +272,9 @@ int sa_sketch_get_device_status(const void* workspace, void* stream);
  * Measurement hook. When both handles are non-null, every later sa_sketch_forward
  * call made by this host thread records `start_event` on its stream just before the
  * main forward kernel (the tcgen05 kernel for bf16, the SIMT kernels for fp32) and
- * `stop_event` just after it; sa_stca_keys_forward calls likewise around their flash
- * kernel. The caller then reads that kernel's own duration with
+ * `stop_event` just after it; the cross-attention calls likewise around their main
+ * kernel (the flash kernel for sa_stca_forward and sa_stca_keys_forward, the tcgen05
+ * backward kernel for sa_stca_backward and sa_stca_keys_backward). The caller then reads that kernel's own duration with
  * cudaEventElapsedTime. Both handles are cudaEvent_t passed as void*; the caller owns
  * them. Passing two nulls turns the hook off. Returns SA_OK, or SA_ERR_INVALID_ARG if
  * exactly one handle is null.
@@ -312,16 +313,16 @@ int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M
  *   lse          [n_cand]     fp32, device   output, nullable
  * d in {64, 128}; 1 <= k <= SA_MAX_K; n_cand <= INT32_MAX; pointers 16-byte aligned.
  * A user without candidates reads nothing. R k_pad <= INT32_MAX (k_pad = k rounded up to
- * a multiple of 128). The forward runs sa_stca_keys_forward's flash kernel with the
- * bf16 sketch as the key rows. Precision: Q Wq WK^T / sqrt(d) is formed in fp32 and
- * enters the tensor cores as a bf16 pair hi + lo; the sketch and the attention weights
- * enter as bf16; accumulation is fp32. The backward (below) computes with Q Wq WK^T in
- * bf16 and forms the weights over the k rows in bf16 (2 k bytes per candidate).
+ * a multiple of 128). Both directions run sa_stca_keys_forward's and
+ * sa_stca_keys_backward's kernels with the bf16 sketch as the key rows. Precision:
+ * Q Wq WK^T / sqrt(d) is formed in fp32 and enters the tensor cores as a bf16 pair
+ * hi + lo; the sketch and the attention weights (and in the backward their gradients)
+ * enter as bf16; accumulation is fp32.
  * The workspace (sa_stca_workspace_size bytes, 256-aligned, caller-owned) holds the bf16
- * sketch and, per candidate, Q Wq WK^T and the unprojected output (forward) or the
- * weights and their gradients (backward); errors follow sa_sketch_forward's
- * conventions, and the device status word in the workspace is read with
- * sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
+ * sketch (2 k_pad d bytes per user), per candidate Q Wq WK^T and the unprojected output,
+ * and for the backward the gradient over the padded sketch rows; errors follow
+ * sa_sketch_forward's conventions, and the device status word in the workspace is read
+ * with sa_sketch_get_device_status. Enqueues on `stream`, never synchronises.
  */
 size_t sa_stca_workspace_size(int R, int64_t n_cand, int k, int d, int backward);
 int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand, int d,
@@ -336,10 +337,9 @@ int sa_stca_forward(const void* Q, const int64_t* cand_offsets, int R, int64_t n
  *                                   sketch (Sketch Attention's dsketch); zero for users
  *                                   without candidates
  *   dWq, dWK, dWV [d, d] fp32, device, summed over users
- * All outputs are overwritten. cand_offsets_host is a HOST copy of cand_offsets (the
- * per-user gradient of the sketch is one GEMM per user, sized on the host); it is
- * checked before anything is launched (SA_ERR_BAD_OFFSETS). The forward is recomputed
- * inside. Workspace: sa_stca_workspace_size(..., backward = 1) bytes. Other arguments,
+ * All outputs are overwritten. cand_offsets_host is a HOST copy of cand_offsets; it is
+ * checked on the host before anything is launched (SA_ERR_BAD_OFFSETS). The forward is
+ * recomputed inside. Workspace: sa_stca_workspace_size(..., backward = 1) bytes. Other arguments,
  * precision and conventions as for sa_stca_forward.
  */
 int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* cand_offsets_host,

@@ -421,13 +421,12 @@ int sa_stca_backward(const void* Q, const int64_t* cand_offsets, const int64_t* 
   a.workspace = workspace;
   StcaGrads g;
   g.dout = dout;
-  g.coff_host = cand_offsets_host;
   g.dQ = dQ;
   g.dS = dS;
   g.dWq = dWq;
   g.dWK = dWK;
   g.dWV = dWV;
-  return cuda_status(launch_stca_backward(a, g, static_cast<cudaStream_t>(stream_)));
+  return cuda_status(launch_stca_backward(a, g, dev.sms, static_cast<cudaStream_t>(stream_)));
 }
 
 namespace {

@@ -199,16 +199,11 @@ struct GemmArgs {
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 
 // ---- candidate-to-sketch cross attention (sa_stca.cu)
-struct StcaPlan {  // workspace layout (byte offsets, 256-aligned)
-  int k_pad = 0, nparts = 0, splits = 0;
-  size_t hdr = 0, ts = 0, sb = 0, mt = 0, qp = 0, dpart = 0, lse2 = 0, ab = 0, o = 0, ohi = 0,
-         olo = 0, total = 0;
-  // forward: the ragged-key attention's workspace first (its header is the status word),
-  // then the bf16 sketch and every user's row range within it
-  size_t kb = 0, ke = 0;
-  // backward only
-  size_t mts = 0, qn = 0, do_f = 0, do_b = 0, dd = 0, czero = 0, dz = 0, g1 = 0, g1hi = 0,
-         g1lo = 0, gb = 0, ob = 0, ghi = 0, glo = 0, part = 0, dm = 0;
+struct StcaPlan {  // workspace layout (byte offsets, 256-aligned): the ragged-key
+                   // attention's workspace first (its header is the status word), then the
+                   // bf16 sketch, every user's row range within it and (backward) dKx
+  int k_pad = 0;
+  size_t hdr = 0, sb = 0, kb = 0, ke = 0, dkx = 0, total = 0;
 };
 size_t stca_plan(int R, long long n_cand, int k, int d, bool backward, int sms, StcaPlan* p);
 struct StcaArgs {
@@ -228,12 +223,11 @@ struct StcaArgs {
 cudaError_t launch_stca_forward(const StcaArgs& a, cudaStream_t s);
 struct StcaGrads {
   const float* dout;          // [n_cand, d]
-  const int64_t* coff_host;   // [R + 1], host copy of the candidate offsets
   float* dQ;                  // [n_cand, d]
   float* dS;                  // [R, k, d]
   float *dWq, *dWK, *dWV;     // [d, d]
 };
-cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& g, cudaStream_t s);
+cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& g, int sms, cudaStream_t s);
 
 // shared pieces of the cross attention (sa_stca.cu)
 cudaError_t stca_split_hilo(const float* x, long long n, __nv_bfloat16* hi, __nv_bfloat16* lo,

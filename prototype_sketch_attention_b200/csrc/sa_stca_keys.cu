@@ -654,7 +654,9 @@ cudaError_t launch_stca_keys_backward(const StcaKeysArgs& a, const StcaKeysGrads
     k.Dd = f32(p.dd);
     k.G1 = f32(p.g1);
     k.dKx = gr.dKx;
+    if ((e = prof_mark_start(s)) != cudaSuccess) return e;
     if ((e = launch_stca_keys_bwd_kernel(k, s)) != cudaSuccess) return e;
+    if ((e = prof_mark_stop(s)) != cudaSuccess) return e;
   } else if ((e = cudaMemsetAsync(f32(p.g1), 0, (size_t)n * d * sizeof(float), s)) != cudaSuccess) {
     return e;
   }

@@ -95,58 +95,56 @@ def test_composition_model_catches_a_swapped_fold():
     assert err > 5e-2, err
 
 
-def model_backward(cw, G):
-    """The backward's launch sequence in sa_stca.cu, step by step, with its roundings."""
+def model_backward(cw, G, ln2=math.log(2.0)):
+    """The backward: the sketch as the key rows of sa_stca_keys.cu's backward (the forward
+    recomputed, dO' and dW_V on the GEMM, the tcgen05 kernel's G1 and dKx = dS, then dQ,
+    dW_q, dW_K), step by step with its roundings."""
     Q = cw.Q.float().numpy().astype(np.float64)
     S = cw.S.numpy().astype(np.float64)
     Wq, WK, WV = (t.float().numpy().astype(np.float64) for t in (cw.Wq, cw.WK, cw.WV))
     R, k, d = S.shape
-    k_pad = (k + 127) // 128 * 128
     coff = cw.cand_offsets.numpy()
     n = Q.shape[0]
     isd = 1.0 / math.sqrt(d)
-    Sb = np.zeros((R, k_pad, d))
-    Sb[:, :k] = bf16(S)
-    Mt = fold(WK, Wq, 1.0, True)
-    Qp = fold(Q, Mt, math.log2(math.e) * isd, True)
-    A = np.zeros((n, k_pad))
+    log2e = math.log2(math.e)
+    Sb = bf16(S)
+    M = fold(Wq, WK, 1.0, False)
+    Qp = fold(Q, M.T, log2e * isd, False)
+    hq = bf16(Qp)
+    lq = bf16(Qp - hq)
     O = np.zeros((n, d))
-    for u in range(R):
+    lse2 = np.zeros(n)
+    for u in range(R):                                         # the forward, recomputed
         a, b = int(coff[u]), int(coff[u + 1])
         if a == b:
             continue
-        z = Qp[a:b] @ Sb[u].T
-        z[:, k:] = -np.inf
+        z = (hq[a:b] + lq[a:b]) @ Sb[u].T
         m = z.max(axis=1, keepdims=True)
-        lse2 = m + np.log2(np.exp2(z - m).sum(axis=1, keepdims=True))
-        A[a:b] = bf16(np.exp2(z - lse2))
-        O[a:b] = (A[a:b] @ Sb[u]).astype(np.float32)
+        e = np.exp2(z - m)
+        l = e.sum(axis=1, keepdims=True)
+        O[a:b] = (bf16(e) @ Sb[u] / l).astype(np.float32)
+        lse2[a:b] = m[:, 0] + np.log2(l[:, 0])
     Gh, Gl = bf16(G), bf16(G - bf16(G))
     dO = (Gh @ bf16(WV).T + Gl @ bf16(WV).T).astype(np.float32).astype(np.float64)
     dWV = bf16(O).T @ bf16(G)
-    D = (dO * O).sum(axis=1)
     dOb = bf16(dO)
-    dZ = np.zeros((n, k_pad))
+    D = (dOb * O).sum(axis=1)                                  # keys_rowdot_kernel
     G1 = np.zeros((n, d))
-    for u in range(R):
+    dS = np.zeros((R, k, d))
+    for u in range(R):                                         # stca_keys_bwd_kernel
         a, b = int(coff[u]), int(coff[u + 1])
         if a == b:
             continue
-        dZ[a:b] = bf16(A[a:b] * (dOb[a:b] @ Sb[u].T - D[a:b, None]))
-        G1[a:b] = (dZ[a:b] @ Sb[u]).astype(np.float32)
+        A = np.exp2((hq[a:b] + lq[a:b]) @ Sb[u].T - lse2[a:b, None])
+        dz = A * (dOb[a:b] @ Sb[u].T - D[a:b, None])
+        G1[a:b] = (bf16(dz) @ Sb[u]).astype(np.float32)
+        dS[u] = ln2 * (bf16(dz).T @ hq[a:b] + bf16(A * log2e).T @ dOb[a:b])
     Mts = fold(WK, Wq, isd, True)
     G1h, G1l = bf16(G1), bf16(G1 - bf16(G1))
     dQ = G1h @ Mts + G1l @ Mts
     dM = isd * (Q.T @ bf16(G1))
     dWq = dM @ WK
     dWK = dM.T @ Wq
-    Qn = fold(Q, Mt, isd, True)
-    dS = np.zeros((R, k, d))
-    for u in range(R):
-        a, b = int(coff[u]), int(coff[u + 1])
-        if a == b:
-            continue
-        dS[u] = (dZ[a:b].T @ Qn[a:b] + A[a:b].T @ dOb[a:b])[:k]
     return {"dQ": dQ, "dS": dS, "dWq": dWq, "dWK": dWK, "dWV": dWV}
 
 
@@ -162,3 +160,15 @@ def test_backward_composition_model_meets_the_oracle(counts, k, d):
         e = np.linalg.norm(got[key] - r) / max(np.linalg.norm(r), 1e-30)
         assert e <= 1e-2, (key, e)
         assert np.abs(got[key] - r).max() <= 5e-2 * max(np.abs(r).max(), 1e-30), (key, "max-abs")
+
+
+def test_backward_model_catches_a_missing_ln2():
+    """The backward check has teeth: dKx = dS without the ln 2 that turns the log2-unit
+    Q' back into natural units fails it."""
+    cw = inputs.make_cross_workload([40, 9], 256, 64, seed=602)
+    G = np.random.default_rng(603).standard_normal((49, 64))
+    got = model_backward(cw, G, ln2=1.0)
+    f = cw.to_f64()
+    ref = oracle.stca_backward(f["Q"], f["cand_offsets"], f["S"], f["Wq"], f["WK"], f["WV"], G)
+    err = np.linalg.norm(got["dS"] - ref["dS"]) / np.linalg.norm(ref["dS"])
+    assert err > 5e-2, err
