@@ -378,6 +378,20 @@ def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> di
             raise RuntimeError(binding.sa_status_string(st))
         bwd_ms = sum(e4[0].elapsed_time(e4[1]) for e4 in bev) / nb
         bwd_kern_ms = sum(event_ms(e4[2], e4[3]) for e4 in bev) / nb
+        # the same backward adding into an existing history gradient (no zeroing of X's rows)
+        dX = torch.zeros(X.shape, dtype=torch.float32, device=dev)
+        binding.stca_keys_backward(Q, coff, X, kb, ke, Wq, WK, WV, G, dKx=dX, ws=g["_ws"])
+        aev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(nb)]
+        torch.cuda.synchronize()
+        for a0, a1 in aev:
+            flush.zero_()
+            a0.record(stream)
+            binding.stca_keys_backward(Q, coff, X, kb, ke, Wq, WK, WV, G, dKx=dX, ws=g["_ws"])
+            a1.record(stream)
+        torch.cuda.synchronize()
+        acc_ms = sum(a0.elapsed_time(a1) for a0, a1 in aev) / nb
+        del dX
         flop = 4.0 * d * pairs  # scores and weighted sum, per (candidate, key) pair
         achieved = flop / (kern_ms / 1e3) / 1e12
         bflop = 10.0 * d * pairs  # scores, dP, G1 and dKx (two terms), per pair
@@ -389,7 +403,8 @@ def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> di
                 "kernel_tflops": achieved, "kernel_frac": achieved / peak,
                 "flop_per_pair": 4 * d,
                 "tensor_flop_per_pair": 6 * d,  # the score MMA runs twice (Q' hi and lo)
-                "backward_ms": bwd_ms, "backward_kernel": "stca_keys_bwd_kernel<128>",
+                "backward_ms": bwd_ms, "backward_accumulate_ms": acc_ms,
+                "backward_kernel": "stca_keys_bwd_kernel<128>",
                 "backward_kernel_ms": bwd_kern_ms, "backward_kernel_tflops": bachieved,
                 "backward_kernel_frac": bachieved / peak, "backward_flop_per_pair": 10 * d,
                 "note": "forward: M and Q' folds, flash kernel, O' split, O' W_V GEMM; the "

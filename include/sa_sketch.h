@@ -392,15 +392,18 @@ int sa_stca_keys_forward(const void* Q, const int64_t* cand_offsets, int R, int6
  *                                   into the history rows; 0 on rows no range covers, a
  *                                   sum over users on rows several ranges cover
  *   dWq, dWK, dWV [d, d] fp32, device, summed over users
- * All outputs are overwritten. The forward is recomputed inside. Workspace:
+ * All outputs are overwritten, except dKx when accumulate is non-zero: then the
+ * gradient is added into the caller's dKx (for the recent branch, straight into the
+ * history gradient that sa_sketch_backward wrote, without zeroing n_keys x d floats
+ * first). The forward is recomputed inside. Workspace:
  * sa_stca_keys_workspace_size(..., backward = 1) bytes. Other arguments, precision and
  * conventions as for sa_stca_keys_forward.
  */
 int sa_stca_keys_backward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand,
                           int d, const void* Kx, int64_t n_keys, const int64_t* key_begin,
                           const int64_t* key_end, const void* Wq, const void* WK, const void* WV,
-                          const float* dout, float* dQ, float* dKx, float* dWq, float* dWK,
-                          float* dWV, void* workspace, size_t ws_bytes, void* stream);
+                          const float* dout, float* dQ, float* dKx, int accumulate, float* dWq,
+                          float* dWK, float* dWV, void* workspace, size_t ws_bytes, void* stream);
 
 /*
  * The recent branch's key ranges over a history X laid out as for sa_sketch_forward: user

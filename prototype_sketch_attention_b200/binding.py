@@ -105,7 +105,7 @@ def _load() -> ctypes.CDLL:
                                          vp, vp, sz, vp]
     lib.sa_stca_keys_backward.restype = i32
     lib.sa_stca_keys_backward.argtypes = [vp, vp, i32, i64, i32, vp, i64, vp, vp, vp, vp, vp, vp,
-                                          vp, vp, vp, vp, vp, vp, sz, vp]
+                                          vp, vp, i32, vp, vp, vp, vp, sz, vp]
     lib.sa_stca_recent_ranges.restype = i32
     lib.sa_stca_recent_ranges.argtypes = [vp, i32, i64, vp, vp, vp]
     return lib
@@ -168,10 +168,11 @@ def sa_stca_keys_forward(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin, k
 
 
 def sa_stca_keys_backward(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin, key_end, Wq, WK,
-                          WV, dout, dQ, dKx, dWq, dWK, dWV, workspace, ws_bytes, stream) -> int:
+                          WV, dout, dQ, dKx, accumulate, dWq, dWK, dWV, workspace, ws_bytes,
+                          stream) -> int:
     return int(_lib.sa_stca_keys_backward(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin,
-                                          key_end, Wq, WK, WV, dout, dQ, dKx, dWq, dWK, dWV,
-                                          workspace, ws_bytes, stream))
+                                          key_end, Wq, WK, WV, dout, dQ, dKx, int(accumulate),
+                                          dWq, dWK, dWV, workspace, ws_bytes, stream))
 
 
 def sa_stca_recent_ranges(offsets, R, L, key_begin, key_end, stream) -> int:
@@ -618,16 +619,21 @@ def stca_keys_forward(Q: torch.Tensor, cand_offsets: torch.Tensor, Kx: torch.Ten
 def stca_keys_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, Kx: torch.Tensor,
                        key_begin: torch.Tensor, key_end: torch.Tensor, Wq: torch.Tensor,
                        WK: torch.Tensor, WV: torch.Tensor, dout: torch.Tensor, *,
-                       ws: torch.Tensor | None = None, stream=None) -> dict:
+                       dKx: torch.Tensor | None = None, ws: torch.Tensor | None = None,
+                       stream=None) -> dict:
     """Gradients of stca_keys_forward given dL/dout [n_cand, d] fp32: dQ, dKx [n_keys, d]
-    (into the key rows), dWq, dWK, dWV. Inputs as for stca_keys_forward."""
+    (into the key rows), dWq, dWK, dWV. Inputs as for stca_keys_forward. With dKx given
+    (fp32 [n_keys, d]), the key rows' gradient is added into it instead of a new tensor
+    (for the recent branch: into the history gradient)."""
     where = "stca_keys_backward"
     n_cand, d, R, n_keys, dev = _check_keys_inputs(where, Q, cand_offsets, Kx, key_begin, key_end,
                                                    Wq, WK, WV)
     f32 = torch.float32
     _check_tensor(where, "dout", dout, (n_cand, d), f32, dev)
+    _check_tensor(where, "dKx", dKx, (n_keys, d), f32, dev, optional=True)
+    accumulate = dKx is not None
     out = {"dQ": torch.empty(n_cand, d, device=dev, dtype=f32),
-           "dKx": torch.empty(n_keys, d, device=dev, dtype=f32),
+           "dKx": dKx if accumulate else torch.empty(n_keys, d, device=dev, dtype=f32),
            "dWq": torch.empty(d, d, device=dev, dtype=f32),
            "dWK": torch.empty(d, d, device=dev, dtype=f32),
            "dWV": torch.empty(d, d, device=dev, dtype=f32)}
@@ -639,7 +645,7 @@ def stca_keys_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, Kx: torch.Te
             ws = torch.empty(nb, dtype=torch.uint8, device=dev)
         st = sa_stca_keys_backward(_ptr(Q), _ptr(cand_offsets), R, n_cand, d, _ptr(Kx), n_keys,
                                    _ptr(key_begin), _ptr(key_end), _ptr(Wq), _ptr(WK), _ptr(WV),
-                                   _ptr(dout), _ptr(out["dQ"]), _ptr(out["dKx"]),
+                                   _ptr(dout), _ptr(out["dQ"]), _ptr(out["dKx"]), accumulate,
                                    _ptr(out["dWq"]), _ptr(out["dWK"]), _ptr(out["dWV"]),
                                    _ptr(ws), ws.nbytes, _stream(stream, dev))
     if st != SA_OK:

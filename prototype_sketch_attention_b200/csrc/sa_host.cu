@@ -496,8 +496,8 @@ int sa_stca_keys_forward(const void* Q, const int64_t* cand_offsets, int R, int6
 int sa_stca_keys_backward(const void* Q, const int64_t* cand_offsets, int R, int64_t n_cand,
                           int d, const void* Kx, int64_t n_keys, const int64_t* key_begin,
                           const int64_t* key_end, const void* Wq, const void* WK, const void* WV,
-                          const float* dout, float* dQ, float* dKx, float* dWq, float* dWK,
-                          float* dWV, void* workspace, size_t ws_bytes, void* stream_) {
+                          const float* dout, float* dQ, float* dKx, int accumulate, float* dWq,
+                          float* dWK, float* dWV, void* workspace, size_t ws_bytes, void* stream_) {
   int st = check_keys_args(Q, cand_offsets, R, n_cand, d, Kx, n_keys, key_begin, key_end, Wq, WK,
                            WV);
   if (st != SA_OK) return st;
@@ -531,6 +531,7 @@ int sa_stca_keys_backward(const void* Q, const int64_t* cand_offsets, int R, int
   g.dout = dout;
   g.dQ = dQ;
   g.dKx = dKx;
+  g.accumulate = accumulate != 0;
   g.dWq = dWq;
   g.dWK = dWK;
   g.dWV = dWV;

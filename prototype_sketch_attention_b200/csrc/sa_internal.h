@@ -271,6 +271,7 @@ struct StcaKeysGrads {
   const float* dout;      // [n_cand, d]
   float* dQ;              // [n_cand, d]
   float* dKx;             // [n_keys, d]
+  bool accumulate;        // add into dKx instead of overwriting it
   float *dWq, *dWK, *dWV; // [d, d]
 };
 cudaError_t launch_stca_keys_forward(const StcaKeysArgs& a, cudaStream_t s);

@@ -250,6 +250,7 @@ cudaError_t launch_stca_backward(const StcaArgs& a, const StcaGrads& gr, int sms
   g.dout = gr.dout;
   g.dQ = gr.dQ;
   g.dKx = reinterpret_cast<float*>(static_cast<uint8_t*>(a.workspace) + a.plan.dkx);
+  g.accumulate = false;
   g.dWq = gr.dWq;
   g.dWK = gr.dWK;
   g.dWV = gr.dWV;

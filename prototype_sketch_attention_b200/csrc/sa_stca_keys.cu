@@ -398,30 +398,92 @@ __global__ void keys_empty_kernel(long long n, int d, float* __restrict__ O, flo
   }
 }
 
-// M[f][e] = sum_g W_q[f][g] W_K[e][g] in fp32 (block f, thread e).
-__global__ void keys_mfold_kernel(const __nv_bfloat16* __restrict__ Wq,
-                                  const __nv_bfloat16* __restrict__ WK, int d, float* __restrict__ M) {
-  const int f = blockIdx.x, e = threadIdx.x;
-  float acc = 0.f;
-  for (int g = 0; g < d; ++g)
-    acc = fmaf(__bfloat162float(Wq[f * d + g]), __bfloat162float(WK[e * d + g]), acc);
-  M[f * d + e] = acc;
+// M[f][e] = sum_g W_q[f][g] W_K[e][g] in fp32. Block b owns the rows f in [8b, 8b + 8):
+// W_K goes to shared memory transposed ([g][e], fp32, rows padded by one), the block's
+// W_q rows beside it, and thread e forms column e of those rows (conflict-free rows of
+// W_K^T, broadcast W_q).
+template <int D>
+__global__ void __launch_bounds__(D) keys_mfold_kernel(const __nv_bfloat16* __restrict__ Wq,
+                                                       const __nv_bfloat16* __restrict__ WK,
+                                                       float* __restrict__ M) {
+  extern __shared__ float fsm[];
+  float* wkt = fsm;                  // [D][D + 1]: wkt[g][e] = W_K[e][g] (padded rows)
+  float* wq = fsm + D * (D + 1);     // [8][D]
+  const int e = threadIdx.x, f0 = blockIdx.x * 8;
+  for (int i = e; i < D * D; i += D) wkt[(i % D) * (D + 1) + i / D] = __bfloat162float(WK[i]);
+  for (int i = e; i < 8 * D; i += D) wq[i] = __bfloat162float(Wq[f0 * D + i]);
+  __syncthreads();
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  for (int g = 0; g < D; ++g) {
+    const float w = wkt[g * (D + 1) + e];
+#pragma unroll
+    for (int r = 0; r < 8; ++r) acc[r] = fmaf(wq[r * D + g], w, acc[r]);
+  }
+#pragma unroll
+  for (int r = 0; r < 8; ++r) M[(f0 + r) * D + e] = acc[r];
 }
 
-// Q'_c = scale Q_c M in fp32, stored as hi = bf16(Q'_c) and lo = bf16(Q'_c - hi) (block per
-// candidate, thread e).
-__global__ void keys_qfold_kernel(const __nv_bfloat16* __restrict__ Q, const float* __restrict__ M,
-                                  long long n, int d, float scale, __nv_bfloat16* __restrict__ hi,
-                                  __nv_bfloat16* __restrict__ lo) {
-  const int e = threadIdx.x;
-  for (long long c = blockIdx.x; c < n; c += gridDim.x) {
-    float acc = 0.f;
-    for (int f = 0; f < d; ++f) acc = fmaf(__bfloat162float(Q[c * d + f]), M[f * d + e], acc);
-    const float v = acc * scale;
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    hi[c * d + e] = h;
-    lo[c * d + e] = __float2bfloat16_rn(v - __bfloat162float(h));
+// Q'_c = scale Q_c M in fp32, stored as hi = bf16(Q'_c) and lo = bf16(Q'_c - hi). Each
+// block keeps M in shared memory and walks groups of 32 candidates: their Q rows are
+// staged in shared memory (fp32, padded), and thread t forms column t mod D of 32 / (256 / D)
+// of the group's rows (broadcast Q, conflict-free rows of M).
+template <int D>
+__global__ void __launch_bounds__(256) keys_qfold_kernel(const __nv_bfloat16* __restrict__ Q,
+                                                         const float* __restrict__ M, long long n,
+                                                         float scale,
+                                                         __nv_bfloat16* __restrict__ hi,
+                                                         __nv_bfloat16* __restrict__ lo) {
+  constexpr int kRows = 32, kPer = kRows * D / 256;  // rows per thread: 16 at d = 128
+  extern __shared__ float fsm[];
+  float* ms = fsm;               // [D][D]
+  float* qs = fsm + D * D;       // [kRows][D + 1]
+  const int t = threadIdx.x, e = t % D, r0 = (t / D) * kPer;
+  for (int i = t; i < D * D; i += 256) ms[i] = M[i];
+  for (long long c0 = (long long)blockIdx.x * kRows; c0 < n; c0 += (long long)gridDim.x * kRows) {
+    __syncthreads();
+    for (int i = t; i < kRows * D; i += 256) {
+      const int r = i / D, f = i % D;
+      qs[r * (D + 1) + f] = c0 + r < n ? __bfloat162float(Q[(c0 + r) * D + f]) : 0.f;
+    }
+    __syncthreads();
+    float acc[kPer];
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) acc[r] = 0.f;
+    for (int f = 0; f < D; ++f) {
+      const float m = ms[f * D + e];
+#pragma unroll
+      for (int r = 0; r < kPer; ++r) acc[r] = fmaf(qs[(r0 + r) * (D + 1) + f], m, acc[r]);
+    }
+#pragma unroll
+    for (int r = 0; r < kPer; ++r) {
+      const long long c = c0 + r0 + r;
+      if (c < n) {
+        const float v = acc[r] * scale;
+        const __nv_bfloat16 h = __float2bfloat16_rn(v);
+        hi[c * D + e] = h;
+        lo[c * D + e] = __float2bfloat16_rn(v - __bfloat162float(h));
+      }
+    }
   }
+}
+
+template <int D>
+cudaError_t launch_folds(const void* Wq, const void* WK, const void* Q, long long n, float scale,
+                         float* M, __nv_bfloat16* Qh, __nv_bfloat16* Ql, cudaStream_t s) {
+  const size_t m_smem = (size_t)(D * (D + 1) + 8 * D) * sizeof(float);
+  const size_t q_smem = (size_t)(D * D + 32 * (D + 1)) * sizeof(float);
+  cudaError_t e;
+  if ((e = cudaFuncSetAttribute(keys_mfold_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)m_smem)) != cudaSuccess ||
+      (e = cudaFuncSetAttribute(keys_qfold_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)q_smem)) != cudaSuccess)
+    return e;
+  keys_mfold_kernel<D><<<D / 8, D, m_smem, s>>>(static_cast<const __nv_bfloat16*>(Wq),
+                                                static_cast<const __nv_bfloat16*>(WK), M);
+  const long long groups = (n + 31) / 32;
+  keys_qfold_kernel<D><<<(unsigned)std::min<long long>(groups, 148LL * 2), 256, q_smem, s>>>(
+      static_cast<const __nv_bfloat16*>(Q), M, n, scale, Qh, Ql);
+  return cudaGetLastError();
 }
 
 // D_c = sum_e bf16(dO'_ce) O'_ce, one warp per candidate.
@@ -496,11 +558,10 @@ cudaError_t keys_core(const StcaKeysArgs& a, float* lse, bool fwd_call, cudaStre
   float* M = at<float>(a.workspace, p.mt);
   __nv_bfloat16* Qh = at<__nv_bfloat16>(a.workspace, p.qh);
   __nv_bfloat16* Ql = at<__nv_bfloat16>(a.workspace, p.ql);
-  keys_mfold_kernel<<<d, d, 0, s>>>(static_cast<const __nv_bfloat16*>(a.Wq),
-                                    static_cast<const __nv_bfloat16*>(a.WK), d, M);
-  keys_qfold_kernel<<<(unsigned)std::min<long long>(n, 148LL * 32), d, 0, s>>>(
-      static_cast<const __nv_bfloat16*>(a.Q), M, n, d, kLog2e / std::sqrt((float)d), Qh, Ql);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  const float qscale = kLog2e / std::sqrt((float)d);
+  if ((e = d == 64 ? launch_folds<64>(a.Wq, a.WK, a.Q, n, qscale, M, Qh, Ql, s)
+                   : launch_folds<128>(a.Wq, a.WK, a.Q, n, qscale, M, Qh, Ql, s)) != cudaSuccess)
+    return e;
   CUtensorMap tqh, tql, tk;
   if (!tmap_rows_bf16(&tqh, Qh, (uint64_t)n, d) || !tmap_rows_bf16(&tql, Ql, (uint64_t)n, d) ||
       !tmap_rows_bf16(&tk, a.Kx, (uint64_t)a.n_keys, d))
@@ -610,7 +671,7 @@ cudaError_t launch_stca_keys_backward(const StcaKeysArgs& a, const StcaKeysGrads
   const float isd = 1.0f / std::sqrt((float)d);
   cudaError_t e;
   if ((e = keys_core(a, nullptr, false, s)) != cudaSuccess) return e;
-  if (a.n_keys > 0 &&
+  if (a.n_keys > 0 && !gr.accumulate &&
       (e = cudaMemsetAsync(gr.dKx, 0, (size_t)a.n_keys * d * sizeof(float), s)) != cudaSuccess)
     return e;
   if (n == 0) {

@@ -13,7 +13,9 @@
 // Per key tile j:
 //   S = (Q'_hi + Q'_lo) Kx_j^T and dP = dO' Kx_j^T on the tensor cores (TMEM, candidate =
 //   lane); two elementwise warpgroups (64 key columns each, thread = candidate) form
-//   a and dz and store dz and a log2(e) as bf16 [candidate][key] tiles in shared memory;
+//   a and dz, park them as bf16 pairs in TMEM over the dP columns they read (so the next
+//   tile's score MMAs can start), and once the previous tile's MMAs have read the shared
+//   dz / a tiles, store dz and a log2(e) there as bf16 [candidate][key] tiles;
 //   then G1 += dz Kx_j (dz K-major, Kx_j MN-major) accumulates in TMEM over the whole walk,
 //   and dKx_part = dz^T Q'_hi + (a log2 e)^T dO' (both A operands MN-major, K = the
 //   candidates) goes to TMEM, from where an epilogue warpgroup adds ln(2) dKx_part into
@@ -21,8 +23,9 @@
 //   whose ranges overlap, meet there). G1 is written once at the end (each candidate tile
 //   has one owner).
 // Roles: warp 0 TMA (the candidate tile's Q'_hi, Q'_lo and dO' once, the key tiles in a
-// ring), warp 1 TMEM allocation and every MMA, warps 4-11 the elementwise step, warps
-// 12-15 the dKx epilogue. Every mbarrier wait is bounded.
+// ring), warp 1 TMEM allocation and every MMA, warps 2-9 the elementwise step, warps
+// 10-13 the dKx epilogue (a warp reads the TMEM lanes of quadrant warp mod 4). Every
+// mbarrier wait is bounded.
 #include <cuda.h>
 
 #include "sa_common.cuh"
@@ -32,7 +35,8 @@ namespace sa {
 namespace {
 
 constexpr int kBox = 16384;  // 128 rows x 128 bytes (64 bf16), 128B swizzle
-constexpr int kThreads = 512;
+constexpr int kThreads = 448;  // 14 warps; at most 128 registers each, since a sub-partition
+                               // (16,384 registers) hosts four of them
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColP = 128, kColG = 256, kColK = 384;
 constexpr float kLn2 = 0.6931471805599453f;
@@ -59,7 +63,7 @@ struct BSmem {
 
 struct BBars {
   uint64_t q_full, k_full[3], k_empty[3];
-  uint64_t sd_full, sd_empty, ew_full, ew_empty, dk_full, dk_empty;
+  uint64_t sd_full, s_empty, p_empty, ew_full, ew_empty, dk_full, dk_empty;
   uint64_t drain;
   uint32_t tmem_base;
 };
@@ -109,7 +113,8 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
       mbar_init(smem_u32(&bars->k_empty[s]), 1);
     }
     mbar_init(smem_u32(&bars->sd_full), 1);
-    mbar_init(smem_u32(&bars->sd_empty), 8);
+    mbar_init(smem_u32(&bars->s_empty), 8);
+    mbar_init(smem_u32(&bars->p_empty), 8);
     mbar_init(smem_u32(&bars->ew_full), 8);
     mbar_init(smem_u32(&bars->ew_empty), 1);
     mbar_init(smem_u32(&bars->dk_full), 1);
@@ -196,7 +201,7 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
       for (int j = 0; ok && j < nkt; ++j) {
         const int st = j % NK;
         ok = mbar_wait(smem_u32(&bars->k_full[st]), (uint32_t)((j / NK) & 1), status, budget) &&
-             (j == 0 || mbar_wait(smem_u32(&bars->sd_empty), (uint32_t)((j - 1) & 1), status, budget));
+             (j == 0 || mbar_wait(smem_u32(&bars->s_empty), (uint32_t)((j - 1) & 1), status, budget));
         if (!ok) break;
         tc_fence_after();
         const uint64_t dk = smem_desc(sbase + L::oK + st * L::kTile, 16, 1024, kSwizzle128B);
@@ -210,6 +215,11 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
           const uint64_t koff = (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4);
           tc_mma_f16(tmem + kColS, dql + koff, dk + koff, id_s, 1u);
         }
+        // dP(j) once the elementwise step has moved the previous tile's packed dz and a out
+        // of the dP columns
+        ok = j == 0 || mbar_wait(smem_u32(&bars->p_empty), (uint32_t)((j - 1) & 1), status, budget);
+        if (!ok) break;
+        tc_fence_after();
 #pragma unroll
         for (int ks = 0; ks < KS_D; ++ks) {
           const uint64_t koff = (uint64_t)((((ks >> 2) * kBox) + (ks & 3) * 32) >> 4);
@@ -222,10 +232,10 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
       tc_commit(smem_u32(&bars->drain));
       mbar_wait_drain(smem_u32(&bars->drain), 0, budget);
     }
-  } else if (warp >= 4 && warp < 12) {
+  } else if (warp >= 2 && warp < 10) {
     // ================= elementwise: thread = candidate row, warpgroup w = key columns
-    // [64w, 64w + 64)
-    const int w = (warp - 4) >> 2;
+    // [64w, 64w + 64); warps 2-5 and 6-9 each cover the four TMEM lane quadrants
+    const int w = (warp - 2) >> 2;
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
@@ -237,43 +247,58 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
     bool ok = true;
     for (int j = 0; ok && j < nkt; ++j) {
       const int nk = (int)min(128LL, k1 - k0 - 128LL * j);
-      ok = mbar_wait_warp(smem_u32(&bars->sd_full), (uint32_t)(j & 1), status, budget) &&
-           mbar_wait_warp(smem_u32(&bars->ew_empty), (uint32_t)((j & 1) ^ 1), status, budget);
-      if (!ok) break;
+      if (!mbar_wait_warp(smem_u32(&bars->sd_full), (uint32_t)(j & 1), status, budget)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      // dz and a log2(e) of this thread's 64 key columns as bf16 pairs, 16 columns at a
+      // time, written back into TMEM over the dP columns just read (8 + 8 per 16 columns)
+#pragma unroll 1
+      for (int q = 0; q < 4; ++q) {
+        const int col = 64 * w + 16 * q;
+        uint32_t sv[16], pv[16], pk[16];
+        tmem_ld16(tmem + lane_off + kColS + col, sv);
+        tmem_ld16(tmem + lane_off + kColP + col, pv);
+        tmem_wait16(sv);
+        tmem_wait16(pv);
+#pragma unroll
+        for (int x = 0; x < 8; ++x) {
+          const bool v0 = row_ok && col + 2 * x < nk, v1 = row_ok && col + 2 * x + 1 < nk;
+          const float a0 = v0 ? ex2_approx(__uint_as_float(sv[2 * x]) - l2) : 0.f;
+          const float a1 = v1 ? ex2_approx(__uint_as_float(sv[2 * x + 1]) - l2) : 0.f;
+          pk[x] = cvt_bf16x2(a0 * (__uint_as_float(pv[2 * x]) - dc),
+                             a1 * (__uint_as_float(pv[2 * x + 1]) - dc));
+          pk[8 + x] = cvt_bf16x2(a0 * kLog2e, a1 * kLog2e);
+        }
+        tmem_st16(tmem + lane_off + kColP + col, pk);
+      }
+      asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+      // S is read: the next tile's score MMAs may overwrite it
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty));
+      // the previous tile's G1 and dKx MMAs have read dz and a: store this tile's
+      if (!mbar_wait_warp(smem_u32(&bars->ew_empty), (uint32_t)((j & 1) ^ 1), status, budget)) {
+        ok = false;
+        break;
+      }
       tc_fence_after();
 #pragma unroll 1
-      for (int h = 0; h < 2; ++h) {
-        const int col = 64 * w + 32 * h;
-        uint32_t s[32], p[32];
-        tmem_ld32_raw(tmem + lane_off + kColS + col, s);
-        tmem_ld32_raw(tmem + lane_off + kColP + col, p);
-        tmem_wait_tie(s);
-        tie32(p);
-        if (h == 1) {  // every TMEM read of S and dP of this tile is done
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(smem_u32(&bars->sd_empty));
-        }
-        uint32_t zp[16], ap[16];
-#pragma unroll
-        for (int x = 0; x < 16; ++x) {
-          const bool v0 = row_ok && col + 2 * x < nk, v1 = row_ok && col + 2 * x + 1 < nk;
-          const float a0 = v0 ? ex2_approx(__uint_as_float(s[2 * x]) - l2) : 0.f;
-          const float a1 = v1 ? ex2_approx(__uint_as_float(s[2 * x + 1]) - l2) : 0.f;
-          zp[x] = cvt_bf16x2(a0 * (__uint_as_float(p[2 * x]) - dc),
-                             a1 * (__uint_as_float(p[2 * x + 1]) - dc));
-          ap[x] = cvt_bf16x2(a0 * kLog2e, a1 * kLog2e);
-        }
-#pragma unroll
-        for (int cc = 0; cc < 4; ++cc) {
-          const int ch = h * 4 + cc;
-          const int off = (ch ^ (r & 7)) << 4;
-          *reinterpret_cast<uint4*>(dzrow + off) =
-              make_uint4(zp[4 * cc], zp[4 * cc + 1], zp[4 * cc + 2], zp[4 * cc + 3]);
-          *reinterpret_cast<uint4*>(arow + off) =
-              make_uint4(ap[4 * cc], ap[4 * cc + 1], ap[4 * cc + 2], ap[4 * cc + 3]);
-        }
+      for (int q = 0; q < 4; ++q) {
+        uint32_t pk[16];
+        tmem_ld16(tmem + lane_off + kColP + 64 * w + 16 * q, pk);
+        tmem_wait16(pk);
+        const int o0 = ((2 * q) ^ (r & 7)) << 4, o1 = ((2 * q + 1) ^ (r & 7)) << 4;
+        *reinterpret_cast<uint4*>(dzrow + o0) = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+        *reinterpret_cast<uint4*>(dzrow + o1) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        *reinterpret_cast<uint4*>(arow + o0) = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+        *reinterpret_cast<uint4*>(arow + o1) = make_uint4(pk[12], pk[13], pk[14], pk[15]);
       }
+      // the dP columns are free for the next tile's dP MMA
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&bars->p_empty));
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&bars->ew_full));
@@ -301,7 +326,7 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
                           __uint_as_float(v[x + 2]), __uint_as_float(v[x + 3]));
       }
     }
-  } else if (warp >= 12) {
+  } else {
     // ================= dKx epilogue: thread = key row of the tile; dKx += ln(2) dKx_part
     const int q4 = warp & 3;
     const int r = q4 * 32 + lane;

@@ -219,3 +219,24 @@ def test_recent_branch_backward_full_compare(lengths, counts, d, L):
         a, b = int(coff[u]), int(coff[u + 1])
         if a < b and np.any(ref["dQ"][a:b]):
             assert rel_l2(got["dQ"][a:b], ref["dQ"][a:b]) <= BF16_REL, u
+
+
+def test_backward_accumulates_into_a_given_history_gradient():
+    """With dKx given, the key rows' gradient is added into it: the result equals the
+    buffer's previous contents plus the overwriting call's dKx, bitwise, since with one
+    candidate tile per user every row receives exactly one addition in both calls."""
+    from prototype_sketch_attention_b200 import binding
+    rw = inputs.make_recent_workload([3000, 500, 0], [64, 7, 3], 128, 1000, seed=930)
+    G = torch.randn(74, 128, generator=torch.Generator().manual_seed(931))
+    dev = _dev()
+    kb, ke = _ranges(rw)
+    args = (rw.Q.to(dev), rw.cand_offsets.to(dev), rw.X.to(dev), kb, ke, rw.Wq.to(dev),
+            rw.WK.to(dev), rw.WV.to(dev), G.to(dev))
+    plain = binding.stca_keys_backward(*args)
+    base = torch.randn(3500, 128, generator=torch.Generator().manual_seed(932)).to(dev)
+    acc = binding.stca_keys_backward(*args, dKx=base.clone())
+    assert binding.device_status(acc["_ws"]) == 0
+    expect = base + plain["dKx"]
+    assert torch.equal(acc["dKx"], expect)
+    for key in ("dQ", "dWq", "dWK", "dWV"):
+        assert torch.equal(acc[key], plain[key]), key
