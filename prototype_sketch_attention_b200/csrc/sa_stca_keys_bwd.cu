@@ -19,8 +19,9 @@
 //   then G1 += dz Kx_j (dz K-major, Kx_j MN-major) accumulates in TMEM over the whole walk,
 //   and dKx_part = dz^T Q'_hi + (a log2 e)^T dO' (both A operands MN-major, K = the
 //   candidates) goes to TMEM, from where an epilogue warpgroup adds ln(2) dKx_part into
-//   dKx in global memory with vector reductions (the user's candidate tiles, and users
-//   whose ranges overlap, meet there). G1 is written once at the end (each candidate tile
+//   dKx in global memory with vector reductions at L2, regrouped by warp shuffles so that
+//   each reduction instruction covers whole 128-byte row segments (the user's candidate
+//   tiles, and users whose ranges overlap, meet there). G1 is written once at the end (each candidate tile
 //   has one owner).
 // Roles: warp 0 TMA (the candidate tile's Q'_hi, Q'_lo and dO' once, the key tiles in a
 // ring), warp 1 TMEM allocation and every MMA, warps 2-9 the elementwise step, warps
@@ -67,6 +68,27 @@ struct BBars {
   uint64_t drain;
   uint32_t tmem_base;
 };
+
+// One stage of a butterfly that regroups a warp's 32 x 32 block (lane = row, register =
+// column): lanes l and l ^ 2^LB swap the 4-register groups whose index bit GB differs from
+// lane bit LB. After the stages (LB, GB) = (4, 2), (3, 1), (2, 0), register group s of
+// lane l holds row 4 s + (l mod 4), columns 4 (l / 4) .. 4 (l / 4) + 3, so one vector
+// reduction over the warp covers 4 rows x 128 contiguous bytes.
+template <int LB, int GB>
+__device__ __forceinline__ void regroup_stage(float (&v)[32], int lane) {
+  const bool hi = (lane >> LB) & 1;
+#pragma unroll
+  for (int gi = 0; gi < 8; ++gi) {
+    if ((gi >> GB) & 1) continue;
+    const int gj = gi | (1 << GB);
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+      const float send = hi ? v[4 * gi + c] : v[4 * gj + c];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, 1 << LB);
+      if (hi) v[4 * gi + c] = recv; else v[4 * gj + c] = recv;
+    }
+  }
+}
 
 // dst[0..3] += v (fp32, one vector reduction performed at L2)
 __device__ __forceinline__ void red_add_v4(float* dst, float a, float b, float c, float d) {
@@ -327,9 +349,9 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
       }
     }
   } else {
-    // ================= dKx epilogue: thread = key row of the tile; dKx += ln(2) dKx_part
+    // ================= dKx epilogue: dKx += ln(2) dKx_part, warp = 32 key rows of the tile
+    // (TMEM lane quadrant warp mod 4), regrouped so that each reduction is coalesced
     const int q4 = warp & 3;
-    const int r = q4 * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q4 * 32) << 16;
     bool ok = true;
     for (int j = 0; ok && j < nkt; ++j) {
@@ -337,23 +359,29 @@ stca_keys_bwd_kernel(const __grid_constant__ CUtensorMap tmap_qh,
       ok = mbar_wait_warp(smem_u32(&bars->dk_full), (uint32_t)(j & 1), status, budget);
       if (!ok) break;
       tc_fence_after();
-      float* drow = dKx + (k0 + 128LL * j + r) * D;
+      float* dtile = dKx + (k0 + 128LL * j + q4 * 32) * D;  // this warp's 32 rows
 #pragma unroll 1
       for (int c = 0; c < D / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32_raw(tmem + lane_off + kColK + 32 * c, v);
-        tmem_wait_tie(v);
+        uint32_t u[32];
+        tmem_ld32_raw(tmem + lane_off + kColK + 32 * c, u);
+        tmem_wait_tie(u);
         if (c == D / 32 - 1) {  // dKx_part of this tile has been read
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(smem_u32(&bars->dk_empty));
         }
-        if (r < nk) {
+        float v[32];
 #pragma unroll
-          for (int x = 0; x < 32; x += 4)
-            red_add_v4(drow + 32 * c + x, __uint_as_float(v[x]) * kLn2,
-                       __uint_as_float(v[x + 1]) * kLn2, __uint_as_float(v[x + 2]) * kLn2,
-                       __uint_as_float(v[x + 3]) * kLn2);
+        for (int x = 0; x < 32; ++x) v[x] = __uint_as_float(u[x]) * kLn2;
+        regroup_stage<4, 2>(v, lane);
+        regroup_stage<3, 1>(v, lane);
+        regroup_stage<2, 0>(v, lane);
+#pragma unroll
+        for (int g = 0; g < 8; ++g) {
+          const int row = 4 * g + (lane & 3);  // within the warp's 32 rows
+          if (q4 * 32 + row < nk)
+            red_add_v4(dtile + row * D + 32 * c + 4 * (lane >> 2), v[4 * g], v[4 * g + 1],
+                       v[4 * g + 2], v[4 * g + 3]);
         }
       }
     }
