@@ -297,10 +297,13 @@ def time_other_workloads(binding, inputs, dev, steps: int, peak: float) -> list:
                 raise RuntimeError(binding.sa_status_string(st))
             step_ms = sum(e4[0].elapsed_time(e4[1]) for e4 in ev) / steps
             kern_ms = sum(event_ms(e4[2], e4[3]) for e4 in ev) / steps
+            graph_ms = graph_replay_ms(lambda: binding.forward(X, off, P, Wk, Wv, ws=o["_ws"], out=o),
+                                       steps, flush)
             n = w.n_total
             achieved = 4.0 * w.k * w.d * n / (kern_ms / 1e3) / 1e12
             out.append({"workload": desc, "n_total": n, "steps": steps,
                         "ms_per_step": step_ms, "tokens_per_s": n / (step_ms / 1e3),
+                        "graph_ms_per_step": graph_ms,
                         "kernel_ms": kern_ms, "kernel_tflops": achieved,
                         "kernel_frac": achieved / peak, "l2": "256 MB flush between steps"})
             del X, off, P, Wk, Wv, o
@@ -313,6 +316,37 @@ def time_other_workloads(binding, inputs, dev, steps: int, peak: float) -> list:
 
 
 RECENT_L, RECENT_CANDIDATES = 10000, 300
+
+
+def graph_replay_ms(fn, steps: int, flush=None) -> float:
+    """fn captured once into a CUDA graph (after a warm-up call on a side stream), then the
+    mean time of its replays from CUDA events (with the L2 flush between replays, outside
+    the events, when given). The library's calls allocate nothing and never synchronise,
+    so they capture as plain kernel and memset nodes."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        fn()
+    torch.cuda.current_stream().wait_stream(side)
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    for _ in range(3):
+        g.replay()
+    stream = torch.cuda.current_stream()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(steps)]
+    torch.cuda.synchronize()
+    for a, b in ev:
+        if flush is not None:
+            flush.zero_()
+        a.record(stream)
+        g.replay()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return sum(a.elapsed_time(b) for a, b in ev) / steps
 
 
 def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> dict:
@@ -358,6 +392,9 @@ def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> di
             raise RuntimeError(binding.sa_status_string(st))
         fwd_ms = sum(e4[0].elapsed_time(e4[1]) for e4 in ev) / steps
         kern_ms = sum(event_ms(e4[2], e4[3]) for e4 in ev) / steps
+        fwd_graph_ms = graph_replay_ms(
+            lambda: binding.stca_keys_forward(Q, coff, X, kb, ke, Wq, WK, WV, ws=o["_ws"]), steps,
+            flush)
         nb = 5
         bev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(nb)]
         for e4 in bev:
@@ -398,7 +435,8 @@ def time_recent_branch(binding, dev, X, off, peak: float, steps: int = 20) -> di
         bachieved = bflop / (bwd_kern_ms / 1e3) / 1e12
         return {"workload": f"{R} users x {RECENT_CANDIDATES} candidates over the last "
                             f"{RECENT_L} of {X.shape[0] // R} history rows each, d={d}",
-                "pairs": pairs, "forward_ms": fwd_ms, "pairs_per_s": pairs / (fwd_ms / 1e3),
+                "pairs": pairs, "forward_ms": fwd_ms, "forward_graph_ms": fwd_graph_ms,
+                "pairs_per_s": pairs / (fwd_ms / 1e3),
                 "kernel": "stca_keys_fwd_kernel<128>", "kernel_ms": kern_ms,
                 "kernel_tflops": achieved, "kernel_frac": achieved / peak,
                 "flop_per_pair": 4 * d,
@@ -429,7 +467,8 @@ def time_sketch_branch(binding, dev, sketch, peak: float, hbm_gbs: float, steps:
         gen = torch.Generator().manual_seed(78)
         R, k, d = sketch.shape
         n_cand = R * RECENT_CANDIDATES
-        coff = torch.arange(0, n_cand + 1, RECENT_CANDIDATES, dtype=torch.int64).to(dev)
+        coff_h = torch.arange(0, n_cand + 1, RECENT_CANDIDATES, dtype=torch.int64)
+        coff = coff_h.to(dev)
         Q = torch.randn(n_cand, d, generator=gen).to(torch.bfloat16).to(dev)
         Wq, WK, WV = ((torch.randn(d, d, generator=gen) / d ** 0.5).to(torch.bfloat16).to(dev)
                       for _ in range(3))
@@ -452,9 +491,15 @@ def time_sketch_branch(binding, dev, sketch, peak: float, hbm_gbs: float, steps:
             return sum(a.elapsed_time(b) for a, b in ev) / n
 
         o = binding.stca_forward(Q, coff, sketch, Wq, WK, WV)
-        g = binding.stca_backward(Q, coff, sketch, Wq, WK, WV, G)
+        g = binding.stca_backward(Q, coff, sketch, Wq, WK, WV, G, cand_offsets_host=coff_h)
         fwd_ms = timed(lambda: binding.stca_forward(Q, coff, sketch, Wq, WK, WV, ws=o["_ws"]), steps)
-        bwd_ms = timed(lambda: binding.stca_backward(Q, coff, sketch, Wq, WK, WV, G, ws=g["_ws"]), 5)
+        bwd_ms = timed(lambda: binding.stca_backward(Q, coff, sketch, Wq, WK, WV, G,
+                                                     cand_offsets_host=coff_h, ws=g["_ws"]), 5)
+        fwd_graph_ms = graph_replay_ms(
+            lambda: binding.stca_forward(Q, coff, sketch, Wq, WK, WV, ws=o["_ws"]), steps, flush)
+        bwd_graph_ms = graph_replay_ms(
+            lambda: binding.stca_backward(Q, coff, sketch, Wq, WK, WV, G, cand_offsets_host=coff_h,
+                                          ws=g["_ws"]), 5, flush)
         for ws in (o["_ws"], g["_ws"]):
             st = binding.device_status(ws)
             if st != 0:
@@ -466,6 +511,7 @@ def time_sketch_branch(binding, dev, sketch, peak: float, hbm_gbs: float, steps:
             "forward_ms": fwd_ms, "forward_tflops": flop / (fwd_ms / 1e3) / 1e12,
             "forward_frac": flop / (fwd_ms / 1e3) / 1e12 / peak,
             "backward_ms": bwd_ms,
+            "forward_graph_ms": fwd_graph_ms, "backward_graph_ms": bwd_graph_ms,
             "note": "the recent branch's kernels with the bf16 sketch rows as the keys; "
                     "4kd FLOP per candidate; one sketch read per user",
             "l2": "256 MB flush before every timed call"}

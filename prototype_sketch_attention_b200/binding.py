@@ -504,9 +504,12 @@ def stca_forward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, W
 
 def stca_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, Wq: torch.Tensor,
                   WK: torch.Tensor, WV: torch.Tensor, dout: torch.Tensor, *,
+                  cand_offsets_host: torch.Tensor | None = None,
                   ws: torch.Tensor | None = None, stream=None) -> dict:
     """Gradients of stca_forward given dL/dout [n_cand, d] fp32: dQ, dS (into each
-    user's sketch), dWq, dWK, dWV. Inputs as for stca_forward."""
+    user's sketch), dWq, dWK, dWV. Inputs as for stca_forward; cand_offsets_host, a CPU
+    copy of cand_offsets, saves the device-to-host copy (and lets the call be captured
+    into a CUDA graph)."""
     where = "stca_backward"
     _require(isinstance(Q, torch.Tensor) and Q.dim() == 2, where, "Q must be a 2-D tensor")
     _require(isinstance(S, torch.Tensor) and S.dim() == 3, where, "S must be a 3-D tensor")
@@ -523,7 +526,12 @@ def stca_backward(Q: torch.Tensor, cand_offsets: torch.Tensor, S: torch.Tensor, 
         _check_tensor(where, name, W, (d, d), bf, dev)
     _check_tensor(where, "dout", dout, (n_cand, d), f32, dev)
     _check_cuda(where, Q)
-    coff_h = cand_offsets.cpu().contiguous()
+    if cand_offsets_host is None:
+        coff_h = cand_offsets.cpu().contiguous()
+    else:
+        _check_tensor(where, "cand_offsets_host", cand_offsets_host, (R + 1,), torch.int64,
+                      torch.device("cpu"))
+        coff_h = cand_offsets_host
     out = {"dQ": torch.empty(n_cand, d, device=dev, dtype=f32),
            "dS": torch.empty(R, k, d, device=dev, dtype=f32),
            "dWq": torch.empty(d, d, device=dev, dtype=f32),
