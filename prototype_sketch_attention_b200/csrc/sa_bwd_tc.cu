@@ -91,7 +91,6 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
     t.a[1] = op(b.Gtlo, (uint64_t)R * k_pad, (uint64_t)d, false);
     t.b[1] = op(b.Wv, (uint64_t)d, (uint64_t)d, false);
     t.k_tiles[0] = t.k_tiles[1] = (d + 63) / 64;
-    t.user_mode = 0;
     t.M = R * k_pad;
     t.N = d;
     t.m_tiles_bound = (R * k_pad + 127) / 128;
@@ -113,7 +112,6 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
     t.a[0] = op(a.Ub, (uint64_t)R * k_pad, (uint64_t)d, true);
     t.b[0] = op(b.Gtb, (uint64_t)R * k_pad, (uint64_t)d, true);
     t.k_tiles[0] = (int)(((long long)R * k_pad + 63) / 64);
-    t.user_mode = 0;
     t.M = d;
     t.N = d;
     t.m_tiles_bound = 1;
@@ -141,17 +139,12 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s) {
       return e;
     GemmArgs l = {};
     l.hdr = b.hdr;
-    l.tile_start = b.tile_start;
-    l.offsets = b.offsets;
-    l.R = R;
-    l.k_pad = k_pad;
     l.k_valid = k;
     l.splits = 1;
     l.phases = 1;
     l.a[0] = op(b.X, (uint64_t)n, (uint64_t)d, false);
     l.b[0] = op(a.pn2, (uint64_t)k_pad, (uint64_t)d, false);
     l.k_tiles[0] = (d + 63) / 64;
-    l.user_mode = 0;
     l.M = (int)n;
     l.N = k_pad;
     l.m_tiles_bound = (int)((n + 127) / 128);

@@ -1,4 +1,6 @@
-// Tensor-core GEMM building block for the Sketch Attention backward (sm_100a).
+// Tensor-core GEMM building block (sm_100a): the finalize's W_v product, the backward's
+// Gh, dW_v and log-sum-exp GEMMs, and the cross attention's projections and weight
+// gradients.
 //
 //   C[128 x 128 tile] = sum over phases p, K tiles k of  A_p[m, k] . B_p[n, k]
 //
@@ -8,19 +10,12 @@
 // operand is either K-major (stored [M or N rows][K], K contiguous) or MN-major (stored
 // [K rows][M or N], M/N contiguous), so A B^T, A^T B and A B are all one kernel.
 //
-// Row tiles are either plain (128 consecutive rows of M) or user tiles: tile g covers
-// the tokens of one user only (the forward's schedule: tile_start prefix sums), so an
-// operand that depends on the user (B_p with a per-user row offset) is well defined.
+// Row tiles are 128 consecutive rows of M.
 //
 // Epilogues:
-//   kEpiStoreF32  out[row][n] = acc (+ add_in[row][n]) in fp32, or a split-K partial at
-//                 split * split_stride
-//   kEpiAExp      a = bf16(2^(acc - lse_scale * lse[row])), 0 for columns n >= k_valid;
-//                 out_bf16[row][n] = a and, with c given, dpart[row][2 tile + h] = the
-//                 row sum of a * c[user][n] over half h (64 columns) of the tile
+//   kEpiStoreF32  out[row][n] = acc in fp32, or a split-K partial at split * split_stride
 //   kEpiLse       dpart[row][2 tile + h] = log2 sum of 2^acc over half h of the tile
 //                 (columns n < k_valid)
-//   kEpiDS        out_bf16[row][n] = bf16(A[row][n] (acc - c[user][n] - drow[row]))
 //   kEpiStoreBf16 out_bf16[row][n] = bf16(acc)
 // Waits on mbarriers are bounded like every other kernel of the library.
 #include <cuda.h>
@@ -40,31 +35,17 @@ struct GemmParams {
   CUtensorMap ta[2], tb[2];
   int a_mn[2], b_mn[2];
   int k_tiles[2];
-  int b_user_rows[2];
   int phases;
-  int user_mode;
   int M, N;
   int splits;
   const WsHeader* hdr;
-  const long long* tile_start;
-  const int64_t* offsets;
-  int R;
   float* out_f32;
   long long ld_out;
   long long split_stride;
   __nv_bfloat16* out_bf16;
-  const float* lse2;
-  float lse_scale;
   int k_valid;
-  const __nv_bfloat16* a_in;
-  long long ld_a_in;
-  const float* c_user;
-  int k_pad;
   float* dpart;
   int dpart_ld;
-  const float* add_in;
-  long long ld_add;
-  const float* drow;
   long long budget;
 };
 
@@ -108,21 +89,9 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
   const unsigned n_tiles = (unsigned)(p.N + kBN - 1) / kBN;
   const int n_tile = (int)(blockIdx.x % n_tiles);
   const long long m_tile = (long long)(blockIdx.x / n_tiles);
-  int row0 = 0, nrows = 0, user = 0;
-  if (p.user_mode) {
-    const long long T = p.hdr->total_tiles;
-    const long long g = m_tile;
-    if (g >= T || read_status(status) != 0) return;
-    user = user_of_tile(p.tile_start, p.R, g);
-    const long long local = g - p.tile_start[user];
-    row0 = (int)(p.offsets[user] + local * kBM);
-    const long long n = p.offsets[user + 1] - row0;
-    nrows = n >= kBM ? kBM : (int)n;
-  } else {
-    row0 = (int)(m_tile * kBM);
-    nrows = min(kBM, p.M - row0);
-    if (nrows <= 0) return;
-  }
+  const int row0 = (int)(m_tile * kBM);
+  const int nrows = min(kBM, p.M - row0);
+  if (nrows <= 0) return;
   const int n0 = n_tile * kBN;
   // K tiles of this CTA: phase 0 is split evenly across gridDim.y; phase 1 is not split
   const int z = blockIdx.y;
@@ -165,11 +134,8 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
         const uint32_t fb = smem_u32(&bars->full[st]);
         mbar_arrive_expect_tx(fb, kStageBytes);
         const uint32_t sa = sbase + st * kStageBytes;
-        const int bu = p.b_user_rows[ph] * user;
         load_operand(sa, &p.ta[ph], p.a_mn[ph], row0, kt * kBK, fb);
-        // B's per-user offset applies to its row dimension: N for K-major, K for MN-major
-        if (!p.b_mn[ph]) load_operand(sa + kBM * kBK * 2, &p.tb[ph], 0, bu + n0, kt * kBK, fb);
-        else load_operand(sa + kBM * kBK * 2, &p.tb[ph], 1, n0, bu + kt * kBK, fb);
+        load_operand(sa + kBM * kBK * 2, &p.tb[ph], p.b_mn[ph], n0, kt * kBK, fb);
       }
       // the last stages' loads must land before exit
       for (int j = total_kt > kStages ? total_kt - kStages : 0; j < total_kt; ++j)
@@ -207,8 +173,7 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
     const int half = (warp - 2) >> 2;
     const int r = q * 32 + lane;
     const uint32_t lane_off = (uint32_t)(q * 32) << 16;
-    float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33 + 64);  // [32][33]
-    float* cst = stg + 32 * 33;  // this warp's 64 values of c[user][n]
+    float* stg = reinterpret_cast<float*>(smem) + (warp - 2) * (32 * 33);  // [32][33]
     const bool have = total_kt > 0 &&
                       mbar_wait_warp(smem_u32(&bars->done), 0, status, p.budget);
     if (have) {
@@ -216,18 +181,7 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
       const bool valid = r < nrows;
       const long long row = (long long)row0 + r;
       const int wrow0 = q * 32;  // first tile row of this warp
-      float rowv = 0.f;          // per-row scalar input: lse2 or D
-      if (valid) {
-        if (EPI == kEpiAExp) rowv = p.lse2[row] * p.lse_scale;
-        if (EPI == kEpiDS) rowv = p.drow[row];
-      }
-      float csum = 0.f, lmax = -INFINITY, lsum = 0.f;
-      if ((EPI == kEpiDS || EPI == kEpiAExp) && p.c_user != nullptr) {
-        const int n = n0 + half * 64 + lane;
-        cst[lane] = n < p.k_valid ? p.c_user[(long long)user * p.k_pad + n] : 0.f;
-        cst[lane + 32] = n + 32 < p.k_valid ? p.c_user[(long long)user * p.k_pad + n + 32] : 0.f;
-        __syncwarp();
-      }
+      float lmax = -INFINITY, lsum = 0.f;
 #pragma unroll 1
       for (int c = half * 2; c < half * 2 + 2; ++c) {
         uint32_t u[32];
@@ -254,59 +208,6 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
           }
           continue;
         }
-        // elementwise input (bf16 A for kEpiDS, fp32 addend for kEpiStoreF32), staged
-        const bool has_in = EPI == kEpiDS || (EPI == kEpiStoreF32 && p.add_in != nullptr);
-        if (has_in) {
-          __syncwarp();
-          if (EPI == kEpiDS) {  // 32 rows x 64 B: 4 lanes per row, 8 rows per instruction
-#pragma unroll
-            for (int it = 0; it < 4; ++it) {
-              const int rr = it * 8 + (lane >> 2), cc = (lane & 3) * 8;
-              uint4 w = make_uint4(0, 0, 0, 0);
-              if (wrow0 + rr < nrows && nb + cc < p.N)
-                w = *reinterpret_cast<const uint4*>(p.a_in + (row0 + wrow0 + rr) * p.ld_a_in + nb + cc);
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int h = 0; h < 4; ++h) {
-                stg[rr * 33 + cc + 2 * h] = __uint_as_float(ww[h] << 16);
-                stg[rr * 33 + cc + 2 * h + 1] = __uint_as_float(ww[h] & 0xFFFF0000u);
-              }
-            }
-          } else {  // 32 rows x 128 B: 8 lanes per row, 4 rows per instruction
-#pragma unroll
-            for (int it = 0; it < 8; ++it) {
-              const int rr = it * 4 + (lane >> 3), cc = (lane & 7) * 4;
-              float4 w = make_float4(0.f, 0.f, 0.f, 0.f);
-              if (wrow0 + rr < nrows && nb + cc < p.N)
-                w = *reinterpret_cast<const float4*>(p.add_in + (row0 + wrow0 + rr) * p.ld_add + nb + cc);
-              stg[rr * 33 + cc] = w.x;
-              stg[rr * 33 + cc + 1] = w.y;
-              stg[rr * 33 + cc + 2] = w.z;
-              stg[rr * 33 + cc + 3] = w.w;
-            }
-          }
-          __syncwarp();
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const float e = stg[lane * 33 + x];
-            if (EPI == kEpiDS) {
-              const float cu = cst[(c & 1) * 32 + x];
-              v[x] = e * (v[x] - cu - rowv);
-            } else {
-              v[x] += e;
-            }
-          }
-        }
-        if (EPI == kEpiAExp) {
-#pragma unroll
-          for (int x = 0; x < 32; ++x) {
-            const float a = nb + x < p.k_valid ? ex2_approx(v[x] - rowv) : 0.f;
-            // the value the later GEMMs see is bf16(a): sum c against that
-            const float ab = __bfloat162float(__float2bfloat16_rn(a));
-            if (p.c_user != nullptr) csum = fmaf(ab, cst[(c & 1) * 32 + x], csum);
-            v[x] = ab;
-          }
-        }
         // stage this warp's 32 x 32 outputs, then store them row by row
         __syncwarp();
 #pragma unroll
@@ -322,7 +223,7 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
                   make_float4(stg[rr * 33 + cc], stg[rr * 33 + cc + 1], stg[rr * 33 + cc + 2],
                               stg[rr * 33 + cc + 3]);
           }
-        } else {  // bf16 outputs (A, dS)
+        } else {  // bf16 output
 #pragma unroll
           for (int it = 0; it < 4; ++it) {
             const int rr = it * 8 + (lane >> 2), cc = (lane & 3) * 8;
@@ -338,8 +239,6 @@ sa_gemm_kernel(const __grid_constant__ GemmParams p) {
       if (EPI == kEpiLse && valid)
         p.dpart[row * p.dpart_ld + 2 * n_tile + half] =
             lmax > -INFINITY ? lmax + lg2_approx(lsum) : -INFINITY;
-      if (EPI == kEpiAExp && valid && p.c_user != nullptr)
-        p.dpart[row * p.dpart_ld + 2 * n_tile + half] = csum;
     }
   }
   tc_fence_before();
@@ -365,7 +264,7 @@ bool make_operand_map(CUtensorMap* m, const GemmOperandDesc& o) {
 
 template <int EPI, int NST>
 cudaError_t launch_st(const GemmParams& p, dim3 grid, cudaStream_t s) {
-  static_assert(8 * (32 * 33 + 64) * 4 <= NST * kStageBytes, "epilogue staging fits the stages");
+  static_assert(8 * (32 * 33) * 4 <= NST * kStageBytes, "epilogue staging fits the stages");
   const size_t smem = 1024 + NST * kStageBytes + sizeof(GemmBars<NST>);
   cudaError_t e = cudaFuncSetAttribute(sa_gemm_kernel<EPI, NST>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -390,37 +289,23 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     p.a_mn[ph] = g.a[ph].mn_major ? 1 : 0;
     p.b_mn[ph] = g.b[ph].mn_major ? 1 : 0;
     p.k_tiles[ph] = g.k_tiles[ph];
-    p.b_user_rows[ph] = g.b_user_rows[ph];
   }
   if (g.phases == 1) {
     p.ta[1] = p.ta[0];
     p.tb[1] = p.tb[0];
   }
   p.phases = g.phases;
-  p.user_mode = g.user_mode;
   p.M = g.M;
   p.N = g.N;
   p.splits = g.splits < 1 ? 1 : g.splits;
   p.hdr = g.hdr;
-  p.tile_start = g.tile_start;
-  p.offsets = g.offsets;
-  p.R = g.R;
   p.out_f32 = g.out_f32;
   p.ld_out = g.ld_out;
   p.split_stride = g.split_stride;
   p.out_bf16 = g.out_bf16;
-  p.lse2 = g.lse2;
-  p.lse_scale = g.lse_scale;
   p.k_valid = g.k_valid;
-  p.a_in = g.a_in;
-  p.ld_a_in = g.ld_a_in;
-  p.c_user = g.c_user;
-  p.k_pad = g.k_pad;
   p.dpart = g.dpart;
   p.dpart_ld = g.dpart_ld;
-  p.add_in = g.add_in;
-  p.ld_add = g.ld_add;
-  p.drow = g.drow;
   p.budget = kDefaultWaitBudget;
   const long long tiles = (long long)g.m_tiles_bound * ((g.N + kBN - 1) / kBN);
   if (tiles > 0x7FFFFFFFLL || p.splits > 65535) return cudaErrorInvalidValue;
@@ -428,8 +313,6 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   if (grid.x == 0) return cudaSuccess;
   switch (g.epi) {
     case kEpiStoreF32: return launch_t<kEpiStoreF32>(p, grid, s);
-    case kEpiAExp: return launch_t<kEpiAExp>(p, grid, s);
-    case kEpiDS: return launch_t<kEpiDS>(p, grid, s);
     case kEpiLse: return launch_t<kEpiLse>(p, grid, s);
     case kEpiStoreBf16: return launch_t<kEpiStoreBf16>(p, grid, s);
     default: return cudaErrorInvalidValue;

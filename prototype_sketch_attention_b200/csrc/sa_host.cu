@@ -691,7 +691,6 @@ int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M
   g.b[0] = {B, (uint64_t)(b_mn ? K : N), (uint64_t)(b_mn ? N : K), b_mn != 0};
   g.phases = 1;
   g.k_tiles[0] = (K + 63) / 64;
-  g.user_mode = 0;
   g.M = M;
   g.N = N;
   g.m_tiles_bound = (M + 127) / 128;

@@ -159,7 +159,7 @@ cudaError_t launch_bwd_tc(const BwdTcArgs& a, cudaStream_t s);
 int bwd_tc_wv_splits(int sms, int R, int k_pad);
 
 // ---- tensor-core GEMM (backward building block, sa_gemm_sm100.cu)
-enum GemmEpi { kEpiStoreF32 = 0, kEpiAExp = 1, kEpiDS = 2, kEpiLse = 3, kEpiStoreBf16 = 4 };
+enum GemmEpi { kEpiStoreF32 = 0, kEpiLse = 3, kEpiStoreBf16 = 4 };
 struct GemmOperandDesc {  // one bf16 operand, row-major in memory
   const void* base;
   uint64_t rows, cols;
@@ -169,32 +169,18 @@ struct GemmArgs {
   GemmOperandDesc a[2], b[2];  // operand pairs, accumulated into one result
   int phases;                  // 1 or 2
   int k_tiles[2];              // 64-wide K tiles of each pair
-  int b_user_rows[2];          // user tiles: B's row offset per user (0: shared B)
-  int user_mode;               // 0: plain 128-row tiles of M; 1: one user per tile
-  int M, N;                    // rows (plain mode) and output columns
-  int m_tiles_bound;           // grid x (user mode: an upper bound; extra CTAs exit)
+  int M, N;                    // rows and output columns
+  int m_tiles_bound;           // grid x: 128-row tiles of M
   int splits;                  // split-K over pair 0's K tiles (grid z)
   int epi;
-  const WsHeader* hdr;         // status word (and the tile count in user mode)
-  const long long* tile_start;
-  const int64_t* offsets;
-  int R;
+  const WsHeader* hdr;         // status word
   float* out_f32;
   long long ld_out;
   long long split_stride;
   __nv_bfloat16* out_bf16;
-  const float* lse2;
-  float lse_scale;             // kEpiAExp: lse2 = lse_scale * lse2[row]
-  int k_valid;                 // kEpiAExp / kEpiLse: columns n >= k_valid are padding
-  const __nv_bfloat16* a_in;
-  long long ld_a_in;
-  const float* c_user;
-  int k_pad;
+  int k_valid;                 // kEpiLse: columns n >= k_valid are padding
   float* dpart;
   int dpart_ld;
-  const float* add_in;         // kEpiStoreF32: added elementwise (nullable)
-  long long ld_add;
-  const float* drow;           // kEpiDS: per-row D
 };
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s);
 

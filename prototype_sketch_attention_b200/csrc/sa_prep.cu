@@ -467,7 +467,6 @@ cudaError_t launch_finalize_tc(const FinalizeArgs& a, cudaStream_t s) {
   g.b[1] = g.b[0];
   g.phases = 2;
   g.k_tiles[0] = g.k_tiles[1] = a.d / 64;
-  g.user_mode = 0;
   g.M = (int)rows;
   g.N = a.d;
   g.m_tiles_bound = (int)((rows + 127) / 128);

@@ -148,7 +148,6 @@ cudaError_t gemm_hilo(const WsHeader* hdr, const __nv_bfloat16* hi, const __nv_b
   t.b[1] = bop;
   t.phases = 2;
   t.k_tiles[0] = t.k_tiles[1] = d / 64;
-  t.user_mode = 0;
   t.M = (int)n;
   t.N = d;
   t.m_tiles_bound = (int)((n + 127) / 128);
@@ -169,7 +168,6 @@ cudaError_t gemm_tn_sum(const WsHeader* hdr, const __nv_bfloat16* A, const __nv_
   t.a[0] = opd(A, (uint64_t)n, (uint64_t)d, true);
   t.b[0] = opd(B, (uint64_t)n, (uint64_t)d, true);
   t.k_tiles[0] = (int)((n + 63) / 64);
-  t.user_mode = 0;
   t.M = d;
   t.N = d;
   t.m_tiles_bound = (d + 127) / 128;
