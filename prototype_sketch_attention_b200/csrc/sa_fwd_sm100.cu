@@ -588,11 +588,6 @@ int stages_for(int d, int C) { return d == 64 ? 4 : (C <= 8 ? 4 : 3); }
 
 }  // namespace
 
-size_t fwd_sm100_smem_bytes(int d, int C) {
-  if (d == 64) return FwdSmem<64, 4, 2>::bytes(C);
-  return stages_for(d, C) == 4 ? FwdSmem<128, 4, 1>::bytes(C) : FwdSmem<128, 3, 1>::bytes(C);
-}
-
 cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
   if (d == 64) return max_clusters_t<64, 4, 2>(C, n);
   return stages_for(d, C) == 4 ? max_clusters_t<128, 4, 1>(C, n) : max_clusters_t<128, 3, 1>(C, n);

@@ -61,7 +61,6 @@ struct FwdSm100Args {
   float* lse;
   long long budget;
 };
-size_t fwd_sm100_smem_bytes(int d, int C);
 cudaError_t fwd_sm100_max_clusters(int d, int C, int* n);
 cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream);
 
