@@ -251,14 +251,19 @@ int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, int R, int6
                               float* xsketch, int* device_status, void* stream);
 
 /*
- * Launch shape of the bf16 forward on the current device: the persistent grid holds
- * *clusters clusters of *cluster_size CTAs (one CTA per 128 prototypes), and cluster g
- * walks tiles [g T / clusters, (g + 1) T / clusters) of the T 128-token tiles of the
- * batch (users' tiles concatenated). A user whose tiles straddle one of those bounds is
- * accumulated by two clusters and summed in the finalize. For fp32 inputs (CUDA-core
- * path) both are set to 0. Returns SA_OK, or the argument codes of sa_sketch_forward.
+ * Launch shape of the bf16 forward on the current device. The persistent grid holds
+ * *clusters clusters of *cluster_size CTAs (one CTA per 128 prototypes); when those
+ * leave SMs free, *helpers helper CTAs (one per free SM, no cluster) run beside them and
+ * take *helper_share / 1024 of the tiles. With T 128-token tiles in the batch (users'
+ * tiles concatenated), Th = floor(T * helper_share / 1024) and T1 = T - Th, cluster g
+ * walks tiles [g T1 / clusters, (g + 1) T1 / clusters) and helper b walks
+ * [T1 + b Th / helpers, T1 + (b + 1) Th / helpers). A user whose tiles straddle one of
+ * those bounds is accumulated by two of them and summed in the finalize. For fp32
+ * inputs (CUDA-core path) all four are set to 0. `helpers` and `helper_share` may be
+ * null. Returns SA_OK, or the argument codes of sa_sketch_forward.
  */
-int sa_sketch_forward_grid(int k, int d, sa_dtype dt, int* clusters, int* cluster_size);
+int sa_sketch_forward_grid(int k, int d, sa_dtype dt, int* clusters, int* cluster_size,
+                           int* helpers, int* helper_share);
 
 /*
  * Reads the device status word that the last call using `workspace` left behind.

@@ -95,7 +95,7 @@ def _load() -> ctypes.CDLL:
     lib.sa_sketch_forward_host_status.restype = i32
     lib.sa_sketch_forward_host_status.argtypes = [vp, i32, i64, i32, i32, i32, i32, vp]
     lib.sa_sketch_forward_grid.restype = i32
-    lib.sa_sketch_forward_grid.argtypes = [i32, i32, i32, vp, vp]
+    lib.sa_sketch_forward_grid.argtypes = [i32, i32, i32, vp, vp, vp, vp]
     lib.sa_sketch_host_parts.restype = i32
     lib.sa_sketch_host_parts.argtypes = [vp, i32, i32, vp]
     lib.sa_stca_keys_workspace_size.restype = sz
@@ -196,18 +196,20 @@ def sa_sketch_forward_host_status(device_buffer, R, n_total, k, d, dt, parts, st
                                                   stream))
 
 
-def sa_sketch_forward_grid(k, d, dt, clusters, cluster_size) -> int:
-    return int(_lib.sa_sketch_forward_grid(k, d, dt, clusters, cluster_size))
+def sa_sketch_forward_grid(k, d, dt, clusters, cluster_size, helpers=None, helper_share=None) -> int:
+    return int(_lib.sa_sketch_forward_grid(k, d, dt, clusters, cluster_size, helpers, helper_share))
 
 
-def forward_grid(k: int, d: int, dtype=torch.bfloat16) -> tuple[int, int]:
-    """(clusters, cluster_size) of the bf16 forward's persistent grid on the current device."""
-    c, s = ctypes.c_int(0), ctypes.c_int(0)
+def forward_grid(k: int, d: int, dtype=torch.bfloat16) -> tuple[int, int, int, int]:
+    """(clusters, cluster_size, helpers, helper_share) of the bf16 forward on the current
+    device: tile ranges as sa_sketch_forward_grid describes."""
+    c, s, h, f = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
     st = sa_sketch_forward_grid(k, d, SA_BF16 if dtype == torch.bfloat16 else SA_F32,
-                                ctypes.addressof(c), ctypes.addressof(s))
+                                ctypes.addressof(c), ctypes.addressof(s), ctypes.addressof(h),
+                                ctypes.addressof(f))
     if st != SA_OK:
         raise SketchAttentionError(st, "sa_sketch_forward_grid")
-    return c.value, s.value
+    return c.value, s.value, h.value, f.value
 
 
 def sa_sketch_host_parts(offsets_host, R, parts, bounds) -> int:

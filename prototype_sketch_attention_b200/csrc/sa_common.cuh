@@ -382,6 +382,44 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// ---------------------------------------------------------------- tile ranges
+// The forward splits the token tiles [0, T) into G cluster ranges over [0, T1) and H helper
+// ranges over [T1, T) (helper CTAs run on the SMs that no cluster fits on). The helpers'
+// share is `share` / 1024 of the tiles: Th = floor(T share / 1024), T1 = T - Th. Range
+// g < G is [g T1 / G, (g + 1) T1 / G); range G + b is [T1 + b Th / H, T1 + (b + 1) Th / H).
+// The forward kernels and the finalize take the ranges from this one definition.
+struct TileRanges {
+  long long T1, Th;
+  int G, H;
+  __device__ TileRanges(long long T, int G_, int H_, int share)
+      : T1(T - (H_ > 0 ? (T * share) >> 10 : 0)), Th(H_ > 0 ? (T * share) >> 10 : 0), G(G_),
+        H(H_) {}
+  __device__ long long start(long long g) const {
+    return g <= G ? g * T1 / G : T1 + (g - G) * Th / H;
+  }
+  // the range holding tile x (0 <= x < T1 + Th); empty ranges are never returned
+  __device__ int of_tile(long long x) const {
+    const bool helper = x >= T1;
+    const long long base = helper ? T1 : 0, n = helper ? Th : T1;
+    const int m = helper ? H : G;
+    const long long y = x - base;
+    long long g = y * m / n;
+    if (g >= m) g = m - 1;
+    while (g + 1 < m && (g + 1) * n / m <= y) ++g;
+    while (g > 0 && g * n / m > y) --g;
+    return (int)g + (helper ? G : 0);
+  }
+};
+
+// Programmatic dependent launch. launch_dependents: the grid queued after this one with
+// the programmatic stream serialization attribute may start once every CTA of this grid
+// has executed it (or exited). wait: blocks until the grids this one depends on that way
+// have completed and their memory operations are visible.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // Token tile -> user lookup: the user whose tile range contains tile `g`
 // (tile_start is the exclusive prefix sum of per-user tile counts, length R+1).
 __device__ __forceinline__ int user_of_tile(const long long* tile_start, int R, long long g) {

@@ -32,6 +32,8 @@
 // bounded (see sa_common.cuh).
 #include <cuda.h>
 
+#include <cmath>
+
 #include "sa_common.cuh"
 #include "sa_internal.h"
 
@@ -155,6 +157,17 @@ __device__ __forceinline__ float exp2_and_sum(float (&v)[kProtoSlice]) {
   return z0 + z1;
 }
 
+// sum over the 128 scores of 2^(v - m), v left unchanged (four packed accumulators).
+__device__ __forceinline__ float sum_exp2(const float (&v)[kProtoSlice], float m) {
+  uint64_t za[4] = {0ull, 0ull, 0ull, 0ull};
+#pragma unroll
+  for (int p = 0; p < kProtoSlice / 2; ++p)
+    za[p & 3] = f2_add(za[p & 3], f2_pack(ex2_approx(v[2 * p] - m), ex2_approx(v[2 * p + 1] - m)));
+  float z0, z1;
+  f2_unpack(f2_add(f2_add(za[0], za[1]), f2_add(za[2], za[3])), z0, z1);
+  return z0 + z1;
+}
+
 // Maximum of the 128 scores: four independent chains of 3-input max.
 __device__ __forceinline__ float row_max(const float (&v)[kProtoSlice]) {
   float mc[4];
@@ -207,7 +220,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
                     const int64_t* __restrict__ offsets, int R, int k_valid, int C, int k_pad,
                     WsHeader* hdr, const long long* __restrict__ tile_start,
                     float* __restrict__ part_u, float* __restrict__ part_m,
-                    float* __restrict__ lse_out, long long budget) {
+                    float* __restrict__ lse_out, int H, int share, long long budget) {
   using L = FwdSmem<D, NS, NA>;
   constexpr int KSTEPS1 = D / 16;           // MMA1 K steps (over d)
   constexpr int KSTEPS2 = kTileTokens / 16;  // MMA2 K steps (over tokens)
@@ -262,11 +275,14 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
   __syncthreads();
   cluster_sync();  // peers' barriers are initialised before any st.async arrives
   tc_fence_after();
+  // every CTA is resident: the helper grid queued behind this one may take the free SMs
+  griddep_launch_dependents();
   const uint32_t tmem = bars->tmem_base;
 
-  // this cluster's share of the token tiles
+  // this cluster's range of the token tiles
   const long long T = read_status(status) == 0 ? hdr->total_tiles : 0;
-  const long long ta = (long long)cid * T / ncl, tb = (long long)(cid + 1) * T / ncl;
+  const TileRanges rg(T, (int)ncl, H, share);
+  const long long ta = rg.start(cid), tb = rg.start(cid + 1);
 
   if (warp == 0) {
     // ================= TMA producer (+ L2 prefetch of upcoming tiles by rank 0)
@@ -533,6 +549,447 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
   }
 }
 
+// ---------------------------------------------------------------------------- helper CTAs
+// Clusters of C CTAs do not tile the SMs exactly (C = 8: 15 clusters on 120 of 148 SMs).
+// The SMs left over run helper CTAs, one per SM and without a cluster, on the tail ranges
+// of the token tiles (TileRanges: range G + b belongs to helper b). Without a cluster a
+// CTA cannot exchange partial log-sums with the CTAs that hold the other prototype slices,
+// so a helper does all C slices of its tiles itself, in chunks of kChunk tiles and two
+// passes per chunk:
+//   pass 1, for each slice s and tile: S = X P'_s^T (MMA1) and the slice's partial
+//     l_s = m + log2 sum_j 2^(S_j - m); the token's running lse2 = log2 sum_s 2^(l_s) is
+//     kept in shared memory, one float per token;
+//   pass 2, for each slice s and tile: S again, A = 2^(S - lse2) and
+//     [U_s | mass_s] += A [X | 1] (MMA2) in TMEM; when the slice's pass over the chunk ends,
+//     or the tile stream crosses a user boundary, the partial is stored into (first time)
+//     or added to the workspace segment (range G + b, user).
+// The scores are computed twice, so a helper tile costs about 1.5 times a cluster CTA's
+// share of one. The kChunk X tiles of a chunk come from HBM once and from L2 for the
+// other 2C - 1 passes.
+//
+// Ownership rules that make the shared-memory and workspace accesses race-free: tile t of
+// a chunk is handled by softmax warpgroup (t & 1) in every pass, so a token's running lse2
+// is read and written by one thread only; every segment epilogue is done by warpgroup 0,
+// so each workspace row is read and written by one thread only, in program order.
+// The score buffers alternate with the tile's parity too, and every role counts each
+// buffer's uses itself (chunks may have an odd number of tiles).
+constexpr int kChunk = 32;  // tiles per chunk
+// Register split: the softmax warpgroups hold a token's 128 scores through both passes'
+// sums, so they take 224 registers and the producer / MMA warpgroup gives up all but 56.
+// setmaxnreg.inc waits until the block's launch allocation covers it, so the split adds up
+// to exactly 384 threads x 168 registers, and the launch refuses a build compiled to fewer.
+constexpr int kHelperRegsLaunch = 168, kHelperRegsControl = 56, kHelperRegsSoftmax = 224;
+static_assert(128 * kHelperRegsControl + 256 * kHelperRegsSoftmax <= kThreads * kHelperRegsLaunch,
+              "register split exceeds the launch allocation");
+
+template <int D>
+struct HelperSmem {
+  using X = FwdSmem<D, 3, 1>;  // the three-stage clustered layout: X stages, A tile, ones atom
+  static constexpr int oP0 = X::oP;                 // P' slice, buffer 0
+  static constexpr int oP1 = X::oP + X::kPBytes;    // P' slice, buffer 1
+  static constexpr int oL = oP1 + X::kPBytes;       // running lse2, [kChunk][128] floats
+  static constexpr int oBars = oL + kChunk * kTileTokens * 4;
+};
+
+struct HBars {
+  uint64_t x_full[3], x_empty[3];
+  uint64_t s_full[2], s_empty[2];
+  uint64_t p_full[2], p_empty[2];
+  uint64_t a_full, a_empty[4];  // a_empty[i2 mod 4]: MMA2 of pass-2 step i2 has completed
+  uint64_t u_full, u_empty;
+  uint64_t m2iss[4];
+  uint64_t drain, drain2;
+  uint32_t tmem_base;
+};
+
+template <int D>
+constexpr size_t helper_smem_bytes() {
+  return 1024 + HelperSmem<D>::oBars + sizeof(HBars);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kThreads, 1)
+sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
+                           const __grid_constant__ CUtensorMap tmap_p,
+                           const int64_t* __restrict__ offsets, int R, int k_valid, int C,
+                           int k_pad, WsHeader* hdr, const long long* __restrict__ tile_start,
+                           float* __restrict__ part_u, float* __restrict__ part_m,
+                           float* __restrict__ lse_out, int G, int H, int share,
+                           long long budget) {
+  using L = FwdSmem<D, 3, 1>;
+  using HS = HelperSmem<D>;
+  constexpr int NS = 3;
+  constexpr int KSTEPS1 = D / 16;
+  constexpr int KSTEPS2 = kTileTokens / 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                             ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  HBars* bars = reinterpret_cast<HBars*>(smem + HS::oBars);
+  float* lsm = reinterpret_cast<float*>(smem + HS::oL);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  int* status = &hdr->status;
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(smem_u32(&bars->x_full[s]), 1);
+      mbar_init(smem_u32(&bars->x_empty[s]), 1);
+    }
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(smem_u32(&bars->s_full[s]), 1);
+      mbar_init(smem_u32(&bars->s_empty[s]), 4);
+      mbar_init(smem_u32(&bars->p_full[s]), 1);
+      mbar_init(smem_u32(&bars->p_empty[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->a_full), 4);
+    for (int s = 0; s < 4; ++s) {
+      mbar_init(smem_u32(&bars->a_empty[s]), 1);
+      mbar_init(smem_u32(&bars->m2iss[s]), 1);
+    }
+    mbar_init(smem_u32(&bars->u_full), 1);
+    mbar_init(smem_u32(&bars->u_empty), 4);
+    mbar_init(smem_u32(&bars->drain), 1);
+    mbar_init(smem_u32(&bars->drain2), 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(&bars->tmem_base), kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp >= 4) {
+    uint32_t* ones = reinterpret_cast<uint32_t*>(smem + L::oOnes);
+    for (int w = threadIdx.x - 128; w < L::kSlot / 4; w += kThreads - 128) ones[w] = 0x3F803F80u;
+    fence_proxy_async_smem();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars->tmem_base;
+
+  const long long T = read_status(status) == 0 ? hdr->total_tiles : 0;
+  const TileRanges rg(T, G, H, share);
+  const long long ra = rg.start(G + (long long)blockIdx.x), rb = rg.start(G + (long long)blockIdx.x + 1);
+
+  // each warp changes its register count inside its own role's branch, so that the
+  // compiler budgets every role's code for that role's count
+  if (warp == 0) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegsControl));
+    // ================= TMA producer: per (pass, slice) the P' slice, per step the X tile;
+    // the next chunk's tiles are prefetched into L2 during the current chunk's last slice
+    if (lane == 0 && ra < rb) {
+      tma_prefetch_desc(&tmap_x);
+      tma_prefetch_desc(&tmap_p);
+      TileIter base, ahead, it;
+      base.init(tile_start, offsets, R, ra, rb);
+      ahead = base;
+      for (int j = 0; j < kChunk && ahead.valid(); ++j, ahead.next())
+        for (int b = 0; b < L::kXBoxes; ++b) tma_prefetch_l2_2d(&tmap_x, b * 64, (int)ahead.t0());
+      int i = 0, q = 0;
+      bool ok = true;
+      for (long long c0 = ra; ok && c0 < rb; c0 += kChunk) {
+        const int K = (int)(rb - c0 < kChunk ? rb - c0 : kChunk);
+        for (int ph = 0; ok && ph < 2; ++ph) {
+          for (int s = 0; ok && s < C; ++s) {
+            const int pb = q & 1;
+            if (!mbar_wait(smem_u32(&bars->p_empty[pb]), (uint32_t)(((q >> 1) & 1) ^ 1), status, budget)) {
+              ok = false;
+              break;
+            }
+            const uint32_t pf = smem_u32(&bars->p_full[pb]);
+            mbar_arrive_expect_tx(pf, L::kPBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_2d(sbase + (pb ? HS::oP1 : HS::oP0) + b * L::kSlot, &tmap_p, b * 64,
+                          s * kProtoSlice, pf);
+            ++q;
+            const bool track = ph == 0 && s == 0, pref = ph == 1 && s == C - 1;
+            if (track) ahead = base;
+            it = base;
+            for (int tl = 0; tl < K; ++tl, it.next(), ++i) {
+              const int st = i % NS;
+              if (!mbar_wait(smem_u32(&bars->x_empty[st]), (uint32_t)(((i / NS) & 1) ^ 1), status,
+                             budget)) {
+                ok = false;
+                break;
+              }
+              const uint32_t fb = smem_u32(&bars->x_full[st]);
+              mbar_arrive_expect_tx(fb, L::kXBytes);
+              for (int b = 0; b < L::kXBoxes; ++b)
+                tma_load_2d(sbase + L::xbox(st, b), &tmap_x, b * 64, (int)it.t0(), fb);
+              if (track) {
+                ahead.next();
+              } else if (pref && ahead.valid()) {
+                for (int b = 0; b < L::kXBoxes; ++b)
+                  tma_prefetch_l2_2d(&tmap_x, b * 64, (int)ahead.t0());
+                ahead.next();
+              }
+            }
+          }
+        }
+        base = it;
+      }
+      // drain: the last NS X loads and the last two P' loads have landed before exit
+      for (int j = (i > NS ? i - NS : 0); j < i; ++j)
+        mbar_wait_drain(smem_u32(&bars->x_full[j % NS]), (uint32_t)((j / NS) & 1), budget);
+      for (int g = (q > 2 ? q - 2 : 0); g < q; ++g)
+        mbar_wait_drain(smem_u32(&bars->p_full[g & 1]), (uint32_t)((g >> 1) & 1), budget);
+    }
+  } else if (warp == 1) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegsControl));
+    // ================= MMA1 issuer: S[tile parity] = X P'_s^T for every step of both passes.
+    // In pass 2, MMA1 of step i2 waits until MMA2(i2 - 3) is issued (so that an accumulate
+    // MMA never queues behind a score MMA) and MMA2(i2 - 4) has completed (which bounds how
+    // far the A buffer's barriers can lag behind a softmax warpgroup's wait).
+    if (lane == 0 && ra < rb) {
+      const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);
+      const uint64_t dp0 = smem_desc(sbase + HS::oP0, 16, 1024, kSwizzle128B);
+      const uint64_t dp1 = smem_desc(sbase + HS::oP1, 16, 1024, kSwizzle128B);
+      int i = 0, q = 0, i2 = 0, nb0 = 0, nb1 = 0;
+      bool ok = true;
+      for (long long c0 = ra; ok && c0 < rb; c0 += kChunk) {
+        const int K = (int)(rb - c0 < kChunk ? rb - c0 : kChunk);
+        for (int ph = 0; ok && ph < 2; ++ph) {
+          for (int s = 0; ok && s < C; ++s, ++q) {
+            const int pb = q & 1;
+            if (!mbar_wait(smem_u32(&bars->p_full[pb]), (uint32_t)((q >> 1) & 1), status, budget)) {
+              ok = false;
+              break;
+            }
+            const uint64_t dp = pb ? dp1 : dp0;
+            for (int tl = 0; tl < K; ++tl, ++i) {
+              const int st = i % NS, sb = tl & 1;
+              const int nbs = sb ? nb1 : nb0;
+              ok = mbar_wait(smem_u32(&bars->x_full[st]), (uint32_t)((i / NS) & 1), status, budget) &&
+                   mbar_wait(smem_u32(&bars->s_empty[sb]), (uint32_t)((nbs & 1) ^ 1), status, budget);
+              if (ok && ph == 1 && i2 >= 3)
+                ok = mbar_wait(smem_u32(&bars->m2iss[(i2 - 3) & 3]), (uint32_t)(((i2 - 3) >> 2) & 1),
+                               status, budget);
+              if (ok && ph == 1 && i2 >= 4)
+                ok = mbar_wait(smem_u32(&bars->a_empty[(i2 - 4) & 3]), (uint32_t)(((i2 - 4) >> 2) & 1),
+                               status, budget);
+              if (!ok) break;
+              tc_fence_after();
+              uint64_t xd[L::kXBoxes];
+#pragma unroll
+              for (int b = 0; b < L::kXBoxes; ++b)
+                xd[b] = smem_desc(sbase + L::xbox(st, b), 16, 1024, kSwizzle128B);
+#pragma unroll
+              for (int ks = 0; ks < KSTEPS1; ++ks) {
+                const uint32_t koff = (ks >> 2) * L::kSlot + (ks & 3) * 32;
+                tc_mma_f16(tmem + (sb ? kColS1 : kColS0), xd[ks >> 2] + (uint64_t)(((ks & 3) * 32) >> 4),
+                           dp + (uint64_t)(koff >> 4), idesc1, ks > 0 ? 1u : 0u);
+              }
+              tc_commit(smem_u32(&bars->s_full[sb]));
+              if (ph == 0) tc_commit(smem_u32(&bars->x_empty[st]));  // pass 1: X is done
+              if (tl == K - 1) tc_commit(smem_u32(&bars->p_empty[pb]));
+              if (sb) ++nb1; else ++nb0;
+              if (ph == 1) ++i2;
+            }
+          }
+        }
+      }
+      tc_commit(smem_u32(&bars->drain));
+      mbar_wait_drain(smem_u32(&bars->drain), 0, budget);
+    }
+  } else if (warp == 2) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegsControl));
+    // ================= MMA2 issuer (pass 2 only): [U | mass] += A [X | 1]
+    if (lane == 0 && ra < rb) {
+      const uint32_t idesc2 = idesc_bf16_f32(128, D + 16, 1, 1);
+      const uint64_t da =
+          smem_desc(sbase + L::abox(0, 0), L::abox(0, 1) - L::abox(0, 0), 1024, kSwizzle128B);
+      TileIter base, it;
+      base.init(tile_start, offsets, R, ra, rb);
+      int i = 0, i2 = 0, seg = 0;
+      bool ok = true;
+      for (long long c0 = ra; ok && c0 < rb; c0 += kChunk) {
+        const int K = (int)(rb - c0 < kChunk ? rb - c0 : kChunk);
+        i += C * K;  // pass 1 steps: MMA1 releases their X stages
+        for (int s = 0; ok && s < C; ++s) {
+          it = base;
+          int prev_u = -1;
+          for (int tl = 0; tl < K; ++tl, it.next(), ++i, ++i2) {
+            const int st = i % NS;
+            const bool first = tl == 0 || it.u != prev_u, last = tl == K - 1 || it.last();
+            prev_u = it.u;
+            ok = mbar_wait(smem_u32(&bars->a_full), (uint32_t)(i2 & 1), status, budget) &&
+                 (!first || mbar_wait(smem_u32(&bars->u_empty), (uint32_t)((seg & 1) ^ 1), status, budget));
+            if (!ok) break;
+            tc_fence_after();
+            const uint64_t xd = smem_desc(sbase + L::xbox(st, 0), L::stage_a(st) * L::kSlot, 1024,
+                                          kSwizzle128B);
+#pragma unroll
+            for (int ks = 0; ks < KSTEPS2; ++ks)
+              tc_mma_f16(tmem + kColU, da + (uint64_t)((ks * 2048) >> 4), xd + (uint64_t)((ks * 2048) >> 4),
+                         idesc2, (first && ks == 0) ? 0u : 1u);
+            tc_commit(smem_u32(&bars->x_empty[st]));
+            tc_commit(smem_u32(&bars->a_empty[i2 & 3]));
+            if (last) {
+              tc_commit(smem_u32(&bars->u_full));
+              ++seg;
+            }
+            mbar_arrive(smem_u32(&bars->m2iss[i2 & 3]));
+          }
+        }
+        base = it;
+      }
+      tc_commit(smem_u32(&bars->drain2));
+      mbar_wait_drain(smem_u32(&bars->drain2), 0, budget);
+    }
+  } else if (warp == 3) {
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegsControl));
+  } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHelperRegsSoftmax));
+    // ================= softmax warpgroups (tile parity) + segment epilogues (warpgroup 0)
+    const int wg = (warp >> 2) - 1;
+    const int qd = warp & 3;
+    const int r = qd * 32 + lane;
+    const uint32_t lane_off = (uint32_t)(qd * 32) << 16;
+    TileIter base, it;
+    base.init(tile_start, offsets, R, ra, rb);
+    int nbw = 0, i2 = 0, useg = 0;
+    long long run_g0 = 0;
+    bool ok = true;
+    for (long long c0 = ra; ok && c0 < rb; c0 += kChunk) {
+      const int K = (int)(rb - c0 < kChunk ? rb - c0 : kChunk);
+      for (int ph = 0; ok && ph < 2; ++ph) {
+        for (int s = 0; ok && s < C; ++s) {
+          const int pbase = s * kProtoSlice;
+          const bool partial_slice = pbase + kProtoSlice > k_valid;
+          it = base;
+          int prev_u = -1;
+          for (int tl = 0; tl < K; ++tl, it.next()) {
+            const int sb = tl & 1;
+            if (ph == 1 && (tl == 0 || it.u != prev_u)) run_g0 = it.g;
+            prev_u = it.u;
+            if (sb == wg) {
+              if (!mbar_wait_warp(smem_u32(&bars->s_full[sb]), (uint32_t)(nbw & 1), status, budget)) {
+                ok = false;
+                break;
+              }
+              ++nbw;
+              tc_fence_after();
+              float v[kProtoSlice];
+              load_scores(tmem + lane_off + (sb ? kColS1 : kColS0), v);
+              // the scores are in registers: the buffer goes back to MMA1 at once, so the
+              // score MMA of this warpgroup's next tile overlaps the exponentials below
+              tc_fence_before();
+              __syncwarp();
+              if (lane == 0) mbar_arrive(smem_u32(&bars->s_empty[sb]));
+              if (partial_slice) {
+#pragma unroll
+                for (int c = 0; c < kProtoSlice; ++c)
+                  if (pbase + c >= k_valid) v[c] = -INFINITY;
+              }
+              const bool valid = r < it.nvalid();
+              float* lp = lsm + tl * kTileTokens + r;
+              if (ph == 0) {
+                // l = m + log2 sum 2^(s - m): no shift (m = 0) unless a lane's sum leaves
+                // [2^-100, 2^100], as in the clustered kernel; only the sum is kept
+                float m = 0.f;
+                float z = sum_exp2(v, 0.f);
+                if (!__all_sync(0xffffffffu, z >= 0x1p-100f && z <= 0x1p100f)) {
+                  m = row_max(v);
+                  z = sum_exp2(v, m);
+                }
+                const float l = valid ? m + lg2_approx(z) : 0.f;
+                if (s == 0) {
+                  *lp = l;
+                } else {  // lse2 <- log2(2^lse2 + 2^l)
+                  const float o = *lp;
+                  const float hi = fmaxf(o, l), lo = fminf(o, l);
+                  *lp = hi + lg2_approx(1.f + ex2_approx(lo - hi));
+                }
+              } else {
+                // A = 2^(s - lse2) <= 1 directly (lse2 >= every score); rows past the
+                // user's last token get A = 0
+                const float lse2 = *lp;
+                if (s == 0 && valid && lse_out != nullptr)
+                  lse_out[it.t0() + r] = lse2 * 0.69314718055994530942f;
+                const float off = valid ? -lse2 : -INFINITY;
+                const uint64_t off2 = f2_pack(off, off);
+                uint32_t pa0[32], pa1[32];
+#pragma unroll
+                for (int p = 0; p < 32; ++p) {
+                  float a, b;
+                  f2_unpack(f2_add(f2_pack(v[2 * p], v[2 * p + 1]), off2), a, b);
+                  pa0[p] = cvt_bf16x2(ex2_approx(a), ex2_approx(b));
+                  f2_unpack(f2_add(f2_pack(v[64 + 2 * p], v[64 + 2 * p + 1]), off2), a, b);
+                  pa1[p] = cvt_bf16x2(ex2_approx(a), ex2_approx(b));
+                }
+                // A(i2) may overwrite the buffer once MMA2(i2 - 1) has read it; MMA1(i2) was
+                // issued after MMA2(i2 - 4) completed, so this barrier is at most one phase
+                // behind the awaited one
+                if (!mbar_wait_warp(smem_u32(&bars->a_empty[(i2 - 1) & 3]),
+                                    (uint32_t)(((i2 - 1) >> 2) & 1), status, budget)) {
+                  ok = false;
+                  break;
+                }
+                store_a_block(smem + L::abox(0, 0) + r * 128, r, pa0);
+                store_a_block(smem + L::abox(0, 1) + r * 128, r, pa1);
+                fence_proxy_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->a_full));
+              }
+            }
+            if (ph == 1) {
+              if (wg == 0 && (tl == K - 1 || it.last())) {
+                // ---- epilogue of the run that ends at this tile: U_s, mass_s into segment
+                // (range G + b, user); stored by the segment's first run, added after that
+                if (!mbar_wait_warp(smem_u32(&bars->u_full), (uint32_t)(useg & 1), status, budget)) {
+                  ok = false;
+                  break;
+                }
+                ++useg;
+                tc_fence_after();
+                const long long sgid = (long long)G + blockIdx.x + it.u;
+                const bool seg_first = run_g0 == ra || run_g0 == tile_start[it.u];
+                float* dst = part_u + ((size_t)sgid * k_pad + pbase + r) * D;
+#pragma unroll
+                for (int c = 0; c < D / 32; ++c) {
+                  uint32_t u32[32];
+                  tmem_ld32_raw(tmem + lane_off + kColU + c * 32, u32);
+                  tmem_wait_tie(u32);
+#pragma unroll
+                  for (int x = 0; x < 32; x += 4) {
+                    float4 o = make_float4(__uint_as_float(u32[x]), __uint_as_float(u32[x + 1]),
+                                           __uint_as_float(u32[x + 2]), __uint_as_float(u32[x + 3]));
+                    float4* p4 = reinterpret_cast<float4*>(dst + c * 32 + x);
+                    if (!seg_first) {
+                      const float4 w4 = *p4;
+                      o.x += w4.x; o.y += w4.y; o.z += w4.z; o.w += w4.w;
+                    }
+                    *p4 = o;
+                  }
+                }
+                const float ms = tmem_ld1(tmem + lane_off + kColU + D);
+                tc_wait_ld();
+                float* pm = part_m + (size_t)sgid * k_pad + pbase + r;
+                *pm = seg_first ? ms : *pm + ms;
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(smem_u32(&bars->u_empty));
+              }
+              ++i2;
+            }
+          }
+        }
+      }
+      base = it;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  // complete only after the clustered grid: work queued behind this grid sees its results
+  griddep_wait();
+}
+
 template <int D, int NS, int NA>
 cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
   auto kern = sa_fwd_sm100_kernel<D, NS, NA>;
@@ -556,7 +1013,8 @@ cudaError_t launch_fwd_sm100_t(const FwdSm100Args& a, cudaStream_t stream) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   return cudaLaunchKernelEx(&cfg, kern, *a.tmap_x, *a.tmap_p, a.offsets, a.R, a.k_valid, a.C,
-                            a.k_pad, a.hdr, a.tile_start, a.part_u, a.part_m, a.lse, a.budget);
+                            a.k_pad, a.hdr, a.tile_start, a.part_u, a.part_m, a.lse, a.H,
+                            a.share, a.budget);
 }
 
 template <int D, int NS, int NA>
@@ -593,10 +1051,50 @@ cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
   return stages_for(d, C) == 4 ? max_clusters_t<128, 4, 1>(C, n) : max_clusters_t<128, 3, 1>(C, n);
 }
 
+// The helpers' share of the tiles balances the two grids: a cluster takes a tile in the
+// time one helper takes kHelperCost of a slice of it (measured at k = 1024, d = 128:
+// 2 C passes of scores, C of them with the accumulate).
+constexpr double kHelperCost = 1.86;
+
+void fwd_sm100_helpers(int d, int C, int G, int sms, int* H, int* share) {
+  *H = 0;
+  *share = 0;
+  const int free_sms = sms - G * C;
+  if (d != 128 || C < 2 || free_sms < 4) return;
+  const double rate = (double)free_sms / (C * kHelperCost);  // helper tiles per cluster tile
+  *H = free_sms;
+  *share = (int)std::lround(1024.0 * rate / (G + rate));
+}
+
 cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream) {
   if (a.d == 64) return launch_fwd_sm100_t<64, 4, 2>(a, stream);
-  return stages_for(a.d, a.C) == 4 ? launch_fwd_sm100_t<128, 4, 1>(a, stream)
-                                   : launch_fwd_sm100_t<128, 3, 1>(a, stream);
+  cudaError_t e = stages_for(a.d, a.C) == 4 ? launch_fwd_sm100_t<128, 4, 1>(a, stream)
+                                            : launch_fwd_sm100_t<128, 3, 1>(a, stream);
+  if (e != cudaSuccess || a.H <= 0) return e;
+  // the helper grid, queued behind the clustered one with programmatic serialization: it
+  // starts once every cluster is resident (their CTAs trigger it after setup), so it can
+  // only take the SMs that no cluster fits on, and it completes after the clustered grid
+  auto kern = sa_fwd_sm100_helper_kernel<128>;
+  cudaFuncAttributes fa;
+  e = cudaFuncGetAttributes(&fa, kern);
+  if (e != cudaSuccess) return e;
+  if (fa.numRegs < kHelperRegsLaunch) return cudaErrorInvalidConfiguration;  // see the split
+  const size_t smem = helper_smem_bytes<128>();
+  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)a.H);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, *a.tmap_x, *a.tmap_p, a.offsets, a.R, a.k_valid, a.C,
+                            a.k_pad, a.hdr, a.tile_start, a.part_u, a.part_m, a.lse, a.G, a.H,
+                            a.share, a.budget);
 }
 
 }  // namespace sa

@@ -70,6 +70,7 @@ sa_status tc_clusters(const Device& dev, int d, int C, int* G, int which = 0) {
 struct Plan {
   bool tc = false;  // tcgen05 path
   int C = 0, k_pad = 0, G = 0, Gb = 0;
+  int H = 0, share = 0;  // forward helper CTAs and their share of the tiles (1/1024)
   size_t hdr = 0, ts = 0, pf = 0, pu = 0, pm = 0, lse2 = 0;
   size_t pn = 0, gt = 0, gh = 0, cj = 0, lseb = 0, db = 0, dppp = 0, dpp = 0, wvp = 0;
   // tensor-core finalize (bf16 forward, k a multiple of 128): U / mass as bf16 hi + lo
@@ -100,6 +101,7 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
     q.C = (k + 127) / 128;
     q.k_pad = q.C * 128;
     if ((st = tc_clusters(dev, d, q.C, &q.G)) != SA_OK) return st;
+    fwd_sm100_helpers(d, q.C, q.G, dev.sms, &q.H, &q.share);
   } else {
     q.k_pad = (k + 31) / 32 * 32;
     const int pblocks = q.k_pad / 32;
@@ -116,7 +118,7 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
   q.ts = take((size_t)(R + 1) * sizeof(long long));
   if (!backward) {
     q.pf = take((size_t)q.k_pad * d * (dt == SA_BF16 ? 2 : 4));
-    const size_t segs = (size_t)q.G + (size_t)R;
+    const size_t segs = (size_t)q.G + (size_t)q.H + (size_t)R;
     q.pu = take(segs * q.k_pad * d * sizeof(float));
     q.pm = take(segs * q.k_pad * sizeof(float));
     if (!q.tc) q.lse2 = take((size_t)n_total * sizeof(float));
@@ -284,6 +286,8 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
       a.k_pad = p.k_pad;
       a.d = d;
       a.G = p.G;
+      a.H = p.H;
+      a.share = p.share;
       a.hdr = hdr;
       a.tile_start = ts;
       a.part_u = pu;
@@ -327,6 +331,8 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   f.k_pad = p.k_pad;
   f.d = d;
   f.G = p.G;
+  f.H = p.H;
+  f.share = p.share;
   f.mass_lanes = 1;
   f.sketch = sketch;
   f.mass = mass;
@@ -703,7 +709,8 @@ int sa_sketch_debug_gemm(const void* A, int a_mn, const void* B, int b_mn, int M
   return cuda_status(launch_gemm(g, static_cast<cudaStream_t>(stream_)));
 }
 
-int sa_sketch_forward_grid(int k, int d, sa_dtype dt, int* clusters, int* cluster_size) {
+int sa_sketch_forward_grid(int k, int d, sa_dtype dt, int* clusters, int* cluster_size,
+                           int* helpers, int* helper_share) {
   if (!clusters || !cluster_size) return SA_ERR_INVALID_ARG;
   sa_status st = check_sizes(0, 0, k, d, dt);
   if (st != SA_OK) return st;
@@ -713,6 +720,8 @@ int sa_sketch_forward_grid(int k, int d, sa_dtype dt, int* clusters, int* cluste
   if ((st = make_plan(dev, 0, 0, k, d, dt, false, &p)) != SA_OK) return st;
   *clusters = p.tc ? p.G : 0;
   *cluster_size = p.tc ? p.C : 0;
+  if (helpers) *helpers = p.tc ? p.H : 0;
+  if (helper_share) *helper_share = p.tc ? p.share : 0;
   return SA_OK;
 }
 

@@ -31,6 +31,7 @@ struct FinalizeArgs {
   const void* Wv;
   sa_dtype dt;
   int R, k, k_pad, d, G;
+  int H = 0, share = 0;  // helper ranges and their share of the tiles (TileRanges)
   int mass_lanes;       // partial masses per prototype and segment, summed in order
   float* sketch;
   float* mass;
@@ -54,6 +55,7 @@ struct FwdSm100Args {
   const CUtensorMap* tmap_p;
   const int64_t* offsets;
   int R, k_valid, C, k_pad, d, G;
+  int H = 0, share = 0;  // helper CTAs and their share of the tiles (TileRanges); 0: none
   WsHeader* hdr;
   const long long* tile_start;
   float* part_u;
@@ -62,6 +64,10 @@ struct FwdSm100Args {
   long long budget;
 };
 cudaError_t fwd_sm100_max_clusters(int d, int C, int* n);
+// Helper CTAs for the SMs that G clusters of C CTAs leave free, and their share of the
+// tiles in 1/1024 (H = 0: none).
+void fwd_sm100_helpers(int d, int C, int G, int sms, int* H, int* share);
+// The clustered grid, then (a.H > 0) the helper grid, both on `stream`.
 cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream);
 
 // ---- SIMT fp32 forward

@@ -79,20 +79,9 @@ template <>
 __device__ __forceinline__ float to_f<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
 
 // ------------------------------------------------------------------ finalize (helpers)
-// A user's segments are the clusters whose tile range intersects the user's tiles; their
-// partials are added in cluster order, so the result does not depend on timing. Then
-// sketch_j = (U_j Wv) / mass_j, with mass_j = 0 -> 0.
-__device__ __forceinline__ long long range_start(long long g, long long T, int G) {
-  return g * T / G;
-}
-
-__device__ int cluster_of_tile(long long x, long long T, int G) {
-  long long g = x * G / T;
-  if (g >= G) g = G - 1;
-  while (g + 1 < G && range_start(g + 1, T, G) <= x) ++g;
-  while (g > 0 && range_start(g, T, G) > x) --g;
-  return (int)g;
-}
+// A user's segments are the tile ranges (TileRanges: clusters, then helper CTAs) that
+// intersect the user's tiles; their partials are added in range order, so the result does
+// not depend on timing. Then sketch_j = (U_j Wv) / mass_j, with mass_j = 0 -> 0.
 
 // ------------------------------------------------------------------ tiled row GEMM
 // out[j][e] = sum_c lr[j][c] * rm[c][e] for a tile of 64 rows j and D columns e, both
@@ -212,7 +201,7 @@ __global__ void __launch_bounds__(256) fold_tiled_kernel(const TIn* __restrict__
 }
 
 // finalize, tiled: block = (user u, 64 prototypes). Adds the user's segment partials in
-// cluster order (deterministic), writes xsketch = U and mass, then sketch = U Wv / mass.
+// range order (deterministic), writes xsketch = U and mass, then sketch = U Wv / mass.
 template <int D, typename TIn>
 __global__ void __launch_bounds__(256) finalize_tiled_kernel(FinalizeArgs a, const TIn* __restrict__ Wv) {
   using S = TileShape<D>;
@@ -231,9 +220,10 @@ __global__ void __launch_bounds__(256) finalize_tiled_kernel(FinalizeArgs a, con
 #pragma unroll
   for (int q = 0; q < kRowTile * kV / 256; ++q) us[q] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (x1 > x0) {
-    const int g0 = cluster_of_tile(x0, T, a.G), g1 = cluster_of_tile(x1 - 1, T, a.G);
+    const TileRanges rg(T, a.G, a.H, a.share);
+    const int g0 = rg.of_tile(x0), g1 = rg.of_tile(x1 - 1);
     for (int g = g0; g <= g1; ++g) {
-      if (range_start(g, T, a.G) == range_start(g + 1, T, a.G)) continue;  // empty range
+      if (rg.start(g) == rg.start(g + 1)) continue;  // empty range
       const size_t seg = (size_t)g + u;
       const float4* src = reinterpret_cast<const float4*>(a.part_u + (seg * a.k_pad + j0) * D);
 #pragma unroll
@@ -281,7 +271,7 @@ __global__ void __launch_bounds__(256) finalize_tiled_kernel(FinalizeArgs a, con
 }
 
 // finalize, split: block = (user u, 64 prototypes). Adds the user's segment partials in
-// cluster order (deterministic), writes xsketch = U and mass, and U / mass (0 where
+// range order (deterministic), writes xsketch = U and mass, and U / mass (0 where
 // mass = 0) as a bf16 pair hi + lo with hi + lo = U / mass to about 16 bits; the product
 // with Wv runs on the tensor cores as two accumulated GEMM phases (hi Wv + lo Wv).
 template <int D>
@@ -299,9 +289,10 @@ __global__ void __launch_bounds__(256) finalize_split_kernel(FinalizeArgs a) {
 #pragma unroll
   for (int q = 0; q < kQ; ++q) us[q] = make_float4(0.f, 0.f, 0.f, 0.f);
   if (x1 > x0) {
-    const int g0 = cluster_of_tile(x0, T, a.G), g1 = cluster_of_tile(x1 - 1, T, a.G);
+    const TileRanges rg(T, a.G, a.H, a.share);
+    const int g0 = rg.of_tile(x0), g1 = rg.of_tile(x1 - 1);
     for (int g = g0; g <= g1; ++g) {
-      if (range_start(g, T, a.G) == range_start(g + 1, T, a.G)) continue;  // empty range
+      if (rg.start(g) == rg.start(g + 1)) continue;  // empty range
       const size_t seg = (size_t)g + u;
       const float4* src = reinterpret_cast<const float4*>(a.part_u + (seg * a.k_pad + j0) * D);
 #pragma unroll

@@ -26,6 +26,13 @@ pytestmark = pytest.mark.gpu
     ([130], 64, 64),
     ([4100, 3], 512, 128),
     ([100, 200, 129, 60, 300, 1, 128, 257, 90, 5000, 2, 383, 384, 385], 1024, 128),
+    # launches with helper CTAs beside the clusters (C = 8; C = 5 and 6 where clusters of
+    # that size leave SMs free): users cut between clusters and helpers, and a user without
+    # tokens in the helper ranges
+    ([20000, 0, 15000, 129, 7000], 1024, 128),
+    ([30000, 700, 20000], 640, 128),
+    ([9000, 25000, 1, 12000], 768, 128),
+    ([11000, 4000, 0, 9000], 1000, 128),
 ])
 def test_bf16_small_full_compare(lengths, k, d):
     w = inputs.make_workload(lengths, d, k, "bf16", seed=11 + k + d + len(lengths))
@@ -62,19 +69,38 @@ def _unit_mass_all_users(w, out):
     np.testing.assert_allclose(mass, n, rtol=2e-3)
 
 
-def _boundary_users(w, k, d):
-    """Users whose tiles straddle a bound between two clusters' tile ranges of the
-    persistent forward grid: two clusters accumulate parts of them, which the finalize
-    sums. Longest first."""
+def _range_bounds(T, k, d):
+    """Inner bounds between the forward's tile ranges (clusters, then helper CTAs), from
+    the launch shape the library reports."""
     from prototype_sketch_attention_b200 import binding
-    G, _ = binding.forward_grid(k, d)
+    G, _, H, share = binding.forward_grid(k, d)
+    Th = (T * share) >> 10 if H > 0 else 0
+    T1 = T - Th
+    bounds = [g * T1 // G for g in range(1, G)]
+    if Th > 0:
+        bounds += [T1] + [T1 + b * Th // H for b in range(1, H)]
+    return bounds, T1
+
+
+def _boundary_users(w, k, d):
+    """Users whose tiles straddle a bound between two tile ranges of the persistent
+    forward grid: two clusters (or helper CTAs) accumulate parts of them, which the
+    finalize sums. Longest first."""
     tiles = (np.diff(w.offsets.numpy()) + 127) // 128
     ts = np.concatenate([[0], np.cumsum(tiles)])
-    T = int(ts[-1])
-    bounds = [g * T // G for g in range(1, G)]
+    bounds, _ = _range_bounds(int(ts[-1]), k, d)
     users = {int(np.searchsorted(ts, b, side="right") - 1) for b in bounds}
     users = [u for u in users if any(ts[u] < b < ts[u + 1] for b in bounds)]
     return sorted(users, key=lambda u: -int(tiles[u]))
+
+
+def _helper_users(w, k, d):
+    """The user cut at the first helper tile and the users whose tiles are all helper
+    tiles (empty when the launch has no helper CTAs)."""
+    tiles = (np.diff(w.offsets.numpy()) + 127) // 128
+    ts = np.concatenate([[0], np.cumsum(tiles)])
+    _, T1 = _range_bounds(int(ts[-1]), k, d)
+    return [u for u in range(w.R) if tiles[u] > 0 and ts[u + 1] > T1]
 
 
 def test_config3_sampled_users():
@@ -85,7 +111,9 @@ def test_config3_sampled_users():
     order = np.argsort(w.lengths)
     cut = _boundary_users(w, w.k, w.d)
     assert cut, "the batch spans several clusters"
+    helper = _helper_users(w, w.k, w.d)
     users = {int(order[0]), int(order[len(order) // 2]), int(order[-1]), cut[0]}
+    users |= set(helper[:1] + helper[-1:])
     check_forward(w, out, users=sorted(users))
 
 
@@ -98,7 +126,8 @@ def test_config5_forward_sampled_users():
     _unit_mass_all_users(w, out)
     cut = _boundary_users(w, w.k, w.d)
     assert len(cut) >= 2, "the batch spans several clusters"
-    check_forward(w, out, users=sorted({0, 19, 39, cut[0], cut[-1]}))
+    helper = _helper_users(w, w.k, w.d)
+    check_forward(w, out, users=sorted({0, 19, 39, cut[0], cut[-1]} | set(helper[:2])))
 
 
 @pytest.mark.parametrize("k", [256, 512, 1024, 2048])
@@ -214,3 +243,12 @@ def test_bf16_extreme_scores_take_the_shifted_path():
     normal[idx.numpy()] = False
     assert np.abs(lse[normal] - ref["lse"][normal]).max() <= BF16_ABS
     assert np.abs(lse[~normal] - ref["lse"][~normal]).max() <= 1.0  # same dominant score
+
+
+def test_headline_launch_has_helper_ctas():
+    """k = 1024 on a B200: clusters of 8 leave SMs free, and helper CTAs take them (the
+    parity cases above with k = 1024 therefore cover the helper kernel)."""
+    from prototype_sketch_attention_b200 import binding
+    G, C, H, share = binding.forward_grid(1024, 128)
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert C == 8 and H == sms - G * C and H > 0 and 0 < share < 1024
