@@ -563,7 +563,7 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
 //     [U_s | mass_s] += A [X | 1] (MMA2) in TMEM; when the slice's pass over the chunk ends,
 //     or the tile stream crosses a user boundary, the partial is stored into (first time)
 //     or added to the workspace segment (range G + b, user).
-// The scores are computed twice, so a helper tile costs about 1.5 times a cluster CTA's
+// The scores are computed twice, so a helper tile costs about 1.7 times a cluster CTA's
 // share of one. The kChunk X tiles of a chunk come from HBM once and from L2 for the
 // other 2C - 1 passes.
 //
@@ -578,23 +578,25 @@ constexpr int kChunk = 32;  // tiles per chunk
 // sums, so they take 224 registers and the producer / MMA warpgroup gives up all but 56.
 // setmaxnreg.inc waits until the block's launch allocation covers it, so the split adds up
 // to exactly 384 threads x 168 registers, and the launch refuses a build compiled to fewer.
-constexpr int kHelperRegsLaunch = 168, kHelperRegsControl = 56, kHelperRegsSoftmax = 224;
+constexpr int kHelperRegsLaunch = 168, kHelperRegsControl = 64, kHelperRegsSoftmax = 216;
 static_assert(128 * kHelperRegsControl + 256 * kHelperRegsSoftmax <= kThreads * kHelperRegsLaunch,
               "register split exceeds the launch allocation");
 
+// Shared memory: the clustered kernel's four-stage layout (X stages, A tile, ones atom,
+// P' slice), then the running lse2. In pass 2 an X stage is held until the accumulate MMA
+// has read it, so the next loads need four stages to hide their L2 latency; that leaves
+// room for one P' buffer, which warp 3 reloads between (pass, slice) groups.
 template <int D>
 struct HelperSmem {
-  using X = FwdSmem<D, 3, 1>;  // the three-stage clustered layout: X stages, A tile, ones atom
-  static constexpr int oP0 = X::oP;                 // P' slice, buffer 0
-  static constexpr int oP1 = X::oP + X::kPBytes;    // P' slice, buffer 1
-  static constexpr int oL = oP1 + X::kPBytes;       // running lse2, [kChunk][128] floats
+  using X = FwdSmem<D, 4, 1>;
+  static constexpr int oL = X::oP + X::kPBytes;  // running lse2, [kChunk][128] floats
   static constexpr int oBars = oL + kChunk * kTileTokens * 4;
 };
 
 struct HBars {
-  uint64_t x_full[3], x_empty[3];
+  uint64_t x_full[4], x_empty[4];
   uint64_t s_full[2], s_empty[2];
-  uint64_t p_full[2], p_empty[2];
+  uint64_t p_full, p_empty;
   uint64_t a_full, a_empty[4];  // a_empty[i2 mod 4]: MMA2 of pass-2 step i2 has completed
   uint64_t u_full, u_empty;
   uint64_t m2iss[4];
@@ -616,9 +618,9 @@ sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
                            float* __restrict__ part_u, float* __restrict__ part_m,
                            float* __restrict__ lse_out, int G, int H, int share,
                            long long budget) {
-  using L = FwdSmem<D, 3, 1>;
+  using L = FwdSmem<D, 4, 1>;
   using HS = HelperSmem<D>;
-  constexpr int NS = 3;
+  constexpr int NS = 4;
   constexpr int KSTEPS1 = D / 16;
   constexpr int KSTEPS2 = kTileTokens / 16;
   extern __shared__ uint8_t smem_raw[];
@@ -639,9 +641,9 @@ sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
     for (int s = 0; s < 2; ++s) {
       mbar_init(smem_u32(&bars->s_full[s]), 1);
       mbar_init(smem_u32(&bars->s_empty[s]), 4);
-      mbar_init(smem_u32(&bars->p_full[s]), 1);
-      mbar_init(smem_u32(&bars->p_empty[s]), 1);
     }
+    mbar_init(smem_u32(&bars->p_full), 1);
+    mbar_init(smem_u32(&bars->p_empty), 1);
     mbar_init(smem_u32(&bars->a_full), 4);
     for (int s = 0; s < 4; ++s) {
       mbar_init(smem_u32(&bars->a_empty[s]), 1);
@@ -675,33 +677,21 @@ sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
   // compiler budgets every role's code for that role's count
   if (warp == 0) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegsControl));
-    // ================= TMA producer: per (pass, slice) the P' slice, per step the X tile;
-    // the next chunk's tiles are prefetched into L2 during the current chunk's last slice
+    // ================= X producer: per step the X tile; the next chunk's tiles are
+    // prefetched into L2 during the current chunk's last slice
     if (lane == 0 && ra < rb) {
       tma_prefetch_desc(&tmap_x);
-      tma_prefetch_desc(&tmap_p);
       TileIter base, ahead, it;
       base.init(tile_start, offsets, R, ra, rb);
       ahead = base;
       for (int j = 0; j < kChunk && ahead.valid(); ++j, ahead.next())
         for (int b = 0; b < L::kXBoxes; ++b) tma_prefetch_l2_2d(&tmap_x, b * 64, (int)ahead.t0());
-      int i = 0, q = 0;
+      int i = 0;
       bool ok = true;
       for (long long c0 = ra; ok && c0 < rb; c0 += kChunk) {
         const int K = (int)(rb - c0 < kChunk ? rb - c0 : kChunk);
         for (int ph = 0; ok && ph < 2; ++ph) {
           for (int s = 0; ok && s < C; ++s) {
-            const int pb = q & 1;
-            if (!mbar_wait(smem_u32(&bars->p_empty[pb]), (uint32_t)(((q >> 1) & 1) ^ 1), status, budget)) {
-              ok = false;
-              break;
-            }
-            const uint32_t pf = smem_u32(&bars->p_full[pb]);
-            mbar_arrive_expect_tx(pf, L::kPBytes);
-            for (int b = 0; b < D / 64; ++b)
-              tma_load_2d(sbase + (pb ? HS::oP1 : HS::oP0) + b * L::kSlot, &tmap_p, b * 64,
-                          s * kProtoSlice, pf);
-            ++q;
             const bool track = ph == 0 && s == 0, pref = ph == 1 && s == C - 1;
             if (track) ahead = base;
             it = base;
@@ -728,11 +718,9 @@ sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
         }
         base = it;
       }
-      // drain: the last NS X loads and the last two P' loads have landed before exit
+      // drain: the last NS X loads have landed before exit
       for (int j = (i > NS ? i - NS : 0); j < i; ++j)
         mbar_wait_drain(smem_u32(&bars->x_full[j % NS]), (uint32_t)((j / NS) & 1), budget);
-      for (int g = (q > 2 ? q - 2 : 0); g < q; ++g)
-        mbar_wait_drain(smem_u32(&bars->p_full[g & 1]), (uint32_t)((g >> 1) & 1), budget);
     }
   } else if (warp == 1) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegsControl));
@@ -742,20 +730,17 @@ sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
     // far the A buffer's barriers can lag behind a softmax warpgroup's wait).
     if (lane == 0 && ra < rb) {
       const uint32_t idesc1 = idesc_bf16_f32(128, kProtoSlice, 0, 0);
-      const uint64_t dp0 = smem_desc(sbase + HS::oP0, 16, 1024, kSwizzle128B);
-      const uint64_t dp1 = smem_desc(sbase + HS::oP1, 16, 1024, kSwizzle128B);
+      const uint64_t dp = smem_desc(sbase + L::oP, 16, 1024, kSwizzle128B);
       int i = 0, q = 0, i2 = 0, nb0 = 0, nb1 = 0;
       bool ok = true;
       for (long long c0 = ra; ok && c0 < rb; c0 += kChunk) {
         const int K = (int)(rb - c0 < kChunk ? rb - c0 : kChunk);
         for (int ph = 0; ok && ph < 2; ++ph) {
           for (int s = 0; ok && s < C; ++s, ++q) {
-            const int pb = q & 1;
-            if (!mbar_wait(smem_u32(&bars->p_full[pb]), (uint32_t)((q >> 1) & 1), status, budget)) {
+            if (!mbar_wait(smem_u32(&bars->p_full), (uint32_t)(q & 1), status, budget)) {
               ok = false;
               break;
             }
-            const uint64_t dp = pb ? dp1 : dp0;
             for (int tl = 0; tl < K; ++tl, ++i) {
               const int st = i % NS, sb = tl & 1;
               const int nbs = sb ? nb1 : nb0;
@@ -781,7 +766,7 @@ sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
               }
               tc_commit(smem_u32(&bars->s_full[sb]));
               if (ph == 0) tc_commit(smem_u32(&bars->x_empty[st]));  // pass 1: X is done
-              if (tl == K - 1) tc_commit(smem_u32(&bars->p_empty[pb]));
+              if (tl == K - 1) tc_commit(smem_u32(&bars->p_empty));  // P' slice is done
               if (sb) ++nb1; else ++nb0;
               if (ph == 1) ++i2;
             }
@@ -838,6 +823,26 @@ sa_fwd_sm100_helper_kernel(const __grid_constant__ CUtensorMap tmap_x,
     }
   } else if (warp == 3) {
     asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kHelperRegsControl));
+    // ================= P' producer: the slice of each (pass, slice) group, once MMA1 has
+    // finished with the previous group's
+    if (lane == 0 && ra < rb) {
+      tma_prefetch_desc(&tmap_p);
+      int q = 0;
+      bool ok = true;
+      for (long long c0 = ra; ok && c0 < rb; c0 += kChunk)
+        for (int ph = 0; ok && ph < 2; ++ph)
+          for (int s = 0; s < C; ++s, ++q) {
+            if (!mbar_wait(smem_u32(&bars->p_empty), (uint32_t)((q & 1) ^ 1), status, budget)) {
+              ok = false;
+              break;
+            }
+            const uint32_t pf = smem_u32(&bars->p_full);
+            mbar_arrive_expect_tx(pf, L::kPBytes);
+            for (int b = 0; b < D / 64; ++b)
+              tma_load_2d(sbase + L::oP + b * L::kSlot, &tmap_p, b * 64, s * kProtoSlice, pf);
+          }
+      if (q > 0) mbar_wait_drain(smem_u32(&bars->p_full), (uint32_t)((q - 1) & 1), budget);
+    }
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kHelperRegsSoftmax));
     // ================= softmax warpgroups (tile parity) + segment epilogues (warpgroup 0)
@@ -1052,9 +1057,11 @@ cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
 }
 
 // The helpers' share of the tiles balances the two grids: a cluster takes a tile in the
-// time one helper takes kHelperCost of a slice of it (measured at k = 1024, d = 128:
-// 2 C passes of scores, C of them with the accumulate).
-constexpr double kHelperCost = 1.86;
+// time one helper takes kHelperCost of a slice of it (2 C passes of scores, C of them
+// with the accumulate). Measured on a B200 at k = 1024, d = 128: a helper tile takes
+// 17.2 us against 1.27 us per tile for a cluster, so 1.70 per slice; a larger share makes
+// the helpers finish last, a smaller one the clusters.
+constexpr double kHelperCost = 1.70;
 
 void fwd_sm100_helpers(int d, int C, int G, int sms, int* H, int* share) {
   *H = 0;

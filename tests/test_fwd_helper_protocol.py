@@ -1,8 +1,9 @@
 """CPU model of the forward helper kernel's barrier protocol (csrc/sa_fwd_sm100.cu,
 sa_fwd_sm100_helper_kernel): one helper CTA walks its tile range in chunks; per chunk,
 pass 1 runs the score MMA and the partial log-sums for every (slice, tile), pass 2 the
-score MMA again, the A store and the accumulate MMA. Roles as coroutines: the TMA
-producer (P' slice per (pass, slice), X tile per step), the score-MMA and accumulate-MMA
+score MMA again, the A store and the accumulate MMA. Roles as coroutines: the X producer
+(four stages, one tile per step), the P' producer (one buffer, one slice per (pass,
+slice) group), the score-MMA and accumulate-MMA
 issuers (one in-order tensor pipe), and the two softmax warpgroups (tile parity), of
 which warpgroup 0 also runs every segment epilogue; a warpgroup hands its score buffer
 back as soon as it has read the scores. TMA landings and pipe completions
@@ -31,7 +32,7 @@ def run_helper(owner, ra, rb, C, chunk, seed, single_a_barrier=False, epilogue_b
     """owner[g]: user of global tile g; the CTA's range is tiles [ra, rb)."""
     rnd = random.Random(seed)
     later, issue, run = _engine(rnd)
-    NS = 3
+    NS = 4
     first_tile = {}
     for g, u in enumerate(owner):
         first_tile.setdefault(u, g)
@@ -43,10 +44,10 @@ def run_helper(owner, ra, rb, C, chunk, seed, single_a_barrier=False, epilogue_b
                 for tl in range(K):
                     step_of[(ci, ph, s, tl)] = len(step_of)
     st = dict(x_full=[Bar(1) for _ in range(NS)], x_empty=[Bar(1) for _ in range(NS)],
-              s_full=[Bar(1), Bar(1)], s_empty=[Bar(4), Bar(4)], p_full=[Bar(1), Bar(1)],
-              p_empty=[Bar(1), Bar(1)], a_full=Bar(4), a_empty=[Bar(1) for _ in range(4)],
+              s_full=[Bar(1), Bar(1)], s_empty=[Bar(4), Bar(4)], p_full=Bar(1),
+              p_empty=Bar(1), a_full=Bar(4), a_empty=[Bar(1) for _ in range(4)],
               u_full=Bar(1), u_empty=Bar(4), m2iss=[Bar(1) for _ in range(4)],
-              xstage=[None] * NS, xuse=[0] * NS, pbuf=[None, None], puse=[0, 0],
+              xstage=[None] * NS, xuse=[0] * NS, pbuf=[None], puse=[0],
               S=[None, None], s_held=[False, False], A=[None], a_use=[0],
               U=dict(seg=None, done=False, read=True), L={}, out={})
 
@@ -54,20 +55,10 @@ def run_helper(owner, ra, rb, C, chunk, seed, single_a_barrier=False, epilogue_b
         return tl == K - 1 or g == rb - 1 or owner[g + 1] != owner[g]
 
     def producer():
-        i = q = 0
+        i = 0
         for ci, (c0, K) in enumerate(chunks):
             for ph in range(2):
                 for s in range(C):
-                    pb = q & 1
-                    yield lambda: st["p_empty"][pb].passes(((q >> 1) & 1) ^ 1)
-                    st["p_full"][pb].arrive_expect_tx(1)
-
-                    def land_p(q=q, pb=pb):
-                        check(st["puse"][pb] == 0, f"P' load of group {q} overwrote buffer {pb} in use")
-                        st["pbuf"][pb] = q
-                        st["p_full"][pb].complete_tx(1)
-                    later(land_p)
-                    q += 1
                     for tl in range(K):
                         sg = i % NS
                         yield lambda: st["x_empty"][sg].passes(((i // NS) & 1) ^ 1)
@@ -80,14 +71,29 @@ def run_helper(owner, ra, rb, C, chunk, seed, single_a_barrier=False, epilogue_b
                         later(land)
                         i += 1
 
+    def p_producer():
+        q = 0
+        for ci, (c0, K) in enumerate(chunks):
+            for ph in range(2):
+                for s in range(C):
+                    yield lambda: st["p_empty"].passes((q & 1) ^ 1)
+                    st["p_full"].arrive_expect_tx(1)
+
+                    def land_p(q=q):
+                        check(st["puse"][0] == 0, f"P' load of group {q} overwrote the buffer in use")
+                        st["pbuf"][0] = q
+                        st["p_full"].complete_tx(1)
+                    later(land_p)
+                    q += 1
+
     def mma1():
         i = q = i2 = 0
         nb = [0, 0]
         for ci, (c0, K) in enumerate(chunks):
             for ph in range(2):
                 for s in range(C):
-                    pb = q & 1
-                    yield lambda: st["p_full"][pb].passes((q >> 1) & 1)
+                    pb = 0
+                    yield lambda: st["p_full"].passes(q & 1)
                     for tl in range(K):
                         sg, sb = i % NS, tl & 1
                         nbs = nb[sb]
@@ -112,7 +118,7 @@ def run_helper(owner, ra, rb, C, chunk, seed, single_a_barrier=False, epilogue_b
                             if ph == 0:
                                 st["x_empty"][sg].arrive()
                             if lastp:
-                                st["p_empty"][pb].arrive()
+                                st["p_empty"].arrive()
                         issue(start, finish)
                         nb[sb] += 1
                         i += 1
@@ -217,7 +223,7 @@ def run_helper(owner, ra, rb, C, chunk, seed, single_a_barrier=False, epilogue_b
                                 st["u_empty"].arrive(4)
                             i2 += 1
 
-    run([producer(), mma1(), mma2(), softmax(0), softmax(1)])
+    run([producer(), p_producer(), mma1(), mma2(), softmax(0), softmax(1)])
     want = {}
     for g in range(ra, rb):
         for s in range(C):
