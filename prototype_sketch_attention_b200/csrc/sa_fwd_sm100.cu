@@ -575,9 +575,9 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
 // buffer's uses itself (chunks may have an odd number of tiles).
 constexpr int kChunk = 32;  // tiles per chunk
 // Register split: the softmax warpgroups hold a token's 128 scores through both passes'
-// sums, so they take 224 registers and the producer / MMA warpgroup gives up all but 56.
-// setmaxnreg.inc waits until the block's launch allocation covers it, so the split adds up
-// to exactly 384 threads x 168 registers, and the launch refuses a build compiled to fewer.
+// sums, so they take 216 registers and the producer / MMA warpgroup gives up all but 64.
+// setmaxnreg.inc waits until the block's launch allocation covers it, so the split stays
+// within 384 threads x 168 registers, and the launch refuses a build compiled to fewer.
 constexpr int kHelperRegsLaunch = 168, kHelperRegsControl = 64, kHelperRegsSoftmax = 216;
 static_assert(128 * kHelperRegsControl + 256 * kHelperRegsSoftmax <= kThreads * kHelperRegsLaunch,
               "register split exceeds the launch allocation");
