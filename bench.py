@@ -13,8 +13,10 @@ batch (users are independent; no collective on the data path), so scaling is wea
 `value` is total tokens / max-over-ranks time.
 
 The JSON line also carries:
-  roofline      the tcgen05 forward kernel alone: algorithmic FLOP per launch
-                (4*k*d per token) / its CUDA-event duration vs the measured bf16 peak
+  roofline      the tcgen05 forward kernels alone (the clustered grid and, on the SMs
+                clusters of 8 leave free, the helper grid beside it): algorithmic FLOP
+                per launch (4*k*d per token) / their CUDA-event duration vs the measured
+                bf16 peak
   e2e           the same metric through the C ABI with host buffers
                 (sa_sketch_forward_host): the per-step H2D of X and offsets and the D2H
                 of sketch and mass inside the timed region
@@ -718,6 +720,7 @@ def run_ours(args) -> None:
     peak, peak_src = measured_peak()
     flop_per_launch = 4.0 * k * d * n_total
     achieved = flop_per_launch / (kern_ms / 1e3) / 1e12
+    n_clusters, cluster_size, n_helpers, helper_share = binding.forward_grid(k, d)
     step_tflops = 4.0 * k * d * total_tokens / (ms_per_step / 1e3) / 1e12
     h2d = X.numel() * X.element_size() + off.numel() * 8
     d2h = R * k * d * 4 + R * k * 4  # sketch and mass back to the host
@@ -759,16 +762,20 @@ def run_ours(args) -> None:
         "step_tflops": step_tflops,
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": profiled_traffic(),
-                     "kernel": "sa_fwd_sm100_kernel<128>", "kernel_ms": kern_ms,
+                     "kernel": "sa_fwd_sm100_kernel<128,4,1> (%d clusters of %d) + "
+                               "sa_fwd_sm100_helper_kernel<128> (%d CTAs, %d/1024 of the tiles), "
+                               "concurrent" % (n_clusters, cluster_size, n_helpers, helper_share),
+                     "kernel_ms": kern_ms,
                      "peak_source": peak_src, "flop_per_launch": flop_per_launch,
                      "frac_of_sustained": (achieved / sustained_peak()
                                            if sustained_peak() else None),
                      "frac_of_datasheet": achieved / DATASHEET_BF16_TFLOPS},
         "e2e": {"value": total_tokens / (e2e_ms / 1e3), "unit": UNIT, "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
-        # per forward: schedule, fold, the tcgen05 kernel, then the finalize (segment sums
-        # and the U Wv GEMM on the tensor cores when k is a multiple of 128, else one kernel)
-        "gpu_launches": (5 if k % 128 == 0 else 4) * args.steps,
+        # per forward: schedule, fold, the tcgen05 kernel (and the helper grid when the
+        # clusters leave SMs free), then the finalize (segment sums and the U Wv GEMM on the
+        # tensor cores when k is a multiple of 128, else one kernel)
+        "gpu_launches": ((5 if k % 128 == 0 else 4) + (1 if n_helpers > 0 else 0)) * args.steps,
         "clocks": clk.summary(),
     }
     if cpu is not None:
