@@ -255,7 +255,8 @@ int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, int R, int6
  * *clusters clusters of *cluster_size CTAs (one CTA per 128 prototypes); when those
  * leave SMs free, *helpers helper CTAs (one per free SM, no cluster) run beside them and
  * take *helper_share / 1024 of the tiles. With T 128-token tiles in the batch (users'
- * tiles concatenated), Th = floor(T * helper_share / 1024) and T1 = T - Th, cluster g
+ * tiles concatenated), Th = floor(T * helper_share / 1024) (0 when that is less than
+ * 32 * helpers: the helpers take work only in full 32-tile chunks) and T1 = T - Th, cluster g
  * walks tiles [g T1 / clusters, (g + 1) T1 / clusters) and helper b walks
  * [T1 + b Th / helpers, T1 + (b + 1) Th / helpers). A user whose tiles straddle one of
  * those bounds is accumulated by two of them and summed in the finalize. For fp32

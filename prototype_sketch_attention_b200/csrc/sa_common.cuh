@@ -385,15 +385,22 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 // ---------------------------------------------------------------- tile ranges
 // The forward splits the token tiles [0, T) into G cluster ranges over [0, T1) and H helper
 // ranges over [T1, T) (helper CTAs run on the SMs that no cluster fits on). The helpers'
-// share is `share` / 1024 of the tiles: Th = floor(T share / 1024), T1 = T - Th. Range
-// g < G is [g T1 / G, (g + 1) T1 / G); range G + b is [T1 + b Th / H, T1 + (b + 1) Th / H).
-// The forward kernels and the finalize take the ranges from this one definition.
+// share is `share` / 1024 of the tiles: Th = floor(T share / 1024), T1 = T - Th, except
+// that the helpers take no tiles (Th = 0) unless each gets at least kHelperMinTiles: a
+// helper pays a fixed cost per (pass, slice) group of a chunk, which only full chunks
+// amortise. Range g < G is [g T1 / G, (g + 1) T1 / G); range G + b is
+// [T1 + b Th / H, T1 + (b + 1) Th / H). The forward kernels and the finalize take the
+// ranges from this one definition.
+constexpr long long kHelperMinTiles = 32;
+__device__ __forceinline__ long long helper_tiles(long long T, int H, int share) {
+  const long long th = H > 0 ? (T * share) >> 10 : 0;
+  return th >= kHelperMinTiles * H ? th : 0;
+}
 struct TileRanges {
   long long T1, Th;
   int G, H;
   __device__ TileRanges(long long T, int G_, int H_, int share)
-      : T1(T - (H_ > 0 ? (T * share) >> 10 : 0)), Th(H_ > 0 ? (T * share) >> 10 : 0), G(G_),
-        H(H_) {}
+      : T1(T - helper_tiles(T, H_, share)), Th(helper_tiles(T, H_, share)), G(G_), H(H_) {}
   __device__ long long start(long long g) const {
     return g <= G ? g * T1 / G : T1 + (g - G) * Th / H;
   }

@@ -563,8 +563,8 @@ sa_fwd_sm100_kernel(const __grid_constant__ CUtensorMap tmap_x,
 //     [U_s | mass_s] += A [X | 1] (MMA2) in TMEM; when the slice's pass over the chunk ends,
 //     or the tile stream crosses a user boundary, the partial is stored into (first time)
 //     or added to the workspace segment (range G + b, user).
-// The scores are computed twice, so a helper tile costs about 1.7 times a cluster CTA's
-// share of one. The kChunk X tiles of a chunk come from HBM once and from L2 for the
+// The scores are computed twice, so a helper tile costs about 1.7 to 1.9 times a cluster
+// CTA's share of one. The kChunk X tiles of a chunk come from HBM once and from L2 for the
 // other 2C - 1 passes.
 //
 // Ownership rules that make the shared-memory and workspace accesses race-free: tile t of
@@ -1058,10 +1058,12 @@ cudaError_t fwd_sm100_max_clusters(int d, int C, int* n) {
 
 // The helpers' share of the tiles balances the two grids: a cluster takes a tile in the
 // time one helper takes kHelperCost of a slice of it (2 C passes of scores, C of them
-// with the accumulate). Measured on a B200 at k = 1024, d = 128: a helper tile takes
-// 17.2 us against 1.27 us per tile for a cluster, so 1.70 per slice; a larger share makes
-// the helpers finish last, a smaller one the clusters.
-constexpr double kHelperCost = 1.70;
+// with the accumulate). Measured on a B200 at k = 1024, d = 128: alone, a helper tile
+// takes 17.2 us against 1.27 us per tile for a cluster (1.70 per slice); beside the
+// clusters (shared L2 and power) the fastest split was 1.86, 114/1024 of the tiles
+// (shares 107 to 156 timed). A larger share makes the helpers finish last, a smaller one
+// the clusters.
+constexpr double kHelperCost = 1.86;
 
 void fwd_sm100_helpers(int d, int C, int G, int sms, int* H, int* share) {
   *H = 0;

@@ -26,9 +26,8 @@ pytestmark = pytest.mark.gpu
     ([130], 64, 64),
     ([4100, 3], 512, 128),
     ([100, 200, 129, 60, 300, 1, 128, 257, 90, 5000, 2, 383, 384, 385], 1024, 128),
-    # launches with helper CTAs beside the clusters (C = 8; C = 5 and 6 where clusters of
-    # that size leave SMs free): users cut between clusters and helpers, and a user without
-    # tokens in the helper ranges
+    # cluster sizes C = 5, 6 and 8 with more users and tiles per cluster (batches this
+    # small leave the helper grid idle: the full-size tests below cover it)
     ([20000, 0, 15000, 129, 7000], 1024, 128),
     ([30000, 700, 20000], 640, 128),
     ([9000, 25000, 1, 12000], 768, 128),
@@ -75,6 +74,8 @@ def _range_bounds(T, k, d):
     from prototype_sketch_attention_b200 import binding
     G, _, H, share = binding.forward_grid(k, d)
     Th = (T * share) >> 10 if H > 0 else 0
+    if Th < 32 * H:  # helpers take work only when each gets a full 32-tile chunk
+        Th = 0
     T1 = T - Th
     bounds = [g * T1 // G for g in range(1, G)]
     if Th > 0:
@@ -112,6 +113,7 @@ def test_config3_sampled_users():
     cut = _boundary_users(w, w.k, w.d)
     assert cut, "the batch spans several clusters"
     helper = _helper_users(w, w.k, w.d)
+    assert helper, "the batch reaches the helper grid"
     users = {int(order[0]), int(order[len(order) // 2]), int(order[-1]), cut[0]}
     users |= set(helper[:1] + helper[-1:])
     check_forward(w, out, users=sorted(users))
@@ -127,20 +129,24 @@ def test_config5_forward_sampled_users():
     cut = _boundary_users(w, w.k, w.d)
     assert len(cut) >= 2, "the batch spans several clusters"
     helper = _helper_users(w, w.k, w.d)
+    assert helper, "the batch reaches the helper grid"
     check_forward(w, out, users=sorted({0, 19, 39, cut[0], cut[-1]} | set(helper[:2])))
 
 
-@pytest.mark.parametrize("k", [256, 512, 1024, 2048])
+@pytest.mark.parametrize("k", [256, 512, 640, 768, 1024, 2048])
 def test_config4_sampled_users(k):
-    """The two shortest users, the median, the longest, and the longest user cut between
-    clusters."""
+    """The two shortest users, the median, the longest, the longest user cut between
+    clusters, and (where the launch has helper CTAs) the users cut at the first helper
+    tile and at the last."""
     w = inputs.make_config(4, k=k)
     _, out = gpu_forward(w)
     _unit_mass_all_users(w, out)
     order = np.argsort(w.lengths)
     cut = _boundary_users(w, k, w.d)
     assert cut, "the batch spans several clusters"
+    helper = _helper_users(w, k, w.d)
     users = {int(order[0]), int(order[1]), int(order[150]), int(order[-1]), cut[0]}
+    users |= set(helper[:1] + helper[-1:])
     check_forward(w, out, users=sorted(users))
 
 
