@@ -37,8 +37,8 @@ template <typename TIn>
 __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a, const TIn* __restrict__ Wv) {
   extern __shared__ float sm[];
   const int d = a.d, ld = d + 1;
-  float* wv = sm;              // [d][d+1]  wv[c][e] = Wv[c][e]
-  float* gt = wv + d * ld;     // [32][d]
+  float* gt = sm;              // [32][d]
+  float* wv = sm + kCP * d;    // [d][d+1]  wv[c][e] = Wv[c][e] (only without Gtlo)
   const int u = blockIdx.x, j0 = blockIdx.y * kCP;
   if (!a.Gtlo)  // W_v is needed here only when this kernel computes Gh itself
     for (int i = threadIdx.x; i < d * d; i += blockDim.x) wv[(i / d) * ld + (i % d)] = ldf(Wv, i);
@@ -66,14 +66,20 @@ __global__ void __launch_bounds__(256) bwd_prep_kernel(BwdArgs a, const TIn* __r
     if (a.Gh) a.Gh[o] = acc;
     if (a.Ghb) a.Ghb[o] = __float2bfloat16_rn(acc);
   }
-  if (threadIdx.x < kCP) {
-    const int j = j0 + threadIdx.x;
+  // c_j = Gt_j . sketch_j - dmass_j: each warp takes kCP / 8 rows, its lanes read the
+  // sketch row coalesced, and a shuffle tree adds the lanes
+  for (int jj = threadIdx.x >> 5; jj < kCP; jj += blockDim.x >> 5) {
+    const int j = j0 + jj, lane = threadIdx.x & 31;
     float v = 0.f;
-    if (j < a.k) {
-      for (int e = 0; e < d; ++e) v = fmaf(gt[threadIdx.x * d + e], a.sketch[((size_t)u * a.k + j) * d + e], v);
-      if (a.dmass) v -= a.dmass[(size_t)u * a.k + j];
+    if (j < a.k)
+      for (int e = lane; e < d; e += 32)
+        v = fmaf(gt[jj * d + e], a.sketch[((size_t)u * a.k + j) * d + e], v);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) {
+      if (j < a.k && a.dmass) v -= a.dmass[(size_t)u * a.k + j];
+      a.cj[(size_t)u * a.k_pad + j] = j < a.k ? v : 0.f;
     }
-    a.cj[(size_t)u * a.k_pad + j] = v;
   }
 }
 
@@ -348,32 +354,63 @@ __global__ void __launch_bounds__(256) bwd_wv_part_kernel(BwdArgs a) {
     a.wv_part[((size_t)blockIdx.x * d + cg + cs * i) * d + e] = acc[i];
 }
 
-// ---- finish: dWv = sum of chunks; dP = dPn Wk / sqrt(d); dWk = dPn^T P / sqrt(d)
+// ---- finish: dWv = sum of chunks; dP = dPn Wk / sqrt(d); dWk = dPn^T P / sqrt(d).
+// 256 threads; lane l covers the columns l + 32 q (q < d / 32), so each thread carries
+// d / 32 independent sums and loads. blockIdx.y = 0: dWv row blockIdx.x, the 8 warps
+// taking the chunks in turn; 1: dWk row blockIdx.x, the warps splitting the prototypes;
+// 2: dP rows 8 blockIdx.x + warp. Partial sums across warps are added in warp order.
 template <typename TIn>
-__global__ void bwd_finish_kernel(BwdArgs a, const TIn* __restrict__ P, const TIn* __restrict__ Wk,
-                                  int nchunks, float inv_sqrt_d) {
+__global__ void __launch_bounds__(256) bwd_finish_kernel(BwdArgs a, const TIn* __restrict__ P,
+                                                          const TIn* __restrict__ Wk, int nchunks,
+                                                          float inv_sqrt_d) {
   if (read_status(&a.hdr->status) != 0) return;
-  const int d = a.d;
-  const int which = blockIdx.y;  // 0: dWv rows, 1: dWk rows, 2: dP rows
-  const int row = blockIdx.x;
-  const int e = threadIdx.x;
-  if (e >= d) return;
-  if (which == 0) {
-    if (row >= d) return;
-    float v = 0.f;
-    for (int ch = 0; ch < nchunks; ++ch) v += a.wv_part[((size_t)ch * d + row) * d + e];
-    a.dWv[(size_t)row * d + e] = v;
-  } else if (which == 1) {
-    if (row >= d) return;
-    float v = 0.f;
-    for (int j = 0; j < a.k; ++j) v = fmaf(a.dpp[(size_t)j * d + row], ldf(P, (size_t)j * d + e), v);
-    a.dWk[(size_t)row * d + e] = v * inv_sqrt_d;
-  } else {
-    for (int j = row; j < a.k; j += gridDim.x) {
-      float v = 0.f;
-      for (int c = 0; c < d; ++c) v = fmaf(a.dpp[(size_t)j * d + c], ldf(Wk, (size_t)c * d + e), v);
-      a.dP[(size_t)j * d + e] = v * inv_sqrt_d;
+  __shared__ float red[8][128];
+  const int d = a.d, nq = d / 32;
+  const int which = blockIdx.y, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  if (which == 2) {
+    const int j = blockIdx.x * 8 + warp;
+    if (j >= a.k) return;
+#pragma unroll 4
+    for (int c = 0; c < d; ++c) {
+      const float g = a.dpp[(size_t)j * d + c];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < nq) acc[q] = fmaf(g, ldf(Wk, (size_t)c * d + lane + 32 * q), acc[q]);
     }
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      if (q < nq) a.dP[(size_t)j * d + lane + 32 * q] = acc[q] * inv_sqrt_d;
+    return;
+  }
+  const int row = blockIdx.x;
+  if (row >= d) return;  // uniform over the block
+  if (which == 0) {
+    for (int ch = warp; ch < nchunks; ch += 8)
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < nq) acc[q] += a.wv_part[((size_t)ch * d + row) * d + lane + 32 * q];
+  } else {
+    const int per = (a.k + 7) / 8, j0 = warp * per, j1 = min(a.k, j0 + per);
+#pragma unroll 4
+    for (int j = j0; j < j1; ++j) {
+      const float g = a.dpp[(size_t)j * d + row];
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        if (q < nq) acc[q] = fmaf(g, ldf(P, (size_t)j * d + lane + 32 * q), acc[q]);
+    }
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    if (q < nq) red[warp][lane + 32 * q] = acc[q];
+  __syncthreads();
+  if ((int)threadIdx.x < d) {
+    float v = 0.f;
+    for (int w = 0; w < 8; ++w) v += red[w][threadIdx.x];
+    if (which == 0)
+      a.dWv[(size_t)row * d + threadIdx.x] = v;
+    else
+      a.dWk[(size_t)row * d + threadIdx.x] = v * inv_sqrt_d;
   }
 }
 
@@ -397,7 +434,8 @@ template <typename TIn>
 static cudaError_t launch_prep(const BwdArgs& a, cudaStream_t s) {
   if (a.R == 0) return cudaSuccess;
   const int d = a.d;
-  const size_t smem = (size_t)(d * (d + 1) + kCP * d) * sizeof(float);
+  // W_v is staged only when this kernel forms Gh itself (no Gtlo)
+  const size_t smem = (size_t)((a.Gtlo ? 0 : d * (d + 1)) + kCP * d) * sizeof(float);
   cudaError_t e =
       cudaFuncSetAttribute(bwd_prep_kernel<TIn>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
@@ -420,7 +458,8 @@ static cudaError_t launch_tail(const BwdArgs& a, int wv_parts, cudaStream_t s) {
     bwd_wv_part_kernel<<<(unsigned)nch, 256, smem_w, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  bwd_finish_kernel<TIn><<<dim3((unsigned)d, 3), 128, 0, s>>>(
+  const int fx = d > (a.k + 7) / 8 ? d : (a.k + 7) / 8;  // d rows of dWv / dWk, k / 8 of dP
+  bwd_finish_kernel<TIn><<<dim3((unsigned)fx, 3), 256, 0, s>>>(
       a, static_cast<const TIn*>(a.P), static_cast<const TIn*>(a.Wk), nch, 1.0f / sqrtf((float)d));
   return cudaGetLastError();
 }
