@@ -258,3 +258,19 @@ def test_headline_launch_has_helper_ctas():
     G, C, H, share = binding.forward_grid(1024, 128)
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     assert C == 8 and H == sms - G * C and H > 0 and 0 < share < 1024
+
+
+@pytest.mark.parametrize("k", [1000, 1024])
+def test_helper_ranges_with_empty_and_short_users(k):
+    """A batch just large enough for the helper grid (each helper gets a full chunk),
+    whose helper ranges hold empty users, users shorter than one tile, a user cut at the
+    first helper tile and a long one; at k = 1000 the last prototype slice is partial.
+    Every user the helpers touch is compared with the oracle."""
+    lengths = [100000] * 10 + [0, 5, 0, 130, 2000, 0, 50000]
+    w = inputs.make_workload(lengths, 128, k, "bf16", seed=91 + k)
+    _, out = gpu_forward(w)
+    _unit_mass_all_users(w, out)
+    helper = _helper_users(w, k, w.d)
+    assert helper and helper[0] <= 9, "the helper ranges start inside the tenth long user"
+    users = set(range(helper[0], w.R))
+    check_forward(w, out, users=sorted(users))
