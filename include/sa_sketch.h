@@ -74,6 +74,10 @@ typedef enum {
  * sa_sketch_backward (backward = 1) needs for these sizes on the current device.
  * The plan depends on the device's SM count, so query it with the device current
  * that will run the call. Returns 0 if the sizes are unsupported.
+ * For the bf16 forward this is the plan with the helper grid (sa_sketch_forward_grid),
+ * whose helper CTAs add H segments of k_pad x (d + 1) floats. Given less than that but
+ * at least the plan without them, sa_sketch_forward runs the clustered grid alone
+ * (slower; same results to rounding).
  */
 size_t sa_sketch_workspace_size(int R, int64_t n_total, int k, int d, sa_dtype dt,
                                 int backward);
@@ -235,6 +239,8 @@ int sa_sketch_combine(const float* xsketch, const float* mass, int R, int k, int
  *    Serialise them, for instance on one stream.
  *  - Sizes whose plan needs more than SA_NOALLOC_SCRATCH_BYTES are rejected with
  *    SA_ERR_WORKSPACE before anything is launched (at k = 1024, d = 128 on a B200 about 24 users).
+ *    When the scratch holds the plan without the helper grid but not with it, the call
+ *    runs the clustered grid alone (see sa_sketch_forward's workspace).
  *  - It calls no cudaMalloc, cudaFree or allocating library routine.
  *  - device_status: nullable HOST pointer. When given, the call waits for `stream` and
  *    stores the device status word there (SA_OK, SA_ERR_BAD_OFFSETS, SA_ERR_TIMEOUT), since

@@ -91,8 +91,10 @@ sa_status check_sizes(int R, int64_t n_total, int k, int d, sa_dtype dt) {
   return SA_OK;
 }
 
+// helpers = false plans the bf16 forward without the helper grid (a smaller workspace:
+// no helper segments).
 sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_dtype dt,
-                    bool backward, Plan* p) {
+                    bool backward, Plan* p, bool helpers = true) {
   sa_status st = check_sizes(R, n_total, k, d, dt);
   if (st != SA_OK) return st;
   Plan q;
@@ -101,7 +103,7 @@ sa_status make_plan(const Device& dev, int R, int64_t n_total, int k, int d, sa_
     q.C = (k + 127) / 128;
     q.k_pad = q.C * 128;
     if ((st = tc_clusters(dev, d, q.C, &q.G)) != SA_OK) return st;
-    fwd_sm100_helpers(d, q.C, q.G, dev.sms, &q.H, &q.share);
+    if (helpers) fwd_sm100_helpers(d, q.C, q.G, dev.sms, &q.H, &q.share);
   } else {
     q.k_pad = (k + 31) / 32 * 32;
     const int pblocks = q.k_pad / 32;
@@ -215,6 +217,15 @@ cudaError_t prof_mark_stop(cudaStream_t s) {
   return g_prof_stop ? cudaEventRecord(g_prof_stop, s) : cudaSuccess;
 }
 
+// The forward's smallest workspace: the plan without the helper grid.
+size_t forward_workspace_min(int R, int64_t n_total, int k, int d, sa_dtype dt) {
+  Device dev;
+  if (current_device(&dev) != SA_OK) return 0;
+  Plan p;
+  if (make_plan(dev, R, n_total, k, d, dt, false, &p, false) != SA_OK) return 0;
+  return p.total;
+}
+
 // cuTensorMapEncodeTiled through the runtime's driver entry point (no -lcuda needed).
 PFN_cuTensorMapEncodeTiled_v12000 tmap_encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -257,6 +268,11 @@ int sa_sketch_forward(const void* X, const int64_t* offsets, int R, int64_t n_to
   if ((st = current_device(&dev)) != SA_OK) return st;
   Plan p;
   if ((st = make_plan(dev, R, n_total, k, d, dt, false, &p)) != SA_OK) return st;
+  // a workspace too small for the helper grid's segments but large enough without them
+  // runs the clustered grid alone
+  if (ws_bytes < p.total && p.H > 0 &&
+      (st = make_plan(dev, R, n_total, k, d, dt, false, &p, false)) != SA_OK)
+    return st;
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) % kAlign) != 0 || ws_bytes < p.total)
     return SA_ERR_WORKSPACE;
   cudaStream_t s = static_cast<cudaStream_t>(stream_);

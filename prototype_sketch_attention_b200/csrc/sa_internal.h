@@ -69,6 +69,9 @@ cudaError_t fwd_sm100_max_clusters(int d, int C, int* n);
 void fwd_sm100_helpers(int d, int C, int G, int sms, int* H, int* share);
 // The clustered grid, then (a.H > 0) the helper grid, both on `stream`.
 cudaError_t launch_fwd_sm100(const FwdSm100Args& a, cudaStream_t stream);
+// The smallest workspace sa_sketch_forward accepts for these sizes (no helper grid); 0 if
+// there is no plan.
+size_t forward_workspace_min(int R, int64_t n_total, int k, int d, sa_dtype dt);
 
 // ---- SIMT fp32 forward
 struct FwdSimtArgs {

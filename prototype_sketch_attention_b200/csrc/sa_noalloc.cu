@@ -12,6 +12,7 @@
 
 #include <mutex>
 
+#include "sa_internal.h"
 #include "sa_sketch.h"
 
 namespace {
@@ -55,7 +56,8 @@ extern "C" int sa_sketch_forward_noalloc(const void* X, const int64_t* offsets, 
                                          const void* Wk, const void* Wv, sa_dtype dt,
                                          float* sketch, float* mass, float* lse,
                                          float* xsketch, int* device_status, void* stream) {
-  const size_t need = sa_sketch_workspace_size(R, n_total, k, d, dt, 0);
+  // the forward runs without the helper grid when the scratch cannot hold its segments
+  const size_t need = sa::forward_workspace_min(R, n_total, k, d, dt);
   // No plan for these arguments: the regular forward fails the same checks before any
   // launch (it never reads a workspace it was not given) and returns their exact code.
   if (need == 0)

@@ -100,3 +100,29 @@ def test_noalloc_rejects_sizes_beyond_its_scratch():
         binding.SA_BF16, out.data_ptr(), m.data_ptr(), None, None, None,
         torch.cuda.current_stream().cuda_stream)
     assert rc == binding.SA_ERR_WORKSPACE
+
+
+def test_noalloc_runs_without_the_helper_grid_when_the_scratch_is_short():
+    """20 users x 60K tokens at k = 1024: with the helper grid's segments the plan needs
+    more than the 32 MiB scratch, without them it fits, so the call runs the clustered grid
+    alone. The regular forward (with the helper grid) and the oracle agree with it."""
+    from parity_util import check_forward
+    w = inputs.make_workload([60000] * 20, 128, 1024, "bf16", seed=4444)
+    g = {n: getattr(w, n).cuda() for n in ("X", "offsets", "P", "Wk", "Wv")}
+    R, n_total, d, k = w.R, w.n_total, w.d, w.k
+    _, _, H, _ = binding.forward_grid(k, d)
+    assert H > 0
+    assert binding.sa_sketch_workspace_size(R, n_total, k, d, binding.SA_BF16, 0) > (32 << 20)
+    out = {"sketch": torch.full((R, k, d), float("nan"), device="cuda"),
+           "mass": torch.full((R, k), float("nan"), device="cuda"),
+           "lse": torch.full((n_total,), float("nan"), device="cuda"),
+           "xsketch": torch.full((R, k, d), float("nan"), device="cuda")}
+    rc, st = _noalloc(g, R, n_total, d, k, out)
+    assert rc == binding.SA_OK and st == binding.SA_OK, (rc, st)
+    ref = binding.forward(g["X"], g["offsets"], g["P"], g["Wk"], g["Wv"])
+    for key in ("sketch", "mass"):
+        got = out[key].cpu().double().numpy()
+        exp = ref[key].cpu().double().numpy()
+        for u in range(R):
+            assert rel_l2(got[u], exp[u]) <= BF16_REL, (key, u)
+    check_forward(w, out, users=[0, R - 1])
