@@ -98,3 +98,26 @@ def test_sketch_branch_calls_replay_from_a_graph():
     for key in ("dQ", "dWq", "dWK", "dWV"):
         assert torch.equal(bout[key], ref_b[key]), key
     assert torch.allclose(bout["dS"], ref_b["dS"], rtol=1e-5, atol=1e-6)
+
+
+def test_forward_with_the_helper_grid_replays_from_a_graph():
+    """A batch large enough for the helper grid: the helper launch (programmatic stream
+    serialization behind the clustered grid) is captured with the rest and replayed."""
+    dev = torch.device("cuda")
+    lengths = [100000] * 10 + [50000]
+    from prototype_sketch_attention_b200 import binding as b
+    G, C, H, share = b.forward_grid(1024, 128)
+    T = sum((n + 127) // 128 for n in lengths)
+    assert H > 0 and (T * share) >> 10 >= 32 * H, "the batch reaches the helper grid"
+    w = inputs.make_workload(lengths, 128, 1024, "bf16", seed=71)
+    X, off = w.X.to(dev), w.offsets.to(dev)
+    P, Wk, Wv = w.P.to(dev), w.Wk.to(dev), w.Wv.to(dev)
+    ws = binding.forward(X, off, P, Wk, Wv)["_ws"]
+    g, out = _capture(lambda: binding.forward(X, off, P, Wk, Wv, ws=ws))
+    X.copy_(inputs.make_workload(lengths, 128, 1024, "bf16", seed=72).X.to(dev))
+    g.replay()
+    torch.cuda.synchronize()
+    assert binding.device_status(ws) == 0
+    ref = binding.forward(X, off, P, Wk, Wv)
+    for key in ("sketch", "mass", "lse"):
+        assert torch.equal(out[key], ref[key]), key
